@@ -1,0 +1,180 @@
+/*
+ * la.h - C ABI of the retention_scan_b200 library: causal linear attention
+ * with an optional decay, on NVIDIA B200 (sm_100a), one GPU.
+ *
+ * What is computed (per batch b and head h, tokens t = 1..T):
+ *
+ *     S_t = g_t * S_{t-1} + k_t v_t^T          state, [Dk, Dv], fp32
+ *     z_t = g_t * z_{t-1} + k_t                key sum, [Dk], fp32 (normalised only)
+ *     y_t = q_t^T S_t                          unnormalised output
+ *     y_t = (q_t^T S_t) / (q_t^T z_t)          normalised output
+ *
+ * Sources:
+ *   - The recurrence with g = 1, a zero start and the current token included
+ *     in y_t: "CS336 L04 linear attention duality" exercise page (tensortonic),
+ *     problem statement and its three worked examples.
+ *   - g_t as a per-step decay factor, state <- state * factor + value, and
+ *     g = gamma (per-head constant) for retention: Jamie-Stirling/RetNet
+ *     issue 21, "Proposed improvement/collaboration: removing the O(T^2)
+ *     training cost", the cumulative_ema listing and the retention(Q,K,gamma,V)
+ *     listing that follows it.
+ *   - Decays kept as log values so that every factor is exp(x) with x <= 0:
+ *     BlinkDL/RWKV-LM discussion 189, "Numerically stable parallel
+ *     cumsum-based WKV", second bullet (exponentially weighted
+ *     parameterisation).
+ *   - The normaliser QKV / QK1, the carried KV state ("cache") and the carried
+ *     key sum ("Z-state", cum_k, shape [B,H,1,D]): flash-linear-attention
+ *     issue 268, "[Linear Attention] Update fused_recurrent.py for inference
+ *     with nomalization=true", the opening comment and yiyousong's two
+ *     explanations (the cache identity and the cum_k argument), and the reply
+ *     recommending that the Z-state stay separate from the memory state.
+ *
+ * Readings where the pages are silent (each is fixed here, not guessed per
+ * call):
+ *   - g_1 decays the initial state: S_1 = g_1 S_0 + k_1 v_1^T.
+ *   - z decays with the same g_t as S.
+ *   - The denominator has no epsilon: IEEE division.  The caller keeps
+ *     q^T z positive (for instance with the feature map elu(x)+1).
+ *   - Feature maps and the q scale are applied by the caller.
+ *   - out has the dtype of q; state and key sum are always fp32.
+ *
+ * Layouts (all dense, row-major, innermost index last):
+ *   q, k            [B, H, T, Dk]   dtype
+ *   v, out          [B, H, T, Dv]   dtype
+ *   state           [B, H, Dk, Dv]  fp32  (Dv fastest)
+ *   z               [B, H, Dk]      fp32
+ *   decode q, k     [B, H, Dk]      dtype
+ *   decode v, out   [B, H, Dv]      dtype
+ *
+ * Ownership: every pointer is a device pointer owned by the caller.  The
+ * library allocates no device memory, keeps no per-call state and never
+ * prints.  It may be called from several host threads.
+ *
+ * Execution: every entry point enqueues its work on `stream` and returns; a
+ * device-side failure surfaces at the caller's next synchronisation.  A
+ * kernel that gives up waiting on one of its own barriers sets a device
+ * error word, which la_device_error() reads and clears.
+ */
+#ifndef RETENTION_SCAN_B200_LA_H
+#define RETENTION_SCAN_B200_LA_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no
+ * CUDA header.  NULL is the legacy default stream. */
+typedef struct CUstream_st* la_stream_t;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,   /* null required pointer, bad size, misaligned pointer, bad decay kind */
+    LA_ERR_UNSUPPORTED = 2,   /* valid request that this build has no kernel for */
+    LA_ERR_CUDA = 3           /* a CUDA call or kernel launch failed */
+} la_status;
+
+typedef enum {
+    LA_F32 = 0,               /* q, k, v, out are float32 */
+    LA_BF16 = 1               /* q, k, v, out are bfloat16 */
+} la_dtype;
+
+typedef enum {
+    LA_DECAY_NONE = 0,        /* g = 1: plain linear attention; log_g ignored */
+    LA_DECAY_PER_HEAD = 1,    /* g_t = exp(log_g[h]) for every t; log_g is [H] */
+    LA_DECAY_PER_STEP = 2     /* g_t = exp(log_g[b,h,t]); log_g is [B,H,T] ([B,H] for decode) */
+} la_decay_kind;
+
+/* Decay descriptor.  log_g holds natural logs of the decay factors, finite
+ * and <= 0, fp32, on the device.  A NULL descriptor means LA_DECAY_NONE.
+ * The page's per-head retention decay gamma_h enters as log(gamma_h). */
+typedef struct {
+    int kind;                 /* an la_decay_kind value */
+    const float* log_g;       /* device pointer, see kind for the shape */
+} la_decay;
+
+/*
+ * la_chunk_forward - the whole sequence forward pass.
+ *
+ * Computes out[b,h,t,:] = y_t for t = 1..T from the recurrence above, and
+ * optionally the state and key sum after token T.
+ *
+ *   q, k, v        inputs, layouts above, `dtype`.  Required (for T > 0).
+ *   decay          NULL or a descriptor (see la_decay).
+ *   normalize      0: y_t = q_t^T S_t.  1: y_t = q_t^T S_t / q_t^T z_t.
+ *   init_state     NULL (zeros) or S_0, [B,H,Dk,Dv] fp32.
+ *   init_z         NULL (zeros) or z_0, [B,H,Dk] fp32; read only if normalize.
+ *   out            output y, [B,H,T,Dv], `dtype`.  Required (for T > 0).
+ *   final_state    NULL (not written) or S_T, [B,H,Dk,Dv] fp32.
+ *   final_z        NULL (not written) or z_T, [B,H,Dk] fp32; written only if normalize.
+ *   B, H, T        batch, heads, tokens; each >= 0.  B*H == 0 is a no-op.
+ *                  T == 0 writes final_state = S_0 and final_z = z_0.
+ *   Dk, Dv         key and value widths, >= 1.
+ *   stream         CUDA stream.
+ *
+ * Aliasing: outputs must not overlap inputs; final_state must not overlap
+ * init_state, nor final_z init_z.
+ *
+ * Errors (returned synchronously, nothing is enqueued):
+ *   LA_ERR_INVALID_ARG  a required pointer is NULL; a size is negative or
+ *                       Dk, Dv < 1; a pointer is not 16-byte aligned; decay
+ *                       kind out of range or its log_g NULL; normalize with
+ *                       init_state given but init_z NULL (a carried state
+ *                       without its key sum gives a wrong denominator: the
+ *                       defect described in flash-linear-attention issue 268).
+ *   LA_ERR_UNSUPPORTED  LA_F32 with Dk or Dv > 128; LA_BF16 with Dk or Dv not
+ *                       in {16, 32, 64, 128}.
+ *   LA_ERR_CUDA         a launch or CUDA runtime call failed.
+ *
+ * bf16 runs on tcgen05 tensor cores with fp32 accumulation (chunks of 128
+ * tokens); fp32 runs a recurrent kernel on fp32 FMA units (no TF32).
+ */
+la_status la_chunk_forward(const void* q, const void* k, const void* v,
+                           const la_decay* decay, int normalize,
+                           const float* init_state, const float* init_z,
+                           void* out, float* final_state, float* final_z,
+                           int B, int H, int T, int Dk, int Dv,
+                           la_dtype dtype, la_stream_t stream);
+
+/*
+ * la_decode_step - one token of the recurrence, state updated in place.
+ *
+ *   S <- g S + k v^T;  z <- g z + k (if normalize);  out = q^T S  (/ q^T z).
+ *
+ * This is the token-by-token inference path that carries the KV state and,
+ * with normalisation, the key sum between calls (flash-linear-attention
+ * issue 268: the generation case where only the last token is passed).
+ *
+ *   q, k           [B,H,Dk], `dtype`.  v, out: [B,H,Dv], `dtype`.
+ *   decay          NULL, LA_DECAY_PER_HEAD (log_g [H]) or LA_DECAY_PER_STEP
+ *                  (log_g [B,H], this token's decay).
+ *   state          [B,H,Dk,Dv] fp32, read and written in place.  Required.
+ *   z              [B,H,Dk] fp32, read and written in place.  Required if
+ *                  normalize, ignored otherwise.
+ *
+ * Errors as for la_chunk_forward; LA_ERR_UNSUPPORTED if Dk or Dv > 128.
+ */
+la_status la_decode_step(const void* q, const void* k, const void* v,
+                         const la_decay* decay, int normalize,
+                         float* state, float* z, void* out,
+                         int B, int H, int Dk, int Dv,
+                         la_dtype dtype, la_stream_t stream);
+
+/* A static string naming a status code. */
+const char* la_status_string(la_status status);
+
+/*
+ * la_device_error - reads and clears the device error word of the current
+ * device.  *code receives 0 if no kernel of this library gave up since the
+ * last call, else a nonzero code naming the wait that timed out.  Synchronises
+ * with `stream` first.  Returns LA_ERR_CUDA if that fails.
+ */
+la_status la_device_error(int* code, la_stream_t stream);
+
+/* Library version, "MAJOR.MINOR.PATCH". */
+const char* la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_SCAN_B200_LA_H */

@@ -1,0 +1,113 @@
+"""The oracle: float64 CPU implementations of causal linear attention.
+
+TEST INFRASTRUCTURE.  Only tests/, __graft_entry__.smoke() and bench.py's
+cpu_baseline / reference legs may import this package.  The CUDA library
+(retention_scan_b200) never imports it and shares no code with it.
+
+  forward(...)           recurrent definition, plain C (la_ref.c), token by token
+  decode_step(...)       one token of the same recurrence, in place
+  parallel_forward(...)  brute-force O(T^2) parallel form, numpy (parallel.py)
+
+Every array argument is converted to contiguous float64; bf16 and fp32
+inputs up-cast exactly, so the oracle reads the same input bits as the GPU.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+from .parallel import parallel_forward  # noqa: F401
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "la_ref.c")
+_LIB_PATH = os.path.join(_HERE, "liblaref.so")
+_libs = {}
+
+DECAY_KINDS = {None: 0, "none": 0, "per_head": 1, "per_step": 2}
+
+
+def build(force=False):
+    """Compile la_ref.c into liblaref.so beside it (gcc -O2, pthreads)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load_library(path=None):
+    """ctypes handle of the compiled oracle (default: liblaref.so, built on
+    demand).  Tests pass another path to load a deliberately broken copy."""
+    path = build() if path is None else path
+    if path not in _libs:
+        lib = ctypes.CDLL(path)
+        d = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        lib.la_ref_forward.argtypes = [d, d, d, i, d, i, d, d, d, d, d, i, i, i, i, i, i]
+        lib.la_ref_forward.restype = i
+        lib.la_ref_decode_step.argtypes = [d, d, d, i, d, i, d, d, d, i, i, i, i]
+        lib.la_ref_decode_step.restype = i
+        _libs[path] = lib
+    return _libs[path]
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor: exact up-cast on the CPU
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _kind(decay_kind):
+    return DECAY_KINDS[decay_kind] if not isinstance(decay_kind, int) else decay_kind
+
+
+def forward(q, k, v, decay_kind=0, log_g=None, normalize=False,
+            init_state=None, init_z=None, nthreads=None, lib=None):
+    """Recurrent float64 forward.  Shapes as in include/la.h.
+
+    Returns (y [B,H,T,Dv], final_state [B,H,Dk,Dv], final_z [B,H,Dk]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    log_g, init_state, init_z = _f64(log_g), _f64(init_state), _f64(init_z)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    y = np.zeros((B, H, T, Dv))
+    S = np.zeros((B, H, Dk, Dv))
+    z = np.zeros((B, H, Dk))
+    nt = nthreads if nthreads else (os.cpu_count() or 1)
+    rc = (lib or load_library()).la_ref_forward(_ptr(q), _ptr(k), _ptr(v), _kind(decay_kind), _ptr(log_g),
+                                int(bool(normalize)), _ptr(init_state), _ptr(init_z),
+                                _ptr(y), _ptr(S), _ptr(z), B, H, T, Dk, Dv, nt)
+    if rc != 0:
+        raise ValueError("la_ref_forward rejected its arguments")
+    if not normalize:
+        z = None
+    return y, S, z
+
+
+def decode_step(q, k, v, state, z=None, decay_kind=0, log_g=None, normalize=False, lib=None):
+    """One token; q, k [B,H,Dk], v [B,H,Dv].  Returns (y, new_state, new_z)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    log_g = _f64(log_g)
+    state = _f64(state).copy()
+    z = _f64(z).copy() if z is not None else None
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    y = np.zeros((B, H, Dv))
+    rc = (lib or load_library()).la_ref_decode_step(_ptr(q), _ptr(k), _ptr(v), _kind(decay_kind), _ptr(log_g),
+                                    int(bool(normalize)), _ptr(state), _ptr(z), _ptr(y),
+                                    B, H, Dk, Dv)
+    if rc != 0:
+        raise ValueError("la_ref_decode_step rejected its arguments")
+    return y, state, z

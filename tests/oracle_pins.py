@@ -1,0 +1,295 @@
+"""Pins of the oracle: checks that tie it to the pages and to mathematics, not
+to itself.  Each check takes the oracle's forward / decode callables, so the
+same checks run against the real oracle (test_oracle_pins.py) and against
+deliberately broken copies of it (test_oracle_mutants.py).
+
+What pins what:
+  worked_examples      exact values printed on the tensortonic "CS336 L04
+                       linear attention duality" page (golden fixture)
+  parallel_form        the O(T^2) (Q K^T * D) V form of RetNet issue 21 via
+                       numpy matmuls, all decay kinds, normaliser, carried state
+  cumsum_form          g = 1: S_t is the prefix sum of k_s v_s^T (numpy cumsum)
+  t1_closed_form       T = 1: y = (q.k) v + g q^T S_0
+  t2_closed_form       T = 2 written out by hand
+  one_hot_keys         k_t = e_{i_t}: row i of S_T is a decayed sum of v's,
+                       decay written as explicit products of g's
+  zero_keys            k = 0: y_t = (prod_{r<=t} g_r) q_t^T S_0
+  scalar_powers        Dk = Dv = 1, constant gamma: sum of gamma^(t-s) k_s v_s
+                       with integer powers
+  normaliser_unity     Dv = 1, v = 1, S_0 = z_0: y = 1 exactly
+  normaliser_scale     normalised output is invariant to scaling q
+  split_carry          run(T) == run(T1) -> carry (S, z) -> run(T - T1)
+                       (flash-linear-attention issue 268: cache and Z-state)
+  ema_operator         segment summaries folded with RetNet issue 21's
+                       (xa, fa) o (xb, fb) = (xa fb + xb, fa fb) in random
+                       bracketings equal the full run's final state
+  decode_matches       decode step == forward with T = 1; n steps == forward
+                       over n tokens; page example 1 through decode
+"""
+import json
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                      "linear_attention_duality_examples.json")
+TOL = 1e-11
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} (scale {scale:.3e})"
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def _log_g(rng, kind, B, H, T):
+    if kind == 0:
+        return None
+    if kind == 1:
+        return np.log(rng.uniform(0.5, 0.99, size=H))
+    return np.log(rng.uniform(0.5, 1.0, size=(B, H, T)))
+
+
+def _positive(rng, *shape):
+    x = rng.standard_normal(shape)
+    return np.where(x > 0, x + 1.0, np.exp(x))  # elu(x) + 1
+
+
+# -- checks ---------------------------------------------------------------
+
+def worked_examples(fwd, dec):
+    ex = json.load(open(GOLDEN))["examples"]
+    for e in ex:
+        q = np.array(e["q"], np.float64)[:, None]  # (B,S,D) -> (B,1,S,D)
+        k = np.array(e["k"], np.float64)[:, None]
+        v = np.array(e["v"], np.float64)[:, None]
+        y, S, _ = fwd(q, k, v)
+        _close(y[:, 0], e["output"], 0.0, e["name"] + " output")
+        _close(S[:, 0], e["final_state"], 0.0, e["name"] + " final_state")
+    # example 1 token by token: the state is 6 then 36
+    e = ex[0]
+    q = np.array(e["q"], np.float64)[:, None]
+    k = np.array(e["k"], np.float64)[:, None]
+    v = np.array(e["v"], np.float64)[:, None]
+    S = np.zeros((1, 1, 1, 1))
+    for t, want in enumerate(e["states_after_each_token"]):
+        y, S, _ = dec(q[:, :, t], k[:, :, t], v[:, :, t], S)
+        _close(S.reshape(()), want, 0.0, "example 1 state after token")
+        _close(y.reshape(()), np.array(e["output"]).reshape(-1)[t], 0.0, "example 1 decode output")
+
+
+def parallel_form(fwd, dec, parallel):
+    rng = np.random.default_rng(11)
+    for kind in (0, 1, 2):
+        for normalize in (False, True):
+            for with_init in (False, True):
+                B, H, T, Dk, Dv = 2, 3, 37, 5, 4
+                if normalize:
+                    q, k = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk)
+                else:
+                    q, k = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk)
+                v = _rand(rng, B, H, T, Dv)
+                lg = _log_g(rng, kind, B, H, T)
+                S0 = _rand(rng, B, H, Dk, Dv) if with_init else None
+                z0 = np.abs(_rand(rng, B, H, Dk)) if (with_init and normalize) else None
+                y, S, z = fwd(q, k, v, kind, lg, normalize, S0, z0)
+                yp, Sp, zp = parallel(q, k, v, kind, lg, normalize, S0, z0)
+                tag = f"kind={kind} norm={normalize} init={with_init}"
+                _close(y, yp, 1e-10, "parallel y " + tag)
+                _close(S, Sp, 1e-10, "parallel S " + tag)
+                if normalize:
+                    _close(z, zp, 1e-10, "parallel z " + tag)
+
+
+def cumsum_form(fwd, dec):
+    rng = np.random.default_rng(12)
+    B, H, T, Dk, Dv = 1, 2, 23, 3, 4
+    q, k, v = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dv)
+    y, S, _ = fwd(q, k, v)
+    outer = k[..., :, None] * v[..., None, :]          # [B,H,T,Dk,Dv]
+    states = np.cumsum(outer, axis=2)
+    _close(y, np.einsum("bhti,bhtij->bhtj", q, states), TOL, "cumsum y")
+    _close(S, states[:, :, -1], TOL, "cumsum final state")
+
+
+def t1_closed_form(fwd, dec):
+    rng = np.random.default_rng(13)
+    Dk, Dv = 4, 3
+    q, k, v = _rand(rng, 1, 1, 1, Dk), _rand(rng, 1, 1, 1, Dk), _rand(rng, 1, 1, 1, Dv)
+    S0 = _rand(rng, 1, 1, Dk, Dv)
+    g = 0.7
+    y, S, _ = fwd(q, k, v, 1, np.array([np.log(g)]), False, S0)
+    qv, kv, vv, S0v = q[0, 0, 0], k[0, 0, 0], v[0, 0, 0], S0[0, 0]
+    _close(y[0, 0, 0], (qv @ kv) * vv + g * (qv @ S0v), TOL, "T=1 output")
+    _close(S[0, 0], g * S0v + np.outer(kv, vv), TOL, "T=1 state")
+
+
+def t2_closed_form(fwd, dec):
+    rng = np.random.default_rng(14)
+    Dk, Dv = 3, 2
+    q, k, v = _rand(rng, 1, 1, 2, Dk), _rand(rng, 1, 1, 2, Dk), _rand(rng, 1, 1, 2, Dv)
+    S0 = _rand(rng, 1, 1, Dk, Dv)
+    z0 = np.abs(_rand(rng, 1, 1, Dk))
+    g1, g2 = 0.9, 0.6
+    lg = np.log(np.array([g1, g2]))[None, None]
+    q1, q2 = q[0, 0]
+    k1, k2 = k[0, 0]
+    v1, v2 = v[0, 0]
+    S0v, z0v = S0[0, 0], z0[0, 0]
+    y, S, _ = fwd(q, k, v, 2, lg, False, S0)
+    y1 = g1 * (q1 @ S0v) + (q1 @ k1) * v1
+    y2 = g1 * g2 * (q2 @ S0v) + g2 * (q2 @ k1) * v1 + (q2 @ k2) * v2
+    _close(y[0, 0, 0], y1, TOL, "T=2 y1")
+    _close(y[0, 0, 1], y2, TOL, "T=2 y2")
+    _close(S[0, 0], g1 * g2 * S0v + g2 * np.outer(k1, v1) + np.outer(k2, v2), TOL, "T=2 state")
+    qp, kp = np.abs(q) + 0.1, np.abs(k) + 0.1
+    q1, q2 = qp[0, 0]
+    k1, k2 = kp[0, 0]
+    y, S, z = fwd(qp, kp, v, 2, lg, True, S0, z0)
+    d2 = g1 * g2 * (q2 @ z0v) + g2 * (q2 @ k1) + (q2 @ k2)
+    n2 = g1 * g2 * (q2 @ S0v) + g2 * (q2 @ k1) * v1 + (q2 @ k2) * v2
+    _close(y[0, 0, 1], n2 / d2, TOL, "T=2 normalised y2")
+    _close(z[0, 0], g1 * g2 * z0v + g2 * k1 + k2, TOL, "T=2 key sum")
+
+
+def one_hot_keys(fwd, dec):
+    rng = np.random.default_rng(15)
+    T, Dk, Dv = 17, 4, 3
+    idx = rng.integers(0, Dk, size=T)
+    k = np.zeros((1, 1, T, Dk))
+    k[0, 0, np.arange(T), idx] = 1.0
+    q, v = _rand(rng, 1, 1, T, Dk), _rand(rng, 1, 1, T, Dv)
+    g = rng.uniform(0.5, 1.0, size=T)
+    y, S, _ = fwd(q, k, v, 2, np.log(g)[None, None])
+    want = np.zeros((Dk, Dv))
+    for t in range(T):
+        want[idx[t]] += np.prod(g[t + 1:]) * v[0, 0, t]
+    _close(S[0, 0], want, TOL, "one-hot keys state")
+
+
+def zero_keys(fwd, dec):
+    rng = np.random.default_rng(16)
+    T, Dk, Dv = 9, 3, 5
+    q, v = _rand(rng, 1, 1, T, Dk), _rand(rng, 1, 1, T, Dv)
+    k = np.zeros((1, 1, T, Dk))
+    S0 = _rand(rng, 1, 1, Dk, Dv)
+    g = rng.uniform(0.3, 1.0, size=T)
+    y, S, _ = fwd(q, k, v, 2, np.log(g)[None, None], False, S0)
+    for t in range(T):
+        _close(y[0, 0, t], np.prod(g[:t + 1]) * (q[0, 0, t] @ S0[0, 0]), TOL, "zero keys y")
+
+
+def scalar_powers(fwd, dec):
+    rng = np.random.default_rng(17)
+    T, gamma = 25, 0.85
+    q, k, v = _rand(rng, 1, 1, T, 1), _rand(rng, 1, 1, T, 1), _rand(rng, 1, 1, T, 1)
+    S0 = _rand(rng, 1, 1, 1, 1)
+    y, S, _ = fwd(q, k, v, 1, np.array([np.log(gamma)]), False, S0)
+    kk, vv, qq, s0 = k[0, 0, :, 0], v[0, 0, :, 0], q[0, 0, :, 0], S0.item()
+    for t in range(T):
+        st = sum(gamma ** (t - s) * kk[s] * vv[s] for s in range(t + 1)) + gamma ** (t + 1) * s0
+        _close(y[0, 0, t, 0], qq[t] * st, TOL, "scalar EMA y")
+
+
+def normaliser_unity(fwd, dec):
+    rng = np.random.default_rng(18)
+    for kind in (0, 1, 2):
+        B, H, T, Dk = 1, 2, 31, 6
+        q, k = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk)
+        v = np.ones((B, H, T, 1))
+        z0 = np.abs(_rand(rng, B, H, Dk))
+        lg = _log_g(rng, kind, B, H, T)
+        y, S, z = fwd(q, k, v, kind, lg, True, z0[..., None], z0)
+        _close(y, np.ones_like(y), 1e-13, f"v=1 gives y=1 (kind {kind})")
+        _close(S[..., 0], z, 1e-13, f"v=1 state equals key sum (kind {kind})")
+
+
+def normaliser_scale(fwd, dec):
+    rng = np.random.default_rng(19)
+    B, H, T, Dk, Dv = 1, 2, 13, 4, 3
+    q, k, v = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk), _rand(rng, B, H, T, Dv)
+    y1, _, _ = fwd(q, k, v, 0, None, True)
+    y2, _, _ = fwd(q * 8.0, k, v, 0, None, True)
+    _close(y1, y2, 1e-13, "normalised output invariant to q scale")
+    y3, _, _ = fwd(q, k, v, 0, None, False)
+    assert np.max(np.abs(y3 - y1)) > 1e-3, "normalize flag has no effect"
+
+
+def split_carry(fwd, dec):
+    rng = np.random.default_rng(20)
+    for kind in (0, 1, 2):
+        for normalize in (False, True):
+            B, H, T, Dk, Dv, T1 = 2, 2, 29, 4, 3, 11
+            q, k = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk)
+            v = _rand(rng, B, H, T, Dv)
+            lg = _log_g(rng, kind, B, H, T)
+            lg1 = lg[..., :T1] if kind == 2 else lg
+            lg2 = lg[..., T1:] if kind == 2 else lg
+            y, S, z = fwd(q, k, v, kind, lg, normalize)
+            ya, Sa, za = fwd(q[:, :, :T1], k[:, :, :T1], v[:, :, :T1], kind, lg1, normalize)
+            yb, Sb, zb = fwd(q[:, :, T1:], k[:, :, T1:], v[:, :, T1:], kind, lg2, normalize, Sa, za)
+            tag = f"kind={kind} norm={normalize}"
+            _close(np.concatenate([ya, yb], axis=2), y, 1e-12, "split y " + tag)
+            _close(Sb, S, 1e-12, "split S " + tag)
+            if normalize:
+                _close(zb, z, 1e-12, "split z " + tag)
+
+
+def ema_operator(fwd, dec):
+    rng = np.random.default_rng(21)
+    T, Dk, Dv, nseg = 40, 3, 2, 5
+    q, k, v = _rand(rng, 1, 1, T, Dk), _rand(rng, 1, 1, T, Dk), _rand(rng, 1, 1, T, Dv)
+    lg = np.log(rng.uniform(0.6, 1.0, size=(1, 1, T)))
+    _, S_full, _ = fwd(q, k, v, 2, lg)
+    cuts = np.sort(rng.choice(np.arange(1, T), size=nseg - 1, replace=False))
+    bounds = [0, *cuts.tolist(), T]
+    segs = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        _, Sx, _ = fwd(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], 2, lg[..., a:b])
+        segs.append((Sx[0, 0], float(np.exp(lg[0, 0, a:b].sum()))))
+
+    def op(x, y):  # (xa, fa) o (xb, fb) = (xa * fb + xb, fa * fb)
+        return (x[0] * y[1] + y[0], x[1] * y[1])
+
+    def fold(items):  # a random bracketing of the ordered sequence
+        if len(items) == 1:
+            return items[0]
+        m = int(rng.integers(1, len(items)))
+        return op(fold(items[:m]), fold(items[m:]))
+
+    for _ in range(4):
+        Sx, _ = fold(segs)
+        _close(Sx, S_full[0, 0], 1e-12, "EMA operator bracketing")
+
+
+def decode_matches(fwd, dec):
+    rng = np.random.default_rng(22)
+    for kind in (0, 1, 2):
+        for normalize in (False, True):
+            B, H, n, Dk, Dv = 2, 3, 7, 4, 5
+            q, k = _positive(rng, B, H, n, Dk), _positive(rng, B, H, n, Dk)
+            v = _rand(rng, B, H, n, Dv)
+            S0 = _rand(rng, B, H, Dk, Dv)
+            z0 = np.abs(_rand(rng, B, H, Dk)) if normalize else None
+            lg = _log_g(rng, kind, B, H, n)
+            y, S, z = fwd(q, k, v, kind, lg, normalize, S0, z0)
+            St, zt = S0, z0
+            for t in range(n):
+                lgt = lg[..., t] if kind == 2 else lg
+                yt, St, zt = dec(q[:, :, t], k[:, :, t], v[:, :, t], St, zt, kind, lgt, normalize)
+                _close(yt, y[:, :, t], 1e-12, f"decode step {t} kind={kind} norm={normalize}")
+            _close(St, S, 1e-12, "decode final state")
+            if normalize:
+                _close(zt, z, 1e-12, "decode final key sum")
+
+
+ALL = [worked_examples, cumsum_form, t1_closed_form, t2_closed_form, one_hot_keys,
+       zero_keys, scalar_powers, normaliser_unity, normaliser_scale, split_carry,
+       ema_operator, decode_matches]
