@@ -1,0 +1,492 @@
+"""Benchmark of the causal-linear-attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of the workload:
+
+  config 2 (default): retention, per-head gamma_h = 1 - 2^(-5-h), bf16,
+      B=4, H=8, T=2048, Dk=Dv=64 -> one la_chunk_forward call
+  config 1: plain linear attention, fp32, B=1, H=1, T=64, D=16
+  config 3: normalised, elu+1 feature map, carried state, B=8, H=16, T=4096, D=128
+  config 4: gated per-step decay, B=1, H=32, T=65536, D=128
+  config 5: decode, B=256, H=32, D=128, normalised, 1024 la_decode_step calls
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
+buffer before every step whose inputs fit in L2, outside the events.  A
+barrier and a device synchronisation bracket the timed region; the time is
+the maximum over ranks.  Under torchrun every rank runs the same per-GPU
+workload (weak scaling, no collective on the data path).
+
+Extra keys: roofline (dominant kernel, algorithmic bytes / event time against
+the measured HBM copy bandwidth), e2e (the same metric through the public API
+with pinned host buffers and the host<->device copies inside the timed
+region), clocks (nvidia-smi sampled during the timed region), cpu_baseline
+(the float64 oracle on the host cores, a bounded sample, rank 0 at N=1).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "linear-attn forward tokens/s (B·H·T/s) and % of roofline (tensor TFLOP/s or HBM GB/s)"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 512 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- workload accounting
+
+def algorithmic_bytes(wl, cfg):
+    """Bytes the hot path must move once: inputs read, outputs written, state
+    in/out (fp32), decays; per launch of the dominant kernel."""
+    es = 4 if wl.dtype == "f32" else 2
+    if cfg == 5:
+        per_bh = 2 * 4 * wl.Dk * wl.Dv + 2 * 4 * wl.Dk + (2 * wl.Dk + wl.Dv) * es + wl.Dv * es
+        return wl.B * wl.H * per_bh  # per decode call
+    BH, T = wl.B * wl.H, wl.T
+    b = BH * T * ((2 * wl.Dk + wl.Dv) * es + wl.Dv * es)
+    if wl.decay == "per_step":
+        b += BH * T * 4
+    b += BH * wl.Dk * wl.Dv * 4  # final state written
+    if wl.prefix_T:
+        b += BH * wl.Dk * wl.Dv * 4 + 2 * BH * wl.Dk * 4  # initial state, key sums in and out
+    return b
+
+
+def algorithmic_flops(wl, cfg):
+    n = wl.B * wl.H * (1 if cfg == 5 else wl.T)
+    return 4 * wl.Dk * wl.Dv * n
+
+
+def tokens_per_step(wl, cfg):
+    return wl.B * wl.H * (wl.steps if cfg == 5 else wl.T)
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "retention_scan_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload_name):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(workload_name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_sha") != kernel_source_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 100 ms; keeps (wall time, row) pairs."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = bus_id.lower()
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        mine = [r for (t, r) in self.rows if r and r[0].lower().endswith(self.bus_id[-12:])]
+        window = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15
+                  and r and r[0].lower().endswith(self.bus_id[-12:])]
+        use = window or mine[-5:]
+        if not use:
+            return None
+
+        def num(x):
+            try:
+                return float(x.split()[0])
+            except (ValueError, IndexError):
+                return float("nan")
+        sm = [num(r[1]) for r in use if len(r) > 1]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in use for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(num(r[2]) for r in use if len(r) > 2),
+                "reasons": reasons, "samples": len(use), "in_window": bool(window)}
+
+
+def bus_id_of(device):
+    p = torch.cuda.get_device_properties(device)
+    try:
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except AttributeError:
+        return ""
+
+
+# ---------------------------------------------------------------- our arm
+
+class Job:
+    """Device-resident inputs and the step function of one workload."""
+
+    def __init__(self, cfg, device):
+        import retention_scan_b200 as la
+        self.la = la
+        self.cfg = cfg
+        self.wl = wl = W.WORKLOADS[cfg]
+        self.dev = device
+        if cfg == 5:
+            S0, z0 = W.decode_initial_state(wl)
+            self.S0, self.z0 = S0.to(device), z0.to(device)
+            self.S, self.z = self.S0.clone(), self.z0.clone()
+            self.q, self.k, self.v = W.decode_pool_device(wl, wl.steps, device)
+            self.log_g = W.per_head_log_gamma(wl.H).to(device)
+            self.out = torch.empty(wl.B, wl.H, wl.Dv, dtype=wl.torch_dtype, device=device)
+            return
+        inp = W.forward_inputs(wl)
+        self.host = inp
+        self.q, self.k, self.v = (inp[n].to(device) for n in ("q", "k", "v"))
+        self.kind = inp["decay_kind"]
+        self.log_g = inp["log_g"].to(device) if inp["log_g"] is not None else None
+        self.out = torch.empty(wl.B, wl.H, wl.T, wl.Dv, dtype=wl.torch_dtype, device=device)
+        self.S = torch.empty(wl.B, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=device)
+        self.z = torch.empty(wl.B, wl.H, wl.Dk, dtype=torch.float32, device=device) if wl.normalize else None
+        self.S0 = self.z0 = None
+        if wl.prefix_T:
+            # carried state of the workload: the library's own forward over the seeded prefix
+            pre = W.prefix_inputs(wl)
+            _, self.S0, self.z0 = la.chunk_forward(pre["q"].to(device), pre["k"].to(device),
+                                                   pre["v"].to(device), pre["decay_kind"], None, True)
+
+    def step(self):
+        la, wl = self.la, self.wl
+        if self.cfg == 5:
+            for t in range(wl.steps):
+                la.decode_step(self.q[t], self.k[t], self.v[t], self.S, self.z, 1, self.log_g, True,
+                               out=self.out)
+            return wl.steps
+        la.chunk_forward(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
+                         out=self.out, final_state=self.S, final_z=self.z)
+        return 1
+
+    E2E_DECODE_TOKENS = 64
+
+    def e2e_step(self, pinned, stream):
+        """Public API with host buffers: copy this step's inputs in, run, read
+        the result back.  Returns the tokens processed."""
+        la, wl = self.la, self.wl
+        if self.cfg == 5:
+            for t in range(self.E2E_DECODE_TOKENS):
+                q = pinned["q"][t].to(self.dev, non_blocking=True)
+                k = pinned["k"][t].to(self.dev, non_blocking=True)
+                v = pinned["v"][t].to(self.dev, non_blocking=True)
+                y = la.decode_step(q, k, v, self.S, self.z, 1, self.log_g, True, out=self.out)
+                pinned["y"][t].copy_(y, non_blocking=True)
+            return wl.B * wl.H * self.E2E_DECODE_TOKENS
+        q, k, v = (pinned[n].to(self.dev, non_blocking=True) for n in ("q", "k", "v"))
+        lg = pinned["log_g"].to(self.dev, non_blocking=True) if pinned.get("log_g") is not None else None
+        y, S, _ = la.chunk_forward(q, k, v, self.kind, lg, wl.normalize, self.S0, self.z0,
+                                   out=self.out, final_state=self.S, final_z=self.z)
+        pinned["y"].copy_(y, non_blocking=True)
+        pinned["S"].copy_(S, non_blocking=True)
+        return tokens_per_step(wl, self.cfg)
+
+    def make_pinned(self):
+        wl = self.wl
+        if self.cfg == 5:
+            n_tok = self.E2E_DECODE_TOKENS
+            p = {n: getattr(self, n)[:n_tok].cpu().pin_memory() for n in ("q", "k", "v")}
+            p["y"] = torch.empty(n_tok, wl.B, wl.H, wl.Dv, dtype=wl.torch_dtype).pin_memory()
+            h2d = sum(p[n].numel() * p[n].element_size() for n in ("q", "k", "v"))
+            d2h = p["y"].numel() * p["y"].element_size()
+            return p, h2d, d2h
+        p = {n: self.host[n].pin_memory() for n in ("q", "k", "v")}
+        p["log_g"] = self.host["log_g"].pin_memory() if self.host["log_g"] is not None else None
+        p["y"] = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        p["S"] = torch.empty(self.S.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(p[n].numel() * p[n].element_size() for n in ("q", "k", "v", "log_g") if p[n] is not None)
+        d2h = p["y"].numel() * p["y"].element_size() + p["S"].numel() * 4
+        return p, h2d, d2h
+
+
+def barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, dist_on, device):
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(job, steps, flush, dist_on, device):
+    """Sum of per-step CUDA-event times (ms) over `steps` steps; L2 flushed
+    before each step outside the events when `flush` is not None."""
+    stream = torch.cuda.current_stream(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    barrier(dist_on)
+    wall0 = time.time()
+    for i in range(steps):
+        if flush is not None:
+            flush.add_(1)
+        starts[i].record(stream)
+        launches += job.step()
+        ends[i].record(stream)
+    barrier(dist_on)
+    wall1 = time.time()
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return per, launches, wall0, wall1
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    """The float64 oracle, as it stands, on a bounded sample of the workload:
+    whole (b, h) sequences (every token) until about budget_s of CPU work."""
+    import oracle
+    wl = W.WORKLOADS[cfg]
+    oracle.build()
+    cores = os.cpu_count() or 1
+    if cfg == 5:
+        # a sample of heads for a sample of decode tokens
+        nh = min(wl.B * wl.H, 64 * cores)
+        heads = list(range(nh))
+        S, z = W.decode_initial_state(wl, heads=heads)
+        S, z = S.double().numpy(), z.double().numpy()
+        inps = [W.decode_step_inputs(wl, s, heads=heads) for s in range(4)]
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            inp = inps[n % len(inps)]
+            _, S, z = oracle.decode_step(inp["q"], inp["k"], inp["v"], S, z, 1, inp["log_g"], True)
+            n += 1
+            if time.perf_counter() - t0 > budget_s / 2:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": nh * n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"{nh} of {wl.B * wl.H} (b,h) states, {n} decode tokens, single thread"}
+    total = wl.B * wl.H
+    # estimate: ~1 GFLOP/s per core for the plain f64 loops
+    per_head_s = 4.0 * wl.Dk * wl.Dv * (wl.T + wl.prefix_T) / 1e9
+    nh = max(1, min(total, int(budget_s * cores / max(per_head_s, 1e-9))))
+    nh = min(nh, total)
+    heads = list(range(nh))
+    inp = W.forward_inputs(wl, heads=heads)
+    threads = min(cores, nh)
+    init = {}
+    if wl.prefix_T:
+        pre = W.prefix_inputs(wl, heads=heads)
+        _, S0, z0 = oracle.forward(pre["q"], pre["k"], pre["v"], 0, None, True, nthreads=threads)
+        init = dict(init_state=S0, init_z=z0)
+    t0 = time.perf_counter()
+    oracle.forward(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize,
+                   nthreads=threads, **init)
+    dt = time.perf_counter() - t0
+    return {"value": nh * wl.T / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nh} of {total} (b,h) sequences, all {wl.T} tokens each, {threads} threads"}
+
+
+def run_ours(args, rank, world, dist_on, device):
+    cfg = args.config
+    wl = W.WORKLOADS[cfg]
+    job = Job(cfg, device)
+    torch.cuda.synchronize()
+    in_bytes = algorithmic_bytes(wl, cfg) * (wl.steps if cfg == 5 else 1)
+    flush = None
+    if in_bytes < 2 * L2_BYTES and cfg != 5:
+        flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.add_(1)
+        job.step()
+    torch.cuda.synchronize()
+    assert job.la.device_error(device) == 0
+
+    sampler = ClockSampler(bus_id_of(device)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    per, launches, w0, w1 = time_steps(job, args.steps, flush, dist_on, device)
+    if sampler:
+        time.sleep(0.3)
+        sampler.stop()
+    assert job.la.device_error(device) == 0
+    total_ms = max_over_ranks(sum(per), dist_on, device)
+    ms_per_step = total_ms / args.steps
+    tokens = tokens_per_step(wl, cfg) * world
+    value = tokens / (ms_per_step / 1e3)
+
+    # dominant kernel: average duration of one launch (decode: one call)
+    launch_ms = ms_per_step / (wl.steps if cfg == 5 else 1)
+    pk, pk_kind = peaks()
+    bytes_launch = algorithmic_bytes(wl, cfg)
+    achieved_gbs = bytes_launch / (launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved_gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
+                "peak_source": pk_kind,
+                "kernel": "la_decode (decode_vec_kernel)" if cfg == 5 else
+                ("la_fwd_f32 (fwd_f32_kernel)" if wl.dtype == "f32" else "la_fwd_tc (fwd_tc_kernel)"),
+                "algorithmic_bytes_per_launch": bytes_launch,
+                "tensor_frac": round(algorithmic_flops(wl, cfg) / (launch_ms / 1e3) / 1e12 / pk.get("bf16_tflops", 1590.0), 4)}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        pinned, h2d, d2h = job.make_pinned()
+        stream = torch.cuda.current_stream(device)
+        e_steps = max(1, min(args.steps, 20))
+        for _ in range(2):
+            job.e2e_step(pinned, stream)
+        barrier(dist_on)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        e_tokens = 0
+        for _ in range(e_steps):
+            e_tokens += job.e2e_step(pinned, stream)
+        ev1.record(stream)
+        barrier(dist_on)
+        e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist_on, device) / e_steps
+        e2e = {"value": e_tokens / e_steps * world / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
+
+    clocks = sampler.summary(w0, w1) if sampler else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if wl.dtype == "f32" else "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
+                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
+                   "decode_steps": wl.steps if cfg == 5 else None,
+                   "l2": "flushed before every step (512 MB write)" if flush is not None
+                   else "inputs larger than L2",
+                   "parallelism": f"replicas x{world}, (b,h) split across CTAs"},
+        "roofline": roofline, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": launches,
+    }
+    return line
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    cfg = args.config
+    wl = W.WORKLOADS[cfg]
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, budget_s=2.0)
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(cfg, budget_s=8.0))
+    v = statistics.median(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tokens_per_step(wl, cfg) / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
+                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize},
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    args = ap.parse_args()
+    default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3}
+    if args.steps is None:
+        args.steps = default_steps[args.config] if args.impl == "ours" else 3
+    if args.warmup is None:
+        args.warmup = max(3, args.steps // 20) if args.impl == "ours" else 1
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=device,
+                                             timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, dist_on, device)
+        if rank == 0:
+            if world == 1 and not args.skip_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args.config)
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist_on:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -58,6 +58,12 @@
 #ifndef RETENTION_SCAN_B200_LA_H
 #define RETENTION_SCAN_B200_LA_H
 
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -128,7 +134,7 @@ typedef struct {
  * bf16 runs on tcgen05 tensor cores with fp32 accumulation (chunks of 128
  * tokens); fp32 runs a recurrent kernel on fp32 FMA units (no TF32).
  */
-la_status la_chunk_forward(const void* q, const void* k, const void* v,
+LA_API la_status la_chunk_forward(const void* q, const void* k, const void* v,
                            const la_decay* decay, int normalize,
                            const float* init_state, const float* init_z,
                            void* out, float* final_state, float* final_z,
@@ -153,14 +159,14 @@ la_status la_chunk_forward(const void* q, const void* k, const void* v,
  *
  * Errors as for la_chunk_forward; LA_ERR_UNSUPPORTED if Dk or Dv > 128.
  */
-la_status la_decode_step(const void* q, const void* k, const void* v,
+LA_API la_status la_decode_step(const void* q, const void* k, const void* v,
                          const la_decay* decay, int normalize,
                          float* state, float* z, void* out,
                          int B, int H, int Dk, int Dv,
                          la_dtype dtype, la_stream_t stream);
 
 /* A static string naming a status code. */
-const char* la_status_string(la_status status);
+LA_API const char* la_status_string(la_status status);
 
 /*
  * la_device_error - reads and clears the device error word of the current
@@ -168,10 +174,10 @@ const char* la_status_string(la_status status);
  * last call, else a nonzero code naming the wait that timed out.  Synchronises
  * with `stream` first.  Returns LA_ERR_CUDA if that fails.
  */
-la_status la_device_error(int* code, la_stream_t stream);
+LA_API la_status la_device_error(int* code, la_stream_t stream);
 
 /* Library version, "MAJOR.MINOR.PATCH". */
-const char* la_version(void);
+LA_API const char* la_version(void);
 
 #ifdef __cplusplus
 }

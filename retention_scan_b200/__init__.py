@@ -1,0 +1,192 @@
+"""retention_scan_b200: causal linear attention with an optional decay on B200.
+
+Python binding of the C ABI in include/la.h (libla.so, built in-tree by
+``python -m retention_scan_b200.build``).  This module only marshals
+arguments: it checks shapes and dtypes, allocates outputs with torch when the
+caller does not pass them, and hands raw device pointers and the current CUDA
+stream to the library.  Every step of the computation runs in the library's
+CUDA kernels; there is no fallback.  Importing works without a GPU; calling
+a compute function without the built library or without a CUDA device raises.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["chunk_forward", "decode_step", "device_error", "LAError", "lib", "library_path",
+           "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libla.so")
+
+DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
+LA_F32, LA_BF16 = 0, 1
+EXPORTED_SYMBOLS = ("la_chunk_forward", "la_decode_step", "la_status_string", "la_device_error",
+                    "la_version")
+
+
+class LAError(RuntimeError):
+    """A nonzero la_status from the library."""
+
+    def __init__(self, status, message):
+        super().__init__(message)
+        self.status = status
+
+
+class _Decay(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("log_g", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libla.so (ctypes).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ImportError(f"retention_scan_b200: {library_path} is missing; build it with "
+                              "`python -m retention_scan_b200.build`")
+        L = ctypes.CDLL(library_path)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        L.la_chunk_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, vp, vp,
+                                       i, i, i, i, i, i, vp]
+        L.la_chunk_forward.restype = i
+        L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
+                                     i, i, i, i, i, vp]
+        L.la_decode_step.restype = i
+        L.la_status_string.argtypes = [i]
+        L.la_status_string.restype = ctypes.c_char_p
+        L.la_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
+        L.la_device_error.restype = i
+        L.la_version.argtypes = []
+        L.la_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != 0:
+        raise LAError(status, lib().la_status_string(status).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(dt):
+    if dt == torch.float32:
+        return LA_F32
+    if dt == torch.bfloat16:
+        return LA_BF16
+    raise TypeError(f"q, k, v must be float32 or bfloat16, got {dt}")
+
+
+def _need(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _decay(kind, log_g):
+    if kind == DECAY_NONE:
+        return None
+    if log_g is None:
+        raise ValueError("log_g is required for a per-head or per-step decay")
+    return _Decay(kind, log_g.data_ptr())
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
+                  init_state=None, init_z=None, out=None, final_state=None, final_z=None,
+                  return_final=True, stream=None):
+    """Whole-sequence forward (la_chunk_forward).
+
+    q, k: [B,H,T,Dk]; v: [B,H,T,Dv]; float32 or bfloat16 CUDA tensors.
+    decay_kind: DECAY_NONE, DECAY_PER_HEAD (log_g [H]) or DECAY_PER_STEP
+    (log_g [B,H,T]); log_g is fp32 natural log of the decay factor, <= 0.
+    init_state [B,H,Dk,Dv] / init_z [B,H,Dk]: fp32 carried state and key sum.
+    Returns (out, final_state, final_z); final_* are None unless requested
+    (return_final, or passed in), final_z only when normalize.
+    """
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q.dtype)
+    _need(k, "k", (B, H, T, Dk), q.dtype, dev)
+    _need(v, "v", (B, H, T, Dv), q.dtype, dev)
+    _need(q, "q", (B, H, T, Dk), q.dtype, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H, T), torch.float32, dev)
+    _need(init_state, "init_state", (B, H, Dk, Dv), torch.float32, dev)
+    _need(init_z, "init_z", (B, H, Dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, T, Dv), dtype=q.dtype, device=dev)
+    _need(out, "out", (B, H, T, Dv), q.dtype, dev)
+    if final_state is None and return_final:
+        final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
+    if final_z is None and return_final and normalize:
+        final_z = torch.empty((B, H, Dk), dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (B, H, Dk, Dv), torch.float32, dev)
+    _need(final_z, "final_z", (B, H, Dk), torch.float32, dev)
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        _check(lib().la_chunk_forward(
+            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+            _ptr(init_state), _ptr(init_z), _ptr(out), _ptr(final_state), _ptr(final_z),
+            B, H, T, Dk, Dv, code, _stream(stream, dev)))
+    return out, final_state, (final_z if normalize else None)
+
+
+def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,
+                out=None, stream=None):
+    """One token (la_decode_step); state [B,H,Dk,Dv] and z [B,H,Dk] (fp32) are
+    updated in place.  q, k: [B,H,Dk]; v: [B,H,Dv].  Returns out [B,H,Dv]."""
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q.dtype)
+    _need(k, "k", (B, H, Dk), q.dtype, dev)
+    _need(v, "v", (B, H, Dv), q.dtype, dev)
+    _need(state, "state", (B, H, Dk, Dv), torch.float32, dev)
+    if normalize:
+        if z is None:
+            raise ValueError("z is required when normalize")
+        _need(z, "z", (B, H, Dk), torch.float32, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=q.dtype, device=dev)
+    _need(out, "out", (B, H, Dv), q.dtype, dev)
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        _check(lib().la_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+            _ptr(state), _ptr(z if normalize else None), _ptr(out), B, H, Dk, Dv, code,
+            _stream(stream, dev)))
+    return out
+
+
+def device_error(device=None, stream=None):
+    """Read and clear the library's device error word (0 = no kernel gave up
+    waiting).  Synchronises with the stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    code = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        _check(lib().la_device_error(ctypes.byref(code), _stream(stream, dev)))
+    return code.value

@@ -1,0 +1,198 @@
+// la_api.cu - the C ABI (include/la.h): argument validation, dispatch to the
+// kernels, the device error word.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "la.h"
+#include "la_internal.h"
+
+namespace {
+
+// Set by a kernel that gave up waiting on one of its barriers (kErr* codes).
+__device__ int g_err_word;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int*> g_err_ptr[kMaxDevices];
+
+int* err_word_for_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    int* p = g_err_ptr[dev].load();
+    if (!p) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_err_word) != cudaSuccess) return nullptr;
+        p = static_cast<int*>(addr);
+        g_err_ptr[dev].store(p);
+    }
+    return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Host-side fault injection for tests: LA_FAULT_INJECT=launch makes every
+// compute entry point report a failed launch without enqueuing anything.
+bool launch_fault_injected() {
+    const char* e = std::getenv("LA_FAULT_INJECT");
+    return e && std::strcmp(e, "launch") == 0;
+}
+
+bool fits_int(long long x) { return x >= 0 && x <= INT_MAX; }
+
+la_status check_decay(const la_decay* decay, int* kind, const float** log_g) {
+    *kind = LA_DECAY_NONE;
+    *log_g = nullptr;
+    if (!decay) return LA_OK;
+    if (decay->kind < LA_DECAY_NONE || decay->kind > LA_DECAY_PER_STEP) return LA_ERR_INVALID_ARG;
+    *kind = decay->kind;
+    if (*kind != LA_DECAY_NONE) {
+        if (!decay->log_g || !aligned4(decay->log_g)) return LA_ERR_INVALID_ARG;
+        *log_g = decay->log_g;
+    }
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* la_status_string(la_status status) {
+    switch (status) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: no kernel for this shape or dtype";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: a CUDA call or kernel launch failed";
+    }
+    return "unknown la_status";
+}
+
+const char* la_version(void) { return "0.1.0"; }
+
+la_status la_chunk_forward(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                           const float* init_state, const float* init_z, void* out, float* final_state,
+                           float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                           la_stream_t stream) {
+    if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    int kind;
+    const float* log_g;
+    if (check_decay(decay, &kind, &log_g) != LA_OK) return LA_ERR_INVALID_ARG;
+    normalize = normalize ? 1 : 0;
+    if (normalize && init_state && !init_z) return LA_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH * 8)) return LA_ERR_INVALID_ARG;
+    for (const void* p : {static_cast<const void*>(init_state), static_cast<const void*>(final_state)})
+        if (p && !aligned16(p)) return LA_ERR_INVALID_ARG;
+    if (normalize)
+        for (const void* p : {static_cast<const void*>(init_z), static_cast<const void*>(final_z)})
+            if (p && !aligned16(p)) return LA_ERR_INVALID_ARG;
+    if (BH > 0 && T > 0) {
+        if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    }
+    if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
+    if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
+    if (BH == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    if (T == 0) {  // empty sequence: the carried state passes through unchanged
+        const size_t sbytes = sizeof(float) * static_cast<size_t>(BH) * Dk * Dv;
+        const size_t zbytes = sizeof(float) * static_cast<size_t>(BH) * Dk;
+        cudaError_t e = cudaSuccess;
+        if (final_state)
+            e = init_state ? cudaMemcpyAsync(final_state, init_state, sbytes, cudaMemcpyDeviceToDevice, s)
+                           : cudaMemsetAsync(final_state, 0, sbytes, s);
+        if (e == cudaSuccess && normalize && final_z)
+            e = init_z ? cudaMemcpyAsync(final_z, init_z, zbytes, cudaMemcpyDeviceToDevice, s)
+                       : cudaMemsetAsync(final_z, 0, zbytes, s);
+        return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    }
+
+    la::FwdArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.decay_kind = kind;
+    a.log_g = log_g;
+    a.normalize = normalize;
+    a.init_state = init_state;
+    a.init_z = normalize ? init_z : nullptr;
+    a.out = out;
+    a.final_state = final_state;
+    a.final_z = normalize ? final_z : nullptr;
+    a.B = B;
+    a.H = H;
+    a.T = T;
+    a.Dk = Dk;
+    a.Dv = Dv;
+    a.stream = s;
+    a.err_word = err_word_for_current_device();
+    cudaError_t e;
+    if (dtype == LA_F32) {
+        e = la::launch_fwd_f32(a);
+    } else {
+        int split = 0;
+        e = la::launch_fwd_tc(a, 0, &split);
+        if (e == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
+    }
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                         float* state, float* z, void* out, int B, int H, int Dk, int Dv, la_dtype dtype,
+                         la_stream_t stream) {
+    if (B < 0 || H < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    int kind;
+    const float* log_g;
+    if (check_decay(decay, &kind, &log_g) != LA_OK) return LA_ERR_INVALID_ARG;
+    normalize = normalize ? 1 : 0;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH)) return LA_ERR_INVALID_ARG;
+    if (BH > 0) {
+        if (!q || !k || !v || !out || !state) return LA_ERR_INVALID_ARG;
+        if (normalize && !z) return LA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+            return LA_ERR_INVALID_ARG;
+        if (normalize && !aligned16(z)) return LA_ERR_INVALID_ARG;
+    }
+    if (Dk > 128 || Dv > 128) return LA_ERR_UNSUPPORTED;
+    if (BH == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    la::DecodeArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.decay_kind = kind;
+    a.log_g = log_g;
+    a.normalize = normalize;
+    a.state = state;
+    a.z = normalize ? z : nullptr;
+    a.out = out;
+    a.B = B;
+    a.H = H;
+    a.Dk = Dk;
+    a.Dv = Dv;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    return la::launch_decode(a, dtype) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_device_error(int* code, la_stream_t stream) {
+    if (!code) return LA_ERR_INVALID_ARG;
+    *code = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LA_ERR_CUDA;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    *code = v;
+    return LA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,20 @@
+// la_fwd_tc_dk64.cu - instantiations of the tensor-core forward for Dk = 64
+// (one file per key width so that the build compiles them in parallel).
+#include "la_fwd_tc.cuh"
+
+namespace la {
+namespace tc {
+
+cudaError_t launch_dk64(int nv, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                        const Params& p, int grid, cudaStream_t stream) {
+    switch (nv) {
+        case 16: return launch_instance<64, 16>(tmq, tmk, tmv, p, grid, stream);
+        case 32: return launch_instance<64, 32>(tmq, tmk, tmv, p, grid, stream);
+        case 64: return launch_instance<64, 64>(tmq, tmk, tmv, p, grid, stream);
+        case 128: return launch_instance<64, 128>(tmq, tmk, tmv, p, grid, stream);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace tc
+}  // namespace la

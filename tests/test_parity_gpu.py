@@ -1,0 +1,339 @@
+"""GPU parity: the CUDA library (through the C ABI) against the float64 oracle
+on the same seeded input bits.  Bar: max relative error 1e-4 (fp32 inputs),
+2e-2 (bf16 inputs, fp32 accumulation), measured per (b, h) slice."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import workloads as W
+from parity import TOL, oracle_forward, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                      "linear_attention_duality_examples.json")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from retention_scan_b200 import build
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    import retention_scan_b200 as la
+    assert la.device_error() == 0, "a kernel gave up waiting on a barrier"
+
+
+def la():
+    import retention_scan_b200
+    return retention_scan_b200
+
+
+def gen_case(B, H, T, Dk, Dv, dtype=torch.bfloat16, kind=0, normalize=False, seed=0,
+             decay_mean=2.0, init=False):
+    """Random case: q, k ~ elu+1 of N(0,1) when normalised, else N(0,1) with q
+    scaled by Dk^-1/2; v ~ N(0,1); per-step log g = logsigmoid(N(decay_mean,1));
+    per-head log g = log(1 - 2^(-1-h)) (strong decays that the test can see)."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, T, Dk, generator=g)
+    k = torch.randn(B, H, T, Dk, generator=g)
+    v = torch.randn(B, H, T, Dv, generator=g)
+    if normalize:
+        q, k = F.elu(q) + 1, F.elu(k) + 1
+    else:
+        q = q * Dk ** -0.5
+    log_g = None
+    if kind == 1:
+        log_g = torch.tensor([math.log1p(-2.0 ** (-1 - h)) for h in range(H)], dtype=torch.float32)
+    elif kind == 2:
+        log_g = F.logsigmoid(torch.randn(B, H, T, generator=g) + decay_mean)
+    S0 = torch.randn(B, H, Dk, Dv, generator=g) if init else None
+    z0 = (torch.rand(B, H, Dk, generator=g) * 4 + 0.5) if (init and normalize) else None
+    return dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), log_g=log_g, decay_kind=kind), S0, z0
+
+
+def run_gpu(inp, normalize=False, S0=None, z0=None):
+    d = to_dev(inp)
+    out, S, z = la().chunk_forward(d["q"], d["k"], d["v"], d["decay_kind"], d["log_g"], normalize,
+                                   None if S0 is None else S0.cuda(),
+                                   None if z0 is None else z0.cuda())
+    torch.cuda.synchronize()
+    return out, S, z
+
+
+def check_case(inp, normalize=False, S0=None, z0=None, tol=None):
+    tol = tol or TOL[inp["q"].dtype]
+    y, S, z = run_gpu(inp, normalize, S0, z0)
+    yr, Sr, zr = oracle_forward(inp, normalize, S0, z0)
+    errs = {"y": rel_err(y, yr), "S": rel_err(S, Sr)}
+    if normalize:
+        errs["z"] = rel_err(z, zr)
+    assert all(e <= tol for e in errs.values()), errs
+    return errs
+
+
+# ---------------------------------------------------------------- page values
+
+def _examples():
+    return json.load(open(GOLDEN))["examples"]
+
+
+@pytest.mark.parametrize("ex", range(3))
+def test_worked_examples_fp32(ex):
+    e = _examples()[ex]
+    q = torch.tensor(e["q"], dtype=torch.float32)[:, None].cuda()
+    k = torch.tensor(e["k"], dtype=torch.float32)[:, None].cuda()
+    v = torch.tensor(e["v"], dtype=torch.float32)[:, None].cuda()
+    y, S, _ = la().chunk_forward(q, k, v)
+    assert torch.equal(y[:, 0].cpu(), torch.tensor(e["output"], dtype=torch.float32))
+    assert torch.equal(S[:, 0].cpu(), torch.tensor(e["final_state"], dtype=torch.float32))
+
+
+@pytest.mark.parametrize("ex", range(3))
+def test_worked_examples_bf16_tensor_cores(ex):
+    # the same integers zero-padded to widths 16: exact in bf16 and in fp32 accumulation
+    e = _examples()[ex]
+    q = torch.tensor(e["q"], dtype=torch.float32)[:, None]
+    k = torch.tensor(e["k"], dtype=torch.float32)[:, None]
+    v = torch.tensor(e["v"], dtype=torch.float32)[:, None]
+    pad = lambda x: F.pad(x, (0, 16 - x.shape[-1])).to(torch.bfloat16).cuda()  # noqa: E731
+    y, S, _ = la().chunk_forward(pad(q), pad(k), pad(v))
+    want_y = torch.tensor(e["output"], dtype=torch.float32)
+    want_S = torch.tensor(e["final_state"], dtype=torch.float32)
+    assert torch.equal(y[:, 0, :, :want_y.shape[-1]].float().cpu(), want_y)
+    assert torch.equal(S[:, 0, :want_S.shape[-2], :want_S.shape[-1]].cpu(), want_S)
+    assert torch.count_nonzero(S[:, 0, want_S.shape[-2]:]) == 0
+
+
+@pytest.mark.parametrize("ex", range(3))
+def test_worked_examples_decode(ex):
+    e = _examples()[ex]
+    q = torch.tensor(e["q"], dtype=torch.float32)[:, None].cuda()
+    k = torch.tensor(e["k"], dtype=torch.float32)[:, None].cuda()
+    v = torch.tensor(e["v"], dtype=torch.float32)[:, None].cuda()
+    B, _, T, Dk = q.shape
+    state = torch.zeros(B, 1, Dk, v.shape[-1], device="cuda")
+    ys = [la().decode_step(q[:, :, t], k[:, :, t], v[:, :, t], state) for t in range(T)]
+    y = torch.stack(ys, dim=2)
+    assert torch.equal(y[:, 0].cpu(), torch.tensor(e["output"], dtype=torch.float32))
+    assert torch.equal(state[:, 0].cpu(), torch.tensor(e["final_state"], dtype=torch.float32))
+
+
+# ---------------------------------------------------------------- fp32 path
+
+def test_plain_workload_fp32():
+    inp = W.forward_inputs(W.PLAIN)
+    errs = check_case(inp)
+    assert errs["y"] <= 1e-4
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+def test_fp32_flags(kind, normalize):
+    inp, S0, z0 = gen_case(2, 3, 77, 8, 12, torch.float32, kind, normalize, seed=kind * 2 + normalize,
+                           init=True)
+    check_case(inp, normalize, S0, z0)
+
+
+# ---------------------------------------------------------------- tensor-core path
+
+WIDTHS = [16, 32, 64, 128]
+
+
+@pytest.mark.parametrize("Dk", WIDTHS)
+@pytest.mark.parametrize("Dv", WIDTHS)
+def test_tc_widths(Dk, Dv):
+    inp, S0, z0 = gen_case(1, 2, 300, Dk, Dv, kind=2, normalize=True, seed=Dk * 1000 + Dv, init=True)
+    check_case(inp, True, S0, z0)
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+@pytest.mark.parametrize("init", [False, True])
+@pytest.mark.parametrize("D", [64, 128])
+def test_tc_flags(kind, normalize, init, D):
+    inp, S0, z0 = gen_case(2, 2, 333, D, D, kind=kind, normalize=normalize, init=init,
+                           seed=100 + kind * 4 + normalize * 2 + init)
+    check_case(inp, normalize, S0, z0)
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 127, 128, 129, 255, 256, 257, 1000])
+def test_tc_ragged_lengths(T):
+    inp, S0, z0 = gen_case(1, 3, T, 64, 64, kind=2, normalize=True, init=True, seed=T)
+    check_case(inp, True, S0, z0)
+
+
+@pytest.mark.parametrize("split", [1, 2, 4, 8])
+def test_tc_value_split(monkeypatch, split):
+    monkeypatch.setenv("LA_DV_SPLIT", str(split))
+    inp, S0, z0 = gen_case(1, 2, 400, 128, 128, kind=2, normalize=True, init=True, seed=7)
+    check_case(inp, True, S0, z0)
+
+
+def test_tc_split_and_carry():
+    # run(T) == run(T1) -> carry (S, z) -> run(T - T1), on the GPU, both against the oracle
+    inp, _, _ = gen_case(2, 2, 700, 64, 64, kind=2, normalize=True, seed=11)
+    T1 = 300
+    y_full, S_full, z_full = run_gpu(inp, True)
+    a = {kk: (vv[:, :, :T1] if kk in ("q", "k", "v", "log_g") else vv) for kk, vv in inp.items()}
+    b = {kk: (vv[:, :, T1:].contiguous() if kk in ("q", "k", "v", "log_g") else vv)
+         for kk, vv in inp.items()}
+    a = {kk: (vv.contiguous() if hasattr(vv, "contiguous") else vv) for kk, vv in a.items()}
+    ya, Sa, za = run_gpu(a, True)
+    yb, Sb, zb = run_gpu(b, True, Sa.cpu(), za.cpu())
+    yr, Sr, zr = oracle_forward(inp, True)
+    assert rel_err(torch.cat([ya, yb], dim=2), yr) <= 2e-2
+    assert rel_err(Sb, Sr) <= 2e-2 and rel_err(zb, zr) <= 2e-2
+    assert rel_err(y_full, yr) <= 2e-2
+
+
+def test_tc_strong_decay_no_nan():
+    # g ~ 1e-13 per step: every decay factor underflows towards 0; nothing may become NaN/inf
+    inp, S0, z0 = gen_case(1, 2, 600, 64, 64, kind=2, normalize=True, init=True, seed=5)
+    inp["log_g"] = torch.full_like(inp["log_g"], -30.0)
+    y, S, z = run_gpu(inp, True, S0, z0)
+    assert torch.isfinite(y.float()).all() and torch.isfinite(S).all() and torch.isfinite(z).all()
+    check_case(inp, True, S0, z0)
+
+
+def test_tc_no_decay_long_sum_matches():
+    # g = 1 over many chunks: the state is a plain prefix sum of k v^T
+    inp, _, _ = gen_case(1, 2, 2048, 128, 128, kind=0, normalize=False, seed=3)
+    check_case(inp)
+
+
+def test_empty_and_zero_sizes():
+    S0 = torch.randn(2, 3, 16, 16, device="cuda")
+    z0 = torch.rand(2, 3, 16, device="cuda")
+    q = torch.zeros(2, 3, 0, 16, device="cuda", dtype=torch.bfloat16)
+    y, S, z = la().chunk_forward(q, q, q, normalize=True, init_state=S0, init_z=z0)
+    torch.cuda.synchronize()
+    assert y.shape == (2, 3, 0, 16) and torch.equal(S, S0) and torch.equal(z, z0)
+    y, S, _ = la().chunk_forward(q, q, q)
+    assert torch.count_nonzero(S) == 0
+    e = torch.zeros(0, 3, 5, 16, device="cuda", dtype=torch.bfloat16)
+    y, S, _ = la().chunk_forward(e, e, e)
+    assert y.shape == (0, 3, 5, 16)
+
+
+def test_invalid_arguments_raise():
+    q = torch.randn(1, 1, 8, 48, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(la().LAError) as ei:
+        la().chunk_forward(q, q, q)
+    assert ei.value.status == 2
+    q = torch.randn(1, 1, 8, 16, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(la().LAError) as ei:
+        la().chunk_forward(q, q, q, normalize=True, init_state=torch.zeros(1, 1, 16, 16, device="cuda"))
+    assert ei.value.status == 1
+
+
+# ---------------------------------------------------------------- workloads
+
+def test_retention_workload_full():
+    inp = W.forward_inputs(W.RETENTION)
+    check_case(inp)
+
+
+def _prefix_state(wl, heads):
+    pre = W.prefix_inputs(wl, heads=heads)
+    _, S0, z0 = oracle_forward(pre, True)
+    return torch.from_numpy(S0).float(), torch.from_numpy(z0).float()
+
+
+def test_normalized_workload_sampled_heads():
+    wl = W.NORMALIZED
+    heads = [0, 37, wl.B * wl.H - 1]
+    # the full-size GPU run, in the launch configuration the benchmark uses
+    full = W.forward_inputs(wl)
+    S0_all = torch.zeros(wl.B, wl.H, wl.Dk, wl.Dv)
+    z0_all = torch.ones(wl.B, wl.H, wl.Dk)
+    S0_s, z0_s = _prefix_state(wl, heads)
+    flat_S, flat_z = S0_all.view(-1, wl.Dk, wl.Dv), z0_all.view(-1, wl.Dk)
+    for i, bh in enumerate(heads):
+        flat_S[bh], flat_z[bh] = S0_s[0, i], z0_s[0, i]
+    y, S, z = run_gpu(full, True, S0_all, z0_all)
+    sub = W.forward_inputs(wl, heads=heads)
+    yr, Sr, zr = oracle_forward(sub, True, S0_s, z0_s)
+    yy = y.view(-1, wl.T, wl.Dv)[heads][None]
+    SS = S.view(-1, wl.Dk, wl.Dv)[heads][None]
+    zz = z.view(-1, wl.Dk)[heads][None]
+    assert rel_err(yy, yr) <= 2e-2 and rel_err(SS, Sr) <= 2e-2 and rel_err(zz, zr) <= 2e-2
+
+
+def test_gated_workload_sampled_heads():
+    wl = W.GATED
+    heads = [0, 31]
+    full = W.forward_inputs(wl)
+    y, S, _ = run_gpu(full)
+    sub = W.forward_inputs(wl, heads=heads)
+    assert torch.equal(full["q"].view(-1, wl.T, wl.Dk)[heads], sub["q"][0])
+    yr, Sr, _ = oracle_forward(sub)
+    yy = y.view(-1, wl.T, wl.Dv)[heads][None]
+    SS = S.view(-1, wl.Dk, wl.Dv)[heads][None]
+    assert rel_err(yy, yr) <= 2e-2 and rel_err(SS, Sr) <= 2e-2
+
+
+# ---------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+@pytest.mark.parametrize("Dk,Dv", [(128, 128), (64, 32), (16, 16), (5, 3), (7, 12)])
+def test_decode_steps_match_oracle(dtype, kind, normalize, Dk, Dv):
+    n = 6
+    inp, S0, z0 = gen_case(3, 4, n, Dk, Dv, dtype, kind, normalize, seed=Dk + Dv + kind, init=True)
+    if z0 is None and normalize:
+        z0 = torch.rand(3, 4, Dk) + 0.5
+    S = S0.clone().cuda()
+    z = z0.clone().cuda() if normalize else None
+    d = to_dev(inp)
+    ys = []
+    for t in range(n):
+        lg = d["log_g"][:, :, t].contiguous() if kind == 2 else d["log_g"]
+        ys.append(la().decode_step(d["q"][:, :, t].contiguous(), d["k"][:, :, t].contiguous(),
+                                   d["v"][:, :, t].contiguous(), S, z, kind, lg, normalize))
+    torch.cuda.synchronize()
+    yr, Sr, zr = oracle_forward(inp, normalize, S0, z0)
+    tol = TOL[dtype]
+    assert rel_err(torch.stack(ys, 2), yr) <= tol
+    assert rel_err(S, Sr) <= 1e-5
+    if normalize:
+        assert rel_err(z, zr) <= 1e-5
+
+
+def test_decode_equals_forward_of_one_token():
+    inp, S0, z0 = gen_case(2, 3, 1, 32, 32, torch.float32, 2, True, seed=9, init=True)
+    d = to_dev(inp)
+    y1, S1, z1 = la().chunk_forward(d["q"], d["k"], d["v"], 2, d["log_g"], True, S0.cuda(), z0.cuda())
+    S, z = S0.clone().cuda(), z0.clone().cuda()
+    y2 = la().decode_step(d["q"][:, :, 0].contiguous(), d["k"][:, :, 0].contiguous(),
+                          d["v"][:, :, 0].contiguous(), S, z, 2, d["log_g"][:, :, 0].contiguous(), True)
+    torch.cuda.synchronize()
+    assert torch.allclose(y1[:, :, 0], y2, rtol=1e-5, atol=1e-6)
+    assert torch.allclose(S1, S, rtol=1e-6, atol=1e-6) and torch.allclose(z1, z, rtol=1e-6, atol=1e-6)
+
+
+def test_decode_workload_sampled_heads():
+    wl = W.DECODE
+    heads = [0, 1000, wl.B * wl.H - 1]
+    S0, z0 = W.decode_initial_state(wl)
+    S, z = S0.cuda(), z0.cuda()
+    Ss, zs = W.decode_initial_state(wl, heads=heads)
+    Sref, zref = Ss.double().numpy(), zs.double().numpy()
+    for step in range(3):
+        inp = W.decode_step_inputs(wl, step)
+        d = to_dev(inp)
+        y = la().decode_step(d["q"], d["k"], d["v"], S, z, 1, d["log_g"], True)
+        sub = W.decode_step_inputs(wl, step, heads=heads)
+        yr, Sref, zref = oracle.decode_step(sub["q"], sub["k"], sub["v"], Sref, zref, 1, sub["log_g"], True)
+        torch.cuda.synchronize()
+        assert rel_err(y.view(-1, wl.Dv)[heads][None], yr) <= 2e-2
+    assert rel_err(S.view(-1, wl.Dk, wl.Dv)[heads][None], Sref) <= 1e-5
+    assert rel_err(z.view(-1, wl.Dk)[heads][None], zref) <= 1e-5
