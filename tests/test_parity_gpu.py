@@ -120,7 +120,9 @@ def test_worked_examples_decode(ex):
     v = torch.tensor(e["v"], dtype=torch.float32)[:, None].cuda()
     B, _, T, Dk = q.shape
     state = torch.zeros(B, 1, Dk, v.shape[-1], device="cuda")
-    ys = [la().decode_step(q[:, :, t], k[:, :, t], v[:, :, t], state) for t in range(T)]
+    # clone: a view into the middle of a row is not 16-byte aligned, which the ABI rejects
+    ys = [la().decode_step(q[:, :, t].clone(), k[:, :, t].clone(), v[:, :, t].clone(), state)
+          for t in range(T)]
     y = torch.stack(ys, dim=2)
     assert torch.equal(y[:, 0].cpu(), torch.tensor(e["output"], dtype=torch.float32))
     assert torch.equal(state[:, 0].cpu(), torch.tensor(e["final_state"], dtype=torch.float32))
