@@ -1,26 +1,27 @@
 // la_fwd_tc.cu - host side of the tensor-core forward: tensor maps, the
 // choice of how many CTAs share one (b, h), and dispatch to the
-// instantiation for (Dk, Dv slice).
+// warp-specialised kernel instantiation for (Dk, Dv slice, normaliser).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdlib>
 
-#include "la_fwd_tc.cuh"
+#include "la_fwd_ws.cuh"
 #include "la_internal.h"
 
 namespace la {
-namespace tc {
-cudaError_t launch_dk16(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const Params&, int,
-                        cudaStream_t);
-cudaError_t launch_dk32(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const Params&, int,
-                        cudaStream_t);
-cudaError_t launch_dk64(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const Params&, int,
-                        cudaStream_t);
-cudaError_t launch_dk128(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const Params&, int,
-                         cudaStream_t);
-}  // namespace tc
+namespace ws {
+#define LA_WS_DECL(DK)                                                                                        \
+    cudaError_t launch_dk##DK(int, bool, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,           \
+                              const Params&, int, cudaStream_t);                                              \
+    bool supported_dk##DK(int, bool);
+LA_WS_DECL(16)
+LA_WS_DECL(32)
+LA_WS_DECL(64)
+LA_WS_DECL(128)
+#undef LA_WS_DECL
+}  // namespace ws
 
 namespace {
 
@@ -58,10 +59,10 @@ bool make_map(CUtensorMap* map, const void* base, int width, int T, int BH, int 
                                 static_cast<cuuint64_t>(BH)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(width) * 2,
                                    static_cast<cuuint64_t>(width) * 2 * static_cast<cuuint64_t>(T)};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(tc::C), 1};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(ws::C), 1};
     const cuuint32_t elem[3] = {1, 1, 1};
     return f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(tc::row_bytes_for(box_inner)),
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(ws::row_bytes_for(box_inner)),
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -78,16 +79,28 @@ int sm_count() {
     return v;
 }
 
+bool instance_ok(int Dk, int nv, bool norm) {
+    switch (Dk) {
+        case 16: return ws::supported_dk16(nv, norm);
+        case 32: return ws::supported_dk32(nv, norm);
+        case 64: return ws::supported_dk64(nv, norm);
+        case 128: return ws::supported_dk128(nv, norm);
+        default: return false;
+    }
+}
+
 // How many CTAs share one (b, h): each owns Dv / split value columns and
-// recomputes the 128 x 128 score tile.  Split until there are enough CTAs to
-// cover most SMs in one wave, keeping slices of at least 16 columns.
-int choose_split(int BH, int Dv) {
+// recomputes the 128 x 128 score tile.  The split is the smallest one whose
+// tiles fit in shared memory, doubled while that leaves most SMs idle
+// (keeping slices of at least 16 columns).
+int choose_split(int BH, int Dk, int Dv, bool norm) {
     if (const char* env = std::getenv("LA_DV_SPLIT")) {
         const int s = std::atoi(env);
-        if (s >= 1 && Dv % s == 0 && width_ok(Dv / s)) return s;
+        if (s >= 1 && Dv % s == 0 && width_ok(Dv / s) && instance_ok(Dk, Dv / s, norm)) return s;
     }
-    const int target = sm_count() * 4 / 5;
     int s = 1;
+    while (!instance_ok(Dk, Dv / s, norm) && Dv / (2 * s) >= 16) s *= 2;
+    const int target = sm_count() * 4 / 5;
     while (static_cast<long long>(BH) * s < target && Dv / (2 * s) >= 16) s *= 2;
     return s;
 }
@@ -98,10 +111,11 @@ bool fwd_tc_supports(int Dk, int Dv) { return width_ok(Dk) && width_ok(Dv); }
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used) {
     if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
+    const bool norm = a.normalize != 0;
     const int BH = a.B * a.H;
-    const int split = dv_split > 0 ? dv_split : choose_split(BH, a.Dv);
+    const int split = dv_split > 0 ? dv_split : choose_split(BH, a.Dk, a.Dv, norm);
     const int nv = a.Dv / split;
-    if (a.Dv % split != 0 || !width_ok(nv)) return cudaErrorNotSupported;
+    if (a.Dv % split != 0 || !width_ok(nv) || !instance_ok(a.Dk, nv, norm)) return cudaErrorNotSupported;
     if (split_used) *split_used = split;
 
     CUtensorMap tmq, tmk, tmv;
@@ -111,10 +125,9 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used) {
         !make_map(&tmv, a.v, a.Dv, a.T, BH, box_v))
         return cudaErrorInvalidValue;
 
-    tc::Params p{};
+    ws::Params p{};
     p.log_g = a.log_g;
     p.decay_kind = a.decay_kind;
-    p.normalize = a.normalize;
     p.init_state = a.init_state;
     p.init_z = a.init_z;
     p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -124,14 +137,14 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used) {
     p.T = a.T;
     p.Dv = a.Dv;
     p.split = split;
-    p.nchunks = (a.T + tc::C - 1) / tc::C;
+    p.nchunks = (a.T + ws::C - 1) / ws::C;
     p.err = a.err_word;
     const int grid = BH * split;
     switch (a.Dk) {
-        case 16: return tc::launch_dk16(nv, tmq, tmk, tmv, p, grid, a.stream);
-        case 32: return tc::launch_dk32(nv, tmq, tmk, tmv, p, grid, a.stream);
-        case 64: return tc::launch_dk64(nv, tmq, tmk, tmv, p, grid, a.stream);
-        case 128: return tc::launch_dk128(nv, tmq, tmk, tmv, p, grid, a.stream);
+        case 16: return ws::launch_dk16(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
+        case 32: return ws::launch_dk32(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
+        case 64: return ws::launch_dk64(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
+        case 128: return ws::launch_dk128(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
         default: return cudaErrorNotSupported;
     }
 }

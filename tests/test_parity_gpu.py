@@ -27,6 +27,10 @@ def built():
     oracle.build()
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     yield
+    out_dir = os.environ.get("LA_PARITY_LOG_DIR")
+    if out_dir and os.path.isdir(out_dir):
+        with open(os.path.join(out_dir, "parity_errors.json"), "w") as f:
+            json.dump(ERRORS, f, indent=0)
     import retention_scan_b200 as la
     assert la.device_error() == 0, "a kernel gave up waiting on a barrier"
 
@@ -68,6 +72,9 @@ def run_gpu(inp, normalize=False, S0=None, z0=None):
     return out, S, z
 
 
+ERRORS = []  # (test id, errors) of every parity check, written out at the end of the module
+
+
 def check_case(inp, normalize=False, S0=None, z0=None, tol=None):
     tol = tol or TOL[inp["q"].dtype]
     y, S, z = run_gpu(inp, normalize, S0, z0)
@@ -75,6 +82,7 @@ def check_case(inp, normalize=False, S0=None, z0=None, tol=None):
     errs = {"y": rel_err(y, yr), "S": rel_err(S, Sr)}
     if normalize:
         errs["z"] = rel_err(z, zr)
+    ERRORS.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], errs))
     assert all(e <= tol for e in errs.values()), errs
     return errs
 
