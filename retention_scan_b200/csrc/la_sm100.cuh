@@ -72,6 +72,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// 2^x with the hardware approximation (ex2.approx.ftz: relative error about
+// 2^-22, denormal results flushed to zero).  Used for decay factors, whose
+// exponents are <= 0 or bounded by the fold limit.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // elect.sync: true in exactly one active lane of the warp.
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
