@@ -174,11 +174,11 @@ def bus_id_of(device):
 class Job:
     """Device-resident inputs and the step function of one workload."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, wl=None, rank=0):
         import retention_scan_b200 as la
         self.la = la
         self.cfg = cfg
-        self.wl = wl = W.WORKLOADS[cfg]
+        self.wl = wl = wl or W.WORKLOADS[cfg]
         self.dev = device
         if cfg == 5:
             S0, z0 = W.decode_initial_state(wl)
@@ -188,7 +188,7 @@ class Job:
             self.log_g = W.per_head_log_gamma(wl.H).to(device)
             self.out = torch.empty(wl.B, wl.H, wl.Dv, dtype=wl.torch_dtype, device=device)
             return
-        inp = W.forward_inputs(wl)
+        inp = W.forward_inputs(wl, seed=rank_seed(wl, rank))
         self.host = inp
         self.q, self.k, self.v = (inp[n].to(device) for n in ("q", "k", "v"))
         self.kind = inp["decay_kind"]
@@ -261,11 +261,18 @@ def barrier(dist_on):
 
 
 def max_over_ranks(x, dist_on, device):
+    """The slowest rank's value (the job's time is set by its slowest GPU)."""
     if not dist_on:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(wl, rank):
+    """Each rank processes its own batch of independent sequences (weak
+    scaling): same shapes and distributions, rank-specific seed."""
+    return wl.seed + 7919 * rank
 
 
 def time_steps(job, steps, flush, dist_on, device):
@@ -335,10 +342,21 @@ def cpu_baseline(cfg, budget_s=15.0):
             "sample": f"{nh} of {total} (b,h) sequences, all {wl.T} tokens each, {threads} threads"}
 
 
+def sized_workload(args):
+    """The workload of --config, with --tokens / --batch overrides (smaller
+    cases for profiler captures); an override renames the workload."""
+    wl = W.WORKLOADS[args.config]
+    if args.tokens and args.config != 5:
+        wl = wl.with_sizes(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
+    if args.batch:
+        wl = wl.with_sizes(B=args.batch, name=f"{wl.name}_B{args.batch}")
+    return wl
+
+
 def run_ours(args, rank, world, dist_on, device):
     cfg = args.config
-    wl = W.WORKLOADS[cfg]
-    job = Job(cfg, device)
+    wl = sized_workload(args)
+    job = Job(cfg, device, wl, rank)
     torch.cuda.synchronize()
     in_bytes = algorithmic_bytes(wl, cfg) * (wl.steps if cfg == 5 else 1)
     flush = None
@@ -452,6 +470,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
+    ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
     args = ap.parse_args()
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3}
     if args.steps is None:
