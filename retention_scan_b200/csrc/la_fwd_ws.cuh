@@ -14,35 +14,38 @@
 //
 // Folded decay.  With v'_s = 2^(-L_s) v_s (the value rows scaled in place) the
 // decay leaves the score tile:
-//   O = causal_mask(Q K^T) V' + Q S,   y_t = 2^(L_t) O_t,
+//   O = Q S + causal_mask(Q K^T) V',   y_t = 2^(L_t) O_t,
 //   S' = 2^(L_C) (S + K^T V').
 // Each factor is bounded by 2^|L_C|; a chunk whose total decay exceeds
 // kFoldLimit (log2 units) is computed in "direct" form instead:
 // P = mask(Q K^T) * 2^(L_t - L_s) per element, Q~ = 2^(L_t) Q,
-// K~ = 2^(L_C - L_s) K, O = P V + Q~ S, S' = 2^(L_C) S + K~^T V.  In both
+// K~ = 2^(L_C - L_s) K, O = Q~ S + P V, S' = 2^(L_C) S + K~^T V.  In both
 // forms no exponent exceeds kFoldLimit and no factor can overflow (RWKV-LM
 // discussion 189: use an exponentially weighted representation, never an
 // unbounded w^(t-1) scale).
 //
-// Normaliser.  Two extra 16-column MMAs give the denominator in TMEM:
-// P [w_hi w_lo 0 ..] plus Q [z_hi z_lo 0 ..], where w_s = 2^(-L_s) (1 in the
-// direct form, whose P already holds the decay) and z are split into two
+// Normaliser.  Two extra 16-column MMAs give the denominator in TMEM, next to
+// O: Q [z_hi z_lo 0 ..] plus P [w_hi w_lo 0 ..], where w_s = 2^(-L_s) (1 in
+// the direct form, whose P already holds the decay) and z are split into two
 // bf16 parts (about 16 bits).  In the folded form numerator and denominator
 // share the factor 2^(L_t), which cancels.  The key-sum update uses
 // K^T [w_hi w_lo 0 ..].
 //
+// Data flow.  Q and K tiles sit in one TMA ring, V tiles (with the chunk's
+// decay prefix) in another.  The inter-chunk term Q S is accumulated first,
+// so a chunk's Q and K are released as soon as Q K^T, K^T V' and Q S have
+// run, long before its P V; P lives in tensor memory (the A operand of P V
+// is read from TMEM), which keeps shared memory for the rings.
+//
 // Roles (one CTA = one (b, h) and NV of its Dv columns; Dv / NV CTAs share a
 // head and read its q, k through L2):
-//   warp 0       TMA producer: Q, K, V tiles into an NSTG-deep stage ring
-//   warp 1       MMA issuer (one thread) and TMEM owner
-//   warps 2-9    two warpgroups: prep (decay prefix, in-place Q'/K' scaling)
-//                and mask (A -> P, bf16, shared memory); warpgroup 0 owns
-//                score columns 0-63 and the Q rows, warpgroup 1 columns
-//                64-127 and the K rows
-//   warps 10-..  state and epilogue (one warpgroup per 64 value columns):
-//                S, z in fp32 registers, S' from the K'^T V tile, bf16 copy
-//                of S for the next chunk's Q S; then y = O / den of the
-//                previous chunk, bf16, stored to global memory
+//   warp 0       TMA producer of the Q/K ring
+//   warp 1       MMA issuer (one elected lane) and TMEM owner
+//   warps 2-9    two warpgroups: prep (decay prefix, value-row scaling,
+//                normaliser weights) and mask (scores -> P in TMEM); warpgroup
+//                0 owns score columns 0-63, warpgroup 1 columns 64-127
+//   warps 10-..  state and epilogue (one warpgroup per 64 value columns)
+//   last warp    TMA producer of the V ring
 // Every hand-off is an mbarrier; every wait gives up after kWaitLimitNs (then
 // the CTA sets the device error word and unwinds).
 #pragma once
@@ -61,7 +64,6 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kFoldLimit = 64.f;
 constexpr int kSmemLimit = 232448;
-constexpr int B_COUNT_MAX = 31;  // barrier slots used (see Bar)
 
 enum Mode : int { kModeNone = 0, kModeFolded = 1, kModeDirect = 2 };
 
@@ -69,85 +71,101 @@ __host__ __device__ constexpr int row_bytes_for(int width) { return width >= 64 
 __host__ __device__ constexpr int panels_for(int width) { return width >= 64 ? width / 64 : 1; }
 __host__ __device__ constexpr int round1k(int x) { return (x + 1023) / 1024 * 1024; }
 
+// Barrier slots (uint64 each) at the start of the MISC area.
+enum Bar : int {
+    B_QKFULL = 0,    // [4] Q/K tiles landed
+    B_QKEMPTY = 4,   // [4] Q/K stage free (Q K^T, K^T V', Q S done)
+    B_VFULL = 8,     // [4] V tile landed
+    B_VEMPTY = 12,   // [4] V stage free (P V done, its prefix read)
+    B_PREP = 16,     // [4] decay prefix, value scaling, weights done
+    B_AFULL = 20,    // scores in TMEM
+    B_AEMPTY = 21,   // scores read by the mask warps
+    B_PFULL = 22,    // [2] P in TMEM
+    B_PEMPTY = 24,   // [2] P V done reading P
+    B_OFULL = 26,    // [2] O (and den) complete
+    B_OEMPTY = 28,   // [2] epilogue done with O
+    B_DSFULL = 30,   // [2] K^T V' in TMEM
+    B_DSEMPTY = 32,  // [2] state warps done with it
+    B_SBFULL = 34,   // [2] bf16 state copy written
+    B_SBEMPTY = 36,  // [2] Q S done reading it
+    B_DRAIN = 38,
+    B_COUNT = 39
+};
+
 template <int DK, int NV, bool NORM>
 struct Plan {
     static constexpr int WK = row_bytes_for(DK), PK = panels_for(DK);
     static constexpr int WV = row_bytes_for(NV), PV = panels_for(NV);
     static constexpr int Q_BYTES = C * DK * 2;
     static constexpr int V_BYTES = C * NV * 2;
-    // one stage: Q | K | V | W (normaliser weights) | L (float[C], log2 units) | meta
-    static constexpr int ST_Q = 0, ST_K = Q_BYTES, ST_V = 2 * Q_BYTES;
-    static constexpr int ST_W = 2 * Q_BYTES + V_BYTES;                  // [C x 16] bf16, 32-byte swizzle
-    static constexpr int ST_LAM = ST_W + (NORM ? C * 32 : 0);
-    static constexpr int ST_META = ST_LAM + C * 4;  // float L_C, int mode
-    static constexpr int STAGE = round1k(ST_META + 64);
-    static constexpr int P_BYTES = C * C * 2;
+    // Q/K stage: Q | K
+    static constexpr int QK_STAGE = round1k(2 * Q_BYTES);
+    // V stage: V | W (normaliser weights, [C x 16] bf16, 32-byte swizzle) | L (float[C], log2) | meta
+    static constexpr int VS_W = V_BYTES;
+    static constexpr int VS_LAM = VS_W + (NORM ? C * 32 : 0);
+    static constexpr int VS_META = VS_LAM + C * 4;  // float L_C, int mode
+    static constexpr int V_STAGE = round1k(VS_META + 64);
     static constexpr int SB_BYTES = round1k(DK * NV * 2);
     static constexpr int ZB_BYTES = NORM ? round1k(DK * 32) : 0;
-    // barriers and flags, then the output row factors of the last kRowfRing chunks.
-    // prep(c + R) may run once state(c + R - NSTG) is done, and the epilogue
-    // of chunk c runs before that, so R = NSTG + 1 slots would do; 8 covers NSTG <= 4.
+    // barriers and flags, then the output row factors of the last kRowfRing
+    // chunks (not needed with the normaliser, where the factor cancels).
     static constexpr int kRowfRing = 8;
-    static constexpr int MISC = 1024 + (NORM ? 0 : kRowfRing * C * 4);  // normalised: the factor cancels
-    static constexpr bool fits(int ns, int np, int nsb) {
-        return ns * STAGE + np * P_BYTES + nsb * (SB_BYTES + ZB_BYTES) + MISC + 1024 <= kSmemLimit;
+    static constexpr int MISC = 1024 + (NORM ? 0 : kRowfRing * C * 4);
+    static constexpr bool fits(int nqk, int nvs, int nsb) {
+        return nqk * QK_STAGE + nvs * V_STAGE + nsb * (SB_BYTES + ZB_BYTES) + MISC + 1024 <= kSmemLimit;
     }
-    static constexpr int NSTG = fits(4, 2, 2) ? 4 : fits(3, 2, 2) ? 3 : 2;
-    static constexpr int NPB = (fits(NSTG, 2, 2) || fits(NSTG, 2, 1)) ? 2 : 1;
-    static constexpr int NSB = fits(NSTG, NPB, 2) ? 2 : 1;
-    static constexpr bool OK = fits(NSTG, NPB, NSB);
-    static constexpr int OFF_P = NSTG * STAGE;
-    static constexpr int OFF_SB = OFF_P + NPB * P_BYTES;
+    // deepest Q/K ring first, then V ring (at least as deep), then state copies
+    static constexpr int pick() {
+        for (int nqk = 4; nqk >= 2; --nqk)
+            for (int nvs = 4; nvs >= nqk; --nvs)
+                for (int nsb = 2; nsb >= 1; --nsb)
+                    if (fits(nqk, nvs, nsb)) return nqk * 100 + nvs * 10 + nsb;
+        return 0;
+    }
+    static constexpr int PICK = pick();
+    static constexpr bool OK = PICK != 0;
+    static constexpr int NQK = OK ? PICK / 100 : 2;
+    static constexpr int NVS = OK ? (PICK / 10) % 10 : 2;
+    static constexpr int NSB = OK ? PICK % 10 : 1;
+    static constexpr int OFF_V = NQK * QK_STAGE;
+    static constexpr int OFF_SB = OFF_V + NVS * V_STAGE;
     static constexpr int OFF_ZB = OFF_SB + NSB * SB_BYTES;
     static constexpr int OFF_MISC = OFF_ZB + NSB * ZB_BYTES;
     static constexpr int OFF_ROWF = OFF_MISC + 1024;  // float[kRowfRing][C]: 2^(L_t) per token
     static constexpr int SMEM = OFF_MISC + MISC + 1024;
-    // TMEM columns
-    static constexpr int NDS = (256 + 2 * NV + (NORM ? 64 : 0)) <= 512 ? 2 : 1;
-    static constexpr int COL_DS0 = 256;
-    static constexpr int COL_ZS0 = 256 + NDS * NV;
-    static constexpr int COL_QZ0 = COL_ZS0 + (NORM ? 16 * NDS : 0);
-    static constexpr int TMEM_USED = COL_QZ0 + (NORM ? 32 : 0);
+    // TMEM columns: scores [0,128) | P (bf16 pairs) 64 per buffer | O | K^T V'
+    static constexpr int OCOLS = NV + (NORM ? 16 : 0);
+    static constexpr int tmem_need(int npb, int no, int nds) { return 128 + 64 * npb + (no + nds) * OCOLS; }
+    static constexpr int NPB = tmem_need(2, 2, 1) <= 512 ? 2 : 1;
+    static constexpr int NO = tmem_need(NPB, 2, 1) <= 512 ? 2 : 1;
+    static constexpr int NDS = tmem_need(NPB, NO, 2) <= 512 ? 2 : 1;
+    static constexpr int COL_P0 = 128;
+    static constexpr int COL_O0 = COL_P0 + 64 * NPB;
+    static constexpr int COL_DS0 = COL_O0 + NO * OCOLS;
+    static constexpr int TMEM_USED = COL_DS0 + NDS * OCOLS;
     static constexpr int TMEM_COLS = 512;
     // warps
     static constexpr int NSW = NV > 64 ? 2 : 1;
     static constexpr int NVW = NV / NSW;
     static constexpr int W_TMA = 0, W_MMA = 1, W_PM = 2, W_ES = 10;
-    static constexpr int NWARPS = W_ES + 4 * NSW;
+    static constexpr int W_TMAV = W_ES + 4 * NSW;
+    static constexpr int NWARPS = W_TMAV + 1;
     static constexpr int THREADS = 32 * NWARPS;
-    static constexpr int EMPTY_ARRIVALS = 1 + 8 + 4 * NSW;
-    static constexpr uint32_t TX_BYTES = 2 * Q_BYTES + V_BYTES;
+    static constexpr int VEMPTY_ARRIVALS = 1 + 8 + 4 * NSW;
+    static constexpr uint32_t QK_TX = 2 * Q_BYTES;
+    static constexpr uint32_t V_TX = V_BYTES;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NV, 0, 1);
     static constexpr uint32_t IDESC_KV = make_idesc_bf16(128, NV, 1, 1);
     static constexpr uint32_t IDESC_N16 = make_idesc_bf16(128, 16, 0, 1);
     static constexpr uint32_t IDESC_KV16 = make_idesc_bf16(128, 16, 1, 1);
     static_assert(TMEM_USED <= TMEM_COLS, "tensor memory budget");
-    static_assert(kRowfRing >= NSTG + 1, "row factor ring too shallow");
-    static_assert(!OK || OFF_MISC + 8 * B_COUNT_MAX + 8 <= OFF_MISC + 1024, "barrier area");
-    static_assert(!OK || NORM || OFF_ROWF + kRowfRing * C * 4 <= SMEM - 1024, "row factor ring inside allocation");
-    static_assert(!OK || OFF_MISC + MISC + 1024 <= SMEM, "regions inside allocation");
-    static_assert(!OK || SMEM <= kSmemLimit, "shared memory limit");
     static_assert(NV % 16 == 0 && NV >= 16 && NV <= 128, "value slice");
     static_assert(DK == 16 || DK == 32 || DK == 64 || DK == 128, "key width");
-};
-
-// Barrier slots (uint64 each) inside the MISC area.
-enum Bar : int {
-    B_FULL = 0,      // [4] TMA -> consumers
-    B_EMPTY = 4,     // [4] stage free
-    B_PREP = 8,      // [4] decay prefix and in-place scaling done
-    B_AFULL = 12,    // [2] scores in TMEM
-    B_OFULL = 14,    // [2] O (and den) in TMEM
-    B_OEMPTY = 16,   // [2] epilogue done with a TMEM region
-    B_PFULL = 18,    // [2] P in shared memory
-    B_PEMPTY = 20,   // [2] MMA done reading P
-    B_DSFULL = 22,   // [2] K'^T V in TMEM
-    B_DSEMPTY = 24,  // [2] state warps done with it
-    B_SBFULL = 26,   // [2] bf16 state copy written
-    B_SBEMPTY = 28,  // [2] MMA done reading it
-    B_DRAIN = 30,
-    B_COUNT = 31
+    static_assert(kRowfRing >= NVS + 1, "row factor ring too shallow");
+    static_assert(8 * B_COUNT + 8 <= 1024, "barrier area");
+    static_assert(!OK || SMEM <= kSmemLimit, "shared memory limit");
+    static_assert(!OK || NORM || OFF_ROWF + kRowfRing * C * 4 <= SMEM - 1024, "row factor ring inside allocation");
 };
 
 struct Params {
@@ -160,6 +178,14 @@ struct Params {
     float* final_z;
     int H, T, Dv, split, nchunks;
     int* err;
+};
+
+// What every role needs from the kernel prologue (passed by value).
+struct Ctx {
+    const Params* p;
+    uint8_t* sm;
+    uint32_t sa, tmem;
+    int bh, h, j0, slice;
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -235,190 +261,208 @@ __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
             __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&w[i]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 x = __bfloat1622float2(hv[e]);
-                hv[e] = __floats2bfloat162_rn(x.x * f, x.y * f);
+                const float2 v2 = __bfloat1622float2(hv[e]);
+                hv[e] = __floats2bfloat162_rn(v2.x * f, v2.y * f);
             }
             *reinterpret_cast<uint4*>(tile + (ci / (W / 16)) * C * W + swz(row, (ci % (W / 16)) * 16, W)) = w[i];
         }
     }
 }
 
-// Columns 16 piece .. 16 piece + 15 of row t of a P panel (128-byte swizzle):
-// a[e] where 16 piece + e <= lim, else 0; as bf16.
-__device__ __forceinline__ void store_masked16(uint8_t* panel, int t, int piece, const float (&a)[16], int lim) {
-    float m[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) m[e] = (16 * piece + e <= lim) ? a[e] : 0.f;
-    const uint4 w0 = make_uint4(pack2(m[0], m[1]), pack2(m[2], m[3]), pack2(m[4], m[5]), pack2(m[6], m[7]));
-    const uint4 w1 = make_uint4(pack2(m[8], m[9]), pack2(m[10], m[11]), pack2(m[12], m[13]), pack2(m[14], m[15]));
-    *reinterpret_cast<uint4*>(panel + swz(t, 32 * piece, 128)) = w0;
-    *reinterpret_cast<uint4*>(panel + swz(t, 32 * piece + 16, 128)) = w1;
+// Byte offset of 16-element K step kk in a K-major tile (rows of W bytes).
+__host__ __device__ constexpr uint32_t kstep(int kk, int W) {
+    return ((kk * 16) / (W / 2)) * C * W + ((kk * 16) % (W / 2)) * 2;
 }
 
-// What every role needs from the kernel prologue (passed by value).
-struct Ctx {
-    const Params* p;
-    uint8_t* sm;
-    uint32_t sa, tmem;
-    int bh, h, j0, slice;
-};
+#define LA_ROLE_PRELUDE                                                                              \
+    using G = Plan<DK, NV, NORM>;                                                                    \
+    const Params& p = *x.p;                                                                          \
+    uint8_t* const sm = x.sm;                                                                        \
+    const uint32_t sa = x.sa, tmem = x.tmem;                                                         \
+    uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);                             \
+    volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4); \
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;                                      \
+    const int T = p.T, n = p.nchunks;                                                                \
+    (void)sa;                                                                                        \
+    (void)tmem;                                                                                      \
+    (void)warp;                                                                                      \
+    (void)T;                                                                                         \
+    (void)lane;
 
+// ------------------------------------------------------------ TMA producers
 template <int DK, int NV, bool NORM>
-__device__ __noinline__ void role_tma(const Ctx x, const CUtensorMap* tmq_p, const CUtensorMap* tmk_p, const CUtensorMap* tmv_p) {
-    using G = Plan<DK, NV, NORM>;
-    const Params& p = *x.p;
-    uint8_t* const sm = x.sm;
-    const uint32_t sa = x.sa, tmem = x.tmem;
-    uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);
-    volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = x.bh, h = x.h, j0 = x.j0, slice = x.slice;
-    const int T = p.T, n = p.nchunks;
-    auto stage_ptr = [&](int s) { return sm + s * G::STAGE; };
-    auto stage_addr = [&](int s) { return sa + s * G::STAGE; };
-    (void)h; (void)j0; (void)slice; (void)T; (void)lane; (void)warp; (void)tmem; (void)stage_addr; (void)stage_ptr;
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-        int issued = 0;
-        for (int c = 0; c < n; ++c) {
-            const int s = c % G::NSTG;
-            if (c >= G::NSTG && !wait1(&bar[B_EMPTY + s], ((c / G::NSTG) - 1) & 1, abort, p, kErrTmaWait))
-                break;
-            mbar_arrive_expect_tx(&bar[B_FULL + s], G::TX_BYTES);
-            uint8_t* st = stage_ptr(s);
-            for (int pp = 0; pp < G::PK; ++pp) {
-                tma_load_3d(st + G::ST_Q + pp * C * G::WK, tmq_p, &bar[B_FULL + s], pp * 64, c * C, bh);
-                tma_load_3d(st + G::ST_K + pp * C * G::WK, tmk_p, &bar[B_FULL + s], pp * 64, c * C, bh);
-            }
-            for (int pp = 0; pp < G::PV; ++pp)
-                tma_load_3d(st + G::ST_V + pp * C * G::WV, tmv_p, &bar[B_FULL + s], j0 + pp * 64, c * C, bh);
-            ++issued;
+__device__ __noinline__ void role_tma_qk(const Ctx x, const CUtensorMap* tmq, const CUtensorMap* tmk) {
+    LA_ROLE_PRELUDE
+    if (lane != 0) return;
+    int issued = 0;
+    for (int c = 0; c < n; ++c) {
+        const int s = c % G::NQK;
+        if (c >= G::NQK && !wait1(&bar[B_QKEMPTY + s], ((c / G::NQK) - 1) & 1, abort, p, kErrTmaWait)) break;
+        mbar_arrive_expect_tx(&bar[B_QKFULL + s], G::QK_TX);
+        uint8_t* st = sm + s * G::QK_STAGE;
+        for (int pp = 0; pp < G::PK; ++pp) {
+            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QKFULL + s], pp * 64, c * C, x.bh);
+            tma_load_3d(st + G::Q_BYTES + pp * C * G::WK, tmk, &bar[B_QKFULL + s], pp * 64, c * C, x.bh);
         }
-        if (*abort) {
-            // let issued copies land before the CTA's shared memory goes away
-            const int first = issued > G::NSTG ? issued - G::NSTG : 0;
-            for (int c = first; c < issued; ++c)
-                mbar_wait_bounded(&bar[B_FULL + c % G::NSTG], (c / G::NSTG) & 1, kWaitLimitNs);
-        }
+        ++issued;
+    }
+    if (*abort) {  // let issued copies land before the CTA's shared memory goes away
+        for (int c = issued > G::NQK ? issued - G::NQK : 0; c < issued; ++c)
+            mbar_wait_bounded(&bar[B_QKFULL + c % G::NQK], (c / G::NQK) & 1, kWaitLimitNs);
     }
 }
 
 template <int DK, int NV, bool NORM>
+__device__ __noinline__ void role_tma_v(const Ctx x, const CUtensorMap* tmv) {
+    LA_ROLE_PRELUDE
+    if (lane != 0) return;
+    int issued = 0;
+    for (int c = 0; c < n; ++c) {
+        const int s = c % G::NVS;
+        if (c >= G::NVS && !wait1(&bar[B_VEMPTY + s], ((c / G::NVS) - 1) & 1, abort, p, kErrTmaWait)) break;
+        mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
+        uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
+        for (int pp = 0; pp < G::PV; ++pp)
+            tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, c * C, x.bh);
+        ++issued;
+    }
+    if (*abort) {
+        for (int c = issued > G::NVS ? issued - G::NVS : 0; c < issued; ++c)
+            mbar_wait_bounded(&bar[B_VFULL + c % G::NVS], (c / G::NVS) & 1, kWaitLimitNs);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+// Four in-order queues, each issued as soon as its inputs are there:
+//   Q K^T (c)   Q/K tiles and prep of c landed, score region free
+//   K^T V' (j)  after Q K^T (j); a direct-form chunk also after its mask,
+//               which decays Q and K; K^T V' buffer free
+//   Q S (j)     after K^T V' (j); O buffer free; bf16 state after j - 1 written
+//   P V (j)     after Q S (j), which opened the accumulator; P (j) written
+// The warp polls the barriers (never blocking on one while another queue
+// could move) and gives up after kWaitLimitNs without progress.
+template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_mma(const Ctx x) {
-    using G = Plan<DK, NV, NORM>;
-    const Params& p = *x.p;
-    uint8_t* const sm = x.sm;
-    const uint32_t sa = x.sa, tmem = x.tmem;
-    uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);
-    volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = x.bh, h = x.h, j0 = x.j0, slice = x.slice;
-    const int T = p.T, n = p.nchunks;
-    auto stage_ptr = [&](int s) { return sm + s * G::STAGE; };
-    auto stage_addr = [&](int s) { return sa + s * G::STAGE; };
-    (void)h; (void)j0; (void)slice; (void)T; (void)lane; (void)warp; (void)tmem; (void)stage_addr; (void)stage_ptr;
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the schedule (so descriptors stay warp-uniform);
-    // one elected lane issues every MMA and commit.
+    LA_ROLE_PRELUDE
     const bool leader = elect_one();
-    int kv_next = 0;  // K'^T V tiles are issued in chunk order
-    auto kstep = [](int kk, int W) -> uint32_t {  // byte offset of K step kk in a K-major tile
-        return ((kk * 16) / (W / 2)) * C * W + ((kk * 16) % (W / 2)) * 2;
+    auto mode_of = [&](int j) {
+        return *reinterpret_cast<volatile int*>(sm + G::OFF_V + (j % G::NVS) * G::V_STAGE + G::VS_META + 4);
     };
-    auto issue_kv = [&](int c) -> bool {
-        const int s = c % G::NSTG, b = c % G::NDS;
-        if (c >= G::NDS && !waitw(&bar[B_DSEMPTY + b], ((c / G::NDS) - 1) & 1, abort, p, kErrMmaWait))
-            return false;
-        tc_fence_after_sync();
-        // M = 128 key rows; for Dk < 128 a zero panel offset repeats the key panel
-        const uint64_t dk = make_smem_desc(stage_addr(s) + G::ST_K, DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
-        const uint64_t dv = make_smem_desc(stage_addr(s) + G::ST_V, C * G::WV, 8 * G::WV, G::WV);
-        if (leader) {
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + G::COL_DS0 + b * NV, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4),
-                          G::IDESC_KV, kk > 0);
-            if (NORM) {
-                const uint64_t dw = make_smem_desc(stage_addr(s) + G::ST_W, 0, 8 * 32, 32);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + G::COL_ZS0 + b * 16, dk + ((kk * 16 * G::WK) >> 4), dw + ((kk * 16 * 32) >> 4),
-                              G::IDESC_KV16, kk > 0);
-            }
-            umma_commit(&bar[B_DSFULL + b]);
+    auto qk_addr = [&](int j) { return sa + (j % G::NQK) * G::QK_STAGE; };
+    auto v_addr = [&](int j) { return sa + G::OFF_V + (j % G::NVS) * G::V_STAGE; };
+    auto ready = [&](int slot, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(&bar[slot], parity)); };
+
+    int m1 = 0, kv = 0, qs = 0, pv = 0, pseen = 0;  // next chunk of each queue; P (j) seen for j < pseen
+    uint64_t last = global_timer_ns();
+    while (pv < n) {
+        bool moved = false;
+        if (pseen < m1 && ready(B_PFULL + pseen % G::NPB, (pseen / G::NPB) & 1)) {
+            ++pseen;
+            moved = true;
         }
-        __syncwarp();
-        return true;
-    };
-    for (int c = 0; c <= n; ++c) {
-        int mode_c = kModeNone;
-        if (c < n) {
-            const int s = c % G::NSTG, r = c & 1;
-            if (!waitw(&bar[B_PREP + s], (c / G::NSTG) & 1, abort, p, kErrMmaWait)) break;
-            mode_c = *reinterpret_cast<volatile int*>(stage_ptr(s) + G::ST_META + 4);
-            if (c >= 2 && !waitw(&bar[B_OEMPTY + r], ((c >> 1) - 1) & 1, abort, p, kErrMmaWait)) break;
+        if (m1 < n && ready(B_QKFULL + m1 % G::NQK, (m1 / G::NQK) & 1) &&
+            ready(B_PREP + m1 % G::NVS, (m1 / G::NVS) & 1) && (m1 == 0 || ready(B_AEMPTY, (m1 - 1) & 1))) {
             tc_fence_after_sync();
-            const uint64_t dq = make_smem_desc(stage_addr(s) + G::ST_Q, 16, 8 * G::WK, G::WK);
-            const uint64_t dkk = make_smem_desc(stage_addr(s) + G::ST_K, 16, 8 * G::WK, G::WK);
+            const uint64_t dq = make_smem_desc(qk_addr(m1), 16, 8 * G::WK, G::WK);
+            const uint64_t dk = make_smem_desc(qk_addr(m1) + G::Q_BYTES, 16, 8 * G::WK, G::WK);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem + 128 * r, dq + (kstep(kk, G::WK) >> 4), dkk + (kstep(kk, G::WK) >> 4),
-                              G::IDESC_QK, kk > 0);
-                umma_commit(&bar[B_AFULL + r]);
+                    umma_bf16(tmem, dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4), G::IDESC_QK,
+                              kk > 0);
+                umma_commit(&bar[B_AFULL]);
             }
             __syncwarp();
-            if (kv_next == c && mode_c != kModeDirect) {
-                if (!issue_kv(c)) break;
-                ++kv_next;
-            }
+            ++m1;
+            moved = true;
         }
-        if (c >= 1) {
-            const int cp = c - 1, sp = cp % G::NSTG, rp = cp & 1, pb = cp % G::NPB, sbb = cp % G::NSB;
-            if (!waitw(&bar[B_PFULL + pb], (cp / G::NPB) & 1, abort, p, kErrMmaWait)) break;
+        if (kv < m1 && (mode_of(kv) != kModeDirect || kv < pseen) &&
+            (kv < G::NDS || ready(B_DSEMPTY + kv % G::NDS, ((kv / G::NDS) - 1) & 1))) {
+            // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
+            // repeats the key panel when Dk < 128
             tc_fence_after_sync();
-            if (kv_next == cp) {  // direct-form chunk: its keys were decayed by the mask warps
-                if (!issue_kv(cp)) break;
-                ++kv_next;
-            }
-            if (c < n && kv_next == c && mode_c != kModeDirect) {
-                if (!issue_kv(c)) break;
-                ++kv_next;
-            }
-            if (!waitw(&bar[B_SBFULL + sbb], (cp / G::NSB) & 1, abort, p, kErrMmaWait)) break;
-            tc_fence_after_sync();
-            const uint64_t dp = make_smem_desc(sa + G::OFF_P + pb * G::P_BYTES, 16, 8 * 128, 128);
-            const uint64_t dq = make_smem_desc(stage_addr(sp) + G::ST_Q, 16, 8 * G::WK, G::WK);
-            const uint64_t dv = make_smem_desc(stage_addr(sp) + G::ST_V, C * G::WV, 8 * G::WV, G::WV);
-            const uint64_t dsb =
-                make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
+            const int b = kv % G::NDS;
+            const uint64_t dk = make_smem_desc(qk_addr(kv) + G::Q_BYTES, DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
+            const uint64_t dv = make_smem_desc(v_addr(kv), C * G::WV, 8 * G::WV, G::WV);
+            const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + 128 * rp, dp + (kstep(kk, 128) >> 4), dv + ((kk * 16 * G::WV) >> 4),
-                              G::IDESC_PV, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem + 128 * rp, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4),
-                              G::IDESC_PV, 1);
+                    umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
                 if (NORM) {
-                    const uint64_t dzb = make_smem_desc(sa + G::OFF_ZB + sbb * G::ZB_BYTES, 0, 8 * 32, 32);
-                    const uint64_t dw = make_smem_desc(stage_addr(sp) + G::ST_W, 0, 8 * 32, 32);
+                    const uint64_t dw = make_smem_desc(v_addr(kv) + G::VS_W, 0, 8 * 32, 32);
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
-                        umma_bf16(tmem + G::COL_QZ0 + 16 * rp, dp + (kstep(kk, 128) >> 4),
-                                  dw + ((kk * 16 * 32) >> 4), G::IDESC_N16, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16(tmem + G::COL_QZ0 + 16 * rp, dq + (kstep(kk, G::WK) >> 4),
-                                  dzb + ((kk * 16 * 32) >> 4), G::IDESC_N16, 1);
+                        umma_bf16(d + NV, dk + ((kk * 16 * G::WK) >> 4), dw + ((kk * 16 * 32) >> 4), G::IDESC_KV16,
+                                  kk > 0);
                 }
-                umma_commit(&bar[B_OFULL + rp]);
-                umma_commit(&bar[B_PEMPTY + pb]);
-                umma_commit(&bar[B_SBEMPTY + sbb]);
-                umma_commit(&bar[B_EMPTY + sp]);
+                umma_commit(&bar[B_DSFULL + b]);
             }
             __syncwarp();
+            ++kv;
+            moved = true;
+        }
+        if (qs < kv && (qs < G::NO || ready(B_OEMPTY + qs % G::NO, ((qs / G::NO) - 1) & 1)) &&
+            ready(B_SBFULL + qs % G::NSB, (qs / G::NSB) & 1)) {
+            // O = Q S (and den = Q z), opening the accumulator of chunk qs
+            tc_fence_after_sync();
+            const int ro = qs % G::NO, sbb = qs % G::NSB;
+            const uint64_t dq = make_smem_desc(qk_addr(qs), 16, 8 * G::WK, G::WK);
+            const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
+            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
+                if (NORM) {
+                    const uint64_t dzb = make_smem_desc(sa + G::OFF_ZB + sbb * G::ZB_BYTES, 0, 8 * 32, 32);
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16(d + NV, dq + (kstep(kk, G::WK) >> 4), dzb + ((kk * 16 * 32) >> 4), G::IDESC_N16,
+                                  kk > 0);
+                }
+                umma_commit(&bar[B_QKEMPTY + qs % G::NQK]);  // Q K^T, K^T V' and Q S of this chunk have run
+                umma_commit(&bar[B_SBEMPTY + sbb]);
+            }
+            __syncwarp();
+            ++qs;
+            moved = true;
+        }
+        if (pv < qs && pv < pseen) {
+            // P V (and P W) accumulate into the O that Q S opened
+            tc_fence_after_sync();
+            const int pb = pv % G::NPB, ro = pv % G::NO;
+            const uint64_t dv = make_smem_desc(v_addr(pv), C * G::WV, 8 * G::WV, G::WV);
+            const uint32_t pa = tmem + G::COL_P0 + 64 * pb;
+            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
+                if (NORM) {
+                    const uint64_t dw = make_smem_desc(v_addr(pv) + G::VS_W, 0, 8 * 32, 32);
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        umma_bf16_ts(d + NV, pa + 8 * kk, dw + ((kk * 16 * 32) >> 4), G::IDESC_N16, 1);
+                }
+                umma_commit(&bar[B_OFULL + ro]);
+                umma_commit(&bar[B_PEMPTY + pb]);
+                umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
+            }
+            __syncwarp();
+            ++pv;
+            moved = true;
+        }
+        if (moved) {
+            last = global_timer_ns();
+        } else {
+            bool give_up = *abort != 0;
+            if (!give_up && global_timer_ns() - last > kWaitLimitNs) {
+                give_up = true;
+                if (lane == 0) fail(p, abort, kErrMmaWait);
+            }
+            if (__any_sync(0xffffffffu, give_up)) break;
+            __nanosleep(64);
         }
     }
     // everything issued has completed before TMEM is released
@@ -427,28 +471,17 @@ __device__ __noinline__ void role_mma(const Ctx x) {
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
 }
 
+// ------------------------------------------------------------ prep + mask
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_prep_mask(const Ctx x) {
-    using G = Plan<DK, NV, NORM>;
-    const Params& p = *x.p;
-    uint8_t* const sm = x.sm;
-    const uint32_t sa = x.sa, tmem = x.tmem;
-    uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);
-    volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = x.bh, h = x.h, j0 = x.j0, slice = x.slice;
-    const int T = p.T, n = p.nchunks;
-    auto stage_ptr = [&](int s) { return sm + s * G::STAGE; };
-    auto stage_addr = [&](int s) { return sa + s * G::STAGE; };
-    (void)h; (void)j0; (void)slice; (void)T; (void)lane; (void)warp; (void)tmem; (void)stage_addr; (void)stage_ptr;
-    // ------------------------------------------------------------ prep + mask
-    const int wg = (warp - G::W_PM) / 4;  // 0: columns 0-63 and Q rows; 1: columns 64-127 and K rows
+    LA_ROLE_PRELUDE
+    const int wg = (warp - G::W_PM) / 4;  // 0: score columns 0-63, V rows; 1: columns 64-127, weights
     const int wq = warp & 3;
     const int t = 32 * wq + lane;        // TMEM lane = token row
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * wq) << 16);
     const int kind = p.decay_kind;
-    const float* lg = p.log_g + static_cast<size_t>(bh) * T;
-    const float ell_head = kind == LA_DECAY_PER_HEAD ? p.log_g[h] * kLog2e : 0.f;
+    const float* lg = p.log_g + static_cast<size_t>(x.bh) * T;
+    const float ell_head = kind == LA_DECAY_PER_HEAD ? p.log_g[x.h] * kLog2e : 0.f;
     float nxt[4] = {0.f, 0.f, 0.f, 0.f};
     auto fetch = [&](int c) {
 #pragma unroll
@@ -458,64 +491,58 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         }
     };
     fetch(0);
-    // decay prefix of the chunk being prepared (nx_*) and of the chunk being masked (cu_*);
-    // scalars, not arrays indexed by chunk parity, so they stay in registers
+    // decay prefix of the chunk being prepared (nx_*) and of the chunk being masked (cu_*)
     float nx_lt = 0.f, nx_lc = 0.f, cu_lt = 0.f, cu_lc = 0.f;
     int nx_md = kModeNone, cu_md = kModeNone;
 
     auto prep = [&](int c) -> bool {
-        const int s = c % G::NSTG, rem = min(C, T - c * C);
-        float cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+        const int s = c % G::NVS, rem = min(C, T - c * C);
+        const float cur0 = nxt[0], cur1 = nxt[1], cur2 = nxt[2], cur3 = nxt[3];
         fetch(c + 1);
-        if (!waitw(&bar[B_FULL + s], (c / G::NSTG) & 1, abort, p, kErrTmaWait)) return false;
+        if (!waitw(&bar[B_VFULL + s], (c / G::NVS) & 1, abort, p, kErrTmaWait)) return false;
         float lt = 0.f, lc = 0.f;
         if (kind == LA_DECAY_PER_STEP) {
-            float tot[4];
+            float tot0 = cur0 * kLog2e, tot1 = cur1 * kLog2e, tot2 = cur2 * kLog2e, tot3 = cur3 * kLog2e;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float x = cur[i] * kLog2e;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                tot[i] = x;
+            for (int o = 16; o > 0; o >>= 1) {
+                tot0 += __shfl_xor_sync(0xffffffffu, tot0, o);
+                tot1 += __shfl_xor_sync(0xffffffffu, tot1, o);
+                tot2 += __shfl_xor_sync(0xffffffffu, tot2, o);
+                tot3 += __shfl_xor_sync(0xffffffffu, tot3, o);
             }
-            float x = (wq == 0 ? cur[0] : wq == 1 ? cur[1] : wq == 2 ? cur[2] : cur[3]) * kLog2e;
+            float v = (wq == 0 ? cur0 : wq == 1 ? cur1 : wq == 2 ? cur2 : cur3) * kLog2e;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
+                const float y = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += y;
             }
-            float off = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (i < wq) off += tot[i];
-            lt = x + off;
-            lc = tot[0] + tot[1] + tot[2] + tot[3];
+            const float off = (wq > 0 ? tot0 : 0.f) + (wq > 1 ? tot1 : 0.f) + (wq > 2 ? tot2 : 0.f);
+            lt = v + off;
+            lc = tot0 + tot1 + tot2 + tot3;
         } else if (kind == LA_DECAY_PER_HEAD) {
             lt = static_cast<float>(min(t + 1, rem)) * ell_head;
             lc = static_cast<float>(rem) * ell_head;
         }
         const int md = kind == LA_DECAY_NONE ? kModeNone : (-lc <= kFoldLimit ? kModeFolded : kModeDirect);
-        uint8_t* st = stage_ptr(s);
+        uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
         if (wg == 0) {
-            reinterpret_cast<float*>(st + G::ST_LAM)[t] = lt;
+            reinterpret_cast<float*>(st + G::VS_LAM)[t] = lt;
             if (t == 0) {
-                *reinterpret_cast<float*>(st + G::ST_META) = lc;
-                *reinterpret_cast<int*>(st + G::ST_META + 4) = md;
+                *reinterpret_cast<float*>(st + G::VS_META) = lc;
+                *reinterpret_cast<int*>(st + G::VS_META + 4) = md;
             }
-        }
-        if (wg == 0) {
             // output row factor 2^(L_t) of the folded form (1 otherwise); the
             // normalised output does not need it (and has no ring for it)
             if (!NORM)
                 reinterpret_cast<float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] =
                     md == kModeFolded ? ex2_approx(lt) : 1.f;
-            if (md == kModeFolded) scale_row<NV>(st + G::ST_V, t, ex2_approx(-lt));
+            if (md == kModeFolded) scale_row<NV>(st, t, ex2_approx(-lt));
         } else if (NORM) {
             // normaliser weights w_t = 2^(-L_t) (1 unless folded), as a bf16 hi/lo pair
             const float w = md == kModeFolded ? ex2_approx(-lt) : 1.f;
             const float hi = __bfloat162float(__float2bfloat16_rn(w));
-            *reinterpret_cast<uint4*>(st + G::ST_W + swz(t, 0, 32)) = make_uint4(pack2(hi, w - hi), 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(st + G::ST_W + swz(t, 16, 32)) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(st + G::VS_W + swz(t, 0, 32)) = make_uint4(pack2(hi, w - hi), 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(st + G::VS_W + swz(t, 16, 32)) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_async_smem();
         warp_arrive(&bar[B_PREP + s]);
@@ -526,58 +553,65 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     };
 
     auto pmask = [&](int c) -> bool {
-        const int s = c % G::NSTG, pb = c % G::NPB, r = c & 1;
+        const int s = c % G::NVS, pb = c % G::NPB;
         if (c >= G::NPB && !waitw(&bar[B_PEMPTY + pb], ((c / G::NPB) - 1) & 1, abort, p, kErrMmaWait))
             return false;
-        if (!waitw(&bar[B_AFULL + r], (c >> 1) & 1, abort, p, kErrMmaWait)) return false;
-        if (!waitw(&bar[B_PREP + s], (c / G::NSTG) & 1, abort, p, kErrMmaWait)) return false;
+        if (!waitw(&bar[B_AFULL], c & 1, abort, p, kErrMmaWait)) return false;
+        if (!waitw(&bar[B_PREP + s], (c / G::NVS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
-        uint8_t* st = stage_ptr(s);
-        uint8_t* pt = sm + G::OFF_P + pb * G::P_BYTES;  // panel wg holds score columns 64 wg .. 64 wg + 63
-        const float* lam = reinterpret_cast<const float*>(st + G::ST_LAM);
         const float lt = cu_lt, lc = cu_lc;
         const int md = cu_md;
+        const float* lam = reinterpret_cast<const float*>(sm + G::OFF_V + s * G::V_STAGE + G::VS_LAM);
         const bool all_masked = (32 * wq + 31) < 64 * wg;  // every row of this warp precedes these columns
-        uint8_t* prow = pt + wg * C * 128;  // this warpgroup's panel of P
-        if (md != kModeDirect) {
-            // causal mask only: two loads in flight per wait
-            const int lim = all_masked ? -1 : t - 64 * wg;  // keep columns j <= lim of this panel
+        const uint32_t p_addr = lane_addr + G::COL_P0 + 64 * pb + 32 * wg;  // packed pairs of score columns
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float a0[16], a1[16];
-                if (!all_masked) {
-                    tmem_ld16(lane_addr + 128 * r + 64 * wg + 32 * half, a0);
-                    tmem_ld16(lane_addr + 128 * r + 64 * wg + 32 * half + 16, a1);
-                    tmem_wait_ld();
-                }
-                store_masked16(prow, t, 2 * half, a0, lim);
-                store_masked16(prow, t, 2 * half + 1, a1, lim);
-            }
-        } else {
-            // direct form: P = mask(A) * 2^(L_t - L_s), one 16-column piece at a time
-#pragma unroll 1
-            for (int piece = 0; piece < 4; ++piece) {
-                float a[16];
-                if (!all_masked) {
-                    tmem_ld16(lane_addr + 128 * r + 64 * wg + 16 * piece, a);
-                    tmem_wait_ld();
-                }
+        for (int half = 0; half < 2; ++half) {
+            float a0[16], a1[16];
+            if (!all_masked) {
+                tmem_ld16(lane_addr + 64 * wg + 32 * half, a0);
+                tmem_ld16(lane_addr + 64 * wg + 32 * half + 16, a1);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int scol = 64 * wg + 16 * piece + e;
-                    a[e] = (scol <= t && !all_masked) ? a[e] * ex2_approx(lt - lam[scol]) : 0.f;
-                }
-                store_masked16(prow, t, piece, a, 64);
+                for (int e = 0; e < 16; ++e) a0[e] = a1[e] = 0.f;
             }
+            if (half == 1) {  // the score region is free for the next Q K^T
+                tc_fence_before_sync();
+                warp_arrive(&bar[B_AEMPTY]);
+            }
+            const int base = 64 * wg + 32 * half;  // score column of a0[0]
+            uint32_t u[16];
+            if (md != kModeDirect) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s0 = base + 2 * e;
+                    u[e] = pack2(s0 <= t ? a0[2 * e] : 0.f, s0 + 1 <= t ? a0[2 * e + 1] : 0.f);
+                    u[8 + e] = pack2(s0 + 16 <= t ? a1[2 * e] : 0.f, s0 + 17 <= t ? a1[2 * e + 1] : 0.f);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s0 = base + 2 * e;
+                    const float f0 = s0 <= t ? a0[2 * e] * ex2_approx(lt - lam[s0]) : 0.f;
+                    const float f1 = s0 + 1 <= t ? a0[2 * e + 1] * ex2_approx(lt - lam[s0 + 1]) : 0.f;
+                    const float f2 = s0 + 16 <= t ? a1[2 * e] * ex2_approx(lt - lam[s0 + 16]) : 0.f;
+                    const float f3 = s0 + 17 <= t ? a1[2 * e + 1] * ex2_approx(lt - lam[s0 + 17]) : 0.f;
+                    u[e] = pack2(f0, f1);
+                    u[8 + e] = pack2(f2, f3);
+                }
+            }
+            tmem_st16u(p_addr + 16 * half, u);
         }
-        if (md == kModeDirect) {
-            if (wg == 0) scale_row<DK>(st + G::ST_Q, t, ex2_approx(lt));
-            else scale_row<DK>(st + G::ST_K, t, ex2_approx(lc - lt));
+        tmem_wait_st();
+        if (md == kModeDirect) {  // decayed Q and K for this chunk's Q S and K^T V
+            uint8_t* qk = sm + (c % G::NQK) * G::QK_STAGE;
+            if (wg == 0) scale_row<DK>(qk, t, ex2_approx(lt));
+            else scale_row<DK>(qk + G::Q_BYTES, t, ex2_approx(lc - lt));
+            fence_async_smem();
         }
         tc_fence_before_sync();
-        fence_async_smem();
         warp_arrive(&bar[B_PFULL + pb]);
-        warp_arrive(&bar[B_EMPTY + s]);
+        warp_arrive(&bar[B_VEMPTY + s]);
         return true;
     };
 
@@ -592,24 +626,13 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     }
 }
 
+// ------------------------------------------------------------ state + epilogue
+// Warpgroup wg owns value columns [wg NVW, (wg + 1) NVW) of the slice.  Per
+// chunk c: the state update of chunk c (its bf16 copy opens the next chunk's
+// O through Q S) and the epilogue of chunk c - 1.
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_state_epilogue(const Ctx x) {
-    using G = Plan<DK, NV, NORM>;
-    const Params& p = *x.p;
-    uint8_t* const sm = x.sm;
-    const uint32_t sa = x.sa, tmem = x.tmem;
-    uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);
-    volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = x.bh, h = x.h, j0 = x.j0, slice = x.slice;
-    const int T = p.T, n = p.nchunks;
-    auto stage_ptr = [&](int s) { return sm + s * G::STAGE; };
-    auto stage_addr = [&](int s) { return sa + s * G::STAGE; };
-    (void)h; (void)j0; (void)slice; (void)T; (void)lane; (void)warp; (void)tmem; (void)stage_addr; (void)stage_ptr;
-    // ------------------------------------------------------------ state + epilogue
-    // Warpgroup wg owns value columns [wg NVW, (wg + 1) NVW) of the slice.
-    // Per chunk c: the epilogue of chunk c - 1, then the state update of
-    // chunk c (its bf16 copy gates the next chunk's Q S).
+    LA_ROLE_PRELUDE
     const int wg = (warp - G::W_ES) / 4;
     const int wq = warp & 3;
     const int d = 32 * wq + lane;          // key row of S; also token row t of O
@@ -617,6 +640,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     const bool row_ok = d < DK;
     const int cb = wg * G::NVW;            // first column (within the slice) of this warpgroup
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+    const int bh = x.bh, j0 = x.j0;
     float S[G::NVW];
     float z = 0.f;
 #pragma unroll
@@ -625,8 +649,11 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const float* src = p.init_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
 #pragma unroll
         for (int j = 0; j < G::NVW; j += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(src + j);
-            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+            const float4 v4 = *reinterpret_cast<const float4*>(src + j);
+            S[j] = v4.x;
+            S[j + 1] = v4.y;
+            S[j + 2] = v4.z;
+            S[j + 3] = v4.w;
         }
     }
     if (NORM && row_ok && p.init_z) z = p.init_z[static_cast<size_t>(bh) * DK + d];
@@ -645,9 +672,8 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             }
             if (NORM && wg == 0) {
                 const float hi = __bfloat162float(__float2bfloat16_rn(z));
-                const float lo = z - hi;
                 *reinterpret_cast<uint4*>(sm + G::OFF_ZB + buf * G::ZB_BYTES + swz(d, 0, 32)) =
-                    make_uint4(pack2(hi, lo), 0u, 0u, 0u);
+                    make_uint4(pack2(hi, z - hi), 0u, 0u, 0u);
             }
         }
         fence_async_smem();
@@ -655,20 +681,20 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     };
 
     auto state = [&](int c) -> bool {
-        const int s = c % G::NSTG, b = c % G::NDS;
-        if (!waitw(&bar[B_PREP + s], (c / G::NSTG) & 1, abort, p, kErrMmaWait)) return false;
-        const uint8_t* st = stage_ptr(s);
-        const float lc = *reinterpret_cast<const volatile float*>(st + G::ST_META);
-        const int md = *reinterpret_cast<const volatile int*>(st + G::ST_META + 4);
+        const int s = c % G::NVS, b = c % G::NDS;
+        if (!waitw(&bar[B_PREP + s], (c / G::NVS) & 1, abort, p, kErrMmaWait)) return false;
+        const uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
+        const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
+        const int md = *reinterpret_cast<const volatile int*>(st + G::VS_META + 4);
         if (!waitw(&bar[B_DSFULL + b], (c / G::NDS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
-        // S' from the K'^T V tile, 16 columns at a time
         const float e = md == kModeNone ? 1.f : ex2_approx(lc);
+        const uint32_t dsa = lane_addr + G::COL_DS0 + b * G::OCOLS;
         if (warp_rows) {
 #pragma unroll
             for (int j = 0; j < G::NVW; j += 16) {
                 float ds[16];
-                tmem_ld16(lane_addr + G::COL_DS0 + b * NV + cb + j, ds);
+                tmem_ld16(dsa + cb + j, ds);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -679,33 +705,34 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             }
             if (NORM && wg == 0) {
                 float zz[16];
-                tmem_ld16(lane_addr + G::COL_ZS0 + 16 * b, zz);
+                tmem_ld16(dsa + NV, zz);
                 tmem_wait_ld();
-                if (md == kModeFolded) z = e * (z + zz[0]);
-                else if (md == kModeDirect) z = fmaf(e, z, zz[0]);
-                else z += zz[0];
+                const float zs = zz[0] + zz[1];
+                if (md == kModeFolded) z = e * (z + zs);
+                else if (md == kModeDirect) z = fmaf(e, z, zs);
+                else z += zs;
             }
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_DSEMPTY + b]);
-        warp_arrive(&bar[B_EMPTY + s]);
+        warp_arrive(&bar[B_VEMPTY + s]);
         if (c == n - 1) return true;
         const int k = c + 1;
-        if (k >= G::NSB &&
-            !waitw(&bar[B_SBEMPTY + k % G::NSB], ((k / G::NSB) - 1) & 1, abort, p, kErrMmaWait))
+        if (k >= G::NSB && !waitw(&bar[B_SBEMPTY + k % G::NSB], ((k / G::NSB) - 1) & 1, abort, p, kErrMmaWait))
             return false;
         write_copy(k);
         return true;
     };
 
     auto epilogue = [&](int c) -> bool {
-        const int r = c & 1, t = d;
-        if (!waitw(&bar[B_OFULL + r], (c >> 1) & 1, abort, p, kErrMmaWait)) return false;
+        const int ro = c % G::NO, t = d;
+        if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
+        const uint32_t oa = lane_addr + G::COL_O0 + ro * G::OCOLS;
         float inv;  // y = O * inv
         if (NORM) {
             float dd[16];
-            tmem_ld16(lane_addr + G::COL_QZ0 + 16 * r, dd);
+            tmem_ld16(oa + NV, dd);
             tmem_wait_ld();
             inv = 1.f / (dd[0] + dd[1]);
         } else {
@@ -714,12 +741,11 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const int rem = min(C, T - c * C);
         __nv_bfloat16* dst =
             p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(c) * C + t) * p.Dv + j0 + cb;
-        constexpr int NB = G::NVW < 64 ? G::NVW / 16 : 4;  // pieces loaded per wait
 #pragma unroll
         for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
-            tmem_ld16(lane_addr + 128 * r + cb + 16 * piece, o);
-            if (piece % NB == NB - 1) tmem_wait_ld();
+            tmem_ld16(oa + cb + 16 * piece, o);
+            tmem_wait_ld();
             if (t < rem) {
                 uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * piece);
                 d4[0] = make_uint4(pack2(o[0] * inv, o[1] * inv), pack2(o[2] * inv, o[3] * inv),
@@ -729,18 +755,20 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             }
         }
         tc_fence_before_sync();
-        warp_arrive(&bar[B_OEMPTY + r]);
+        warp_arrive(&bar[B_OEMPTY + ro]);
         return true;
     };
 
-    // The epilogue of chunk c - 1 runs before the state update of chunk c:
-    // for a direct-form chunk c the MMA warp issues K~^T V(c) only after
-    // this warpgroup has released the TMEM region of chunk c - 1.
+    // The state update of chunk c gates the next chunk's Q S, so it goes
+    // first, unless both the O buffer and the state copy are single: then
+    // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
+    constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
     write_copy(0);
     bool ok = true;
     for (int c = 0; c < n && ok; ++c) {
-        if (c >= 1) ok = epilogue(c - 1);
+        if (!kStateFirst && c >= 1) ok = epilogue(c - 1);
         if (ok) ok = state(c);
+        if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
     }
     if (ok && n > 0) ok = epilogue(n - 1);
     if (ok && !*abort && row_ok) {
@@ -750,7 +778,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             for (int j = 0; j < G::NVW; j += 4)
                 *reinterpret_cast<float4*>(fs + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
-        if (NORM && p.final_z && slice == 0 && wg == 0) p.final_z[static_cast<size_t>(bh) * DK + d] = z;
+        if (NORM && p.final_z && x.slice == 0 && wg == 0) p.final_z[static_cast<size_t>(bh) * DK + d] = z;
     }
 }
 
@@ -766,27 +794,27 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + G::OFF_MISC + 8 * B_COUNT);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
 
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int tid = threadIdx.x, warp = tid / 32;
     const int bh = blockIdx.x / p.split, slice = blockIdx.x % p.split;
-    const int h = bh % p.H;
-    const int j0 = slice * NV;
-    const int T = p.T, n = p.nchunks;
 
     if (tid == 0) {
         prefetch_tensormap(&tmq);
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
         for (int s = 0; s < 4; ++s) {
-            mbar_init(&bar[B_FULL + s], 1);
-            mbar_init(&bar[B_EMPTY + s], G::EMPTY_ARRIVALS);
+            mbar_init(&bar[B_QKFULL + s], 1);
+            mbar_init(&bar[B_QKEMPTY + s], 1);
+            mbar_init(&bar[B_VFULL + s], 1);
+            mbar_init(&bar[B_VEMPTY + s], G::VEMPTY_ARRIVALS);
             mbar_init(&bar[B_PREP + s], 8);
         }
+        mbar_init(&bar[B_AFULL], 1);
+        mbar_init(&bar[B_AEMPTY], 8);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar[B_AFULL + i], 1);
-            mbar_init(&bar[B_OFULL + i], 1);
-            mbar_init(&bar[B_OEMPTY + i], 4 * G::NSW);
             mbar_init(&bar[B_PFULL + i], 8);
             mbar_init(&bar[B_PEMPTY + i], 1);
+            mbar_init(&bar[B_OFULL + i], 1);
+            mbar_init(&bar[B_OEMPTY + i], 4 * G::NSW);
             mbar_init(&bar[B_DSFULL + i], 1);
             mbar_init(&bar[B_DSEMPTY + i], 4 * G::NSW);
             mbar_init(&bar[B_SBFULL + i], 4 * G::NSW);
@@ -799,8 +827,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_MMA) tmem_alloc(tmem_slot, G::TMEM_COLS);
     if (NORM && warp >= G::W_ES && warp < G::W_ES + 4) {
         // zeroed key-sum tiles (only their first two columns are ever written)
-        const int t = tid - 32 * G::W_ES;
-        for (int i = t; i < G::NSB * G::ZB_BYTES / 16; i += 128)
+        for (int i = tid - 32 * G::W_ES; i < G::NSB * G::ZB_BYTES / 16; i += 128)
             reinterpret_cast<uint4*>(sm + G::OFF_ZB)[i] = make_uint4(0u, 0u, 0u, 0u);
         fence_async_smem();
     }
@@ -808,15 +835,18 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const Ctx x{&p, sm, sa, tmem, bh, h, j0, slice};
+
+    const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice};
     if (warp == G::W_TMA) {
-        role_tma<DK, NV, NORM>(x, &tmq, &tmk, &tmv);
+        role_tma_qk<DK, NV, NORM>(x, &tmq, &tmk);
     } else if (warp == G::W_MMA) {
         role_mma<DK, NV, NORM>(x);
     } else if (warp < G::W_ES) {
         role_prep_mask<DK, NV, NORM>(x);
-    } else {
+    } else if (warp < G::W_TMAV) {
         role_state_epilogue<DK, NV, NORM>(x);
+    } else {
+        role_tma_v<DK, NV, NORM>(x, &tmv);
     }
 
     __syncwarp();  // lanes that idled while lane 0 ran a single-thread role rejoin it
