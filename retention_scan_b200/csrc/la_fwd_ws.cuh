@@ -31,21 +31,22 @@
 // share the factor 2^(L_t), which cancels.  The key-sum update uses
 // K^T [w_hi w_lo 0 ..].
 //
-// Data flow.  Q and K tiles sit in one TMA ring, V tiles (with the chunk's
-// decay prefix) in another.  The inter-chunk term Q S is accumulated first,
-// so a chunk's Q and K are released as soon as Q K^T, K^T V' and Q S have
-// run, long before its P V; P lives in tensor memory (the A operand of P V
-// is read from TMEM), which keeps shared memory for the rings.
+// Data flow.  Q, K and V tiles (the V stage with the chunk's decay prefix)
+// sit in three TMA rings.  A K stage is free once Q K^T and K^T V' have run;
+// a Q stage only after Q S, which waits for the state of the previous chunk,
+// so the Q ring is the deeper one.  The inter-chunk term Q S is accumulated
+// first, long before P V; P lives in tensor memory (the A operand of P V is
+// read from TMEM), which keeps shared memory for the rings.
 //
 // Roles (one CTA = one (b, h) and NV of its Dv columns; Dv / NV CTAs share a
 // head and read its q, k through L2):
-//   warp 0       TMA producer of the Q/K ring
+//   warp 0       TMA producer of the Q ring
 //   warp 1       MMA issuer (one elected lane) and TMEM owner
 //   warps 2-9    two warpgroups: prep (decay prefix, value-row scaling,
 //                normaliser weights) and mask (scores -> P in TMEM); warpgroup
 //                0 owns score columns 0-63, warpgroup 1 columns 64-127
 //   warps 10-..  state and epilogue (one warpgroup per 64 value columns)
-//   last warp    TMA producer of the V ring
+//   last warp    TMA producer of the K and V rings
 // Every hand-off is an mbarrier; every wait gives up after kWaitLimitNs (then
 // the CTA sets the device error word and unwinds).
 #pragma once
@@ -73,23 +74,25 @@ __host__ __device__ constexpr int round1k(int x) { return (x + 1023) / 1024 * 10
 
 // Barrier slots (uint64 each) at the start of the MISC area.
 enum Bar : int {
-    B_QKFULL = 0,    // [4] Q/K tiles landed
-    B_QKEMPTY = 4,   // [4] Q/K stage free (Q K^T, K^T V', Q S done)
-    B_VFULL = 8,     // [4] V tile landed
-    B_VEMPTY = 12,   // [4] V stage free (P V done, its prefix read)
-    B_PREP = 16,     // [4] decay prefix, value scaling, weights done
-    B_AFULL = 20,    // scores in TMEM
-    B_AEMPTY = 21,   // scores read by the mask warps
-    B_PFULL = 22,    // [2] P in TMEM
-    B_PEMPTY = 24,   // [2] P V done reading P
-    B_OFULL = 26,    // [2] O (and den) complete
-    B_OEMPTY = 28,   // [2] epilogue done with O
-    B_DSFULL = 30,   // [2] K^T V' in TMEM
-    B_DSEMPTY = 32,  // [2] state warps done with it
-    B_SBFULL = 34,   // [2] bf16 state copy written
-    B_SBEMPTY = 36,  // [2] Q S done reading it
-    B_DRAIN = 38,
-    B_COUNT = 39
+    B_QFULL = 0,     // [4] Q tile landed
+    B_QEMPTY = 4,    // [4] Q stage free (Q K^T and Q S done)
+    B_KFULL = 8,     // [4] K tile landed
+    B_KEMPTY = 12,   // [4] K stage free (Q K^T and K^T V' done)
+    B_VFULL = 16,    // [4] V tile landed
+    B_VEMPTY = 20,   // [4] V stage free (P V done, its prefix read)
+    B_PREP = 24,     // [4] decay prefix, value scaling, weights done
+    B_AFULL = 28,    // scores in TMEM
+    B_AEMPTY = 29,   // scores read by the mask warps
+    B_PFULL = 30,    // [2] P in TMEM
+    B_PEMPTY = 32,   // [2] P V done reading P
+    B_OFULL = 34,    // [2] O (and den) complete
+    B_OEMPTY = 36,   // [2] epilogue done with O
+    B_DSFULL = 38,   // [2] K^T V' in TMEM
+    B_DSEMPTY = 40,  // [2] state warps done with it
+    B_SBFULL = 42,   // [2] bf16 state copy written
+    B_SBEMPTY = 44,  // [2] Q S done reading it
+    B_DRAIN = 46,
+    B_COUNT = 47
 };
 
 template <int DK, int NV, bool NORM>
@@ -98,8 +101,8 @@ struct Plan {
     static constexpr int WV = row_bytes_for(NV), PV = panels_for(NV);
     static constexpr int Q_BYTES = C * DK * 2;
     static constexpr int V_BYTES = C * NV * 2;
-    // Q/K stage: Q | K
-    static constexpr int QK_STAGE = round1k(2 * Q_BYTES);
+    // Q and K stages (one tile each)
+    static constexpr int Q_STAGE = round1k(Q_BYTES);
     // V stage: V | W (normaliser weights, [C x 16] bf16, 32-byte swizzle) | L (float[C], log2) | meta
     static constexpr int VS_W = V_BYTES;
     static constexpr int VS_LAM = VS_W + (NORM ? C * 32 : 0);
@@ -111,23 +114,40 @@ struct Plan {
     // chunks (not needed with the normaliser, where the factor cancels).
     static constexpr int kRowfRing = 8;
     static constexpr int MISC = 1024 + (NORM ? 0 : kRowfRing * C * 4);
-    static constexpr bool fits(int nqk, int nvs, int nsb) {
-        return nqk * QK_STAGE + nvs * V_STAGE + nsb * (SB_BYTES + ZB_BYTES) + MISC + 1024 <= kSmemLimit;
+    static constexpr bool fits(int nq, int nk, int nvs, int nsb) {
+        return (nq + nk) * Q_STAGE + nvs * V_STAGE + nsb * (SB_BYTES + ZB_BYTES) + MISC + 1024 <= kSmemLimit;
     }
-    // deepest Q/K ring first, then V ring (at least as deep), then state copies
+    // A ring of depth n whose stages each stay busy for a time L allows one
+    // chunk per L / n.  Rough busy times (arbitrary units): a Q stage from its
+    // load to the chunk's Q S, which waits for the state chain (40); a V stage
+    // to its P V, after Q S (45); a K stage only to K^T V' (25).  A single
+    // state copy adds a little.  The fitting plan with the smallest bound wins.
+    static constexpr int bound(int nq, int nk, int nvs, int nsb) {
+        int b = 400 / nq;
+        if (250 / nk > b) b = 250 / nk;
+        if (450 / nvs > b) b = 450 / nvs;
+        return b + (nsb == 1 ? 20 : 0);
+    }
     static constexpr int pick() {
-        for (int nqk = 4; nqk >= 2; --nqk)
-            for (int nvs = 4; nvs >= nqk; --nvs)
-                for (int nsb = 2; nsb >= 1; --nsb)
-                    if (fits(nqk, nvs, nsb)) return nqk * 100 + nvs * 10 + nsb;
-        return 0;
+        int best = 0, bb = 1 << 30;
+        for (int nq = 4; nq >= 2; --nq)
+            for (int nk = 4; nk >= 2; --nk)
+                for (int nvs = 4; nvs >= 2; --nvs)
+                    for (int nsb = 2; nsb >= 1; --nsb)
+                        if (fits(nq, nk, nvs, nsb) && bound(nq, nk, nvs, nsb) < bb) {
+                            bb = bound(nq, nk, nvs, nsb);
+                            best = nq * 1000 + nk * 100 + nvs * 10 + nsb;
+                        }
+        return best;
     }
     static constexpr int PICK = pick();
     static constexpr bool OK = PICK != 0;
-    static constexpr int NQK = OK ? PICK / 100 : 2;
+    static constexpr int NQ = OK ? PICK / 1000 : 2;
+    static constexpr int NK = OK ? (PICK / 100) % 10 : 2;
     static constexpr int NVS = OK ? (PICK / 10) % 10 : 2;
     static constexpr int NSB = OK ? PICK % 10 : 1;
-    static constexpr int OFF_V = NQK * QK_STAGE;
+    static constexpr int OFF_K = NQ * Q_STAGE;
+    static constexpr int OFF_V = OFF_K + NK * Q_STAGE;
     static constexpr int OFF_SB = OFF_V + NVS * V_STAGE;
     static constexpr int OFF_ZB = OFF_SB + NSB * SB_BYTES;
     static constexpr int OFF_MISC = OFF_ZB + NSB * ZB_BYTES;
@@ -152,7 +172,7 @@ struct Plan {
     static constexpr int NWARPS = W_TMAV + 1;
     static constexpr int THREADS = 32 * NWARPS;
     static constexpr int VEMPTY_ARRIVALS = 1 + 8 + 4 * NSW;
-    static constexpr uint32_t QK_TX = 2 * Q_BYTES;
+    static constexpr uint32_t Q_TX = Q_BYTES;
     static constexpr uint32_t V_TX = V_BYTES;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NV, 0, 1);
@@ -164,6 +184,7 @@ struct Plan {
     static_assert(DK == 16 || DK == 32 || DK == 64 || DK == 128, "key width");
     static_assert(kRowfRing >= NVS + 1, "row factor ring too shallow");
     static_assert(8 * B_COUNT + 8 <= 1024, "barrier area");
+    static_assert(!OK || (OFF_K % 1024 == 0 && OFF_V % 1024 == 0), "stages aligned for 128-byte swizzle");
     static_assert(!OK || SMEM <= kSmemLimit, "shared memory limit");
     static_assert(!OK || NORM || OFF_ROWF + kRowfRing * C * 4 <= SMEM - 1024, "row factor ring inside allocation");
 };
@@ -199,10 +220,10 @@ __device__ __forceinline__ void fail(const Params& p, volatile int* abort, int c
 
 constexpr uint32_t kSleepHintNs = 20000;  // longest single sleep inside a wait
 
-// Single-thread bounded wait; sleeps in the barrier between checks.
-__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
-                                      int code) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow paths of the bounded waits, kept out of line so that the hot loops stay
+// small in the instruction cache.
+static __device__ __noinline__ bool wait1_slow(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
+                                        int code) {
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
@@ -214,11 +235,8 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile i
     }
 }
 
-// Whole-warp bounded wait; every lane gets the same answer.
-__device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
-                                      int code) {
-    bool ok = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, ok)) return true;
+static __device__ __noinline__ bool waitw_slow(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
+                                        int code, bool ok) {
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (!ok) ok = mbar_try_wait_sleep(bar, parity, kSleepHintNs);
@@ -230,6 +248,21 @@ __device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile i
             return false;
         }
     }
+}
+
+// Single-thread bounded wait; sleeps in the barrier between checks.
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
+                                      int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait1_slow(bar, parity, abort, p, code);
+}
+
+// Whole-warp bounded wait; every lane gets the same answer.
+__device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile int* abort, const Params& p,
+                                      int code) {
+    const bool ok = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    return waitw_slow(bar, parity, abort, p, code, ok);
 }
 
 __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
@@ -290,54 +323,85 @@ __host__ __device__ constexpr uint32_t kstep(int kk, int W) {
     (void)lane;
 
 // ------------------------------------------------------------ TMA producers
+// Q ring: one thread, blocking on each stage in turn.
 template <int DK, int NV, bool NORM>
-__device__ __noinline__ void role_tma_qk(const Ctx x, const CUtensorMap* tmq, const CUtensorMap* tmk) {
+__device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
     LA_ROLE_PRELUDE
     if (lane != 0) return;
     int issued = 0;
     for (int c = 0; c < n; ++c) {
-        const int s = c % G::NQK;
-        if (c >= G::NQK && !wait1(&bar[B_QKEMPTY + s], ((c / G::NQK) - 1) & 1, abort, p, kErrTmaWait)) break;
-        mbar_arrive_expect_tx(&bar[B_QKFULL + s], G::QK_TX);
-        uint8_t* st = sm + s * G::QK_STAGE;
-        for (int pp = 0; pp < G::PK; ++pp) {
-            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QKFULL + s], pp * 64, c * C, x.bh);
-            tma_load_3d(st + G::Q_BYTES + pp * C * G::WK, tmk, &bar[B_QKFULL + s], pp * 64, c * C, x.bh);
-        }
+        const int s = c % G::NQ;
+        if (c >= G::NQ && !wait1(&bar[B_QEMPTY + s], ((c / G::NQ) - 1) & 1, abort, p, kErrTmaWait)) break;
+        mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
+        uint8_t* st = sm + s * G::Q_STAGE;
+        for (int pp = 0; pp < G::PK; ++pp)
+            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * 64, c * C, x.bh);
         ++issued;
     }
     if (*abort) {  // let issued copies land before the CTA's shared memory goes away
-        for (int c = issued > G::NQK ? issued - G::NQK : 0; c < issued; ++c)
-            mbar_wait_bounded(&bar[B_QKFULL + c % G::NQK], (c / G::NQK) & 1, kWaitLimitNs);
+        for (int c = issued > G::NQ ? issued - G::NQ : 0; c < issued; ++c)
+            mbar_wait_bounded(&bar[B_QFULL + c % G::NQ], (c / G::NQ) & 1, kWaitLimitNs);
     }
 }
 
+// K and V rings: one thread polls both, so that neither waits behind the
+// other's free stage.  V runs as far ahead as its ring allows: the prep of
+// chunk c + 1 (which needs V) runs before the mask of chunk c.
 template <int DK, int NV, bool NORM>
-__device__ __noinline__ void role_tma_v(const Ctx x, const CUtensorMap* tmv) {
+__device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, const CUtensorMap* tmv) {
     LA_ROLE_PRELUDE
     if (lane != 0) return;
-    int issued = 0;
-    for (int c = 0; c < n; ++c) {
-        const int s = c % G::NVS;
-        if (c >= G::NVS && !wait1(&bar[B_VEMPTY + s], ((c / G::NVS) - 1) & 1, abort, p, kErrTmaWait)) break;
-        mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
-        uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
-        for (int pp = 0; pp < G::PV; ++pp)
-            tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, c * C, x.bh);
-        ++issued;
+    int ck = 0, cv = 0;
+    uint64_t last = global_timer_ns();
+    while (ck < n || cv < n) {
+        bool moved = false;
+        if (ck < n &&
+            (ck < G::NK || mbar_test(&bar[B_KEMPTY + ck % G::NK], ((ck / G::NK) - 1) & 1))) {
+            const int s = ck % G::NK;
+            mbar_arrive_expect_tx(&bar[B_KFULL + s], G::Q_TX);
+            uint8_t* st = sm + G::OFF_K + s * G::Q_STAGE;
+            for (int pp = 0; pp < G::PK; ++pp)
+                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * 64, ck * C, x.bh);
+            ++ck;
+            moved = true;
+        }
+        if (cv < n &&
+            (cv < G::NVS || mbar_test(&bar[B_VEMPTY + cv % G::NVS], ((cv / G::NVS) - 1) & 1))) {
+            const int s = cv % G::NVS;
+            mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
+            uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
+            for (int pp = 0; pp < G::PV; ++pp)
+                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, cv * C, x.bh);
+            ++cv;
+            moved = true;
+        }
+        if (moved) {
+            last = global_timer_ns();
+        } else {
+            if (*abort) break;
+            if (global_timer_ns() - last > kWaitLimitNs) {
+                fail(p, abort, kErrTmaWait);
+                break;
+            }
+            __nanosleep(128);
+        }
     }
     if (*abort) {
-        for (int c = issued > G::NVS ? issued - G::NVS : 0; c < issued; ++c)
+        for (int c = ck > G::NK ? ck - G::NK : 0; c < ck; ++c)
+            mbar_wait_bounded(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, kWaitLimitNs);
+        for (int c = cv > G::NVS ? cv - G::NVS : 0; c < cv; ++c)
             mbar_wait_bounded(&bar[B_VFULL + c % G::NVS], (c / G::NVS) & 1, kWaitLimitNs);
     }
 }
 
 // ------------------------------------------------------------ MMA issuer
 // Four in-order queues, each issued as soon as its inputs are there:
-//   Q K^T (c)   Q/K tiles and prep of c landed, score region free
-//   K^T V' (j)  after Q K^T (j); a direct-form chunk also after its mask,
-//               which decays Q and K; K^T V' buffer free
-//   Q S (j)     after K^T V' (j); O buffer free; bf16 state after j - 1 written
+//   Q K^T (c)   Q and K tiles of c landed, score region free
+//   K^T V' (j)  after Q K^T (j) and the prep of j; a direct-form chunk also
+//               after its mask, which decays Q and K; K^T V' buffer free;
+//               releases the K stage
+//   Q S (j)     after K^T V' (j); O buffer free; bf16 state after j - 1
+//               written; releases the Q stage
 //   P V (j)     after Q S (j), which opened the accumulator; P (j) written
 // The warp polls the barriers (never blocking on one while another queue
 // could move) and gives up after kWaitLimitNs without progress.
@@ -348,7 +412,8 @@ __device__ __noinline__ void role_mma(const Ctx x) {
     auto mode_of = [&](int j) {
         return *reinterpret_cast<volatile int*>(sm + G::OFF_V + (j % G::NVS) * G::V_STAGE + G::VS_META + 4);
     };
-    auto qk_addr = [&](int j) { return sa + (j % G::NQK) * G::QK_STAGE; };
+    auto q_addr = [&](int j) { return sa + (j % G::NQ) * G::Q_STAGE; };
+    auto k_addr = [&](int j) { return sa + G::OFF_K + (j % G::NK) * G::Q_STAGE; };
     auto v_addr = [&](int j) { return sa + G::OFF_V + (j % G::NVS) * G::V_STAGE; };
     auto ready = [&](int slot, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(&bar[slot], parity)); };
 
@@ -360,11 +425,11 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             ++pseen;
             moved = true;
         }
-        if (m1 < n && ready(B_QKFULL + m1 % G::NQK, (m1 / G::NQK) & 1) &&
-            ready(B_PREP + m1 % G::NVS, (m1 / G::NVS) & 1) && (m1 == 0 || ready(B_AEMPTY, (m1 - 1) & 1))) {
+        if (m1 < n && ready(B_QFULL + m1 % G::NQ, (m1 / G::NQ) & 1) && ready(B_KFULL + m1 % G::NK, (m1 / G::NK) & 1) &&
+            (m1 == 0 || ready(B_AEMPTY, (m1 - 1) & 1))) {
             tc_fence_after_sync();
-            const uint64_t dq = make_smem_desc(qk_addr(m1), 16, 8 * G::WK, G::WK);
-            const uint64_t dk = make_smem_desc(qk_addr(m1) + G::Q_BYTES, 16, 8 * G::WK, G::WK);
+            const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
+            const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
@@ -376,13 +441,13 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             ++m1;
             moved = true;
         }
-        if (kv < m1 && (mode_of(kv) != kModeDirect || kv < pseen) &&
+        if (kv < m1 && ready(B_PREP + kv % G::NVS, (kv / G::NVS) & 1) && (mode_of(kv) != kModeDirect || kv < pseen) &&
             (kv < G::NDS || ready(B_DSEMPTY + kv % G::NDS, ((kv / G::NDS) - 1) & 1))) {
             // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
             // repeats the key panel when Dk < 128
             tc_fence_after_sync();
             const int b = kv % G::NDS;
-            const uint64_t dk = make_smem_desc(qk_addr(kv) + G::Q_BYTES, DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
+            const uint64_t dk = make_smem_desc(k_addr(kv), DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
             const uint64_t dv = make_smem_desc(v_addr(kv), C * G::WV, 8 * G::WV, G::WV);
             const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
             if (leader) {
@@ -397,6 +462,7 @@ __device__ __noinline__ void role_mma(const Ctx x) {
                                   kk > 0);
                 }
                 umma_commit(&bar[B_DSFULL + b]);
+                umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
             }
             __syncwarp();
             ++kv;
@@ -407,7 +473,7 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             // O = Q S (and den = Q z), opening the accumulator of chunk qs
             tc_fence_after_sync();
             const int ro = qs % G::NO, sbb = qs % G::NSB;
-            const uint64_t dq = make_smem_desc(qk_addr(qs), 16, 8 * G::WK, G::WK);
+            const uint64_t dq = make_smem_desc(q_addr(qs), 16, 8 * G::WK, G::WK);
             const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
             const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
             if (leader) {
@@ -421,7 +487,7 @@ __device__ __noinline__ void role_mma(const Ctx x) {
                         umma_bf16(d + NV, dq + (kstep(kk, G::WK) >> 4), dzb + ((kk * 16 * 32) >> 4), G::IDESC_N16,
                                   kk > 0);
                 }
-                umma_commit(&bar[B_QKEMPTY + qs % G::NQK]);  // Q K^T, K^T V' and Q S of this chunk have run
+                umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // Q K^T and Q S of this chunk have run
                 umma_commit(&bar[B_SBEMPTY + sbb]);
             }
             __syncwarp();
@@ -472,6 +538,47 @@ __device__ __noinline__ void role_mma(const Ctx x) {
 }
 
 // ------------------------------------------------------------ prep + mask
+// Mask of a direct-form chunk (total decay beyond the fold limit), out of line
+// because it is rare: P = mask(A) * 2^(L_t - L_s), written as bf16 pairs at
+// p_addr; then this thread's row of the chunk's Q tile (warpgroup 0) or K tile
+// (warpgroup 1), given as `tile`, is decayed in place for its Q S and K^T V.
+template <int DK>
+__device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint64_t* aempty, int wg, int t,
+                                         bool all_masked, float lt, float lc, const float* lam, uint8_t* tile) {
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        float a0[16], a1[16];
+        if (!all_masked) {
+            tmem_ld16(s_addr + 32 * half, a0);
+            tmem_ld16(s_addr + 32 * half + 16, a1);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) a0[e] = a1[e] = 0.f;
+        }
+        if (half == 1) {
+            tc_fence_before_sync();
+            warp_arrive(aempty);
+        }
+        const int base = 64 * wg + 32 * half;
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int s0 = base + 2 * e;
+            const float f0 = s0 <= t ? a0[2 * e] * ex2_approx(lt - lam[s0]) : 0.f;
+            const float f1 = s0 + 1 <= t ? a0[2 * e + 1] * ex2_approx(lt - lam[s0 + 1]) : 0.f;
+            const float f2 = s0 + 16 <= t ? a1[2 * e] * ex2_approx(lt - lam[s0 + 16]) : 0.f;
+            const float f3 = s0 + 17 <= t ? a1[2 * e + 1] * ex2_approx(lt - lam[s0 + 17]) : 0.f;
+            u[e] = pack2(f0, f1);
+            u[8 + e] = pack2(f2, f3);
+        }
+        tmem_st16u(p_addr + 16 * half, u);
+    }
+    tmem_wait_st();
+    scale_row<DK>(tile, t, ex2_approx(wg == 0 ? lt : lc - lt));
+    fence_async_smem();
+}
+
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_prep_mask(const Ctx x) {
     LA_ROLE_PRELUDE
@@ -490,19 +597,25 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             nxt[i] = (kind == LA_DECAY_PER_STEP && c < n && row < T) ? lg[row] : 0.f;
         }
     };
-    fetch(0);
-    // decay prefix of the chunk being prepared (nx_*) and of the chunk being masked (cu_*)
-    float nx_lt = 0.f, nx_lc = 0.f, cu_lt = 0.f, cu_lc = 0.f;
-    int nx_md = kModeNone, cu_md = kModeNone;
+    if (wg == 0 || NORM) fetch(0);
 
+    // Warpgroup 0 computes the chunk's decay prefix, writes it (and the
+    // mode) into the V stage, the output row factors and the scaled value
+    // rows; warpgroup 1 writes the normaliser weights, or has nothing to do.
     auto prep = [&](int c) -> bool {
         const int s = c % G::NVS, rem = min(C, T - c * C);
+        if (!NORM && wg == 1) {
+            warp_arrive(&bar[B_PREP + s]);
+            return true;
+        }
         const float cur0 = nxt[0], cur1 = nxt[1], cur2 = nxt[2], cur3 = nxt[3];
         fetch(c + 1);
         if (!waitw(&bar[B_VFULL + s], (c / G::NVS) & 1, abort, p, kErrTmaWait)) return false;
-        float lt = 0.f, lc = 0.f;
+        // chunk-local log2 decay prefix L_t and total L_C
+        float lt, lc;
         if (kind == LA_DECAY_PER_STEP) {
             float tot0 = cur0 * kLog2e, tot1 = cur1 * kLog2e, tot2 = cur2 * kLog2e, tot3 = cur3 * kLog2e;
+            float v = (wq == 0 ? cur0 : wq == 1 ? cur1 : wq == 2 ? cur2 : cur3) * kLog2e;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 tot0 += __shfl_xor_sync(0xffffffffu, tot0, o);
@@ -510,16 +623,14 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                 tot2 += __shfl_xor_sync(0xffffffffu, tot2, o);
                 tot3 += __shfl_xor_sync(0xffffffffu, tot3, o);
             }
-            float v = (wq == 0 ? cur0 : wq == 1 ? cur1 : wq == 2 ? cur2 : cur3) * kLog2e;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, v, o);
                 if (lane >= o) v += y;
             }
-            const float off = (wq > 0 ? tot0 : 0.f) + (wq > 1 ? tot1 : 0.f) + (wq > 2 ? tot2 : 0.f);
-            lt = v + off;
+            lt = v + (wq > 0 ? tot0 : 0.f) + (wq > 1 ? tot1 : 0.f) + (wq > 2 ? tot2 : 0.f);
             lc = tot0 + tot1 + tot2 + tot3;
-        } else if (kind == LA_DECAY_PER_HEAD) {
+        } else {  // per head (ell_head = L per step), or none (ell_head = 0)
             lt = static_cast<float>(min(t + 1, rem)) * ell_head;
             lc = static_cast<float>(rem) * ell_head;
         }
@@ -537,7 +648,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                 reinterpret_cast<float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] =
                     md == kModeFolded ? ex2_approx(lt) : 1.f;
             if (md == kModeFolded) scale_row<NV>(st, t, ex2_approx(-lt));
-        } else if (NORM) {
+        } else {
             // normaliser weights w_t = 2^(-L_t) (1 unless folded), as a bf16 hi/lo pair
             const float w = md == kModeFolded ? ex2_approx(-lt) : 1.f;
             const float hi = __bfloat162float(__float2bfloat16_rn(w));
@@ -546,9 +657,6 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         }
         fence_async_smem();
         warp_arrive(&bar[B_PREP + s]);
-        nx_lt = lt;
-        nx_lc = lc;
-        nx_md = md;
         return true;
     };
 
@@ -559,55 +667,52 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         if (!waitw(&bar[B_AFULL], c & 1, abort, p, kErrMmaWait)) return false;
         if (!waitw(&bar[B_PREP + s], (c / G::NVS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
-        const float lt = cu_lt, lc = cu_lc;
-        const int md = cu_md;
-        const float* lam = reinterpret_cast<const float*>(sm + G::OFF_V + s * G::V_STAGE + G::VS_LAM);
-        const bool all_masked = (32 * wq + 31) < 64 * wg;  // every row of this warp precedes these columns
+        const uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
+        const int md = *reinterpret_cast<const volatile int*>(st + G::VS_META + 4);
         const uint32_t p_addr = lane_addr + G::COL_P0 + 64 * pb + 32 * wg;  // packed pairs of score columns
+        if (md == kModeDirect) {
+            const float* lam = reinterpret_cast<const float*>(st + G::VS_LAM);
+            const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
+            const bool all_masked = (32 * wq + 31) < 64 * wg;  // every row of this warp precedes these columns
+            mask_direct<DK>(lane_addr + 64 * wg, p_addr, &bar[B_AEMPTY], wg, t, all_masked, lam[t], lc, lam,
+                            wg == 0 ? sm + (c % G::NQ) * G::Q_STAGE : sm + G::OFF_K + (c % G::NK) * G::Q_STAGE);
+        } else {
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            float a0[16], a1[16];
-            if (!all_masked) {
-                tmem_ld16(lane_addr + 64 * wg + 32 * half, a0);
-                tmem_ld16(lane_addr + 64 * wg + 32 * half + 16, a1);
-                tmem_wait_ld();
-            } else {
+            for (int half = 0; half < 2; ++half) {
+                // 32 x 32 block (row block wq, column block cb) of the scores:
+                // above the diagonal all zero, below it copied, on it masked
+                const int cb = 2 * wg + half;
+                uint32_t u[16];
+                if (cb > wq) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) a0[e] = a1[e] = 0.f;
-            }
-            if (half == 1) {  // the score region is free for the next Q K^T
-                tc_fence_before_sync();
-                warp_arrive(&bar[B_AEMPTY]);
-            }
-            const int base = 64 * wg + 32 * half;  // score column of a0[0]
-            uint32_t u[16];
-            if (md != kModeDirect) {
+                    for (int e = 0; e < 16; ++e) u[e] = 0u;
+                } else {
+                    float a0[16], a1[16];
+                    tmem_ld16(lane_addr + 32 * cb, a0);
+                    tmem_ld16(lane_addr + 32 * cb + 16, a1);
+                    tmem_wait_ld();
+                    if (cb < wq) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s0 = base + 2 * e;
-                    u[e] = pack2(s0 <= t ? a0[2 * e] : 0.f, s0 + 1 <= t ? a0[2 * e + 1] : 0.f);
-                    u[8 + e] = pack2(s0 + 16 <= t ? a1[2 * e] : 0.f, s0 + 17 <= t ? a1[2 * e + 1] : 0.f);
+                        for (int e = 0; e < 8; ++e) {
+                            u[e] = pack2(a0[2 * e], a0[2 * e + 1]);
+                            u[8 + e] = pack2(a1[2 * e], a1[2 * e + 1]);
+                        }
+                    } else {
+                        const int r = lane;  // column s0 of the block is kept when s0 <= r
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            u[e] = pack2(2 * e <= r ? a0[2 * e] : 0.f, 2 * e + 1 <= r ? a0[2 * e + 1] : 0.f);
+                            u[8 + e] = pack2(2 * e + 16 <= r ? a1[2 * e] : 0.f, 2 * e + 17 <= r ? a1[2 * e + 1] : 0.f);
+                        }
+                    }
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s0 = base + 2 * e;
-                    const float f0 = s0 <= t ? a0[2 * e] * ex2_approx(lt - lam[s0]) : 0.f;
-                    const float f1 = s0 + 1 <= t ? a0[2 * e + 1] * ex2_approx(lt - lam[s0 + 1]) : 0.f;
-                    const float f2 = s0 + 16 <= t ? a1[2 * e] * ex2_approx(lt - lam[s0 + 16]) : 0.f;
-                    const float f3 = s0 + 17 <= t ? a1[2 * e + 1] * ex2_approx(lt - lam[s0 + 17]) : 0.f;
-                    u[e] = pack2(f0, f1);
-                    u[8 + e] = pack2(f2, f3);
+                if (half == 1) {  // the score region is free for the next Q K^T
+                    tc_fence_before_sync();
+                    warp_arrive(&bar[B_AEMPTY]);
                 }
+                tmem_st16u(p_addr + 16 * half, u);
             }
-            tmem_st16u(p_addr + 16 * half, u);
-        }
-        tmem_wait_st();
-        if (md == kModeDirect) {  // decayed Q and K for this chunk's Q S and K^T V
-            uint8_t* qk = sm + (c % G::NQK) * G::QK_STAGE;
-            if (wg == 0) scale_row<DK>(qk, t, ex2_approx(lt));
-            else scale_row<DK>(qk + G::Q_BYTES, t, ex2_approx(lc - lt));
-            fence_async_smem();
+            tmem_wait_st();
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_PFULL + pb]);
@@ -615,14 +720,12 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         return true;
     };
 
-    if (n > 0 && prep(0)) {
-        for (int c = 0; c < n; ++c) {
-            cu_lt = nx_lt;
-            cu_lc = nx_lc;
-            cu_md = nx_md;
-            if (c + 1 < n && !prep(c + 1)) break;
-            if (!pmask(c)) break;
-        }
+    // prep runs one chunk ahead of the mask (one call site each keeps the
+    // loop small in the instruction cache)
+#pragma unroll 1
+    for (int c = -1; c < n; ++c) {
+        if (c + 1 < n && !prep(c + 1)) break;
+        if (c >= 0 && !pmask(c)) break;
     }
 }
 
@@ -688,7 +791,9 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const int md = *reinterpret_cast<const volatile int*>(st + G::VS_META + 4);
         if (!waitw(&bar[B_DSFULL + b], (c / G::NDS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
+        // S' = ca S + cb DS: folded 2^(L_C) (S + K^T V'), direct 2^(L_C) S + K~^T V, none S + K^T V
         const float e = md == kModeNone ? 1.f : ex2_approx(lc);
+        const float ca = e, cbf = md == kModeFolded ? e : 1.f;
         const uint32_t dsa = lane_addr + G::COL_DS0 + b * G::OCOLS;
         if (warp_rows) {
 #pragma unroll
@@ -697,20 +802,13 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
                 tmem_ld16(dsa + cb + j, ds);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    if (md == kModeFolded) S[j + i] = e * (S[j + i] + ds[i]);
-                    else if (md == kModeDirect) S[j + i] = fmaf(e, S[j + i], ds[i]);
-                    else S[j + i] += ds[i];
-                }
+                for (int i = 0; i < 16; ++i) S[j + i] = fmaf(ca, S[j + i], cbf * ds[i]);
             }
             if (NORM && wg == 0) {
                 float zz[16];
                 tmem_ld16(dsa + NV, zz);
                 tmem_wait_ld();
-                const float zs = zz[0] + zz[1];
-                if (md == kModeFolded) z = e * (z + zs);
-                else if (md == kModeDirect) z = fmaf(e, z, zs);
-                else z += zs;
+                z = fmaf(ca, z, cbf * (zz[0] + zz[1]));
             }
         }
         tc_fence_before_sync();
@@ -741,7 +839,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const int rem = min(C, T - c * C);
         __nv_bfloat16* dst =
             p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(c) * C + t) * p.Dv + j0 + cb;
-#pragma unroll
+#pragma unroll 1
         for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
@@ -765,12 +863,12 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
     write_copy(0);
     bool ok = true;
-    for (int c = 0; c < n && ok; ++c) {
+#pragma unroll 1
+    for (int c = 0; c <= n && ok; ++c) {
         if (!kStateFirst && c >= 1) ok = epilogue(c - 1);
-        if (ok) ok = state(c);
+        if (ok && c < n) ok = state(c);
         if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
     }
-    if (ok && n > 0) ok = epilogue(n - 1);
     if (ok && !*abort && row_ok) {
         if (p.final_state) {
             float* fs = p.final_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
@@ -802,8 +900,10 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
         for (int s = 0; s < 4; ++s) {
-            mbar_init(&bar[B_QKFULL + s], 1);
-            mbar_init(&bar[B_QKEMPTY + s], 1);
+            mbar_init(&bar[B_QFULL + s], 1);
+            mbar_init(&bar[B_QEMPTY + s], 1);
+            mbar_init(&bar[B_KFULL + s], 1);
+            mbar_init(&bar[B_KEMPTY + s], 1);
             mbar_init(&bar[B_VFULL + s], 1);
             mbar_init(&bar[B_VEMPTY + s], G::VEMPTY_ARRIVALS);
             mbar_init(&bar[B_PREP + s], 8);
@@ -838,7 +938,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
 
     const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice};
     if (warp == G::W_TMA) {
-        role_tma_qk<DK, NV, NORM>(x, &tmq, &tmk);
+        role_tma_q<DK, NV, NORM>(x, &tmq);
     } else if (warp == G::W_MMA) {
         role_mma<DK, NV, NORM>(x);
     } else if (warp < G::W_ES) {
@@ -846,7 +946,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     } else if (warp < G::W_TMAV) {
         role_state_epilogue<DK, NV, NORM>(x);
     } else {
-        role_tma_v<DK, NV, NORM>(x, &tmv);
+        role_tma_kv<DK, NV, NORM>(x, &tmk, &tmv);
     }
 
     __syncwarp();  // lanes that idled while lane 0 ran a single-thread role rejoin it
