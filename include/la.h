@@ -58,6 +58,8 @@
 #ifndef RETENTION_SCAN_B200_LA_H
 #define RETENTION_SCAN_B200_LA_H
 
+#include <stddef.h>
+
 #if defined(__GNUC__)
 #define LA_API __attribute__((visibility("default")))
 #else
@@ -140,6 +142,47 @@ LA_API la_status la_chunk_forward(const void* q, const void* k, const void* v,
                            void* out, float* final_state, float* final_z,
                            int B, int H, int T, int Dk, int Dv,
                            la_dtype dtype, la_stream_t stream);
+
+/*
+ * la_chunk_forward_workspace_size - scratch bytes that la_chunk_forward_ws
+ * can use for these sizes (0 when the sequence would run as one segment).
+ *
+ * With a workspace, a bf16 forward whose B*H heads would leave most SMs idle
+ * cuts each sequence into T-segments that run side by side: a first pass
+ * computes every earlier segment's own state contribution S_j (from a zero
+ * state) and its total decay G_j, and the main pass starts segment i from
+ * the combination of the earlier ones, S <- G_j S + S_j in order: the
+ * associative pairing of (state, decay) spans that RetNet issue 21 uses for
+ * its cumulative-EMA scan (and RWKV-LM discussion 189 for the parallel WKV
+ * form).  Results equal the unsegmented pass up to fp32 summation order.
+ * The fp32 path ignores the workspace.  Deterministic for given sizes and
+ * environment (LA_SEGMENTS and LA_DV_SPLIT override the choice, for tests).
+ */
+LA_API size_t la_chunk_forward_workspace_size(int B, int H, int T, int Dk, int Dv,
+                                              la_dtype dtype, int normalize);
+
+/*
+ * la_chunk_forward_ws - la_chunk_forward with caller-owned scratch.
+ *
+ *   workspace        NULL, or device memory of workspace_bytes bytes, 16-byte
+ *                    aligned, not overlapping any other argument.  Its
+ *                    contents on entry do not matter; it is used on `stream`
+ *                    only and may be reused once the stream has passed this
+ *                    call.  NULL (or a size below
+ *                    la_chunk_forward_workspace_size) runs one segment per
+ *                    sequence, exactly as la_chunk_forward.
+ *   other arguments  as la_chunk_forward.
+ *
+ * Errors as la_chunk_forward, plus LA_ERR_INVALID_ARG for a non-NULL
+ * workspace that is not 16-byte aligned.
+ */
+LA_API la_status la_chunk_forward_ws(const void* q, const void* k, const void* v,
+                              const la_decay* decay, int normalize,
+                              const float* init_state, const float* init_z,
+                              void* out, float* final_state, float* final_z,
+                              int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                              void* workspace, size_t workspace_bytes,
+                              la_stream_t stream);
 
 /*
  * la_decode_step - one token of the recurrence, state updated in place.

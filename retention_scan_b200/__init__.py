@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "decode_step", "device_error", "LAError", "lib", "library_path",
+__all__ = ["chunk_forward", "workspace_size", "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -21,8 +21,8 @@ library_path = os.path.join(_HERE, "libla.so")
 
 DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
 LA_F32, LA_BF16 = 0, 1
-EXPORTED_SYMBOLS = ("la_chunk_forward", "la_decode_step", "la_status_string", "la_device_error",
-                    "la_version")
+EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
+                    "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
 class LAError(RuntimeError):
@@ -52,6 +52,11 @@ def lib():
         L.la_chunk_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, vp, vp,
                                        i, i, i, i, i, i, vp]
         L.la_chunk_forward.restype = i
+        L.la_chunk_forward_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, vp, vp,
+                                          i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_chunk_forward_ws.restype = i
+        L.la_chunk_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        L.la_chunk_forward_workspace_size.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
                                      i, i, i, i, i, vp]
         L.la_decode_step.restype = i
@@ -108,10 +113,15 @@ def _stream(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def workspace_size(B, H, T, Dk, Dv, dtype=torch.bfloat16, normalize=False):
+    """Scratch bytes chunk_forward can use for these sizes (la_chunk_forward_workspace_size)."""
+    return int(lib().la_chunk_forward_workspace_size(B, H, T, Dk, Dv, _dtype_code(dtype), int(bool(normalize))))
+
+
 def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
                   init_state=None, init_z=None, out=None, final_state=None, final_z=None,
-                  return_final=True, stream=None):
-    """Whole-sequence forward (la_chunk_forward).
+                  return_final=True, stream=None, workspace=True):
+    """Whole-sequence forward (la_chunk_forward_ws).
 
     q, k: [B,H,T,Dk]; v: [B,H,T,Dv]; float32 or bfloat16 CUDA tensors.
     decay_kind: DECAY_NONE, DECAY_PER_HEAD (log_g [H]) or DECAY_PER_STEP
@@ -119,6 +129,9 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     init_state [B,H,Dk,Dv] / init_z [B,H,Dk]: fp32 carried state and key sum.
     Returns (out, final_state, final_z); final_* are None unless requested
     (return_final, or passed in), final_z only when normalize.
+    workspace: True allocates the scratch that lets short-on-heads inputs run
+    as T-segments (a torch allocation on the call's stream), None/False runs
+    without, or a CUDA uint8 tensor to use.
     """
     B, H, T, Dk = q.shape
     Dv = v.shape[-1]
@@ -144,10 +157,21 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     _need(final_z, "final_z", (B, H, Dk), torch.float32, dev)
     d = _decay(decay_kind, log_g)
     with torch.cuda.device(dev):
-        _check(lib().la_chunk_forward(
+        if workspace is True:
+            nbytes = workspace_size(B, H, T, Dk, Dv, q.dtype, normalize)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+            if workspace is not None and stream is not None:
+                workspace.record_stream(stream)
+        elif workspace is False:
+            workspace = None
+        if workspace is not None:
+            if workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+                raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
+        _check(lib().la_chunk_forward_ws(
             _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
             _ptr(init_state), _ptr(init_z), _ptr(out), _ptr(final_state), _ptr(final_z),
-            B, H, T, Dk, Dv, code, _stream(stream, dev)))
+            B, H, T, Dk, Dv, code, _ptr(workspace), 0 if workspace is None else workspace.numel(),
+            _stream(stream, dev)))
     return out, final_state, (final_z if normalize else None)
 
 

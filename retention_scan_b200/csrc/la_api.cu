@@ -73,11 +73,26 @@ const char* la_status_string(la_status status) {
 
 const char* la_version(void) { return "0.1.0"; }
 
+size_t la_chunk_forward_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int normalize) {
+    if (dtype != LA_BF16 || B < 1 || H < 1 || T < 1) return 0;
+    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
+    return la::fwd_tc_workspace_bytes(B, H, T, Dk, Dv, normalize != 0);
+}
+
 la_status la_chunk_forward(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
                            const float* init_state, const float* init_z, void* out, float* final_state,
                            float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
                            la_stream_t stream) {
+    return la_chunk_forward_ws(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T,
+                               Dk, Dv, dtype, nullptr, 0, stream);
+}
+
+la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                              const float* init_state, const float* init_z, void* out, float* final_state,
+                              float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace,
+                              size_t workspace_bytes, la_stream_t stream) {
     if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     int kind;
     const float* log_g;
@@ -137,8 +152,9 @@ la_status la_chunk_forward(const void* q, const void* k, const void* v, const la
     if (dtype == LA_F32) {
         e = la::launch_fwd_f32(a);
     } else {
-        int split = 0;
-        e = la::launch_fwd_tc(a, 0, &split);
+        a.workspace = workspace;
+        a.workspace_bytes = workspace ? workspace_bytes : 0;
+        e = la::launch_fwd_tc(a, nullptr, nullptr);
         if (e == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
     }
     return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;

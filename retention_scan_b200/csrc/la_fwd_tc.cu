@@ -89,34 +89,111 @@ bool instance_ok(int Dk, int nv, bool norm) {
     }
 }
 
-// How many CTAs share one (b, h): each owns Dv / split value columns and
-// recomputes the 128 x 128 score tile.  The split is the smallest one whose
-// tiles fit in shared memory, doubled while that leaves most SMs idle
-// (keeping slices of at least 16 columns).
-int choose_split(int BH, int Dk, int Dv, bool norm) {
-    if (const char* env = std::getenv("LA_DV_SPLIT")) {
-        const int s = std::atoi(env);
-        if (s >= 1 && Dv % s == 0 && width_ok(Dv / s) && instance_ok(Dk, Dv / s, norm)) return s;
-    }
+int env_int(const char* name) {
+    const char* e = std::getenv(name);
+    return e ? std::atoi(e) : 0;
+}
+
+// How the (b, h) sequences are spread over CTAs (one CTA per SM).
+//  split: CTAs sharing one (b, h, segment), each owning Dv / split value
+//         columns and recomputing the 128 x 128 score tile;
+//  nseg:  output segments per (b, h), of seg_chunks chunks each; segment i
+//         starts from the state after segment i - 1, assembled from per_seg
+//         state segments per earlier output segment (computed by a state
+//         pass into the caller's workspace).
+// The split is the smallest one whose tiles fit in shared memory.  While that
+// leaves most SMs idle, the sequences are cut into segments (of at least
+// kMinSegChunks chunks: a segment pays a second launch and a pipeline fill and
+// drain, about as long as a dozen chunks) as long as one wave holds them, and
+// only then the value columns are
+// split further (slices of at least 16 columns): every extra slice reloads
+// and re-multiplies Q and K, a segment only reloads K and V once in the state
+// pass.  The state pass cuts each segment further while SMs stay idle.
+struct Layout {
+    int split, nseg, seg_chunks, per_seg, nS;
+};
+
+constexpr int kMinSegChunks = 16;
+
+Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments) {
+    const int sms = sm_count();
+    const long long target = sms * 4 / 5;
     int s = 1;
     while (!instance_ok(Dk, Dv / s, norm) && Dv / (2 * s) >= 16) s *= 2;
-    const int target = sm_count() * 4 / 5;
-    while (static_cast<long long>(BH) * s < target && Dv / (2 * s) >= 16) s *= 2;
-    return s;
+    const int es = env_int("LA_DV_SPLIT");
+    const bool fixed_split = es >= 1 && Dv % es == 0 && width_ok(Dv / es) && instance_ok(Dk, Dv / es, norm);
+    if (fixed_split) s = es;
+    int nseg = 1;
+    if (segments && nchunks >= 2) {
+        const int eg = env_int("LA_SEGMENTS");
+        if (eg >= 1) {
+            nseg = eg < nchunks ? eg : nchunks;
+        } else if (static_cast<long long>(BH) * s < target) {
+            while (nseg * 2 * kMinSegChunks <= nchunks && static_cast<long long>(BH) * s * nseg * 2 <= sms)
+                nseg *= 2;
+        }
+    }
+    if (!fixed_split)
+        while (static_cast<long long>(BH) * s * nseg < target && Dv / (2 * s) >= 16) s *= 2;
+    Layout L{};
+    L.split = s;
+    L.seg_chunks = (nchunks + nseg - 1) / (nseg > 0 ? nseg : 1);
+    if (L.seg_chunks < 1) L.seg_chunks = 1;
+    L.nseg = (nchunks + L.seg_chunks - 1) / L.seg_chunks;
+    if (L.nseg < 1) L.nseg = 1;
+    L.per_seg = 1;
+    if (L.nseg > 1)
+        while (L.seg_chunks % (2 * L.per_seg) == 0 &&
+               static_cast<long long>(BH) * s * (L.nseg - 1) * L.per_seg * 2 <= sms)
+            L.per_seg *= 2;
+    L.nS = (L.nseg - 1) * L.per_seg;
+    return L;
+}
+
+size_t workspace_bytes_for(int BH, int Dk, int Dv, int nS) {
+    const size_t per = static_cast<size_t>(Dk) * Dv + Dk + 1;
+    const size_t b = sizeof(float) * static_cast<size_t>(BH) * nS * per;
+    return (b + 255) / 256 * 256;
 }
 
 }  // namespace
 
 bool fwd_tc_supports(int Dk, int Dv) { return width_ok(Dk) && width_ok(Dv); }
 
-cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used) {
+size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm) {
+    if (!fwd_tc_supports(Dk, Dv) || B <= 0 || H <= 0 || T <= 0) return 0;
+    const int BH = B * H;
+    const Layout L = plan_layout(BH, (T + ws::C - 1) / ws::C, Dk, Dv, norm, true);
+    return L.nS > 0 ? workspace_bytes_for(BH, Dk, Dv, L.nS) : 0;
+}
+
+namespace {
+
+cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                      const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
+    switch (Dk) {
+        case 16: return ws::launch_dk16(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 32: return ws::launch_dk32(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 64: return ws::launch_dk64(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 128: return ws::launch_dk128(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used) {
     if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
     const bool norm = a.normalize != 0;
     const int BH = a.B * a.H;
-    const int split = dv_split > 0 ? dv_split : choose_split(BH, a.Dk, a.Dv, norm);
-    const int nv = a.Dv / split;
+    const int nchunks = (a.T + ws::C - 1) / ws::C;
+    Layout L = plan_layout(BH, nchunks, a.Dk, a.Dv, norm, a.workspace != nullptr);
+    if (L.nS > 0 && a.workspace_bytes < workspace_bytes_for(BH, a.Dk, a.Dv, L.nS))
+        L = plan_layout(BH, nchunks, a.Dk, a.Dv, norm, false);  // too small: one segment
+    const int split = L.split, nv = a.Dv / split;
     if (a.Dv % split != 0 || !width_ok(nv) || !instance_ok(a.Dk, nv, norm)) return cudaErrorNotSupported;
     if (split_used) *split_used = split;
+    if (segments_used) *segments_used = L.nseg;
 
     CUtensorMap tmq, tmk, tmv;
     const int box_k = a.Dk < 64 ? a.Dk : 64;
@@ -137,16 +214,27 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used) {
     p.T = a.T;
     p.Dv = a.Dv;
     p.split = split;
-    p.nchunks = (a.T + ws::C - 1) / ws::C;
+    p.nchunks = nchunks;
     p.err = a.err_word;
-    const int grid = BH * split;
-    switch (a.Dk) {
-        case 16: return ws::launch_dk16(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
-        case 32: return ws::launch_dk32(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
-        case 64: return ws::launch_dk64(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
-        case 128: return ws::launch_dk128(nv, norm, tmq, tmk, tmv, p, grid, a.stream);
-        default: return cudaErrorNotSupported;
+    if (L.nS > 0) {
+        float* base = static_cast<float*>(a.workspace);
+        p.ws_S = base;
+        p.ws_z = p.ws_S + static_cast<size_t>(BH) * L.nS * a.Dk * a.Dv;
+        p.ws_L = p.ws_z + static_cast<size_t>(BH) * L.nS * a.Dk;
+        p.ws_nS = L.nS;
+        p.ws_per_seg = L.per_seg;
+        // state pass: the contribution of each state segment before the last output segment
+        ws::Params ps = p;
+        ps.state_pass = 1;
+        ps.nseg = L.nS;
+        ps.seg_chunks = L.seg_chunks / L.per_seg;
+        const cudaError_t e = launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, ps, BH * L.nS * split, a.stream);
+        if (e != cudaSuccess) return e;
     }
+    p.state_pass = 0;
+    p.nseg = L.nseg;
+    p.seg_chunks = L.seg_chunks;
+    return launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, p, BH * L.nseg * split, a.stream);
 }
 
 }  // namespace la

@@ -81,18 +81,18 @@ enum Bar : int {
     B_VFULL = 16,    // [4] V tile landed
     B_VEMPTY = 20,   // [4] V stage free (P V done, its prefix read)
     B_PREP = 24,     // [4] decay prefix, value scaling, weights done
-    B_AFULL = 28,    // scores in TMEM
-    B_AEMPTY = 29,   // scores read by the mask warps
-    B_PFULL = 30,    // [2] P in TMEM
-    B_PEMPTY = 32,   // [2] P V done reading P
-    B_OFULL = 34,    // [2] O (and den) complete
-    B_OEMPTY = 36,   // [2] epilogue done with O
-    B_DSFULL = 38,   // [2] K^T V' in TMEM
-    B_DSEMPTY = 40,  // [2] state warps done with it
-    B_SBFULL = 42,   // [2] bf16 state copy written
-    B_SBEMPTY = 44,  // [2] Q S done reading it
-    B_DRAIN = 46,
-    B_COUNT = 47
+    B_AFULL = 28,    // [2] scores in TMEM
+    B_AEMPTY = 30,   // [2] scores read by the mask warps
+    B_PFULL = 32,    // [2] P in TMEM
+    B_PEMPTY = 34,   // [2] P V done reading P
+    B_OFULL = 36,    // [2] O (and den) complete
+    B_OEMPTY = 38,   // [2] epilogue done with O
+    B_DSFULL = 40,   // [2] K^T V' in TMEM
+    B_DSEMPTY = 42,  // [2] state warps done with it
+    B_SBFULL = 44,   // [2] bf16 state copy written
+    B_SBEMPTY = 46,  // [2] Q S done reading it
+    B_DRAIN = 48,
+    B_COUNT = 49
 };
 
 template <int DK, int NV, bool NORM>
@@ -153,13 +153,17 @@ struct Plan {
     static constexpr int OFF_MISC = OFF_ZB + NSB * ZB_BYTES;
     static constexpr int OFF_ROWF = OFF_MISC + 1024;  // float[kRowfRing][C]: 2^(L_t) per token
     static constexpr int SMEM = OFF_MISC + MISC + 1024;
-    // TMEM columns: scores [0,128) | P (bf16 pairs) 64 per buffer | O | K^T V'
+    // TMEM columns: scores 128 per buffer | P (bf16 pairs) 64 per buffer | O | K^T V'.
+    // Double buffers in the order P, O, scores, K^T V' while they fit.
     static constexpr int OCOLS = NV + (NORM ? 16 : 0);
-    static constexpr int tmem_need(int npb, int no, int nds) { return 128 + 64 * npb + (no + nds) * OCOLS; }
-    static constexpr int NPB = tmem_need(2, 2, 1) <= 512 ? 2 : 1;
-    static constexpr int NO = tmem_need(NPB, 2, 1) <= 512 ? 2 : 1;
-    static constexpr int NDS = tmem_need(NPB, NO, 2) <= 512 ? 2 : 1;
-    static constexpr int COL_P0 = 128;
+    static constexpr int tmem_need(int na, int npb, int no, int nds) {
+        return 128 * na + 64 * npb + (no + nds) * OCOLS;
+    }
+    static constexpr int NPB = tmem_need(1, 2, 2, 1) <= 512 ? 2 : 1;
+    static constexpr int NO = tmem_need(1, NPB, 2, 1) <= 512 ? 2 : 1;
+    static constexpr int NA = tmem_need(2, NPB, NO, 1) <= 512 ? 2 : 1;
+    static constexpr int NDS = tmem_need(NA, NPB, NO, 2) <= 512 ? 2 : 1;
+    static constexpr int COL_P0 = 128 * NA;
     static constexpr int COL_O0 = COL_P0 + 64 * NPB;
     static constexpr int COL_DS0 = COL_O0 + NO * OCOLS;
     static constexpr int TMEM_USED = COL_DS0 + NDS * OCOLS;
@@ -199,6 +203,16 @@ struct Params {
     float* final_z;
     int H, T, Dv, split, nchunks;
     int* err;
+    // T-segments: each (b, h, slice) is cut into nseg segments of seg_chunks
+    // chunks, one CTA each.  The output pass starts segment i from the state
+    // after segment i - 1, combined from the workspace; the state pass
+    // (state_pass = 1) only writes each segment's own contribution there.
+    int nseg, seg_chunks, state_pass;
+    float* ws_S;         // [B H][ws_nS][Dk][Dv] state of each state segment, from zero
+    float* ws_z;         // [B H][ws_nS][Dk] key sum of each state segment, from zero
+    float* ws_L;         // [B H][ws_nS] total log2 decay of each state segment
+    int ws_nS;           // state segments per (b, h)
+    int ws_per_seg;      // state segments per output segment
 };
 
 // What every role needs from the kernel prologue (passed by value).
@@ -207,6 +221,7 @@ struct Ctx {
     uint8_t* sm;
     uint32_t sa, tmem;
     int bh, h, j0, slice;
+    int seg, c0, n;  // segment, its first chunk and its number of chunks
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -315,7 +330,7 @@ __host__ __device__ constexpr uint32_t kstep(int kk, int W) {
     uint64_t* const bar = reinterpret_cast<uint64_t*>(sm + G::OFF_MISC);                             \
     volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4); \
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;                                      \
-    const int T = p.T, n = p.nchunks;                                                                \
+    const int T = p.T, n = x.n;                                                                      \
     (void)sa;                                                                                        \
     (void)tmem;                                                                                      \
     (void)warp;                                                                                      \
@@ -327,7 +342,7 @@ __host__ __device__ constexpr uint32_t kstep(int kk, int W) {
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
     LA_ROLE_PRELUDE
-    if (lane != 0) return;
+    if (lane != 0 || p.state_pass) return;  // the state pass reads no queries
     int issued = 0;
     for (int c = 0; c < n; ++c) {
         const int s = c % G::NQ;
@@ -335,7 +350,7 @@ __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
         mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
         uint8_t* st = sm + s * G::Q_STAGE;
         for (int pp = 0; pp < G::PK; ++pp)
-            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * 64, c * C, x.bh);
+            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * 64, (x.c0 + c) * C, x.bh);
         ++issued;
     }
     if (*abort) {  // let issued copies land before the CTA's shared memory goes away
@@ -361,7 +376,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_KFULL + s], G::Q_TX);
             uint8_t* st = sm + G::OFF_K + s * G::Q_STAGE;
             for (int pp = 0; pp < G::PK; ++pp)
-                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * 64, ck * C, x.bh);
+                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * 64, (x.c0 + ck) * C, x.bh);
             ++ck;
             moved = true;
         }
@@ -371,7 +386,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
             uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
             for (int pp = 0; pp < G::PV; ++pp)
-                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, cv * C, x.bh);
+                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, (x.c0 + cv) * C, x.bh);
             ++cv;
             moved = true;
         }
@@ -396,7 +411,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
 
 // ------------------------------------------------------------ MMA issuer
 // Four in-order queues, each issued as soon as its inputs are there:
-//   Q K^T (c)   Q and K tiles of c landed, score region free
+//   Q K^T (c)   Q and K tiles of c landed, its score buffer free
 //   K^T V' (j)  after Q K^T (j) and the prep of j; a direct-form chunk also
 //               after its mask, which decays Q and K; K^T V' buffer free;
 //               releases the K stage
@@ -405,9 +420,52 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
 //   P V (j)     after Q S (j), which opened the accumulator; P (j) written
 // The warp polls the barriers (never blocking on one while another queue
 // could move) and gives up after kWaitLimitNs without progress.
+// State pass: only K^T V' (and K^T W), in order; each also releases its K and
+// V stages.
+template <int DK, int NV, bool NORM>
+__device__ __noinline__ void mma_state_pass(const Ctx x) {
+    LA_ROLE_PRELUDE
+    const bool leader = elect_one();
+    for (int kv = 0; kv < n; ++kv) {
+        const int b = kv % G::NDS;
+        if (!waitw(&bar[B_KFULL + kv % G::NK], (kv / G::NK) & 1, abort, p, kErrMmaWait)) break;
+        if (!waitw(&bar[B_PREP + kv % G::NVS], (kv / G::NVS) & 1, abort, p, kErrMmaWait)) break;
+        if (kv >= G::NDS && !waitw(&bar[B_DSEMPTY + b], ((kv / G::NDS) - 1) & 1, abort, p, kErrMmaWait)) break;
+        tc_fence_after_sync();
+        const uint32_t ka = sa + G::OFF_K + (kv % G::NK) * G::Q_STAGE;
+        const uint32_t va = sa + G::OFF_V + (kv % G::NVS) * G::V_STAGE;
+        const uint64_t dk = make_smem_desc(ka, DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
+        const uint64_t dv = make_smem_desc(va, C * G::WV, 8 * G::WV, G::WV);
+        const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
+        if (leader) {
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
+            if (NORM) {
+                const uint64_t dw = make_smem_desc(va + G::VS_W, 0, 8 * 32, 32);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(d + NV, dk + ((kk * 16 * G::WK) >> 4), dw + ((kk * 16 * 32) >> 4), G::IDESC_KV16,
+                              kk > 0);
+            }
+            umma_commit(&bar[B_DSFULL + b]);
+            umma_commit(&bar[B_KEMPTY + kv % G::NK]);
+            umma_commit(&bar[B_VEMPTY + kv % G::NVS]);
+        }
+        __syncwarp();
+    }
+    if (leader) umma_commit(&bar[B_DRAIN]);
+    __syncwarp();
+    mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
+}
+
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_mma(const Ctx x) {
     LA_ROLE_PRELUDE
+    if (p.state_pass) {
+        mma_state_pass<DK, NV, NORM>(x);
+        return;
+    }
     const bool leader = elect_one();
     auto mode_of = [&](int j) {
         return *reinterpret_cast<volatile int*>(sm + G::OFF_V + (j % G::NVS) * G::V_STAGE + G::VS_META + 4);
@@ -426,16 +484,16 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             moved = true;
         }
         if (m1 < n && ready(B_QFULL + m1 % G::NQ, (m1 / G::NQ) & 1) && ready(B_KFULL + m1 % G::NK, (m1 / G::NK) & 1) &&
-            (m1 == 0 || ready(B_AEMPTY, (m1 - 1) & 1))) {
+            (m1 < G::NA || ready(B_AEMPTY + m1 % G::NA, ((m1 / G::NA) - 1) & 1))) {
             tc_fence_after_sync();
             const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
             const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem, dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4), G::IDESC_QK,
-                              kk > 0);
-                umma_commit(&bar[B_AFULL]);
+                    umma_bf16(tmem + 128 * (m1 % G::NA), dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4),
+                              G::IDESC_QK, kk > 0);
+                umma_commit(&bar[B_AFULL + m1 % G::NA]);
             }
             __syncwarp();
             ++m1;
@@ -593,7 +651,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     auto fetch = [&](int c) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = c * C + 32 * i + lane;
+            const int row = (x.c0 + c) * C + 32 * i + lane;
             nxt[i] = (kind == LA_DECAY_PER_STEP && c < n && row < T) ? lg[row] : 0.f;
         }
     };
@@ -603,8 +661,12 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     // mode) into the V stage, the output row factors and the scaled value
     // rows; warpgroup 1 writes the normaliser weights, or has nothing to do.
     auto prep = [&](int c) -> bool {
-        const int s = c % G::NVS, rem = min(C, T - c * C);
+        const int s = c % G::NVS, rem = min(C, T - (x.c0 + c) * C);
         if (!NORM && wg == 1) {
+            // nothing to prepare; in the state pass (no mask to pace this
+            // warpgroup) wait for the tile so that its arrivals never run a
+            // ring's length ahead
+            if (p.state_pass && !waitw(&bar[B_VFULL + s], (c / G::NVS) & 1, abort, p, kErrTmaWait)) return false;
             warp_arrive(&bar[B_PREP + s]);
             return true;
         }
@@ -648,7 +710,12 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                 reinterpret_cast<float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] =
                     md == kModeFolded ? ex2_approx(lt) : 1.f;
             if (md == kModeFolded) scale_row<NV>(st, t, ex2_approx(-lt));
-        } else {
+            if (md == kModeDirect && p.state_pass) {
+                // no mask in the state pass: decay this key row here, K~ = 2^(L_C - L_t) K
+                if (!waitw(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, abort, p, kErrTmaWait)) return false;
+                scale_row<DK>(sm + G::OFF_K + (c % G::NK) * G::Q_STAGE, t, ex2_approx(lc - lt));
+            }
+        } else if (NORM) {
             // normaliser weights w_t = 2^(-L_t) (1 unless folded), as a bf16 hi/lo pair
             const float w = md == kModeFolded ? ex2_approx(-lt) : 1.f;
             const float hi = __bfloat162float(__float2bfloat16_rn(w));
@@ -664,7 +731,8 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         const int s = c % G::NVS, pb = c % G::NPB;
         if (c >= G::NPB && !waitw(&bar[B_PEMPTY + pb], ((c / G::NPB) - 1) & 1, abort, p, kErrMmaWait))
             return false;
-        if (!waitw(&bar[B_AFULL], c & 1, abort, p, kErrMmaWait)) return false;
+        const int ab = c % G::NA;  // score buffer
+        if (!waitw(&bar[B_AFULL + ab], (c / G::NA) & 1, abort, p, kErrMmaWait)) return false;
         if (!waitw(&bar[B_PREP + s], (c / G::NVS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
         const uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
@@ -674,7 +742,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             const float* lam = reinterpret_cast<const float*>(st + G::VS_LAM);
             const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
             const bool all_masked = (32 * wq + 31) < 64 * wg;  // every row of this warp precedes these columns
-            mask_direct<DK>(lane_addr + 64 * wg, p_addr, &bar[B_AEMPTY], wg, t, all_masked, lam[t], lc, lam,
+            mask_direct<DK>(lane_addr + 128 * ab + 64 * wg, p_addr, &bar[B_AEMPTY + ab], wg, t, all_masked, lam[t], lc, lam,
                             wg == 0 ? sm + (c % G::NQ) * G::Q_STAGE : sm + G::OFF_K + (c % G::NK) * G::Q_STAGE);
         } else {
 #pragma unroll 1
@@ -688,8 +756,8 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                     for (int e = 0; e < 16; ++e) u[e] = 0u;
                 } else {
                     float a0[16], a1[16];
-                    tmem_ld16(lane_addr + 32 * cb, a0);
-                    tmem_ld16(lane_addr + 32 * cb + 16, a1);
+                    tmem_ld16(lane_addr + 128 * ab + 32 * cb, a0);
+                    tmem_ld16(lane_addr + 128 * ab + 32 * cb + 16, a1);
                     tmem_wait_ld();
                     if (cb < wq) {
 #pragma unroll
@@ -706,9 +774,9 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                         }
                     }
                 }
-                if (half == 1) {  // the score region is free for the next Q K^T
+                if (half == 1) {  // the score buffer is free for a later Q K^T
                     tc_fence_before_sync();
-                    warp_arrive(&bar[B_AEMPTY]);
+                    warp_arrive(&bar[B_AEMPTY + ab]);
                 }
                 tmem_st16u(p_addr + 16 * half, u);
             }
@@ -720,6 +788,14 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         return true;
     };
 
+    if (p.state_pass) {  // prep only; nothing reads the V stage's prefix later
+#pragma unroll 1
+        for (int c = 0; c < n; ++c) {
+            if (!prep(c)) break;
+            warp_arrive(&bar[B_VEMPTY + c % G::NVS]);
+        }
+        return;
+    }
     // prep runs one chunk ahead of the mask (one call site each keeps the
     // loop small in the instruction cache)
 #pragma unroll 1
@@ -748,7 +824,8 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     float z = 0.f;
 #pragma unroll
     for (int j = 0; j < G::NVW; ++j) S[j] = 0.f;
-    if (row_ok && p.init_state) {
+    float ltot = 0.f;  // state pass: total log2 decay of the segment
+    if (row_ok && p.init_state && !p.state_pass) {
         const float* src = p.init_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
 #pragma unroll
         for (int j = 0; j < G::NVW; j += 4) {
@@ -759,7 +836,25 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             S[j + 3] = v4.w;
         }
     }
-    if (NORM && row_ok && p.init_z) z = p.init_z[static_cast<size_t>(bh) * DK + d];
+    if (NORM && row_ok && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * DK + d];
+    if (row_ok && !p.state_pass && x.seg > 0) {
+        // state entering this segment: fold in every earlier state segment j,
+        // S <- 2^(L_j) S + S_j (the combination of two consecutive spans)
+        for (int j = 0; j < x.seg * p.ws_per_seg; ++j) {
+            const size_t sj = static_cast<size_t>(bh) * p.ws_nS + j;
+            const float e = ex2_approx(p.ws_L[sj]);
+            const float* src = p.ws_S + (sj * DK + d) * p.Dv + j0 + cb;
+#pragma unroll
+            for (int i = 0; i < G::NVW; i += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(src + i);
+                S[i] = fmaf(e, S[i], v4.x);
+                S[i + 1] = fmaf(e, S[i + 1], v4.y);
+                S[i + 2] = fmaf(e, S[i + 2], v4.z);
+                S[i + 3] = fmaf(e, S[i + 3], v4.w);
+            }
+            if (NORM) z = fmaf(e, z, p.ws_z[sj * DK + d]);
+        }
+    }
 
     auto write_copy = [&](int k) {  // bf16 copy of S (and z) for production index k
         const int buf = k % G::NSB;
@@ -789,6 +884,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
         const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
         const int md = *reinterpret_cast<const volatile int*>(st + G::VS_META + 4);
+        ltot += lc;
         if (!waitw(&bar[B_DSFULL + b], (c / G::NDS) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
         // S' = ca S + cb DS: folded 2^(L_C) (S + K^T V'), direct 2^(L_C) S + K~^T V, none S + K^T V
@@ -814,7 +910,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         tc_fence_before_sync();
         warp_arrive(&bar[B_DSEMPTY + b]);
         warp_arrive(&bar[B_VEMPTY + s]);
-        if (c == n - 1) return true;
+        if (c == n - 1 || p.state_pass) return true;
         const int k = c + 1;
         if (k >= G::NSB && !waitw(&bar[B_SBEMPTY + k % G::NSB], ((k / G::NSB) - 1) & 1, abort, p, kErrMmaWait))
             return false;
@@ -836,9 +932,9 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         } else {
             inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
         }
-        const int rem = min(C, T - c * C);
+        const int rem = min(C, T - (x.c0 + c) * C);
         __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(c) * C + t) * p.Dv + j0 + cb;
+            p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + j0 + cb;
 #pragma unroll 1
         for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
@@ -860,6 +956,24 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     // The state update of chunk c gates the next chunk's Q S, so it goes
     // first, unless both the O buffer and the state copy are single: then
     // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
+    if (p.state_pass) {
+        bool ok = true;
+#pragma unroll 1
+        for (int c = 0; c < n && ok; ++c) ok = state(c);
+        if (ok && !*abort) {
+            const size_t sj = static_cast<size_t>(bh) * p.ws_nS + x.seg;
+            if (row_ok) {
+                float* dst = p.ws_S + (sj * DK + d) * p.Dv + j0 + cb;
+#pragma unroll
+                for (int j = 0; j < G::NVW; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                if (NORM && x.slice == 0 && wg == 0) p.ws_z[sj * DK + d] = z;
+            }
+            if (x.slice == 0 && wg == 0 && d == 0) p.ws_L[sj] = ltot;
+        }
+        return;
+    }
+
     constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
     write_copy(0);
     bool ok = true;
@@ -869,7 +983,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         if (ok && c < n) ok = state(c);
         if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
     }
-    if (ok && !*abort && row_ok) {
+    if (ok && !*abort && row_ok && x.seg == p.nseg - 1) {
         if (p.final_state) {
             float* fs = p.final_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
 #pragma unroll
@@ -893,7 +1007,11 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     volatile int* abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4);
 
     const int tid = threadIdx.x, warp = tid / 32;
-    const int bh = blockIdx.x / p.split, slice = blockIdx.x % p.split;
+    // blockIdx.x = (bh * nseg + seg) * split + slice
+    const int slice = blockIdx.x % p.split, bs = blockIdx.x / p.split;
+    const int seg = bs % p.nseg, bh = bs / p.nseg;
+    const int c0 = seg * p.seg_chunks;
+    const int nloc = max(0, min(p.seg_chunks, p.nchunks - c0));
 
     if (tid == 0) {
         prefetch_tensormap(&tmq);
@@ -908,9 +1026,9 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
             mbar_init(&bar[B_VEMPTY + s], G::VEMPTY_ARRIVALS);
             mbar_init(&bar[B_PREP + s], 8);
         }
-        mbar_init(&bar[B_AFULL], 1);
-        mbar_init(&bar[B_AEMPTY], 8);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar[B_AFULL + i], 1);
+            mbar_init(&bar[B_AEMPTY + i], 8);
             mbar_init(&bar[B_PFULL + i], 8);
             mbar_init(&bar[B_PEMPTY + i], 1);
             mbar_init(&bar[B_OFULL + i], 1);
@@ -936,7 +1054,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice};
+    const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice, seg, c0, nloc};
     if (warp == G::W_TMA) {
         role_tma_q<DK, NV, NORM>(x, &tmq);
     } else if (warp == G::W_MMA) {

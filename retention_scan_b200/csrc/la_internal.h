@@ -29,6 +29,8 @@ struct FwdArgs {
     int B, H, T, Dk, Dv;
     cudaStream_t stream;
     int* err_word;            // device error word of the current device
+    void* workspace;          // scratch for T-segment states (may be null: no segments)
+    size_t workspace_bytes;
 };
 
 struct DecodeArgs {
@@ -49,11 +51,14 @@ struct DecodeArgs {
 cudaError_t launch_fwd_f32(const FwdArgs& a);
 
 // bf16 inputs: chunked kernel on tcgen05 tensor cores (la_fwd_tc.cu).
-// dv_split: number of CTAs sharing one (b, h), each owning Dv / dv_split
-// value columns (0 = choose).  Returns cudaErrorNotSupported for shapes
-// without a kernel; *split_used receives the split that ran.
-cudaError_t launch_fwd_tc(const FwdArgs& a, int dv_split, int* split_used);
+// Returns cudaErrorNotSupported for shapes without a kernel; *split_used and
+// *segments_used (may be null) receive the value split and the number of
+// T-segments that ran.  Segments need a.workspace of at least
+// fwd_tc_workspace_bytes(...) bytes; with less (or none) the sequence runs as
+// one segment.
+cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used);
 bool fwd_tc_supports(int Dk, int Dv);
+size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm);
 
 // Decode step (la_decode.cu).
 cudaError_t launch_decode(const DecodeArgs& a, la_dtype dtype);

@@ -123,3 +123,41 @@ print(r, r2)
     env = dict(os.environ, LA_FAULT_INJECT="launch")
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
     assert out.stdout.split() == ["3", "3"]
+
+
+def _ws_bytes(BH, Dk, Dv, nS):
+    b = 4 * BH * nS * (Dk * Dv + Dk + 1)
+    return (b + 255) // 256 * 256
+
+
+def test_workspace_size_follows_the_segment_plan(L, monkeypatch):
+    # 148 SMs (the B200 count, also the host default without a device).
+    # 32 heads of 16 chunks: too short to cut (segments of at least 16 chunks)
+    monkeypatch.delenv("LA_SEGMENTS", raising=False)
+    monkeypatch.delenv("LA_DV_SPLIT", raising=False)
+    assert L.la_chunk_forward_workspace_size(4, 8, 2048, 64, 64, 1, 0) == 0
+    # 8 heads of 64 chunks, Dk = Dv = 64: four segments of 16 chunks, then
+    # four value slices (8 x 4 x 4 = 128 CTAs); a state pass of 8 x 4 x 3 =
+    # 96 CTAs, one state segment for each of the first three segments
+    assert L.la_chunk_forward_workspace_size(1, 8, 8192, 64, 64, 1, 0) == _ws_bytes(8, 64, 64, 3)
+    # 32 heads of 512 chunks, Dk = Dv = 128: two value slices, two segments,
+    # the first cut into two state segments
+    assert L.la_chunk_forward_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 2)
+    # 128 heads fill the GPU: no segments
+    assert L.la_chunk_forward_workspace_size(8, 16, 4096, 128, 128, 1, 1) == 0
+    # fp32, empty or too short inputs: none
+    assert L.la_chunk_forward_workspace_size(4, 8, 2048, 64, 64, 0, 0) == 0
+    assert L.la_chunk_forward_workspace_size(0, 8, 2048, 64, 64, 1, 0) == 0
+    assert L.la_chunk_forward_workspace_size(4, 8, 0, 64, 64, 1, 0) == 0
+    assert L.la_chunk_forward_workspace_size(4, 8, 128, 64, 64, 1, 0) == 0
+    # an explicit segment count (test override)
+    monkeypatch.setenv("LA_SEGMENTS", "5")
+    assert L.la_chunk_forward_workspace_size(1, 2, 1100, 64, 64, 1, 0) > 0
+
+
+def test_segmented_entry_rejects_misaligned_workspace(L):
+    buf = ctypes.create_string_buffer(64)
+    addr = ctypes.addressof(buf) + 4
+    st = L.la_chunk_forward_ws(None, None, None, None, 0, None, None, None, None, None,
+                               1, 1, 0, 16, 16, 1, ctypes.c_void_p(addr), 60, None)
+    assert st == 1  # LA_ERR_INVALID_ARG

@@ -219,6 +219,69 @@ def test_tc_no_decay_long_sum_matches():
     check_case(inp)
 
 
+# ---------------------------------------------------------------- T-segments
+# A sequence cut into segments: a state pass writes each earlier segment's own
+# state (from zero) and total decay to the workspace; the output pass starts
+# segment i from their ordered combination S <- G_j S + S_j.
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 5, 9])
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+def test_segments(monkeypatch, nseg, kind, normalize):
+    monkeypatch.setenv("LA_SEGMENTS", str(nseg))
+    inp, S0, z0 = gen_case(1, 2, 1100, 64, 64, kind=kind, normalize=normalize, init=True,
+                           seed=900 + nseg * 8 + kind * 2 + normalize)
+    check_case(inp, normalize, S0, z0)
+
+
+@pytest.mark.parametrize("split", [2, 4])
+def test_segments_with_value_split(monkeypatch, split):
+    monkeypatch.setenv("LA_SEGMENTS", "4")
+    monkeypatch.setenv("LA_DV_SPLIT", str(split))
+    inp, S0, z0 = gen_case(1, 2, 1000, 128, 128, kind=2, normalize=True, init=True, seed=910 + split)
+    check_case(inp, True, S0, z0)
+
+
+@pytest.mark.parametrize("decay_mean", [1.0, -30.0])
+def test_segments_direct_form(monkeypatch, decay_mean):
+    # chunks whose total decay passes the fold limit run in the direct form,
+    # in the state pass too (there the key rows are decayed by the prep warps)
+    monkeypatch.setenv("LA_SEGMENTS", "4")
+    inp, S0, z0 = gen_case(1, 2, 1024, 64, 64, kind=2, normalize=True, init=True, seed=920,
+                           decay_mean=decay_mean)
+    if decay_mean < 0:
+        inp["log_g"] = torch.full_like(inp["log_g"], decay_mean)
+    check_case(inp, True, S0, z0)
+
+
+def test_segments_match_one_segment():
+    # the default plan segments this shape; without a workspace it runs as one segment
+    inp, S0, _ = gen_case(1, 4, 4096, 64, 64, kind=1, init=True, seed=930)
+    assert la().workspace_size(1, 4, 4096, 64, 64) > 0
+    d = to_dev(inp)
+    args = (d["q"], d["k"], d["v"], d["decay_kind"], d["log_g"], False, S0.cuda(), None)
+    y1, S1, _ = la().chunk_forward(*args, workspace=None)
+    y2, S2, _ = la().chunk_forward(*args)
+    torch.cuda.synchronize()
+    assert rel_err(y1, y2.cpu().double()) < 2e-3 and rel_err(S1, S2.cpu().double()) < 1e-4
+    check_case(inp, False, S0)
+
+
+def test_workspace_too_small_or_misaligned():
+    inp, S0, _ = gen_case(1, 2, 1024, 64, 64, kind=2, init=True, seed=940)
+    d = to_dev(inp)
+    args = (d["q"], d["k"], d["v"], d["decay_kind"], d["log_g"], False, S0.cuda(), None)
+    small = torch.empty(64, dtype=torch.uint8, device="cuda")  # below the size: one segment
+    y, S, _ = la().chunk_forward(*args, workspace=small)
+    yr, Sr, _ = oracle_forward(inp, False, S0, None)
+    assert rel_err(y, yr) <= TOL[torch.bfloat16] and rel_err(S, Sr) <= TOL[torch.bfloat16]
+    n = la().workspace_size(1, 2, 1024, 64, 64) + 16
+    buf = torch.empty(n, dtype=torch.uint8, device="cuda")
+    with pytest.raises(la().LAError):
+        la().chunk_forward(*args, workspace=buf[4:])
+
+
 def test_empty_and_zero_sizes():
     S0 = torch.randn(2, 3, 16, 16, device="cuda")
     z0 = torch.rand(2, 3, 16, device="cuda")
