@@ -185,6 +185,30 @@ LA_API la_status la_chunk_forward_ws(const void* q, const void* k, const void* v
                               la_stream_t stream);
 
 /*
+ * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
+ * device array inside this library (la_chunk_forward_noalloc_capacity()
+ * bytes, 16 MiB, one per device, reserved when the library's device code is
+ * loaded), so that the call itself allocates no device memory.  The pages
+ * have no counterpart: this is a property of this library's interface only.
+ *
+ * The array is shared by every call on a device: calls on one device must
+ * not overlap in time (issue them on one stream, or synchronise between the
+ * streams).  Arguments, results and errors as la_chunk_forward, plus
+ * LA_ERR_UNSUPPORTED (nothing enqueued) when these sizes would need a larger
+ * workspace than the array holds (la_chunk_forward_workspace_size), and
+ * LA_ERR_CUDA if the array's address cannot be obtained on the current device.
+ */
+LA_API la_status la_chunk_forward_noalloc(const void* q, const void* k, const void* v,
+                                   const la_decay* decay, int normalize,
+                                   const float* init_state, const float* init_z,
+                                   void* out, float* final_state, float* final_z,
+                                   int B, int H, int T, int Dk, int Dv,
+                                   la_dtype dtype, la_stream_t stream);
+
+/* Bytes of the fixed device array that la_chunk_forward_noalloc uses. */
+LA_API size_t la_chunk_forward_noalloc_capacity(void);
+
+/*
  * la_decode_step - one token of the recurrence, state updated in place.
  *
  *   S <- g S + k v^T;  z <- g z + k (if normalize);  out = q^T S  (/ q^T z).
