@@ -473,18 +473,37 @@ __device__ __noinline__ void role_mma(const Ctx x) {
     auto q_addr = [&](int j) { return sa + (j % G::NQ) * G::Q_STAGE; };
     auto k_addr = [&](int j) { return sa + G::OFF_K + (j % G::NK) * G::Q_STAGE; };
     auto v_addr = [&](int j) { return sa + G::OFF_V + (j % G::NVS) * G::V_STAGE; };
-    auto ready = [&](int slot, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(&bar[slot], parity)); };
+    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
 
     int m1 = 0, kv = 0, qs = 0, pv = 0, pseen = 0;  // next chunk of each queue; P (j) seen for j < pseen
-    uint64_t last = global_timer_ns();
+    // One snapshot per pass of every barrier a queue head may wait on: the
+    // issuing lane runs the tests back to back (their latencies overlap; no
+    // test waits for another's answer) and broadcasts the bits to the warp.
+    enum : uint32_t { kP = 1, kQ = 2, kK = 4, kA = 8, kPrep = 16, kDir = 32, kDse = 64, kOe = 128, kSb = 256 };
+    auto snapshot = [&]() -> uint32_t {
+        uint32_t b = 0;
+        if (leader) {
+            b |= mbar_test(&bar[B_PFULL + pseen % G::NPB], (pseen / G::NPB) & 1) ? kP : 0u;
+            b |= mbar_test(&bar[B_QFULL + m1 % G::NQ], (m1 / G::NQ) & 1) ? kQ : 0u;
+            b |= mbar_test(&bar[B_KFULL + m1 % G::NK], (m1 / G::NK) & 1) ? kK : 0u;
+            b |= (m1 < G::NA || mbar_test(&bar[B_AEMPTY + m1 % G::NA], ((m1 / G::NA) - 1) & 1)) ? kA : 0u;
+            b |= mbar_test(&bar[B_PREP + kv % G::NVS], (kv / G::NVS) & 1) ? kPrep : 0u;
+            b |= (kv < G::NDS || mbar_test(&bar[B_DSEMPTY + kv % G::NDS], ((kv / G::NDS) - 1) & 1)) ? kDse : 0u;
+            b |= (qs < G::NO || mbar_test(&bar[B_OEMPTY + qs % G::NO], ((qs / G::NO) - 1) & 1)) ? kOe : 0u;
+            b |= mbar_test(&bar[B_SBFULL + qs % G::NSB], (qs / G::NSB) & 1) ? kSb : 0u;
+            if ((b & kPrep) && mode_of(kv) == kModeDirect) b |= kDir;  // the mode is valid once prep is done
+        }
+        return __shfl_sync(0xffffffffu, b, leader_lane);
+    };
+    uint64_t idle_since = 0;  // start of the current run of passes without progress
     while (pv < n) {
         bool moved = false;
-        if (pseen < m1 && ready(B_PFULL + pseen % G::NPB, (pseen / G::NPB) & 1)) {
+        const uint32_t bits = snapshot();
+        if (pseen < m1 && (bits & kP)) {
             ++pseen;
             moved = true;
         }
-        if (m1 < n && ready(B_QFULL + m1 % G::NQ, (m1 / G::NQ) & 1) && ready(B_KFULL + m1 % G::NK, (m1 / G::NK) & 1) &&
-            (m1 < G::NA || ready(B_AEMPTY + m1 % G::NA, ((m1 / G::NA) - 1) & 1))) {
+        if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA)) {
             tc_fence_after_sync();
             const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
             const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
@@ -499,8 +518,7 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             ++m1;
             moved = true;
         }
-        if (kv < m1 && ready(B_PREP + kv % G::NVS, (kv / G::NVS) & 1) && (mode_of(kv) != kModeDirect || kv < pseen) &&
-            (kv < G::NDS || ready(B_DSEMPTY + kv % G::NDS, ((kv / G::NDS) - 1) & 1))) {
+        if (kv < m1 && (bits & kPrep) && (!(bits & kDir) || kv < pseen) && (bits & kDse)) {
             // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
             // repeats the key panel when Dk < 128
             tc_fence_after_sync();
@@ -526,8 +544,7 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             ++kv;
             moved = true;
         }
-        if (qs < kv && (qs < G::NO || ready(B_OEMPTY + qs % G::NO, ((qs / G::NO) - 1) & 1)) &&
-            ready(B_SBFULL + qs % G::NSB, (qs / G::NSB) & 1)) {
+        if (qs < kv && (bits & kOe) && (bits & kSb)) {
             // O = Q S (and den = Q z), opening the accumulator of chunk qs
             tc_fence_after_sync();
             const int ro = qs % G::NO, sbb = qs % G::NSB;
@@ -578,10 +595,12 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             moved = true;
         }
         if (moved) {
-            last = global_timer_ns();
+            idle_since = 0;
         } else {
+            const uint64_t now = global_timer_ns();
+            if (idle_since == 0) idle_since = now;
             bool give_up = *abort != 0;
-            if (!give_up && global_timer_ns() - last > kWaitLimitNs) {
+            if (!give_up && now - idle_since > kWaitLimitNs) {
                 give_up = true;
                 if (lane == 0) fail(p, abort, kErrMmaWait);
             }
