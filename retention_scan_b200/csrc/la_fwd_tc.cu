@@ -197,7 +197,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
 
     CUtensorMap tmq, tmk, tmv;
     const int box_k = a.Dk < 64 ? a.Dk : 64;
-    const int box_v = nv < 64 ? nv : 64;
+    const int box_v = norm ? 16 : (nv < 64 ? nv : 64);  // the normaliser instances use 16-column panels
     if (!make_map(&tmq, a.q, a.Dk, a.T, BH, box_k) || !make_map(&tmk, a.k, a.Dk, a.T, BH, box_k) ||
         !make_map(&tmv, a.v, a.Dv, a.T, BH, box_v))
         return cudaErrorInvalidValue;

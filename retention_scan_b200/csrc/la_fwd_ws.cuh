@@ -98,7 +98,11 @@ enum Bar : int {
 template <int DK, int NV, bool NORM>
 struct Plan {
     static constexpr int WK = row_bytes_for(DK), PK = panels_for(DK);
-    static constexpr int WV = row_bytes_for(NV), PV = panels_for(NV);
+    // Value tiles (and the bf16 state copy, whose columns are value columns):
+    // with the normaliser, panels of 16 columns (32-byte swizzle), so that the
+    // weight panel W (16 columns) continues V and the key-sum panel continues
+    // S: one MMA of N = NV + 16 then computes both, reading its A operand once.
+    static constexpr int WV = NORM ? 32 : row_bytes_for(NV), PV = NORM ? NV / 16 : panels_for(NV);
     static constexpr int Q_BYTES = C * DK * 2;
     static constexpr int V_BYTES = C * NV * 2;
     // Q and K stages (one tile each)
@@ -108,14 +112,15 @@ struct Plan {
     static constexpr int VS_LAM = VS_W + (NORM ? C * 32 : 0);
     static constexpr int VS_META = VS_LAM + C * 4;  // float L_C, int mode
     static constexpr int V_STAGE = round1k(VS_META + 64);
-    static constexpr int SB_BYTES = round1k(DK * NV * 2);
-    static constexpr int ZB_BYTES = NORM ? round1k(DK * 32) : 0;
+    // bf16 state copy: S panels, then (normaliser) the key-sum panel [z_hi z_lo 0 ..]
+    static constexpr int SB_ZB = DK * NV * 2;  // offset of the key-sum panel
+    static constexpr int SB_BYTES = round1k(DK * NV * 2 + (NORM ? DK * 32 : 0));
     // barriers and flags, then the output row factors of the last kRowfRing
     // chunks (not needed with the normaliser, where the factor cancels).
     static constexpr int kRowfRing = 8;
     static constexpr int MISC = 1024 + (NORM ? 0 : kRowfRing * C * 4);
     static constexpr bool fits(int nq, int nk, int nvs, int nsb) {
-        return (nq + nk) * Q_STAGE + nvs * V_STAGE + nsb * (SB_BYTES + ZB_BYTES) + MISC + 1024 <= kSmemLimit;
+        return (nq + nk) * Q_STAGE + nvs * V_STAGE + nsb * SB_BYTES + MISC + 1024 <= kSmemLimit;
     }
     // A ring of depth n whose stages each stay busy for a time L allows one
     // chunk per L / n.  Rough busy times (arbitrary units): a Q stage from its
@@ -149,8 +154,7 @@ struct Plan {
     static constexpr int OFF_K = NQ * Q_STAGE;
     static constexpr int OFF_V = OFF_K + NK * Q_STAGE;
     static constexpr int OFF_SB = OFF_V + NVS * V_STAGE;
-    static constexpr int OFF_ZB = OFF_SB + NSB * SB_BYTES;
-    static constexpr int OFF_MISC = OFF_ZB + NSB * ZB_BYTES;
+    static constexpr int OFF_MISC = OFF_SB + NSB * SB_BYTES;
     static constexpr int OFF_ROWF = OFF_MISC + 1024;  // float[kRowfRing][C]: 2^(L_t) per token
     static constexpr int SMEM = OFF_MISC + MISC + 1024;
     // TMEM columns: scores 128 per buffer | P (bf16 pairs) 64 per buffer | O | K^T V'.
@@ -179,10 +183,9 @@ struct Plan {
     static constexpr uint32_t Q_TX = Q_BYTES;
     static constexpr uint32_t V_TX = V_BYTES;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
-    static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NV, 0, 1);
-    static constexpr uint32_t IDESC_KV = make_idesc_bf16(128, NV, 1, 1);
-    static constexpr uint32_t IDESC_N16 = make_idesc_bf16(128, 16, 0, 1);
-    static constexpr uint32_t IDESC_KV16 = make_idesc_bf16(128, 16, 1, 1);
+    static constexpr int NOUT = NV + (NORM ? 16 : 0);  // value columns plus the normaliser panel
+    static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NOUT, 0, 1);
+    static constexpr uint32_t IDESC_KV = make_idesc_bf16(128, NOUT, 1, 1);
     static_assert(TMEM_USED <= TMEM_COLS, "tensor memory budget");
     static_assert(NV % 16 == 0 && NV >= 16 && NV <= 128, "value slice");
     static_assert(DK == 16 || DK == 32 || DK == 64 || DK == 128, "key width");
@@ -291,9 +294,11 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 // Multiply the bf16 row `row` of a swizzled [C x width] tile by f, in place.
-template <int WIDTH>
+// W: bytes per swizzled panel row (the tile's layout; by default the widest
+// swizzle for WIDTH columns).
+template <int WIDTH, int W = row_bytes_for(WIDTH)>
 __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
-    constexpr int W = row_bytes_for(WIDTH), NP = panels_for(WIDTH), NCH = NP * W / 16;
+    constexpr int NP = WIDTH * 2 / W, NCH = NP * W / 16;
     constexpr int BATCH = NCH < 4 ? NCH : 4;  // loads in flight before the first store
 #pragma unroll
     for (int i0 = 0; i0 < NCH; i0 += BATCH) {
@@ -350,7 +355,7 @@ __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
         mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
         uint8_t* st = sm + s * G::Q_STAGE;
         for (int pp = 0; pp < G::PK; ++pp)
-            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * 64, (x.c0 + c) * C, x.bh);
+            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * (G::WK / 2), (x.c0 + c) * C, x.bh);
         ++issued;
     }
     if (*abort) {  // let issued copies land before the CTA's shared memory goes away
@@ -376,7 +381,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_KFULL + s], G::Q_TX);
             uint8_t* st = sm + G::OFF_K + s * G::Q_STAGE;
             for (int pp = 0; pp < G::PK; ++pp)
-                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * 64, (x.c0 + ck) * C, x.bh);
+                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * (G::WK / 2), (x.c0 + ck) * C, x.bh);
             ++ck;
             moved = true;
         }
@@ -386,7 +391,8 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
             uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
             for (int pp = 0; pp < G::PV; ++pp)
-                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * 64, (x.c0 + cv) * C, x.bh);
+                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * (G::WV / 2), (x.c0 + cv) * C,
+                            x.bh);
             ++cv;
             moved = true;
         }
@@ -441,13 +447,6 @@ __device__ __noinline__ void mma_state_pass(const Ctx x) {
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
                 umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
-            if (NORM) {
-                const uint64_t dw = make_smem_desc(va + G::VS_W, 0, 8 * 32, 32);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(d + NV, dk + ((kk * 16 * G::WK) >> 4), dw + ((kk * 16 * 32) >> 4), G::IDESC_KV16,
-                              kk > 0);
-            }
             umma_commit(&bar[B_DSFULL + b]);
             umma_commit(&bar[B_KEMPTY + kv % G::NK]);
             umma_commit(&bar[B_VEMPTY + kv % G::NVS]);
@@ -530,13 +529,6 @@ __device__ __noinline__ void role_mma(const Ctx x) {
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
-                if (NORM) {
-                    const uint64_t dw = make_smem_desc(v_addr(kv) + G::VS_W, 0, 8 * 32, 32);
-#pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        umma_bf16(d + NV, dk + ((kk * 16 * G::WK) >> 4), dw + ((kk * 16 * 32) >> 4), G::IDESC_KV16,
-                                  kk > 0);
-                }
                 umma_commit(&bar[B_DSFULL + b]);
                 umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
             }
@@ -549,19 +541,13 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             tc_fence_after_sync();
             const int ro = qs % G::NO, sbb = qs % G::NSB;
             const uint64_t dq = make_smem_desc(q_addr(qs), 16, 8 * G::WK, G::WK);
+            // B = [S | z] panels of the bf16 state copy
             const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
             const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
                     umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
-                if (NORM) {
-                    const uint64_t dzb = make_smem_desc(sa + G::OFF_ZB + sbb * G::ZB_BYTES, 0, 8 * 32, 32);
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16(d + NV, dq + (kstep(kk, G::WK) >> 4), dzb + ((kk * 16 * 32) >> 4), G::IDESC_N16,
-                                  kk > 0);
-                }
                 umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // Q K^T and Q S of this chunk have run
                 umma_commit(&bar[B_SBEMPTY + sbb]);
             }
@@ -580,12 +566,6 @@ __device__ __noinline__ void role_mma(const Ctx x) {
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
-                if (NORM) {
-                    const uint64_t dw = make_smem_desc(v_addr(pv) + G::VS_W, 0, 8 * 32, 32);
-#pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        umma_bf16_ts(d + NV, pa + 8 * kk, dw + ((kk * 16 * 32) >> 4), G::IDESC_N16, 1);
-                }
                 umma_commit(&bar[B_OFULL + ro]);
                 umma_commit(&bar[B_PEMPTY + pb]);
                 umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
@@ -728,7 +708,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             if (!NORM)
                 reinterpret_cast<float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] =
                     md == kModeFolded ? ex2_approx(lt) : 1.f;
-            if (md == kModeFolded) scale_row<NV>(st, t, ex2_approx(-lt));
+            if (md == kModeFolded) scale_row<NV, G::WV>(st, t, ex2_approx(-lt));
             if (md == kModeDirect && p.state_pass) {
                 // no mask in the state pass: decay this key row here, K~ = 2^(L_C - L_t) K
                 if (!waitw(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, abort, p, kErrTmaWait)) return false;
@@ -889,7 +869,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             }
             if (NORM && wg == 0) {
                 const float hi = __bfloat162float(__float2bfloat16_rn(z));
-                *reinterpret_cast<uint4*>(sm + G::OFF_ZB + buf * G::ZB_BYTES + swz(d, 0, 32)) =
+                *reinterpret_cast<uint4*>(sb + G::SB_ZB + swz(d, 0, 32)) =
                     make_uint4(pack2(hi, z - hi), 0u, 0u, 0u);
             }
         }
@@ -1064,8 +1044,9 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_MMA) tmem_alloc(tmem_slot, G::TMEM_COLS);
     if (NORM && warp >= G::W_ES && warp < G::W_ES + 4) {
         // zeroed key-sum tiles (only their first two columns are ever written)
-        for (int i = tid - 32 * G::W_ES; i < G::NSB * G::ZB_BYTES / 16; i += 128)
-            reinterpret_cast<uint4*>(sm + G::OFF_ZB)[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = tid - 32 * G::W_ES; i < G::NSB * DK * 2; i += 128)  // 16-byte pieces
+            reinterpret_cast<uint4*>(sm + G::OFF_SB + (i / (DK * 2)) * G::SB_BYTES + G::SB_ZB)[i % (DK * 2)] =
+                make_uint4(0u, 0u, 0u, 0u);
         fence_async_smem();
     }
     tc_fence_before_sync();
