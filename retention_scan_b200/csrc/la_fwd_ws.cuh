@@ -44,8 +44,10 @@
 //   warp 1       MMA issuer (one elected lane) and TMEM owner
 //   warps 2-9    two warpgroups: prep (decay prefix, value-row scaling,
 //                normaliser weights) and mask (scores -> P in TMEM); warpgroup
-//                0 owns score columns 0-63, warpgroup 1 columns 64-127
-//   warps 10-..  state and epilogue (one warpgroup per 64 value columns)
+//                0 owns score columns 0-63, warpgroup 1 columns 64-127 and
+//                writes the outputs (epilogue)
+//   warps 10-..  state: fp32 S in registers and its bf16 copy (one warpgroup
+//                per 64 value columns)
 //   last warp    TMA producer of the K and V rings
 // Every hand-off is an mbarrier; every wait gives up after kWaitLimitNs (then
 // the CTA sets the device error word and unwinds).
@@ -183,13 +185,16 @@ struct Plan {
     static constexpr uint32_t Q_TX = Q_BYTES;
     static constexpr uint32_t V_TX = V_BYTES;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
+    static constexpr bool EPI_MASK = NORM;  // outputs written by mask warpgroup 1 (else by the state warps)
     static constexpr int NOUT = NV + (NORM ? 16 : 0);  // value columns plus the normaliser panel
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NOUT, 0, 1);
     static constexpr uint32_t IDESC_KV = make_idesc_bf16(128, NOUT, 1, 1);
     static_assert(TMEM_USED <= TMEM_COLS, "tensor memory budget");
     static_assert(NV % 16 == 0 && NV >= 16 && NV <= 128, "value slice");
     static_assert(DK == 16 || DK == 32 || DK == 64 || DK == 128, "key width");
-    static_assert(kRowfRing >= NVS + 1, "row factor ring too shallow");
+    // the epilogue of chunk c runs before the mask of chunk c + 2, so before
+    // the prep of chunk c + 2 + NVS rewrites its row factors
+    static_assert(kRowfRing >= NVS + 3, "row factor ring too shallow");
     static_assert(8 * B_COUNT + 8 <= 1024, "barrier area");
     static_assert(!OK || (OFF_K % 1024 == 0 && OFF_V % 1024 == 0), "stages aligned for 128-byte swizzle");
     static_assert(!OK || SMEM <= kSmemLimit, "shared memory limit");
@@ -787,6 +792,43 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         return true;
     };
 
+    // Epilogue (warpgroup 1, after its mask of the next chunk): y = O times
+    // the row factor 2^(L_t) (or / den_t) for all NV columns of the slice;
+    // 16-byte stores of bf16 pairs, rows past the sequence end skipped.
+    auto epilogue = [&](int c) -> bool {
+        const int ro = c % G::NO;
+        if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
+        tc_fence_after_sync();
+        const uint32_t oa = lane_addr + G::COL_O0 + ro * G::OCOLS;
+        float inv;  // y = O * inv
+        if (NORM) {
+            float dd[16];
+            tmem_ld16(oa + NV, dd);
+            tmem_wait_ld();
+            inv = 1.f / (dd[0] + dd[1]);
+        } else {
+            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
+        }
+        const int rem = min(C, T - (x.c0 + c) * C);
+        __nv_bfloat16* dst =
+            p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + x.j0;
+#pragma unroll 1
+        for (int piece = 0; piece < NV / 16; ++piece) {
+            float o[16];
+            tmem_ld16(oa + 16 * piece, o);
+            tmem_wait_ld();
+            if (t < rem) {
+                uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * piece);
+                d4[0] = make_uint4(pack2(o[0] * inv, o[1] * inv), pack2(o[2] * inv, o[3] * inv),
+                                   pack2(o[4] * inv, o[5] * inv), pack2(o[6] * inv, o[7] * inv));
+                d4[1] = make_uint4(pack2(o[8] * inv, o[9] * inv), pack2(o[10] * inv, o[11] * inv),
+                                   pack2(o[12] * inv, o[13] * inv), pack2(o[14] * inv, o[15] * inv));
+            }
+        }
+        tc_fence_before_sync();
+        warp_arrive(&bar[B_OEMPTY + ro]);
+        return true;
+    };
     if (p.state_pass) {  // prep only; nothing reads the V stage's prefix later
 #pragma unroll 1
         for (int c = 0; c < n; ++c) {
@@ -795,19 +837,20 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         }
         return;
     }
-    // prep runs one chunk ahead of the mask (one call site each keeps the
-    // loop small in the instruction cache)
+    // prep runs one chunk ahead of the mask, the epilogue one chunk behind
+    // it (one call site each keeps the loop small in the instruction cache)
 #pragma unroll 1
-    for (int c = -1; c < n; ++c) {
+    for (int c = -1; c <= n; ++c) {
         if (c + 1 < n && !prep(c + 1)) break;
-        if (c >= 0 && !pmask(c)) break;
+        if (c >= 0 && c < n && !pmask(c)) break;
+        if (G::EPI_MASK && wg == 1 && c >= 1 && !epilogue(c - 1)) break;
     }
 }
 
-// ------------------------------------------------------------ state + epilogue
+// ------------------------------------------------------------ state
 // Warpgroup wg owns value columns [wg NVW, (wg + 1) NVW) of the slice.  Per
-// chunk c: the state update of chunk c (its bf16 copy opens the next chunk's
-// O through Q S) and the epilogue of chunk c - 1.
+// chunk c: the state update of chunk c, then its bf16 copy, which the next
+// chunk's Q S reads.
 template <int DK, int NV, bool NORM>
 __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     LA_ROLE_PRELUDE
@@ -917,6 +960,10 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         return true;
     };
 
+
+    // The state update of chunk c gates the next chunk's Q S, so it goes
+    // first, unless both the O buffer and the state copy are single: then
+    // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO, t = d;
         if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
@@ -951,10 +998,6 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         warp_arrive(&bar[B_OEMPTY + ro]);
         return true;
     };
-
-    // The state update of chunk c gates the next chunk's Q S, so it goes
-    // first, unless both the O buffer and the state copy are single: then
-    // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
     if (p.state_pass) {
         bool ok = true;
 #pragma unroll 1
@@ -973,14 +1016,19 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         return;
     }
 
-    constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
     write_copy(0);
     bool ok = true;
+    if constexpr (G::EPI_MASK) {
 #pragma unroll 1
-    for (int c = 0; c <= n && ok; ++c) {
-        if (!kStateFirst && c >= 1) ok = epilogue(c - 1);
-        if (ok && c < n) ok = state(c);
-        if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
+        for (int c = 0; c < n && ok; ++c) ok = state(c);
+    } else {
+        constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
+#pragma unroll 1
+        for (int c = 0; c <= n && ok; ++c) {
+            if (!kStateFirst && c >= 1) ok = epilogue(c - 1);
+            if (ok && c < n) ok = state(c);
+            if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
+        }
     }
     if (ok && !*abort && row_ok && x.seg == p.nseg - 1) {
         if (p.final_state) {
@@ -1031,7 +1079,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
             mbar_init(&bar[B_PFULL + i], 8);
             mbar_init(&bar[B_PEMPTY + i], 1);
             mbar_init(&bar[B_OFULL + i], 1);
-            mbar_init(&bar[B_OEMPTY + i], 4 * G::NSW);
+            mbar_init(&bar[B_OEMPTY + i], G::EPI_MASK ? 4 : 4 * G::NSW);
             mbar_init(&bar[B_DSFULL + i], 1);
             mbar_init(&bar[B_DSEMPTY + i], 4 * G::NSW);
             mbar_init(&bar[B_SBFULL + i], 4 * G::NSW);
