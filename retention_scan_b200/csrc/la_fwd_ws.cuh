@@ -305,6 +305,10 @@ template <int WIDTH, int W = row_bytes_for(WIDTH)>
 __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
     constexpr int NP = WIDTH * 2 / W, NCH = NP * W / 16;
     constexpr int BATCH = NCH < 4 ? NCH : 4;  // loads in flight before the first store
+    // f = f_hi + f_lo (two bf16 parts): fma(v, f_hi, v f_lo) rounds once, so the
+    // result is the bf16 rounding of v f up to about 2^-17 relative
+    const float fhi = __bfloat162float(__float2bfloat16_rn(f));
+    const __nv_bfloat162 f2h = __float2bfloat162_rn(fhi), f2l = __float2bfloat162_rn(f - fhi);
 #pragma unroll
     for (int i0 = 0; i0 < NCH; i0 += BATCH) {
         uint4 w[BATCH];
@@ -318,10 +322,7 @@ __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
             const int ci = i0 + i;
             __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&w[i]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 v2 = __bfloat1622float2(hv[e]);
-                hv[e] = __floats2bfloat162_rn(v2.x * f, v2.y * f);
-            }
+            for (int e = 0; e < 4; ++e) hv[e] = __hfma2(hv[e], f2h, __hmul2(hv[e], f2l));
             *reinterpret_cast<uint4*>(tile + (ci / (W / 16)) * C * W + swz(row, (ci % (W / 16)) * 16, W)) = w[i];
         }
     }
