@@ -652,11 +652,13 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     const int kind = p.decay_kind;
     const float* lg = p.log_g + static_cast<size_t>(x.bh) * T;
     const float ell_head = kind == LA_DECAY_PER_HEAD ? p.log_g[x.h] * kLog2e : 0.f;
+    // per-step decays: lane l holds rows 4 l .. 4 l + 3 of the chunk (every
+    // warp of warpgroup 0 holds the whole chunk)
     float nxt[4] = {0.f, 0.f, 0.f, 0.f};
     auto fetch = [&](int c) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = (x.c0 + c) * C + 32 * i + lane;
+            const int row = (x.c0 + c) * C + 4 * lane + i;
             nxt[i] = (kind == LA_DECAY_PER_STEP && c < n && row < T) ? lg[row] : 0.f;
         }
     };
@@ -681,22 +683,24 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         // chunk-local log2 decay prefix L_t and total L_C
         float lt, lc;
         if (kind == LA_DECAY_PER_STEP) {
-            float tot0 = cur0 * kLog2e, tot1 = cur1 * kLog2e, tot2 = cur2 * kLog2e, tot3 = cur3 * kLog2e;
-            float v = (wq == 0 ? cur0 : wq == 1 ? cur1 : wq == 2 ? cur2 : cur3) * kLog2e;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                tot0 += __shfl_xor_sync(0xffffffffu, tot0, o);
-                tot1 += __shfl_xor_sync(0xffffffffu, tot1, o);
-                tot2 += __shfl_xor_sync(0xffffffffu, tot2, o);
-                tot3 += __shfl_xor_sync(0xffffffffu, tot3, o);
-            }
+            // prefix of the lane's four rows, an exclusive warp scan of the
+            // lane totals, then each lane of this warp's 32 rows publishes
+            // its four prefixes (rows 32 wq .. 32 wq + 31) and reads its own
+            const float a0 = cur0 * kLog2e, a1 = a0 + cur1 * kLog2e, a2 = a1 + cur2 * kLog2e,
+                        a3 = a2 + cur3 * kLog2e;
+            float incl = a3;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += y;
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
             }
-            lt = v + (wq > 0 ? tot0 : 0.f) + (wq > 1 ? tot1 : 0.f) + (wq > 2 ? tot2 : 0.f);
-            lc = tot0 + tot1 + tot2 + tot3;
+            const float excl = incl - a3;
+            lc = __shfl_sync(0xffffffffu, incl, 31);
+            float* lam = reinterpret_cast<float*>(sm + G::OFF_V + s * G::V_STAGE + G::VS_LAM);
+            if ((lane >> 3) == wq)
+                *reinterpret_cast<float4*>(lam + 4 * lane) = make_float4(excl + a0, excl + a1, excl + a2, excl + a3);
+            __syncwarp();
+            lt = lam[t];
         } else {  // per head (ell_head = L per step), or none (ell_head = 0)
             lt = static_cast<float>(min(t + 1, rem)) * ell_head;
             lc = static_cast<float>(rem) * ell_head;
@@ -961,10 +965,8 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         return true;
     };
 
-
-    // The state update of chunk c gates the next chunk's Q S, so it goes
-    // first, unless both the O buffer and the state copy are single: then
-    // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
+    // Epilogue (unnormalised instances): y = O times the row factor 2^(L_t)
+    // for this warpgroup's columns.
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO, t = d;
         if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
@@ -1023,6 +1025,9 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
 #pragma unroll 1
         for (int c = 0; c < n && ok; ++c) ok = state(c);
     } else {
+        // The state update of chunk c gates the next chunk's Q S, so it goes
+        // first, unless both the O buffer and the state copy are single: then
+        // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
         constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
 #pragma unroll 1
         for (int c = 0; c <= n && ok; ++c) {
