@@ -333,6 +333,21 @@ __host__ __device__ constexpr uint32_t kstep(int kk, int W) {
     return ((kk * 16) / (W / 2)) * C * W + ((kk * 16) % (W / 2)) * 2;
 }
 
+// Store 16 outputs o * inv as bf16 (32 bytes) at dst: one 32-byte store when
+// the output is 32-byte aligned, else two 16-byte stores.
+__device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)[16], float inv, bool wide) {
+    uint32_t u[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[e] = pack2(o[2 * e] * inv, o[2 * e + 1] * inv);
+    if (wide) {
+        st_global_v8(dst, u);
+    } else {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+        d4[0] = make_uint4(u[0], u[1], u[2], u[3]);
+        d4[1] = make_uint4(u[4], u[5], u[6], u[7]);
+    }
+}
+
 #define LA_ROLE_PRELUDE                                                                              \
     using G = Plan<DK, NV, NORM>;                                                                    \
     const Params& p = *x.p;                                                                          \
@@ -815,6 +830,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
         }
         const int rem = min(C, T - (x.c0 + c) * C);
+        const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst =
             p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + x.j0;
 #pragma unroll 1
@@ -822,13 +838,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             float o[16];
             tmem_ld16(oa + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) {
-                uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * piece);
-                d4[0] = make_uint4(pack2(o[0] * inv, o[1] * inv), pack2(o[2] * inv, o[3] * inv),
-                                   pack2(o[4] * inv, o[5] * inv), pack2(o[6] * inv, o[7] * inv));
-                d4[1] = make_uint4(pack2(o[8] * inv, o[9] * inv), pack2(o[10] * inv, o[11] * inv),
-                                   pack2(o[12] * inv, o[13] * inv), pack2(o[14] * inv, o[15] * inv));
-            }
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);
@@ -982,6 +992,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
         }
         const int rem = min(C, T - (x.c0 + c) * C);
+        const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst =
             p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + j0 + cb;
 #pragma unroll 1
@@ -989,13 +1000,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) {
-                uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * piece);
-                d4[0] = make_uint4(pack2(o[0] * inv, o[1] * inv), pack2(o[2] * inv, o[3] * inv),
-                                   pack2(o[4] * inv, o[5] * inv), pack2(o[6] * inv, o[7] * inv));
-                d4[1] = make_uint4(pack2(o[8] * inv, o[9] * inv), pack2(o[10] * inv, o[11] * inv),
-                                   pack2(o[12] * inv, o[13] * inv), pack2(o[14] * inv, o[15] * inv));
-            }
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);

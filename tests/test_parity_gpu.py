@@ -282,6 +282,21 @@ def test_workspace_too_small_or_misaligned():
         la().chunk_forward(*args, workspace=buf[4:])
 
 
+def test_output_only_16_byte_aligned():
+    # outputs 16- but not 32-byte aligned take the 16-byte store path
+    inp, S0, _ = gen_case(1, 2, 300, 64, 64, kind=2, init=True, seed=960)
+    d = to_dev(inp)
+    n = 1 * 2 * 300 * 64
+    buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(1, 2, 300, 64)
+    assert out.data_ptr() % 32 == 16
+    y, S, _ = la().chunk_forward(d["q"], d["k"], d["v"], d["decay_kind"], d["log_g"], False, S0.cuda(), None,
+                                 out=out)
+    torch.cuda.synchronize()
+    yr, Sr, _ = oracle_forward(inp, False, S0, None)
+    assert rel_err(y, yr) <= TOL[torch.bfloat16] and rel_err(S, Sr) <= TOL[torch.bfloat16]
+
+
 def test_empty_and_zero_sizes():
     S0 = torch.randn(2, 3, 16, 16, device="cuda")
     z0 = torch.rand(2, 3, 16, device="cuda")
