@@ -5,8 +5,12 @@ cpu_baseline / reference legs may import this package.  The CUDA library
 (retention_scan_b200) never imports it and shares no code with it.
 
   forward(...)           recurrent definition, plain C (la_ref.c), token by token
+  reverse(...)           the reverse scan, by its definition: forward of the
+                         time-reversed arguments, output reversed back
+  bidirectional(...)     forward + reverse
   decode_step(...)       one token of the same recurrence, in place
   parallel_forward(...)  brute-force O(T^2) parallel form, numpy (parallel.py)
+  parallel_reverse(...)  brute-force O(T^2) anti-causal form, numpy (parallel.py)
 
 Every array argument is converted to contiguous float64; bf16 and fp32
 inputs up-cast exactly, so the oracle reads the same input bits as the GPU.
@@ -17,7 +21,7 @@ import subprocess
 
 import numpy as np
 
-from .parallel import parallel_forward  # noqa: F401
+from .parallel import parallel_forward, parallel_reverse  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "la_ref.c")
@@ -111,3 +115,34 @@ def decode_step(q, k, v, state, z=None, decay_kind=0, log_g=None, normalize=Fals
     if rc != 0:
         raise ValueError("la_ref_decode_step rejected its arguments")
     return y, state, z
+
+
+def _flip_time(a, axis):
+    return None if a is None else np.ascontiguousarray(np.flip(a, axis=axis))
+
+
+def reverse(q, k, v, decay_kind=0, log_g=None, normalize=False,
+            init_state=None, init_z=None, nthreads=None, lib=None):
+    """Reverse scan, float64.  Jamie-Stirling/RetNet issue 21 (the
+    cumulative_ema docstring): with reverse=True the result is the reverse of
+    the non-reversed call on arguments reversed along time.  So, per sequence,
+    S_t = g_t S_{t+1} + k_t v_t^T and z_t = g_t z_{t+1} + k_t for t = T..1,
+    y_t = q_t^T S_t (or / q_t^T z_t).  init_state / init_z enter from beyond
+    token T (decayed by g_T); the returned state is the one at token 1.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    log_g = _f64(log_g)
+    kind = _kind(decay_kind)
+    lg = _flip_time(log_g, 2) if kind == 2 else log_g
+    y, S, z = forward(_flip_time(q, 2), _flip_time(k, 2), _flip_time(v, 2), kind, lg, normalize,
+                      init_state, init_z, nthreads=nthreads, lib=lib)
+    return np.ascontiguousarray(y[:, :, ::-1]), S, z
+
+
+def bidirectional(q, k, v, decay_kind=0, log_g=None, normalize=False, nthreads=None, lib=None):
+    """Bidirectional encoder, float64: the forward scan plus the reverse scan
+    (RetNet issue 21: "combining two", one with reverse=False and one with
+    reverse=True; read as their sum).  No carried state."""
+    yf, _, _ = forward(q, k, v, decay_kind, log_g, normalize, nthreads=nthreads, lib=lib)
+    yr, _, _ = reverse(q, k, v, decay_kind, log_g, normalize, nthreads=nthreads, lib=lib)
+    return yf + yr

@@ -67,3 +67,46 @@ def parallel_forward(q, k, v, decay_kind=0, log_g=None, normalize=False,
             S_T[b, h] = (k[b, h] * w[:, None]).T @ v[b, h] + np.exp(LT) * S0
             z_T[b, h] = (k[b, h] * w[:, None]).sum(axis=0) + np.exp(LT) * z0
     return y, S_T, z_T
+
+
+def parallel_reverse(q, k, v, decay_kind=0, log_g=None, normalize=False,
+                     init_state=None, init_z=None):
+    """Anti-causal parallel form of the reverse scan (S_t = g_t S_{t+1} + k_t
+    v_t^T), float64, stated independently of the recurrent oracle.  With
+    R_t = sum_{r>=t} log g_r (suffix sums) the weight of token s >= t in y_t
+    is prod_{r=t}^{s-1} g_r = exp(R_t - R_s), and the state entering from
+    beyond the end reaches token t with exp(R_t):
+        y_t   = sum_{s>=t} exp(R_t - R_s) (q_t . k_s) v_s + exp(R_t) q_t^T S_0
+        den_t = sum_{s>=t} exp(R_t - R_s) (q_t . k_s)     + exp(R_t) q_t . z_0
+        S_1   = sum_s exp(R_1 - R_s) k_s v_s^T + exp(R_1) S_0   (z_1 likewise)
+    Returns (y, S_1, z_1)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    y = np.zeros((B, H, T, Dv))
+    S_1 = np.zeros((B, H, Dk, Dv))
+    z_1 = np.zeros((B, H, Dk))
+    for b in range(B):
+        for h in range(H):
+            S0 = np.zeros((Dk, Dv)) if init_state is None else init_state[b, h]
+            z0 = np.zeros(Dk) if init_z is None else init_z[b, h]
+            ell = _log_decay(decay_kind, log_g, b, h, T)
+            R = np.cumsum(ell[::-1])[::-1]
+            anti = np.triu(np.ones((T, T), dtype=bool))
+            D = np.zeros((T, T))
+            diff = R[:, None] - R[None, :]
+            D[anti] = np.exp(diff[anti])
+            A = (q[b, h] @ k[b, h].T) * D
+            num = A @ v[b, h] + np.exp(R)[:, None] * (q[b, h] @ S0)
+            if normalize:
+                den = A.sum(axis=1) + np.exp(R) * (q[b, h] @ z0)
+                y[b, h] = num / den[:, None]
+            else:
+                y[b, h] = num
+            R1 = R[0] if T > 0 else 0.0
+            w = np.exp(R1 - R)
+            S_1[b, h] = (k[b, h] * w[:, None]).T @ v[b, h] + np.exp(R1) * S0
+            z_1[b, h] = (k[b, h] * w[:, None]).sum(axis=0) + np.exp(R1) * z0
+    return y, S_1, z_1

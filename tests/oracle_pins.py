@@ -293,3 +293,68 @@ def decode_matches(fwd, dec):
 ALL = [worked_examples, cumsum_form, t1_closed_form, t2_closed_form, one_hot_keys,
        zero_keys, scalar_powers, normaliser_unity, normaliser_scale, split_carry,
        ema_operator, decode_matches]
+
+
+# -- reverse scan (S_t = g_t S_{t+1} + k_t v_t^T) and bidirectional sum -----
+
+def reverse_parallel_form(rev, parallel_rev):
+    rng = np.random.default_rng(31)
+    for kind in (0, 1, 2):
+        for normalize in (False, True):
+            for with_init in (False, True):
+                B, H, T, Dk, Dv = 2, 2, 29, 4, 3
+                if normalize:
+                    q, k = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk)
+                else:
+                    q, k = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk)
+                v = _rand(rng, B, H, T, Dv)
+                lg = _log_g(rng, kind, B, H, T)
+                S0 = _rand(rng, B, H, Dk, Dv) if with_init else None
+                z0 = np.abs(_rand(rng, B, H, Dk)) if (with_init and normalize) else None
+                y, S, z = rev(q, k, v, kind, lg, normalize, S0, z0)
+                yp, Sp, zp = parallel_rev(q, k, v, kind, lg, normalize, S0, z0)
+                tag = f"reverse kind={kind} norm={normalize} init={with_init}"
+                _close(y, yp, 1e-10, "y " + tag)
+                _close(S, Sp, 1e-10, "S " + tag)
+                if normalize:
+                    _close(z, zp, 1e-10, "z " + tag)
+
+
+def reverse_cumsum_form(rev):
+    # g = 1: the state at t is the suffix sum of k_s v_s^T
+    rng = np.random.default_rng(32)
+    B, H, T, Dk, Dv = 1, 2, 19, 3, 4
+    q, k, v = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dv)
+    y, S, _ = rev(q, k, v)
+    outer = k[..., :, None] * v[..., None, :]
+    states = np.flip(np.cumsum(np.flip(outer, 2), axis=2), 2)
+    _close(y, np.einsum("bhti,bhtij->bhtj", q, states), TOL, "reverse cumsum y")
+    _close(S, states[:, :, 0], TOL, "reverse cumsum state at token 1")
+
+
+def reverse_t2_closed_form(rev):
+    # T = 2, per-step g: S_2 = g_2 S0 + k_2 v_2^T, S_1 = g_1 S_2 + k_1 v_1^T
+    rng = np.random.default_rng(33)
+    Dk, Dv = 3, 2
+    q, k, v = _rand(rng, 1, 1, 2, Dk), _rand(rng, 1, 1, 2, Dk), _rand(rng, 1, 1, 2, Dv)
+    S0 = _rand(rng, 1, 1, Dk, Dv)
+    g = np.array([0.6, 0.8])
+    y, S, _ = rev(q, k, v, 2, np.log(g)[None, None, :], False, S0)
+    q1, q2, k1, k2, v1, v2, S0v = q[0, 0, 0], q[0, 0, 1], k[0, 0, 0], k[0, 0, 1], v[0, 0, 0], v[0, 0, 1], S0[0, 0]
+    S2 = g[1] * S0v + np.outer(k2, v2)
+    S1 = g[0] * S2 + np.outer(k1, v1)
+    _close(y[0, 0, 1], q2 @ S2, TOL, "reverse T=2 y_2")
+    _close(y[0, 0, 0], q1 @ S1, TOL, "reverse T=2 y_1")
+    _close(S[0, 0], S1, TOL, "reverse T=2 state at token 1")
+
+
+def bidirectional_closed_form(bi):
+    # g = 1: forward counts s <= t and reverse s >= t, so their sum is
+    # (Q K^T) V plus the diagonal term (q_t . k_t) v_t once more
+    rng = np.random.default_rng(34)
+    B, H, T, Dk, Dv = 1, 2, 17, 3, 4
+    q, k, v = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dv)
+    y = bi(q, k, v)
+    A = np.einsum("bhti,bhsi->bhts", q, k)
+    diag = np.einsum("bhti,bhti->bht", q, k)[..., None] * v
+    _close(y, A @ v + diag, TOL, "bidirectional g=1")

@@ -68,3 +68,23 @@ def test_rejects_bad_arguments(oracle_lib):
         oracle.forward(q, q, q, 3, np.zeros(1))
     with pytest.raises(ValueError):
         oracle.forward(q, q, q, 1, None)
+
+
+# ---------------------------------------------------------------- reverse scan
+def _rev(*a, **kw):
+    return oracle.reverse(*a, nthreads=2, **kw)
+
+
+def test_reverse_matches_anticausal_form(oracle_lib):
+    pins.reverse_parallel_form(_rev, oracle.parallel_reverse)
+
+
+@pytest.mark.parametrize("check", [pins.reverse_cumsum_form, pins.reverse_t2_closed_form],
+                         ids=lambda f: f.__name__)
+def test_reverse_closed_forms(oracle_lib, check):
+    check(_rev)          # the recurrent reverse (forward of the time-reversed arguments)
+    check(oracle.parallel_reverse)  # and the independent anti-causal form
+
+
+def test_bidirectional_closed_form(oracle_lib):
+    pins.bidirectional_closed_form(lambda q, k, v: oracle.bidirectional(q, k, v, nthreads=2))
