@@ -185,6 +185,55 @@ LA_API la_status la_chunk_forward_ws(const void* q, const void* k, const void* v
                               la_stream_t stream);
 
 /*
+ * la_chunk_reverse_ws - the anti-causal (right-to-left) scan.
+ *
+ * The recurrence run from the last token back to the first: RetNet issue 21,
+ * Details (the cumulative EMA's reverse flag: the forward scan of the
+ * time-reversed inputs, reversed back), which gives:
+ *
+ *   S_{T+1} = init_state (or 0),   z_{T+1} = init_z (or 0)
+ *   S_t = g_t S_{t+1} + k_t v_t^T,  z_t = g_t z_{t+1} + k_t,   t = T .. 1
+ *   y_t = q_t^T S_t  (normalize: / q_t^T z_t)
+ *
+ * so y_t sums over s >= t with the weight g_t g_{t+1} ... g_{s-1}; the
+ * decay g_t of token t scales everything after it, mirroring the forward
+ * scan.  final_state / final_z receive S_1 / z_1.  Arguments, layouts,
+ * workspace (sized by la_chunk_forward_workspace_size), aliasing rules and
+ * errors as la_chunk_forward_ws.
+ */
+LA_API la_status la_chunk_reverse_ws(const void* q, const void* k, const void* v,
+                              const la_decay* decay, int normalize,
+                              const float* init_state, const float* init_z,
+                              void* out, float* final_state, float* final_z,
+                              int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                              void* workspace, size_t workspace_bytes,
+                              la_stream_t stream);
+
+/*
+ * la_chunk_bidirectional_ws - the bidirectional (encoder) form:
+ * out = y_forward + y_reverse, both scans from zero states.
+ *
+ * RetNet issue 21, Details (closing remark) builds a bidirectional encoder
+ * from one forward and one reverse retention of the same sequence.  Both
+ * scans include their own token, and the plain reading of that remark -
+ * the sum of the two outputs - counts the s = t term q_t^T k_t v_t twice.  That is what
+ * this computes; with normalize each direction is normalised by its own key
+ * sum before the addition.  Two launches on `stream`: the forward scan
+ * writes out, the reverse scan adds to it (bf16: the sum is formed in fp32
+ * from the stored bf16 forward value and rounded once more).
+ *
+ *   q, k, v, decay, normalize, out, B, H, T, Dk, Dv, dtype, workspace,
+ *   workspace_bytes, stream   as la_chunk_forward_ws.
+ *
+ * Errors as la_chunk_forward_ws; on an error nothing is enqueued.
+ */
+LA_API la_status la_chunk_bidirectional_ws(const void* q, const void* k, const void* v,
+                                    const la_decay* decay, int normalize, void* out,
+                                    int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                                    void* workspace, size_t workspace_bytes,
+                                    la_stream_t stream);
+
+/*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
  * device array inside this library (la_chunk_forward_noalloc_capacity()
  * bytes, 16 MiB, one per device, reserved when the library's device code is

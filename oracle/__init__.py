@@ -141,8 +141,9 @@ def reverse(q, k, v, decay_kind=0, log_g=None, normalize=False,
 
 def bidirectional(q, k, v, decay_kind=0, log_g=None, normalize=False, nthreads=None, lib=None):
     """Bidirectional encoder, float64: the forward scan plus the reverse scan
-    (RetNet issue 21: "combining two", one with reverse=False and one with
-    reverse=True; read as their sum).  No carried state."""
+    (RetNet issue 21, Details, closing remark: an encoder built from one
+    reverse=False and one reverse=True retention; read as their sum, so the
+    diagonal term appears in both).  No carried state."""
     yf, _, _ = forward(q, k, v, decay_kind, log_g, normalize, nthreads=nthreads, lib=lib)
     yr, _, _ = reverse(q, k, v, decay_kind, log_g, normalize, nthreads=nthreads, lib=lib)
     return yf + yr

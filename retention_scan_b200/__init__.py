@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "workspace_size", "decode_step", "device_error", "LAError", "lib", "library_path",
+__all__ = ["chunk_forward", "bidirectional", "workspace_size", "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -22,6 +22,7 @@ library_path = os.path.join(_HERE, "libla.so")
 DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
 LA_F32, LA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
+                    "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -55,6 +56,11 @@ def lib():
         L.la_chunk_forward_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, vp, vp,
                                           i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
         L.la_chunk_forward_ws.restype = i
+        L.la_chunk_reverse_ws.argtypes = L.la_chunk_forward_ws.argtypes
+        L.la_chunk_reverse_ws.restype = i
+        L.la_chunk_bidirectional_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp,
+                                                i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_chunk_bidirectional_ws.restype = i
         L.la_chunk_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_forward_workspace_size.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
@@ -118,10 +124,27 @@ def workspace_size(B, H, T, Dk, Dv, dtype=torch.bfloat16, normalize=False):
     return int(lib().la_chunk_forward_workspace_size(B, H, T, Dk, Dv, _dtype_code(dtype), int(bool(normalize))))
 
 
+def _workspace(workspace, B, H, T, Dk, Dv, dtype, normalize, stream, dev):
+    if workspace is True:
+        nbytes = workspace_size(B, H, T, Dk, Dv, dtype, normalize)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+        if workspace is not None and stream is not None:
+            workspace.record_stream(stream)
+    elif workspace is False:
+        workspace = None
+    if workspace is not None:
+        if workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
+    return workspace
+
+
 def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
                   init_state=None, init_z=None, out=None, final_state=None, final_z=None,
-                  return_final=True, stream=None, workspace=True):
-    """Whole-sequence forward (la_chunk_forward_ws).
+                  return_final=True, stream=None, workspace=True, reverse=False):
+    """Whole-sequence forward (la_chunk_forward_ws), or with reverse=True the
+    anti-causal scan from the last token back (la_chunk_reverse_ws; the
+    carried state then enters after token T and final_* hold the state at
+    token 1).
 
     q, k: [B,H,T,Dk]; v: [B,H,T,Dv]; float32 or bfloat16 CUDA tensors.
     decay_kind: DECAY_NONE, DECAY_PER_HEAD (log_g [H]) or DECAY_PER_STEP
@@ -157,22 +180,43 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     _need(final_z, "final_z", (B, H, Dk), torch.float32, dev)
     d = _decay(decay_kind, log_g)
     with torch.cuda.device(dev):
-        if workspace is True:
-            nbytes = workspace_size(B, H, T, Dk, Dv, q.dtype, normalize)
-            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
-            if workspace is not None and stream is not None:
-                workspace.record_stream(stream)
-        elif workspace is False:
-            workspace = None
-        if workspace is not None:
-            if workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
-                raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
-        _check(lib().la_chunk_forward_ws(
+        workspace = _workspace(workspace, B, H, T, Dk, Dv, q.dtype, normalize, stream, dev)
+        entry = lib().la_chunk_reverse_ws if reverse else lib().la_chunk_forward_ws
+        _check(entry(
             _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
             _ptr(init_state), _ptr(init_z), _ptr(out), _ptr(final_state), _ptr(final_z),
             B, H, T, Dk, Dv, code, _ptr(workspace), 0 if workspace is None else workspace.numel(),
             _stream(stream, dev)))
     return out, final_state, (final_z if normalize else None)
+
+
+def bidirectional(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False, out=None, stream=None,
+                  workspace=True):
+    """Bidirectional encoder output (la_chunk_bidirectional_ws): the forward
+    scan plus the reverse scan, both from zero states.  Arguments as
+    chunk_forward.  Returns out [B,H,T,Dv]."""
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q.dtype)
+    _need(k, "k", (B, H, T, Dk), q.dtype, dev)
+    _need(v, "v", (B, H, T, Dv), q.dtype, dev)
+    _need(q, "q", (B, H, T, Dk), q.dtype, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H, T), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, T, Dv), dtype=q.dtype, device=dev)
+    _need(out, "out", (B, H, T, Dv), q.dtype, dev)
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        workspace = _workspace(workspace, B, H, T, Dk, Dv, q.dtype, normalize, stream, dev)
+        _check(lib().la_chunk_bidirectional_ws(
+            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+            _ptr(out), B, H, T, Dk, Dv, code, _ptr(workspace), 0 if workspace is None else workspace.numel(),
+            _stream(stream, dev)))
+    return out
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,

@@ -57,40 +57,12 @@ la_status check_decay(const la_decay* decay, int* kind, const float** log_g) {
     return LA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* la_status_string(la_status status) {
-    switch (status) {
-        case LA_OK: return "LA_OK";
-        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
-        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: no kernel for this shape or dtype";
-        case LA_ERR_CUDA: return "LA_ERR_CUDA: a CUDA call or kernel launch failed";
-    }
-    return "unknown la_status";
-}
-
-const char* la_version(void) { return "0.1.0"; }
-
-size_t la_chunk_forward_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int normalize) {
-    if (dtype != LA_BF16 || B < 1 || H < 1 || T < 1) return 0;
-    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
-    return la::fwd_tc_workspace_bytes(B, H, T, Dk, Dv, normalize != 0);
-}
-
-la_status la_chunk_forward(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
-                           const float* init_state, const float* init_z, void* out, float* final_state,
-                           float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
-                           la_stream_t stream) {
-    return la_chunk_forward_ws(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T,
-                               Dk, Dv, dtype, nullptr, 0, stream);
-}
-
-la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
-                              const float* init_state, const float* init_z, void* out, float* final_state,
-                              float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace,
-                              size_t workspace_bytes, la_stream_t stream) {
+// One whole-sequence scan, forward (t = 1..T) or reverse (t = T..1), its
+// outputs written to out or (accumulate) added to the values already there.
+la_status scan(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+               const float* init_state, const float* init_z, void* out, float* final_state, float* final_z,
+               int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace, size_t workspace_bytes,
+               la_stream_t stream, int reverse, int accumulate) {
     if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
@@ -148,6 +120,8 @@ la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const
     a.Dv = Dv;
     a.stream = s;
     a.err_word = err_word_for_current_device();
+    a.reverse = reverse;
+    a.accumulate = accumulate;
     cudaError_t e;
     if (dtype == LA_F32) {
         e = la::launch_fwd_f32(a);
@@ -158,6 +132,64 @@ la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const
         if (e == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
     }
     return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* la_status_string(la_status status) {
+    switch (status) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: no kernel for this shape or dtype";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: a CUDA call or kernel launch failed";
+    }
+    return "unknown la_status";
+}
+
+const char* la_version(void) { return "0.1.0"; }
+
+size_t la_chunk_forward_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int normalize) {
+    if (dtype != LA_BF16 || B < 1 || H < 1 || T < 1) return 0;
+    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
+    return la::fwd_tc_workspace_bytes(B, H, T, Dk, Dv, normalize != 0);
+}
+
+la_status la_chunk_forward(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                           const float* init_state, const float* init_z, void* out, float* final_state,
+                           float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                           la_stream_t stream) {
+    return la_chunk_forward_ws(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T,
+                               Dk, Dv, dtype, nullptr, 0, stream);
+}
+
+la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                              const float* init_state, const float* init_z, void* out, float* final_state,
+                              float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace,
+                              size_t workspace_bytes, la_stream_t stream) {
+    return scan(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T, Dk, Dv, dtype,
+                workspace, workspace_bytes, stream, 0, 0);
+}
+
+la_status la_chunk_reverse_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                              const float* init_state, const float* init_z, void* out, float* final_state,
+                              float* final_z, int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace,
+                              size_t workspace_bytes, la_stream_t stream) {
+    return scan(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T, Dk, Dv, dtype,
+                workspace, workspace_bytes, stream, 1, 0);
+}
+
+la_status la_chunk_bidirectional_ws(const void* q, const void* k, const void* v, const la_decay* decay,
+                                    int normalize, void* out, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                                    void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    // the reverse scan's launch is not enqueued unless the forward one was;
+    // the arguments are checked once, by the first call
+    const la_status st = scan(q, k, v, decay, normalize, nullptr, nullptr, out, nullptr, nullptr, B, H, T, Dk, Dv,
+                              dtype, workspace, workspace_bytes, stream, 0, 0);
+    if (st != LA_OK) return st;
+    return scan(q, k, v, decay, normalize, nullptr, nullptr, out, nullptr, nullptr, B, H, T, Dk, Dv, dtype,
+                workspace, workspace_bytes, stream, 1, 1);
 }
 
 la_status la_decode_step(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,

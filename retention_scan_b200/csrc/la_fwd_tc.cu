@@ -216,6 +216,8 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     p.split = split;
     p.nchunks = nchunks;
     p.err = a.err_word;
+    p.reverse = a.reverse;
+    p.accumulate = a.accumulate;
     if (L.nS > 0) {
         float* base = static_cast<float*>(a.workspace);
         p.ws_S = base;

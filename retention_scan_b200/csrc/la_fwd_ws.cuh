@@ -221,6 +221,11 @@ struct Params {
     float* ws_L;         // [B H][ws_nS] total log2 decay of each state segment
     int ws_nS;           // state segments per (b, h)
     int ws_per_seg;      // state segments per output segment
+    // reverse scan (S_t = g_t S_{t+1} + k_t v_t^T): chunks are visited from
+    // the last, and inside a chunk the decay runs from its last token; the
+    // kernel works in scan order, mem_chunk maps it to memory
+    int reverse;
+    int accumulate;      // add y to the values already in out (bf16 read, fp32 add)
 };
 
 // What every role needs from the kernel prologue (passed by value).
@@ -334,11 +339,24 @@ __host__ __device__ constexpr uint32_t kstep(int kk, int W) {
 }
 
 // Store 16 outputs o * inv as bf16 (32 bytes) at dst: one 32-byte store when
-// the output is 32-byte aligned, else two 16-byte stores.
-__device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)[16], float inv, bool wide) {
+// the output is 32-byte aligned, else two 16-byte stores. With acc the bf16
+// values already at dst are added first (in fp32, one rounding to bf16).
+__device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)[16], float inv, bool wide,
+                                            bool acc) {
     uint32_t u[8];
+    if (acc) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(dst);
+        const uint4 h0 = s4[0], h1 = s4[1];
+        const uint32_t old[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) u[e] = pack2(o[2 * e] * inv, o[2 * e + 1] * inv);
+        for (int e = 0; e < 8; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&old[e]));
+            u[e] = pack2(fmaf(o[2 * e], inv, f.x), fmaf(o[2 * e + 1], inv, f.y));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[e] = pack2(o[2 * e] * inv, o[2 * e + 1] * inv);
+    }
     if (wide) {
         st_global_v8(dst, u);
     } else {
@@ -357,6 +375,10 @@ __device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)
     volatile int* const abort = reinterpret_cast<volatile int*>(sm + G::OFF_MISC + 8 * B_COUNT + 4); \
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;                                      \
     const int T = p.T, n = x.n;                                                                      \
+    const auto mem_chunk = [&](int c) { /* memory chunk of the c-th chunk of this segment */         \
+        return p.reverse ? p.nchunks - 1 - (x.c0 + c) : x.c0 + c;                                    \
+    };                                                                                               \
+    (void)mem_chunk;                                                                                 \
     (void)sa;                                                                                        \
     (void)tmem;                                                                                      \
     (void)warp;                                                                                      \
@@ -376,7 +398,7 @@ __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
         mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
         uint8_t* st = sm + s * G::Q_STAGE;
         for (int pp = 0; pp < G::PK; ++pp)
-            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * (G::WK / 2), (x.c0 + c) * C, x.bh);
+            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * (G::WK / 2), mem_chunk(c) * C, x.bh);
         ++issued;
     }
     if (*abort) {  // let issued copies land before the CTA's shared memory goes away
@@ -402,7 +424,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_KFULL + s], G::Q_TX);
             uint8_t* st = sm + G::OFF_K + s * G::Q_STAGE;
             for (int pp = 0; pp < G::PK; ++pp)
-                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * (G::WK / 2), (x.c0 + ck) * C, x.bh);
+                tma_load_3d(st + pp * C * G::WK, tmk, &bar[B_KFULL + s], pp * (G::WK / 2), mem_chunk(ck) * C, x.bh);
             ++ck;
             moved = true;
         }
@@ -412,7 +434,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
             mbar_arrive_expect_tx(&bar[B_VFULL + s], G::V_TX);
             uint8_t* st = sm + G::OFF_V + s * G::V_STAGE;
             for (int pp = 0; pp < G::PV; ++pp)
-                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * (G::WV / 2), (x.c0 + cv) * C,
+                tma_load_3d(st + pp * C * G::WV, tmv, &bar[B_VFULL + s], x.j0 + pp * (G::WV / 2), mem_chunk(cv) * C,
                             x.bh);
             ++cv;
             moved = true;
@@ -622,7 +644,8 @@ __device__ __noinline__ void role_mma(const Ctx x) {
 // (warpgroup 1), given as `tile`, is decayed in place for its Q S and K^T V.
 template <int DK>
 __device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint64_t* aempty, int wg, int t,
-                                         bool all_masked, float lt, float lc, const float* lam, uint8_t* tile) {
+                                         bool all_masked, float lt, float lc, const float* lam, uint8_t* tile,
+                                         bool rev) {
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
         float a0[16], a1[16];
@@ -643,10 +666,11 @@ __device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint6
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int s0 = base + 2 * e;
-            const float f0 = s0 <= t ? a0[2 * e] * ex2_approx(lt - lam[s0]) : 0.f;
-            const float f1 = s0 + 1 <= t ? a0[2 * e + 1] * ex2_approx(lt - lam[s0 + 1]) : 0.f;
-            const float f2 = s0 + 16 <= t ? a1[2 * e] * ex2_approx(lt - lam[s0 + 16]) : 0.f;
-            const float f3 = s0 + 17 <= t ? a1[2 * e + 1] * ex2_approx(lt - lam[s0 + 17]) : 0.f;
+            // kept: s <= t (forward) or s >= t (reverse scan)
+            const float f0 = (rev ? s0 >= t : s0 <= t) ? a0[2 * e] * ex2_approx(lt - lam[s0]) : 0.f;
+            const float f1 = (rev ? s0 + 1 >= t : s0 + 1 <= t) ? a0[2 * e + 1] * ex2_approx(lt - lam[s0 + 1]) : 0.f;
+            const float f2 = (rev ? s0 + 16 >= t : s0 + 16 <= t) ? a1[2 * e] * ex2_approx(lt - lam[s0 + 16]) : 0.f;
+            const float f3 = (rev ? s0 + 17 >= t : s0 + 17 <= t) ? a1[2 * e + 1] * ex2_approx(lt - lam[s0 + 17]) : 0.f;
             u[e] = pack2(f0, f1);
             u[8 + e] = pack2(f2, f3);
         }
@@ -673,7 +697,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     auto fetch = [&](int c) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = (x.c0 + c) * C + 4 * lane + i;
+            const int row = mem_chunk(c) * C + 4 * lane + i;
             nxt[i] = (kind == LA_DECAY_PER_STEP && c < n && row < T) ? lg[row] : 0.f;
         }
     };
@@ -683,7 +707,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     // mode) into the V stage, the output row factors and the scaled value
     // rows; warpgroup 1 writes the normaliser weights, or has nothing to do.
     auto prep = [&](int c) -> bool {
-        const int s = c % G::NVS, rem = min(C, T - (x.c0 + c) * C);
+        const int s = c % G::NVS, rem = min(C, T - mem_chunk(c) * C);
         if (!NORM && wg == 1) {
             // nothing to prepare; in the state pass (no mask to pace this
             // warpgroup) wait for the tile so that its arrivals never run a
@@ -712,12 +736,18 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             const float excl = incl - a3;
             lc = __shfl_sync(0xffffffffu, incl, 31);
             float* lam = reinterpret_cast<float*>(sm + G::OFF_V + s * G::V_STAGE + G::VS_LAM);
-            if ((lane >> 3) == wq)
-                *reinterpret_cast<float4*>(lam + 4 * lane) = make_float4(excl + a0, excl + a1, excl + a2, excl + a3);
+            if ((lane >> 3) == wq) {
+                // forward: inclusive prefix of the row; reverse: inclusive
+                // suffix (the chunk total minus the exclusive prefix)
+                const float4 pre = p.reverse
+                                       ? make_float4(lc - excl, lc - excl - a0, lc - excl - a1, lc - excl - a2)
+                                       : make_float4(excl + a0, excl + a1, excl + a2, excl + a3);
+                *reinterpret_cast<float4*>(lam + 4 * lane) = pre;
+            }
             __syncwarp();
             lt = lam[t];
         } else {  // per head (ell_head = L per step), or none (ell_head = 0)
-            lt = static_cast<float>(min(t + 1, rem)) * ell_head;
+            lt = static_cast<float>(p.reverse ? max(rem - t, 0) : min(t + 1, rem)) * ell_head;
             lc = static_cast<float>(rem) * ell_head;
         }
         const int md = kind == LA_DECAY_NONE ? kModeNone : (-lc <= kFoldLimit ? kModeFolded : kModeDirect);
@@ -765,17 +795,21 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         if (md == kModeDirect) {
             const float* lam = reinterpret_cast<const float*>(st + G::VS_LAM);
             const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
-            const bool all_masked = (32 * wq + 31) < 64 * wg;  // every row of this warp precedes these columns
+            // every row of this warp precedes (reverse: follows) these columns
+            const bool all_masked = p.reverse ? 32 * wq > 64 * wg + 63 : (32 * wq + 31) < 64 * wg;
             mask_direct<DK>(lane_addr + 128 * ab + 64 * wg, p_addr, &bar[B_AEMPTY + ab], wg, t, all_masked, lam[t], lc, lam,
-                            wg == 0 ? sm + (c % G::NQ) * G::Q_STAGE : sm + G::OFF_K + (c % G::NK) * G::Q_STAGE);
+                            wg == 0 ? sm + (c % G::NQ) * G::Q_STAGE : sm + G::OFF_K + (c % G::NK) * G::Q_STAGE,
+                            p.reverse != 0);
         } else {
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 // 32 x 32 block (row block wq, column block cb) of the scores:
                 // above the diagonal all zero, below it copied, on it masked
+                // (the reverse scan keeps the upper triangle instead)
                 const int cb = 2 * wg + half;
+                const bool rev = p.reverse != 0;
                 uint32_t u[16];
-                if (cb > wq) {
+                if (rev ? cb < wq : cb > wq) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) u[e] = 0u;
                 } else {
@@ -783,18 +817,25 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                     tmem_ld16(lane_addr + 128 * ab + 32 * cb, a0);
                     tmem_ld16(lane_addr + 128 * ab + 32 * cb + 16, a1);
                     tmem_wait_ld();
-                    if (cb < wq) {
+                    if (rev ? cb > wq : cb < wq) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             u[e] = pack2(a0[2 * e], a0[2 * e + 1]);
                             u[8 + e] = pack2(a1[2 * e], a1[2 * e + 1]);
                         }
-                    } else {
+                    } else if (!rev) {
                         const int r = lane;  // column s0 of the block is kept when s0 <= r
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             u[e] = pack2(2 * e <= r ? a0[2 * e] : 0.f, 2 * e + 1 <= r ? a0[2 * e + 1] : 0.f);
                             u[8 + e] = pack2(2 * e + 16 <= r ? a1[2 * e] : 0.f, 2 * e + 17 <= r ? a1[2 * e + 1] : 0.f);
+                        }
+                    } else {
+                        const int r = lane;  // column s0 of the block is kept when s0 >= r
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            u[e] = pack2(2 * e >= r ? a0[2 * e] : 0.f, 2 * e + 1 >= r ? a0[2 * e + 1] : 0.f);
+                            u[8 + e] = pack2(2 * e + 16 >= r ? a1[2 * e] : 0.f, 2 * e + 17 >= r ? a1[2 * e + 1] : 0.f);
                         }
                     }
                 }
@@ -829,16 +870,16 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         } else {
             inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
         }
-        const int rem = min(C, T - (x.c0 + c) * C);
+        const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + x.j0;
+            p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(mem_chunk(c)) * C + t) * p.Dv + x.j0;
 #pragma unroll 1
         for (int piece = 0; piece < NV / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide);
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, p.accumulate != 0);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);
@@ -991,16 +1032,16 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         } else {
             inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
         }
-        const int rem = min(C, T - (x.c0 + c) * C);
+        const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(x.c0 + c) * C + t) * p.Dv + j0 + cb;
+            p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(mem_chunk(c)) * C + t) * p.Dv + j0 + cb;
 #pragma unroll 1
         for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide);
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, p.accumulate != 0);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);

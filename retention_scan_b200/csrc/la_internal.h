@@ -31,6 +31,8 @@ struct FwdArgs {
     int* err_word;            // device error word of the current device
     void* workspace;          // scratch for T-segment states (may be null: no segments)
     size_t workspace_bytes;
+    int reverse;              // 1: anti-causal scan, t = T-1 down to 0
+    int accumulate;           // 1: add y to the values already in out
 };
 
 struct DecodeArgs {

@@ -161,3 +161,49 @@ def test_segmented_entry_rejects_misaligned_workspace(L):
     st = L.la_chunk_forward_ws(None, None, None, None, 0, None, None, None, None, None,
                                1, 1, 0, 16, 16, 1, ctypes.c_void_p(addr), 60, None)
     assert st == 1  # LA_ERR_INVALID_ARG
+
+
+def test_reverse_and_bidirectional_validate_like_the_forward(L):
+    vp = ctypes.c_void_p
+
+    def rev(**over):
+        a = dict(q=16, k=16, v=16, out=16, B=1, H=1, T=4, Dk=16, Dv=16, dtype=1, normalize=0,
+                 init_state=None, init_z=None)
+        a.update(over)
+        return L.la_chunk_reverse_ws(vp(a["q"]), vp(a["k"]), vp(a["v"]), None, a["normalize"],
+                                     vp(a["init_state"]), vp(a["init_z"]), vp(a["out"]), None, None,
+                                     a["B"], a["H"], a["T"], a["Dk"], a["Dv"], a["dtype"], None, 0, None)
+
+    def bi(**over):
+        a = dict(q=16, k=16, v=16, out=16, B=1, H=1, T=4, Dk=16, Dv=16, dtype=1, normalize=0, ws=None)
+        a.update(over)
+        return L.la_chunk_bidirectional_ws(vp(a["q"]), vp(a["k"]), vp(a["v"]), None, a["normalize"],
+                                           vp(a["out"]), a["B"], a["H"], a["T"], a["Dk"], a["Dv"], a["dtype"],
+                                           vp(a["ws"]), 64, None)
+    for f in (rev, bi):
+        assert f(q=None) == 1
+        assert f(out=8) == 1
+        assert f(T=-1) == 1
+        assert f(dtype=9) == 1
+        assert f(Dk=48) == 2
+        assert f(dtype=0, Dv=200) == 2
+        assert f(B=0) == 0
+    assert rev(normalize=1, init_state=32, init_z=None) == 1
+    assert bi(ws=4) == 1  # misaligned workspace
+
+
+def test_injected_launch_failure_reverse_and_bidirectional():
+    code = r'''
+import ctypes, sys
+sys.path.insert(0, %r)
+import retention_scan_b200 as la
+L = la.lib()
+vp = ctypes.c_void_p
+r = L.la_chunk_reverse_ws(vp(16), vp(16), vp(16), None, 0, None, None, vp(16), None, None,
+                          1, 1, 4, 16, 16, 1, None, 0, None)
+r2 = L.la_chunk_bidirectional_ws(vp(16), vp(16), vp(16), None, 0, vp(16), 1, 1, 4, 16, 16, 1, None, 0, None)
+print(r, r2)
+''' % ROOT
+    env = dict(os.environ, LA_FAULT_INJECT="launch")
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
+    assert out.stdout.split() == ["3", "3"]

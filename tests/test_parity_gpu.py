@@ -12,7 +12,7 @@ import torch.nn.functional as F
 
 import oracle
 import workloads as W
-from parity import TOL, oracle_forward, rel_err, to_dev
+from parity import TOL, gen_case, oracle_forward, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -38,29 +38,6 @@ def built():
 def la():
     import retention_scan_b200
     return retention_scan_b200
-
-
-def gen_case(B, H, T, Dk, Dv, dtype=torch.bfloat16, kind=0, normalize=False, seed=0,
-             decay_mean=2.0, init=False):
-    """Random case: q, k ~ elu+1 of N(0,1) when normalised, else N(0,1) with q
-    scaled by Dk^-1/2; v ~ N(0,1); per-step log g = logsigmoid(N(decay_mean,1));
-    per-head log g = log(1 - 2^(-1-h)) (strong decays that the test can see)."""
-    g = torch.Generator().manual_seed(seed)
-    q = torch.randn(B, H, T, Dk, generator=g)
-    k = torch.randn(B, H, T, Dk, generator=g)
-    v = torch.randn(B, H, T, Dv, generator=g)
-    if normalize:
-        q, k = F.elu(q) + 1, F.elu(k) + 1
-    else:
-        q = q * Dk ** -0.5
-    log_g = None
-    if kind == 1:
-        log_g = torch.tensor([math.log1p(-2.0 ** (-1 - h)) for h in range(H)], dtype=torch.float32)
-    elif kind == 2:
-        log_g = F.logsigmoid(torch.randn(B, H, T, generator=g) + decay_mean)
-    S0 = torch.randn(B, H, Dk, Dv, generator=g) if init else None
-    z0 = (torch.rand(B, H, Dk, generator=g) * 4 + 0.5) if (init and normalize) else None
-    return dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), log_g=log_g, decay_kind=kind), S0, z0
 
 
 def run_gpu(inp, normalize=False, S0=None, z0=None):
