@@ -1,6 +1,7 @@
 """Benchmark of the causal-linear-attention library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+                    [--direction forward|reverse|bidirectional]
 
 One step is one pass of the hot path over one batch of the workload:
 
@@ -10,6 +11,10 @@ One step is one pass of the hot path over one batch of the workload:
   config 3: normalised, elu+1 feature map, carried state, B=8, H=16, T=4096, D=128
   config 4: gated per-step decay, B=1, H=32, T=65536, D=128
   config 5: decode, B=256, H=32, D=128, normalised, 1024 la_decode_step calls
+
+--direction reverse times the anti-causal scan (la_chunk_reverse_ws) on the
+same inputs; --direction bidirectional the encoder form (forward scan, then
+the reverse scan adding to its output; no carried state).  Configs 1-4.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
@@ -43,15 +48,22 @@ import torch  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "linear-attn forward tokens/s (B·H·T/s) and % of roofline (tensor TFLOP/s or HBM GB/s)"
+
+
+def metric_for(direction):
+    return METRIC if direction == "forward" else METRIC.replace("forward", direction)
 L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 512 * 1024 * 1024
 
 
 # ---------------------------------------------------------------- workload accounting
 
-def algorithmic_bytes(wl, cfg):
+def algorithmic_bytes(wl, cfg, direction="forward"):
     """Bytes the hot path must move once: inputs read, outputs written, state
-    in/out (fp32), decays; per launch of the dominant kernel."""
+    in/out (fp32), decays; per launch of the dominant kernel.  The
+    bidirectional form has no carried state; its minimum is one read of the
+    inputs and one write of the output, although its two scans read the
+    inputs twice (and the output once more)."""
     es = 4 if wl.dtype == "f32" else 2
     if cfg == 5:
         per_bh = 2 * 4 * wl.Dk * wl.Dv + 2 * 4 * wl.Dk + (2 * wl.Dk + wl.Dv) * es + wl.Dv * es
@@ -60,15 +72,17 @@ def algorithmic_bytes(wl, cfg):
     b = BH * T * ((2 * wl.Dk + wl.Dv) * es + wl.Dv * es)
     if wl.decay == "per_step":
         b += BH * T * 4
+    if direction == "bidirectional":
+        return b
     b += BH * wl.Dk * wl.Dv * 4  # final state written
     if wl.prefix_T:
         b += BH * wl.Dk * wl.Dv * 4 + 2 * BH * wl.Dk * 4  # initial state, key sums in and out
     return b
 
 
-def algorithmic_flops(wl, cfg):
+def algorithmic_flops(wl, cfg, direction="forward"):
     n = wl.B * wl.H * (1 if cfg == 5 else wl.T)
-    return 4 * wl.Dk * wl.Dv * n
+    return 4 * wl.Dk * wl.Dv * n * (2 if direction == "bidirectional" else 1)
 
 
 def tokens_per_step(wl, cfg):
@@ -174,10 +188,11 @@ def bus_id_of(device):
 class Job:
     """Device-resident inputs and the step function of one workload."""
 
-    def __init__(self, cfg, device, wl=None, rank=0):
+    def __init__(self, cfg, device, wl=None, rank=0, direction="forward"):
         import retention_scan_b200 as la
         self.la = la
         self.cfg = cfg
+        self.direction = direction
         self.wl = wl = wl or W.WORKLOADS[cfg]
         self.dev = device
         if cfg == 5:
@@ -201,7 +216,9 @@ class Job:
         # library cuts the sequences into T-segments (it asks for a workspace)
         self.fwd_launches = 2 if (wl.dtype != "f32" and la.workspace_size(
             wl.B, wl.H, wl.T, wl.Dk, wl.Dv, wl.torch_dtype, wl.normalize) > 0) else 1
-        if wl.prefix_T:
+        if direction == "bidirectional":
+            self.fwd_launches *= 2  # a forward and a reverse scan
+        if wl.prefix_T and direction != "bidirectional":
             # carried state of the workload: the library's own forward over the seeded prefix
             pre = W.prefix_inputs(wl)
             _, self.S0, self.z0 = la.chunk_forward(pre["q"].to(device), pre["k"].to(device),
@@ -214,8 +231,12 @@ class Job:
                 la.decode_step(self.q[t], self.k[t], self.v[t], self.S, self.z, 1, self.log_g, True,
                                out=self.out)
             return wl.steps
-        la.chunk_forward(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
-                         out=self.out, final_state=self.S, final_z=self.z)
+        if self.direction == "bidirectional":
+            la.bidirectional(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, out=self.out)
+        else:
+            la.chunk_forward(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
+                             out=self.out, final_state=self.S, final_z=self.z,
+                             reverse=self.direction == "reverse")
         return self.fwd_launches
 
     E2E_DECODE_TOKENS = 64
@@ -234,8 +255,13 @@ class Job:
             return wl.B * wl.H * self.E2E_DECODE_TOKENS
         q, k, v = (pinned[n].to(self.dev, non_blocking=True) for n in ("q", "k", "v"))
         lg = pinned["log_g"].to(self.dev, non_blocking=True) if pinned.get("log_g") is not None else None
+        if self.direction == "bidirectional":
+            y = la.bidirectional(q, k, v, self.kind, lg, wl.normalize, out=self.out)
+            pinned["y"].copy_(y, non_blocking=True)
+            return tokens_per_step(wl, self.cfg)
         y, S, _ = la.chunk_forward(q, k, v, self.kind, lg, wl.normalize, self.S0, self.z0,
-                                   out=self.out, final_state=self.S, final_z=self.z)
+                                   out=self.out, final_state=self.S, final_z=self.z,
+                                   reverse=self.direction == "reverse")
         pinned["y"].copy_(y, non_blocking=True)
         pinned["S"].copy_(S, non_blocking=True)
         return tokens_per_step(wl, self.cfg)
@@ -254,7 +280,9 @@ class Job:
         p["y"] = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         p["S"] = torch.empty(self.S.shape, dtype=torch.float32).pin_memory()
         h2d = sum(p[n].numel() * p[n].element_size() for n in ("q", "k", "v", "log_g") if p[n] is not None)
-        d2h = p["y"].numel() * p["y"].element_size() + p["S"].numel() * 4
+        d2h = p["y"].numel() * p["y"].element_size()
+        if self.direction != "bidirectional":
+            d2h += p["S"].numel() * 4
         return p, h2d, d2h
 
 
@@ -300,7 +328,7 @@ def time_steps(job, steps, flush, dist_on, device):
     return per, launches, wall0, wall1
 
 
-def cpu_baseline(cfg, budget_s=15.0):
+def cpu_baseline(cfg, budget_s=15.0, direction="forward"):
     """The float64 oracle, as it stands, on a bounded sample of the workload:
     whole (b, h) sequences (every token) until about budget_s of CPU work."""
     import oracle
@@ -328,19 +356,25 @@ def cpu_baseline(cfg, budget_s=15.0):
     total = wl.B * wl.H
     # estimate: ~1 GFLOP/s per core for the plain f64 loops
     per_head_s = 4.0 * wl.Dk * wl.Dv * (wl.T + wl.prefix_T) / 1e9
+    if direction == "bidirectional":
+        per_head_s *= 2
     nh = max(1, min(total, int(budget_s * cores / max(per_head_s, 1e-9))))
     nh = min(nh, total)
     heads = list(range(nh))
     inp = W.forward_inputs(wl, heads=heads)
     threads = min(cores, nh)
     init = {}
-    if wl.prefix_T:
+    if wl.prefix_T and direction != "bidirectional":
         pre = W.prefix_inputs(wl, heads=heads)
         _, S0, z0 = oracle.forward(pre["q"], pre["k"], pre["v"], 0, None, True, nthreads=threads)
         init = dict(init_state=S0, init_z=z0)
+    fn = {"forward": oracle.forward, "reverse": oracle.reverse}.get(direction)
     t0 = time.perf_counter()
-    oracle.forward(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize,
-                   nthreads=threads, **init)
+    if fn is None:
+        oracle.bidirectional(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize,
+                             nthreads=threads)
+    else:
+        fn(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize, nthreads=threads, **init)
     dt = time.perf_counter() - t0
     return {"value": nh * wl.T / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{nh} of {total} (b,h) sequences, all {wl.T} tokens each, {threads} threads"}
@@ -360,9 +394,9 @@ def sized_workload(args):
 def run_ours(args, rank, world, dist_on, device):
     cfg = args.config
     wl = sized_workload(args)
-    job = Job(cfg, device, wl, rank)
+    job = Job(cfg, device, wl, rank, args.direction)
     torch.cuda.synchronize()
-    in_bytes = algorithmic_bytes(wl, cfg) * (wl.steps if cfg == 5 else 1)
+    in_bytes = algorithmic_bytes(wl, cfg, args.direction) * (wl.steps if cfg == 5 else 1)
     flush = None
     if in_bytes < 2 * L2_BYTES and cfg != 5:
         flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
@@ -392,16 +426,18 @@ def run_ours(args, rank, world, dist_on, device):
     # is a state pass and an output pass of the same kernel, timed together)
     launch_ms = ms_per_step / (wl.steps if cfg == 5 else 1)
     pk, pk_kind = peaks()
-    bytes_launch = algorithmic_bytes(wl, cfg)
+    bytes_launch = algorithmic_bytes(wl, cfg, args.direction)
     achieved_gbs = bytes_launch / (launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved_gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
                 "peak_source": pk_kind,
                 "kernel": "la_decode (decode_vec_kernel)" if cfg == 5 else
                 ("la_fwd_f32 (fwd_f32_kernel)" if wl.dtype == "f32" else
-                 ("fwd_ws_kernel (state pass + output pass)" if job.fwd_launches == 2 else "fwd_ws_kernel")),
+                 ({1: "fwd_ws_kernel", 2: "fwd_ws_kernel (state pass + output pass)"
+                  if args.direction != "bidirectional" else "fwd_ws_kernel (forward + reverse scan)",
+                  4: "fwd_ws_kernel (state + output pass, forward and reverse)"}[job.fwd_launches])),
                 "algorithmic_bytes_per_launch": bytes_launch,
-                "tensor_frac": round(algorithmic_flops(wl, cfg) / (launch_ms / 1e3) / 1e12 / pk.get("bf16_tflops", 1590.0), 4)}
+                "tensor_frac": round(algorithmic_flops(wl, cfg, args.direction) / (launch_ms / 1e3) / 1e12 / pk.get("bf16_tflops", 1590.0), 4)}
 
     # end to end through the public API with host buffers
     e2e = None
@@ -426,16 +462,19 @@ def run_ours(args, rank, world, dist_on, device):
 
     clocks = sampler.summary(w0, w1) if sampler else None
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric_for(args.direction), "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if wl.dtype == "f32" else "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
                    "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
+                   "direction": args.direction,
                    "decode_steps": wl.steps if cfg == 5 else None,
                    "l2": "flushed before every step (512 MB write)" if flush is not None
                    else "inputs larger than L2",
                    "parallelism": f"replicas x{world}; per GPU (b,h) spread over CTAs by value slices"
-                   + (" and T-segments" if cfg != 5 and job.fwd_launches == 2 else "")},
+                   + (" and T-segments" if cfg != 5 and job.fwd_launches in (2, 4) and
+                      (args.direction != "bidirectional" or job.fwd_launches == 4) else "")},
         "roofline": roofline, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches,
     }
@@ -448,20 +487,21 @@ def run_reference(args):
     cfg = args.config
     wl = W.WORKLOADS[cfg]
     for _ in range(args.warmup):
-        cpu_baseline(cfg, budget_s=2.0)
+        cpu_baseline(cfg, budget_s=2.0, direction=args.direction)
     vals = []
     for _ in range(args.steps):
-        vals.append(cpu_baseline(cfg, budget_s=8.0))
+        vals.append(cpu_baseline(cfg, budget_s=8.0, direction=args.direction))
     v = statistics.median(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = v
     return {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "impl": "reference", "metric": metric_for(args.direction), "value": v, "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tokens_per_step(wl, cfg) / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
-                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize},
+                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
+                   "direction": args.direction},
         "cpu_baseline": cb,
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -479,7 +519,10 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
+    ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional"])
     args = ap.parse_args()
+    if args.config == 5 and args.direction != "forward":
+        ap.error("--direction applies to the whole-sequence configs 1-4")
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
@@ -507,7 +550,7 @@ def main():
         line = run_ours(args, rank, world, dist_on, device)
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(args.config)
+                line["cpu_baseline"] = cpu_baseline(args.config, direction=args.direction)
             print(json.dumps(line), flush=True)
     finally:
         if dist_on:

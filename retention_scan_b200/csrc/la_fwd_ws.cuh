@@ -226,6 +226,7 @@ struct Params {
     // kernel works in scan order, mem_chunk maps it to memory
     int reverse;
     int accumulate;      // add y to the values already in out (bf16 read, fp32 add)
+    int pdl;             // (host) launch with programmatic stream serialisation
 };
 
 // What every role needs from the kernel prologue (passed by value).
@@ -364,6 +365,13 @@ __device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)
         d4[0] = make_uint4(u[0], u[1], u[2], u[3]);
         d4[1] = make_uint4(u[4], u[5], u[6], u[7]);
     }
+}
+
+// Ask L2 for the n bf16 values at p (the output row that an accumulating
+// epilogue reads back one chunk later).
+__device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
+    for (int e = 0; e < n; e += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + e));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p + n - 1));
 }
 
 #define LA_ROLE_PRELUDE                                                                              \
@@ -856,8 +864,15 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     // Epilogue (warpgroup 1, after its mask of the next chunk): y = O times
     // the row factor 2^(L_t) (or / den_t) for all NV columns of the slice;
     // 16-byte stores of bf16 pairs, rows past the sequence end skipped.
+    auto out_row = [&](int c) {
+        return p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(mem_chunk(c)) * C + t) * p.Dv + x.j0;
+    };
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO;
+        if (p.accumulate) {  // the rows this epilogue and the next read back
+            if (c == 0 && t < min(C, T - mem_chunk(0) * C)) prefetch_row_l2(out_row(0), NV);
+            if (c + 1 < n && t < min(C, T - mem_chunk(c + 1) * C)) prefetch_row_l2(out_row(c + 1), NV);
+        }
         if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
         const uint32_t oa = lane_addr + G::COL_O0 + ro * G::OCOLS;
@@ -872,8 +887,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         }
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
-        __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(x.bh) * T + static_cast<size_t>(mem_chunk(c)) * C + t) * p.Dv + x.j0;
+        __nv_bfloat16* dst = out_row(c);
 #pragma unroll 1
         for (int piece = 0; piece < NV / 16; ++piece) {
             float o[16];
@@ -1018,8 +1032,15 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
 
     // Epilogue (unnormalised instances): y = O times the row factor 2^(L_t)
     // for this warpgroup's columns.
+    auto out_row = [&](int c) {
+        return p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(mem_chunk(c)) * C + d) * p.Dv + j0 + cb;
+    };
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO, t = d;
+        if (p.accumulate) {  // the rows this epilogue and the next read back
+            if (c == 0 && t < min(C, T - mem_chunk(0) * C)) prefetch_row_l2(out_row(0), G::NVW);
+            if (c + 1 < n && t < min(C, T - mem_chunk(c + 1) * C)) prefetch_row_l2(out_row(c + 1), G::NVW);
+        }
         if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
         tc_fence_after_sync();
         const uint32_t oa = lane_addr + G::COL_O0 + ro * G::OCOLS;
@@ -1034,8 +1055,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         }
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
-        __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(mem_chunk(c)) * C + t) * p.Dv + j0 + cb;
+        __nv_bfloat16* dst = out_row(c);
 #pragma unroll 1
         for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
@@ -1153,6 +1173,13 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // The prologue above may overlap the previous kernel on the stream (the
+    // launch allows programmatic serialisation); no global memory is read or
+    // written before that kernel has completed.  Every CTA signals the next
+    // launch only after its own wait, so a kernel two launches on still
+    // starts after this one's predecessor has finished.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice, seg, c0, nloc};
     if (warp == G::W_TMA) {
@@ -1186,8 +1213,19 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         cudaError_t e =
             cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        fwd_ws_kernel<DK, NV, NORM><<<grid, G::THREADS, smem, stream>>>(tmq, tmk, tmv, p);
-        return cudaGetLastError();
+        // programmatic serialisation: this grid's prologue (barriers, TMEM,
+        // descriptor prefetch) overlaps the tail of the previous kernel
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(G::THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = p.pdl ? 1 : 0;
+        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM>, tmq, tmk, tmv, p);
     }
 }
 
