@@ -9,6 +9,8 @@ cpu_baseline / reference legs may import this package.  The CUDA library
                          time-reversed arguments, output reversed back
   bidirectional(...)     forward + reverse
   decode_step(...)       one token of the same recurrence, in place
+  backward(...)          gradients of a loss through the forward recurrence,
+                         by the chain rule token by token (la_ref.c)
   parallel_forward(...)  brute-force O(T^2) parallel form, numpy (parallel.py)
   parallel_reverse(...)  brute-force O(T^2) anti-causal form, numpy (parallel.py)
 
@@ -54,6 +56,9 @@ def load_library(path=None):
         lib.la_ref_forward.restype = i
         lib.la_ref_decode_step.argtypes = [d, d, d, i, d, i, d, d, d, i, i, i, i]
         lib.la_ref_decode_step.restype = i
+        lib.la_ref_backward.argtypes = [d, d, d, i, d, i, d, d, d, d, d, d, d, d, d, d, d,
+                                        i, i, i, i, i, i]
+        lib.la_ref_backward.restype = i
         _libs[path] = lib
     return _libs[path]
 
@@ -98,6 +103,41 @@ def forward(q, k, v, decay_kind=0, log_g=None, normalize=False,
     if not normalize:
         z = None
     return y, S, z
+
+
+def backward(q, k, v, dy, decay_kind=0, log_g=None, normalize=False, init_state=None, init_z=None,
+             d_final_state=None, d_final_z=None, nthreads=None, lib=None):
+    """Gradients of L = sum_t dy_t . y_t + <d_final_state, S_T> + <d_final_z, z_T>
+    through forward(q, k, v, decay_kind, log_g, normalize, init_state, init_z),
+    float64, by reverse-mode differentiation of the recurrence (la_ref.c).
+
+    Returns (dq, dk, dv, dlog_g, d_init_state, d_init_z): dlog_g has the shape
+    of log_g ([H]: the per-step gradients summed over b and t, since every step
+    of head h shares log g_h; [B,H,T]; None without decay); d_init_z is None
+    unless normalize.
+    """
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    log_g, init_state, init_z = _f64(log_g), _f64(init_state), _f64(init_z)
+    d_final_state, d_final_z = _f64(d_final_state), _f64(d_final_z)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    kind = _kind(decay_kind)
+    dq, dk, dv = np.zeros((B, H, T, Dk)), np.zeros((B, H, T, Dk)), np.zeros((B, H, T, Dv))
+    dlog = np.zeros((B, H, T))
+    dS0, dz0 = np.zeros((B, H, Dk, Dv)), np.zeros((B, H, Dk))
+    nt = nthreads if nthreads else (os.cpu_count() or 1)
+    rc = (lib or load_library()).la_ref_backward(
+        _ptr(q), _ptr(k), _ptr(v), kind, _ptr(log_g), int(bool(normalize)), _ptr(init_state), _ptr(init_z),
+        _ptr(dy), _ptr(d_final_state), _ptr(d_final_z), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog),
+        _ptr(dS0), _ptr(dz0), B, H, T, Dk, Dv, nt)
+    if rc != 0:
+        raise ValueError("la_ref_backward rejected its arguments")
+    dlog_g = None
+    if kind == 1:
+        dlog_g = dlog.sum(axis=(0, 2))
+    elif kind == 2:
+        dlog_g = dlog
+    return dq, dk, dv, dlog_g, dS0, (dz0 if normalize else None)
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=0, log_g=None, normalize=False, lib=None):

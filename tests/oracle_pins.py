@@ -358,3 +358,122 @@ def bidirectional_closed_form(bi):
     A = np.einsum("bhti,bhsi->bhts", q, k)
     diag = np.einsum("bhti,bhti->bht", q, k)[..., None] * v
     _close(y, A @ v + diag, TOL, "bidirectional g=1")
+
+
+# -- backward: gradients of L = sum dy . y + <dS_T, S_T> + <dz_T, z_T> -------
+#
+#   backward_finite_differences  central differences of L through the
+#                                (pinned) forward, every input, all decay kinds,
+#                                normaliser and carried state
+#   backward_t1_closed_form      T = 1 differentiated by hand
+#   backward_parallel_form       g-weighted matrices: dQ = (dY V^T o M) K,
+#                                dK = (dY V^T o M)^T Q, dV = (Q K^T o M)^T dY
+#                                with M_ts = G_t / G_s (s <= t); the decay
+#                                gradient as the suffix sum of
+#                                q_t . dq_t - k_t . dk_t (plus <S_T, dS_T> at T)
+
+def _loss(fwd, normalize, dy, dST, dzT):
+    def L(q, k, v, kind, lg, S0, z0):
+        y, S, z = fwd(q, k, v, kind, lg, normalize, S0, z0)
+        r = float(np.sum(y * dy)) + float(np.sum(S * dST))
+        if normalize:
+            r += float(np.sum(z * dzT))
+        return r
+    return L
+
+
+def backward_finite_differences(bwd, fwd):
+    rng = np.random.default_rng(41)
+    h = 1e-6
+    for kind in (0, 1, 2):
+        for normalize in (False, True):
+            for with_init in (False, True):
+                B, H, T, Dk, Dv = 1, 2, 7, 3, 4
+                if normalize:
+                    q, k = _positive(rng, B, H, T, Dk), _positive(rng, B, H, T, Dk)
+                else:
+                    q, k = _rand(rng, B, H, T, Dk), _rand(rng, B, H, T, Dk)
+                v = _rand(rng, B, H, T, Dv)
+                lg = _log_g(rng, kind, B, H, T)
+                S0 = _rand(rng, B, H, Dk, Dv) if with_init else None
+                z0 = np.abs(_rand(rng, B, H, Dk)) + 0.5 if (with_init and normalize) else None
+                dy, dST = _rand(rng, B, H, T, Dv), _rand(rng, B, H, Dk, Dv)
+                dzT = _rand(rng, B, H, Dk) if normalize else None
+                L = _loss(fwd, normalize, dy, dST, dzT)
+                grads = bwd(q, k, v, dy, kind, lg, normalize, S0, z0, dST, dzT)
+                args = {"q": q, "k": k, "v": v, "lg": lg, "S0": S0, "z0": z0}
+                slot = {"q": 0, "k": 1, "v": 2, "lg": 3, "S0": 4, "z0": 5}
+                tag = f"kind={kind} norm={normalize} init={with_init}"
+                for name, x in args.items():
+                    if x is None:
+                        continue
+                    flat = x.reshape(-1)
+                    for idx in rng.choice(flat.size, size=min(flat.size, 6), replace=False):
+                        a = dict(args)
+                        xp, xm = x.copy(), x.copy()
+                        xp.reshape(-1)[idx] += h
+                        xm.reshape(-1)[idx] -= h
+                        a[name] = xp
+                        lp = L(a["q"], a["k"], a["v"], kind, a["lg"], a["S0"], a["z0"])
+                        a[name] = xm
+                        lm = L(a["q"], a["k"], a["v"], kind, a["lg"], a["S0"], a["z0"])
+                        fd = (lp - lm) / (2 * h)
+                        got = np.asarray(grads[slot[name]]).reshape(-1)[idx]
+                        assert abs(got - fd) <= 1e-6 * max(1.0, abs(fd)), \
+                            f"d{name}[{idx}] {tag}: {got} vs finite difference {fd}"
+
+
+def backward_t1_closed_form(bwd):
+    # y = g q^T S0 + (q.k) v,  S_1 = g S0 + k v^T,  L = dy.y + <dS, S_1>
+    rng = np.random.default_rng(42)
+    Dk, Dv = 3, 4
+    q, k, v, dy = _rand(rng, Dk), _rand(rng, Dk), _rand(rng, Dv), _rand(rng, Dv)
+    S0, dS = _rand(rng, Dk, Dv), _rand(rng, Dk, Dv)
+    g = 0.7
+    sh = lambda x: x[None, None, None]  # noqa: E731
+    dq, dk, dv, dlg, dS0, _ = bwd(sh(q), sh(k), sh(v), sh(dy), 2, np.full((1, 1, 1), np.log(g)), False,
+                                  S0[None, None], None, dS[None, None], None)
+    _close(dq[0, 0, 0], g * S0 @ dy + k * (v @ dy), TOL, "T=1 dq")
+    _close(dk[0, 0, 0], q * (v @ dy) + dS @ v, TOL, "T=1 dk")
+    _close(dv[0, 0, 0], (q @ k) * dy + dS.T @ k, TOL, "T=1 dv")
+    _close(dS0[0, 0], g * (np.outer(q, dy) + dS), TOL, "T=1 dS0")
+    _close(dlg[0, 0, 0], g * (q @ S0 @ dy + np.sum(S0 * dS)), TOL, "T=1 dlog g")
+
+
+def backward_parallel_form(bwd, fwd):
+    rng = np.random.default_rng(43)
+    for kind in (0, 1, 2):
+        for with_init in (False, True):
+            B, H, T, Dk, Dv = 2, 2, 23, 4, 3
+            q, k, v, dy = (_rand(rng, B, H, T, D) for D in (Dk, Dk, Dv, Dv))
+            lg = _log_g(rng, kind, B, H, T)
+            S0 = _rand(rng, B, H, Dk, Dv) if with_init else np.zeros((B, H, Dk, Dv))
+            dST = _rand(rng, B, H, Dk, Dv)
+            dq, dk, dv, dlg, dS0, _ = bwd(q, k, v, dy, kind, lg, False, S0 if with_init else None, None,
+                                          dST, None)
+            _, ST, _ = fwd(q, k, v, kind, lg, False, S0 if with_init else None, None)
+            tag = f"kind={kind} init={with_init}"
+            dA_all = np.zeros((B, H, T))
+            for b in range(B):
+                for hh in range(H):
+                    a = np.zeros(T) if kind == 0 else (np.full(T, lg[hh]) if kind == 1 else lg[b, hh])
+                    A = np.cumsum(a)                      # log of G_t = g_1 ... g_t
+                    M = np.tril(np.exp(A[:, None] - A[None, :]))
+                    Q, K, V, dY = q[b, hh], k[b, hh], v[b, hh], dy[b, hh]
+                    GT = np.exp(A[-1] - A)                # G_T / G_s
+                    eq = (dY @ V.T * M) @ K + np.exp(A)[:, None] * (dY @ S0[b, hh].T)
+                    ek = (dY @ V.T * M).T @ Q + GT[:, None] * (V @ dST[b, hh].T)
+                    ev = (Q @ K.T * M).T @ dY + GT[:, None] * (K @ dST[b, hh])
+                    _close(dq[b, hh], eq, 1e-10, "parallel dq " + tag)
+                    _close(dk[b, hh], ek, 1e-10, "parallel dk " + tag)
+                    _close(dv[b, hh], ev, 1e-10, "parallel dv " + tag)
+                    dS1 = (np.exp(A)[:, None] * Q).T @ dY + np.exp(A[-1]) * dST[b, hh]
+                    _close(dS0[b, hh], dS1, 1e-10, "parallel dS0 " + tag)
+                    dA = np.sum(Q * eq, axis=1) - np.sum(K * ek, axis=1)
+                    dA[-1] += np.sum(ST[b, hh] * dST[b, hh])
+                    dA_all[b, hh] = np.flip(np.cumsum(np.flip(dA)))
+            if kind == 1:
+                _close(dlg, dA_all.sum(axis=(0, 2)), 1e-9, "parallel dlog g " + tag)
+            elif kind == 2:
+                _close(dlg, dA_all, 1e-9, "parallel dlog g " + tag)
+

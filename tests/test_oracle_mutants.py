@@ -17,12 +17,12 @@ MUTANTS = [
      "S[i * Dv + c] = S[i * Dv + c] + kt[i] * vt[c];\n        if (j->normalize)"),
     ("decay applied after the add", "S[i * Dv + c] = g * S[i * Dv + c] + kt[i] * vt[c];\n        if (j->normalize)",
      "S[i * Dv + c] = g * (S[i * Dv + c] + kt[i] * vt[c]);\n        if (j->normalize)"),
-    ("sign of log decay flipped", "return exp(j->log_g[(size_t)bh * j->T + t]);",
-     "return exp(-j->log_g[(size_t)bh * j->T + t]);"),
-    ("per-step decay off by one token", "return exp(j->log_g[(size_t)bh * j->T + t]);",
-     "return exp(j->log_g[(size_t)bh * j->T + (t > 0 ? t - 1 : 0)]);"),
-    ("per-head decay indexed by batch", "return exp(j->log_g[bh % j->H]);",
-     "return exp(j->log_g[(bh / j->H) % j->H]);"),
+    ("sign of log decay flipped", "return exp(log_g[(size_t)bh * T + t]);",
+     "return exp(-log_g[(size_t)bh * T + t]);"),
+    ("per-step decay off by one token", "return exp(log_g[(size_t)bh * T + t]);",
+     "return exp(log_g[(size_t)bh * T + (t > 0 ? t - 1 : 0)]);"),
+    ("per-head decay indexed by batch", "return exp(log_g[bh % H]);",
+     "return exp(log_g[(bh / H) % H]);"),
     ("key sum not decayed", "if (j->normalize)\n            for (int i = 0; i < Dk; ++i) z[i] = g * z[i] + kt[i];",
      "if (j->normalize)\n            for (int i = 0; i < Dk; ++i) z[i] = z[i] + kt[i];"),
     ("initial state ignored", "S[a] = j->init_state ? j->init_state[ss + a] : 0.0;", "S[a] = 0.0;"),
@@ -39,6 +39,21 @@ MUTANTS = [
      "S[i * Dv + c] = S[i * Dv + c] + kt[i] * vt[c];\n        if (normalize)"),
     ("decode per-step decay read per head", "if (decay_kind == 2) g = exp(log_g[bh]);",
      "if (decay_kind == 2) g = exp(log_g[bh % H]);"),
+    # backward
+    ("state gradient not decayed", "for (int a = 0; a < DD; ++a) G[a] *= g;", "(void)0;"),
+    ("key-sum gradient not decayed", "for (int i = 0; i < Dk; ++i) w[i] *= g;", "(void)0;"),
+    ("decay gradient against the current state", "for (int a = 0; a < DD; ++a) dg += G[a] * Sp[a];",
+     "for (int a = 0; a < DD; ++a) dg += G[a] * St[a];"),
+    ("decay gradient without the factor g", "if (j->dlog) j->dlog[(size_t)bh * T + t] = g * dg;",
+     "if (j->dlog) j->dlog[(size_t)bh * T + t] = dg;"),
+    ("key gradient misses the key-sum term", "j->dk[rq + i] = s + (j->normalize ? w[i] : 0.0);",
+     "j->dk[rq + i] = s;"),
+    ("denominator gradient sign flipped", "f = -dn / (den * den);", "f = dn / (den * den);"),
+    ("value gradient from the query", "for (int i = 0; i < Dk; ++i) s += G[i * Dv + c] * kt[i];",
+     "for (int i = 0; i < Dk; ++i) s += G[i * Dv + c] * qt[i];"),
+    ("query gradient from the previous state", "for (int c = 0; c < Dv; ++c) s += St[i * Dv + c] * e[c];",
+     "for (int c = 0; c < Dv; ++c) s += Sp[i * Dv + c] * e[c];"),
+    ("final state gradient ignored", "G[a] = j->d_final_state ? j->d_final_state[ss + a] : 0.0;", "G[a] = 0.0;"),
 ]
 
 
@@ -55,6 +70,15 @@ def _run_all_pins(lib):
         pins.parallel_form(fwd, dec, oracle.parallel_forward)
     except AssertionError:
         failed.append("parallel_form")
+    bwd = lambda *a, **kw: oracle.backward(*a, nthreads=1, lib=lib, **kw)  # noqa: E731
+    real_fwd = lambda *a, **kw: oracle.forward(*a, nthreads=1, **kw)  # noqa: E731
+    for name, run in (("backward_finite_differences", lambda: pins.backward_finite_differences(bwd, real_fwd)),
+                      ("backward_t1_closed_form", lambda: pins.backward_t1_closed_form(bwd)),
+                      ("backward_parallel_form", lambda: pins.backward_parallel_form(bwd, real_fwd))):
+        try:
+            run()
+        except AssertionError:
+            failed.append(name)
     return failed
 
 

@@ -88,3 +88,30 @@ def test_reverse_closed_forms(oracle_lib, check):
 
 def test_bidirectional_closed_form(oracle_lib):
     pins.bidirectional_closed_form(lambda q, k, v: oracle.bidirectional(q, k, v, nthreads=2))
+
+
+# ---------------------------------------------------------------- backward
+def _bwd(*a, **kw):
+    return oracle.backward(*a, nthreads=2, **kw)
+
+
+def test_backward_matches_finite_differences(oracle_lib):
+    pins.backward_finite_differences(_bwd, _fwd)
+
+
+def test_backward_t1_closed_form(oracle_lib):
+    pins.backward_t1_closed_form(_bwd)
+
+
+def test_backward_matches_parallel_form(oracle_lib):
+    pins.backward_parallel_form(_bwd, _fwd)
+
+
+def test_backward_empty_sequence(oracle_lib):
+    rng = np.random.default_rng(5)
+    dST = rng.standard_normal((1, 2, 3, 4))
+    q = np.zeros((1, 2, 0, 3))
+    v = np.zeros((1, 2, 0, 4))
+    dq, dk, dv, dlg, dS0, _ = oracle.backward(q, q, v, v, 2, np.zeros((1, 2, 0)), False, None, None, dST)
+    assert dq.shape == (1, 2, 0, 3) and dv.shape == (1, 2, 0, 4) and dlg.shape == (1, 2, 0)
+    assert np.array_equal(dS0, dST)
