@@ -12,10 +12,13 @@
 
 namespace la {
 namespace ws {
+// instantiated in la_fwd_ws_dk*.cu (one file per key width and direction)
 #define LA_WS_DECL(DK)                                                                                        \
-    cudaError_t launch_dk##DK(int, bool, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,           \
-                              const Params&, int, cudaStream_t);                                              \
-    bool supported_dk##DK(int, bool);
+    extern template cudaError_t launch_dk<DK, false>(int, bool, const CUtensorMap&, const CUtensorMap&,       \
+                                                     const CUtensorMap&, const Params&, int, cudaStream_t);  \
+    extern template cudaError_t launch_dk<DK, true>(int, bool, const CUtensorMap&, const CUtensorMap&,        \
+                                                    const CUtensorMap&, const Params&, int, cudaStream_t);   \
+    extern template bool supported_dk<DK>(int, bool);
 LA_WS_DECL(16)
 LA_WS_DECL(32)
 LA_WS_DECL(64)
@@ -81,10 +84,10 @@ int sm_count() {
 
 bool instance_ok(int Dk, int nv, bool norm) {
     switch (Dk) {
-        case 16: return ws::supported_dk16(nv, norm);
-        case 32: return ws::supported_dk32(nv, norm);
-        case 64: return ws::supported_dk64(nv, norm);
-        case 128: return ws::supported_dk128(nv, norm);
+        case 16: return ws::supported_dk<16>(nv, norm);
+        case 32: return ws::supported_dk<32>(nv, norm);
+        case 64: return ws::supported_dk<64>(nv, norm);
+        case 128: return ws::supported_dk<128>(nv, norm);
         default: return false;
     }
 }
@@ -178,21 +181,31 @@ namespace {
 constexpr int kPdlFirst = 1;
 constexpr int kPdlOutput = 0;
 
-cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                      const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
+template <bool REV>
+cudaError_t launch_dir(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
     switch (Dk) {
-        case 16: return ws::launch_dk16(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 32: return ws::launch_dk32(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 64: return ws::launch_dk64(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 128: return ws::launch_dk128(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 16: return ws::launch_dk<16, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 32: return ws::launch_dk<32, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 64: return ws::launch_dk<64, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 128: return ws::launch_dk<128, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
         default: return cudaErrorNotSupported;
     }
+}
+
+// The direction picks the instance: the forward instances carry no code of
+// the reverse scan (its index mapping, mask and accumulating epilogue).
+cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                      const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
+    return p.reverse ? launch_dir<true>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream)
+                     : launch_dir<false>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used) {
     if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
+    if (a.accumulate && !a.reverse) return cudaErrorNotSupported;  // only the reverse instances accumulate
     const bool norm = a.normalize != 0;
     const int BH = a.B * a.H;
     const int nchunks = (a.T + ws::C - 1) / ws::C;

@@ -223,9 +223,11 @@ struct Params {
     int ws_per_seg;      // state segments per output segment
     // reverse scan (S_t = g_t S_{t+1} + k_t v_t^T): chunks are visited from
     // the last, and inside a chunk the decay runs from its last token; the
-    // kernel works in scan order, mem_chunk maps it to memory
+    // kernel works in scan order, mem_chunk maps it to memory.  The kernel
+    // takes the direction from its REV template argument (the forward
+    // instances carry no reverse-scan code); this field selects the instance.
     int reverse;
-    int accumulate;      // add y to the values already in out (bf16 read, fp32 add)
+    int accumulate;      // reverse instances only: add y to the values already in out (fp32 add)
     int pdl;             // (host) launch with programmatic stream serialisation
 };
 
@@ -384,9 +386,11 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;                                      \
     const int T = p.T, n = x.n;                                                                      \
     const auto mem_chunk = [&](int c) { /* memory chunk of the c-th chunk of this segment */         \
-        return p.reverse ? p.nchunks - 1 - (x.c0 + c) : x.c0 + c;                                    \
+        return REV ? p.nchunks - 1 - (x.c0 + c) : x.c0 + c;                                          \
     };                                                                                               \
     (void)mem_chunk;                                                                                 \
+    const bool accumulate = REV && p.accumulate != 0; /* only the reverse scan accumulates */        \
+    (void)accumulate;                                                                                \
     (void)sa;                                                                                        \
     (void)tmem;                                                                                      \
     (void)warp;                                                                                      \
@@ -395,7 +399,7 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
 
 // ------------------------------------------------------------ TMA producers
 // Q ring: one thread, blocking on each stage in turn.
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
     LA_ROLE_PRELUDE
     if (lane != 0 || p.state_pass) return;  // the state pass reads no queries
@@ -418,7 +422,7 @@ __device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
 // K and V rings: one thread polls both, so that neither waits behind the
 // other's free stage.  V runs as far ahead as its ring allows: the prep of
 // chunk c + 1 (which needs V) runs before the mask of chunk c.
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, const CUtensorMap* tmv) {
     LA_ROLE_PRELUDE
     if (lane != 0) return;
@@ -479,7 +483,7 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
 // could move) and gives up after kWaitLimitNs without progress.
 // State pass: only K^T V' (and K^T W), in order; each also releases its K and
 // V stages.
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void mma_state_pass(const Ctx x) {
     LA_ROLE_PRELUDE
     const bool leader = elect_one();
@@ -509,11 +513,11 @@ __device__ __noinline__ void mma_state_pass(const Ctx x) {
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
 }
 
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void role_mma(const Ctx x) {
     LA_ROLE_PRELUDE
     if (p.state_pass) {
-        mma_state_pass<DK, NV, NORM>(x);
+        mma_state_pass<DK, NV, NORM, REV>(x);
         return;
     }
     const bool leader = elect_one();
@@ -689,7 +693,7 @@ __device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint6
     fence_async_smem();
 }
 
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void role_prep_mask(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_PM) / 4;  // 0: score columns 0-63, V rows; 1: columns 64-127, weights
@@ -747,7 +751,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             if ((lane >> 3) == wq) {
                 // forward: inclusive prefix of the row; reverse: inclusive
                 // suffix (the chunk total minus the exclusive prefix)
-                const float4 pre = p.reverse
+                const float4 pre = REV
                                        ? make_float4(lc - excl, lc - excl - a0, lc - excl - a1, lc - excl - a2)
                                        : make_float4(excl + a0, excl + a1, excl + a2, excl + a3);
                 *reinterpret_cast<float4*>(lam + 4 * lane) = pre;
@@ -755,7 +759,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             __syncwarp();
             lt = lam[t];
         } else {  // per head (ell_head = L per step), or none (ell_head = 0)
-            lt = static_cast<float>(p.reverse ? max(rem - t, 0) : min(t + 1, rem)) * ell_head;
+            lt = static_cast<float>(REV ? max(rem - t, 0) : min(t + 1, rem)) * ell_head;
             lc = static_cast<float>(rem) * ell_head;
         }
         const int md = kind == LA_DECAY_NONE ? kModeNone : (-lc <= kFoldLimit ? kModeFolded : kModeDirect);
@@ -804,10 +808,10 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             const float* lam = reinterpret_cast<const float*>(st + G::VS_LAM);
             const float lc = *reinterpret_cast<const volatile float*>(st + G::VS_META);
             // every row of this warp precedes (reverse: follows) these columns
-            const bool all_masked = p.reverse ? 32 * wq > 64 * wg + 63 : (32 * wq + 31) < 64 * wg;
+            const bool all_masked = REV ? 32 * wq > 64 * wg + 63 : (32 * wq + 31) < 64 * wg;
             mask_direct<DK>(lane_addr + 128 * ab + 64 * wg, p_addr, &bar[B_AEMPTY + ab], wg, t, all_masked, lam[t], lc, lam,
                             wg == 0 ? sm + (c % G::NQ) * G::Q_STAGE : sm + G::OFF_K + (c % G::NK) * G::Q_STAGE,
-                            p.reverse != 0);
+                            REV);
         } else {
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
@@ -815,7 +819,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                 // above the diagonal all zero, below it copied, on it masked
                 // (the reverse scan keeps the upper triangle instead)
                 const int cb = 2 * wg + half;
-                const bool rev = p.reverse != 0;
+                constexpr bool rev = REV;
                 uint32_t u[16];
                 if (rev ? cb < wq : cb > wq) {
 #pragma unroll
@@ -869,7 +873,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     };
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO;
-        if (p.accumulate) {  // the rows this epilogue and the next read back
+        if (accumulate) {  // the rows this epilogue and the next read back
             if (c == 0 && t < min(C, T - mem_chunk(0) * C)) prefetch_row_l2(out_row(0), NV);
             if (c + 1 < n && t < min(C, T - mem_chunk(c + 1) * C)) prefetch_row_l2(out_row(c + 1), NV);
         }
@@ -893,7 +897,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             float o[16];
             tmem_ld16(oa + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, p.accumulate != 0);
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, accumulate);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);
@@ -921,7 +925,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
 // Warpgroup wg owns value columns [wg NVW, (wg + 1) NVW) of the slice.  Per
 // chunk c: the state update of chunk c, then its bf16 copy, which the next
 // chunk's Q S reads.
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_ES) / 4;
@@ -1037,7 +1041,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     };
     auto epilogue = [&](int c) -> bool {
         const int ro = c % G::NO, t = d;
-        if (p.accumulate) {  // the rows this epilogue and the next read back
+        if (accumulate) {  // the rows this epilogue and the next read back
             if (c == 0 && t < min(C, T - mem_chunk(0) * C)) prefetch_row_l2(out_row(0), G::NVW);
             if (c + 1 < n && t < min(C, T - mem_chunk(c + 1) * C)) prefetch_row_l2(out_row(c + 1), G::NVW);
         }
@@ -1061,7 +1065,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
             tmem_wait_ld();
-            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, p.accumulate != 0);
+            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, accumulate);
         }
         tc_fence_before_sync();
         warp_arrive(&bar[B_OEMPTY + ro]);
@@ -1113,7 +1117,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     }
 }
 
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     fwd_ws_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ Params p) {
@@ -1183,15 +1187,15 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
 
     const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice, seg, c0, nloc};
     if (warp == G::W_TMA) {
-        role_tma_q<DK, NV, NORM>(x, &tmq);
+        role_tma_q<DK, NV, NORM, REV>(x, &tmq);
     } else if (warp == G::W_MMA) {
-        role_mma<DK, NV, NORM>(x);
+        role_mma<DK, NV, NORM, REV>(x);
     } else if (warp < G::W_ES) {
-        role_prep_mask<DK, NV, NORM>(x);
+        role_prep_mask<DK, NV, NORM, REV>(x);
     } else if (warp < G::W_TMAV) {
-        role_state_epilogue<DK, NV, NORM>(x);
+        role_state_epilogue<DK, NV, NORM, REV>(x);
     } else {
-        role_tma_kv<DK, NV, NORM>(x, &tmk, &tmv);
+        role_tma_kv<DK, NV, NORM, REV>(x, &tmk, &tmv);
     }
 
     __syncwarp();  // lanes that idled while lane 0 ran a single-thread role rejoin it
@@ -1201,7 +1205,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_MMA) tmem_dealloc(tmem, G::TMEM_COLS);
 }
 
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool REV>
 cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                             const Params& p, int grid, cudaStream_t stream) {
     using G = Plan<DK, NV, NORM>;
@@ -1211,7 +1215,7 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         // at least 116 KB so that one CTA (512 TMEM columns) owns each SM
         const int smem = G::SMEM > 116 * 1024 ? G::SMEM : 116 * 1024;
         cudaError_t e =
-            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         // programmatic serialisation: this grid's prologue (barriers, TMEM,
         // descriptor prefetch) overlaps the tail of the previous kernel
@@ -1225,13 +1229,46 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = p.pdl ? 1 : 0;
-        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM>, tmq, tmk, tmv, p);
+        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM, REV>, tmq, tmk, tmv, p);
     }
 }
 
 template <int DK, int NV, bool NORM>
 constexpr bool supported() {
     return Plan<DK, NV, NORM>::OK;
+}
+
+// Dispatch on the value slice and the normaliser for one key width and one
+// direction; each instantiation file (la_fwd_ws_dk*.cu) instantiates these
+// for its key width, so that the build compiles the widths in parallel.
+template <int DK, bool REV, bool NORM>
+cudaError_t launch_nv(int nv, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                      const Params& p, int grid, cudaStream_t stream) {
+    switch (nv) {
+        case 16: return launch_instance<DK, 16, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
+        case 32: return launch_instance<DK, 32, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
+        case 64: return launch_instance<DK, 64, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
+        case 128: return launch_instance<DK, 128, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <int DK, bool REV>
+cudaError_t launch_dk(int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                      const Params& p, int grid, cudaStream_t stream) {
+    return norm ? launch_nv<DK, REV, true>(nv, tmq, tmk, tmv, p, grid, stream)
+                : launch_nv<DK, REV, false>(nv, tmq, tmk, tmv, p, grid, stream);
+}
+
+template <int DK>
+bool supported_dk(int nv, bool norm) {
+    switch (nv) {
+        case 16: return norm ? supported<DK, 16, true>() : supported<DK, 16, false>();
+        case 32: return norm ? supported<DK, 32, true>() : supported<DK, 32, false>();
+        case 64: return norm ? supported<DK, 64, true>() : supported<DK, 64, false>();
+        case 128: return norm ? supported<DK, 128, true>() : supported<DK, 128, false>();
+        default: return false;
+    }
 }
 
 }  // namespace ws

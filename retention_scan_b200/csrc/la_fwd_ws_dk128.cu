@@ -1,37 +1,14 @@
-// la_fwd_ws_dk128.cu - instantiations of the warp-specialised tensor-core
-// forward for Dk = 128 (one file per key width so the build runs in parallel).
+// la_fwd_ws_dk128.cu - instantiations of the warp-specialised tensor-core kernel for
+// Dk = 128, forward scan (one file per key width and direction, so that
+// the build compiles them in parallel).
 #include "la_fwd_ws.cuh"
 
 namespace la {
 namespace ws {
 
-template <bool NORM>
-static cudaError_t launch_nv(int nv, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                             const Params& p, int grid, cudaStream_t stream) {
-    switch (nv) {
-        case 16: return launch_instance<128, 16, NORM>(tmq, tmk, tmv, p, grid, stream);
-        case 32: return launch_instance<128, 32, NORM>(tmq, tmk, tmv, p, grid, stream);
-        case 64: return launch_instance<128, 64, NORM>(tmq, tmk, tmv, p, grid, stream);
-        case 128: return launch_instance<128, 128, NORM>(tmq, tmk, tmv, p, grid, stream);
-        default: return cudaErrorNotSupported;
-    }
-}
-
-cudaError_t launch_dk128(int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                        const CUtensorMap& tmv, const Params& p, int grid, cudaStream_t stream) {
-    return norm ? launch_nv<true>(nv, tmq, tmk, tmv, p, grid, stream)
-                : launch_nv<false>(nv, tmq, tmk, tmv, p, grid, stream);
-}
-
-bool supported_dk128(int nv, bool norm) {
-    switch (nv) {
-        case 16: return norm ? supported<128, 16, true>() : supported<128, 16, false>();
-        case 32: return norm ? supported<128, 32, true>() : supported<128, 32, false>();
-        case 64: return norm ? supported<128, 64, true>() : supported<128, 64, false>();
-        case 128: return norm ? supported<128, 128, true>() : supported<128, 128, false>();
-        default: return false;
-    }
-}
+template cudaError_t launch_dk<128, false>(int, bool, const CUtensorMap&, const CUtensorMap&,
+                                             const CUtensorMap&, const Params&, int, cudaStream_t);
+template bool supported_dk<128>(int, bool);
 
 }  // namespace ws
 }  // namespace la
