@@ -14,7 +14,10 @@ One step is one pass of the hot path over one batch of the workload:
 
 --direction reverse times the anti-causal scan (la_chunk_reverse_ws) on the
 same inputs; --direction bidirectional the encoder form (forward scan, then
-the reverse scan adding to its output; no carried state).  Configs 1-4.
+the reverse scan adding to its output; no carried state); --direction
+backward the gradients of the unnormalised forward (la_chunk_backward_ws:
+dq, dk, dv, the log-decay gradient and, with a carried state, the initial
+state's) for a seeded upstream gradient dy.  Configs 1-4 (backward: 1, 2, 4).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
@@ -74,6 +77,12 @@ def algorithmic_bytes(wl, cfg, direction="forward"):
         b += BH * T * 4
     if direction == "bidirectional":
         return b
+    if direction == "backward":
+        # read q, k, v, dy; write dq, dk, dv; the log decay read and its gradient written
+        b = BH * T * (2 * wl.Dk + 2 * wl.Dv) * es + BH * T * (2 * wl.Dk + wl.Dv) * es
+        if wl.decay == "per_step":
+            b += BH * T * 8
+        return b
     b += BH * wl.Dk * wl.Dv * 4  # final state written
     if wl.prefix_T:
         b += BH * wl.Dk * wl.Dv * 4 + 2 * BH * wl.Dk * 4  # initial state, key sums in and out
@@ -82,7 +91,7 @@ def algorithmic_bytes(wl, cfg, direction="forward"):
 
 def algorithmic_flops(wl, cfg, direction="forward"):
     n = wl.B * wl.H * (1 if cfg == 5 else wl.T)
-    return 4 * wl.Dk * wl.Dv * n * (2 if direction == "bidirectional" else 1)
+    return 4 * wl.Dk * wl.Dv * n * {"bidirectional": 2, "backward": 3}.get(direction, 1)
 
 
 def tokens_per_step(wl, cfg):
@@ -218,6 +227,19 @@ class Job:
             wl.B, wl.H, wl.T, wl.Dk, wl.Dv, wl.torch_dtype, wl.normalize) > 0) else 1
         if direction == "bidirectional":
             self.fwd_launches *= 2  # a forward and a reverse scan
+        if direction == "backward":
+            g = torch.Generator(device=device).manual_seed(wl.seed + 500 + 7919 * rank)
+            self.dy = torch.randn(wl.B, wl.H, wl.T, wl.Dv, generator=g, device=device).to(wl.torch_dtype)
+            self.grads = (torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v),
+                          torch.empty_like(self.log_g) if self.log_g is not None else None,
+                          torch.empty(wl.B, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=device))
+            self.bws = torch.empty(la.backward_workspace_size(wl.B, wl.H, wl.T, wl.Dk, wl.Dv, wl.torch_dtype,
+                                                              self.kind), dtype=torch.uint8, device=device)
+            # three scans (each a state pass and an output pass when segmented),
+            # the state transpose, the shifted decay, and the decay-gradient kernels
+            scans = 3 * (2 if (wl.dtype != "f32" and la.workspace_size(
+                wl.B, wl.H, wl.T, wl.Dv, wl.Dk, wl.torch_dtype, False) > 0) else 1)
+            self.fwd_launches = scans + (0 if self.kind == 0 else (1 + 1 + 2 + (1 if self.kind == 1 else 0)))
         if wl.prefix_T and direction != "bidirectional":
             # carried state of the workload: the library's own forward over the seeded prefix
             pre = W.prefix_inputs(wl)
@@ -233,6 +255,9 @@ class Job:
             return wl.steps
         if self.direction == "bidirectional":
             la.bidirectional(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, out=self.out)
+        elif self.direction == "backward":
+            la.chunk_backward(self.q, self.k, self.v, self.dy, self.kind, self.log_g, self.S0, None,
+                              workspace=self.bws, out=self.grads)
         else:
             la.chunk_forward(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
                              out=self.out, final_state=self.S, final_z=self.z,
@@ -259,6 +284,14 @@ class Job:
             y = la.bidirectional(q, k, v, self.kind, lg, wl.normalize, out=self.out)
             pinned["y"].copy_(y, non_blocking=True)
             return tokens_per_step(wl, self.cfg)
+        if self.direction == "backward":
+            dy = pinned["dy"].to(self.dev, non_blocking=True)
+            dq, dk, dv, dlg, _ = la.chunk_backward(q, k, v, dy, self.kind, lg, self.S0, None, workspace=self.bws,
+                                                   out=self.grads)
+            for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("dlog", dlg)):
+                if t is not None:
+                    pinned[n].copy_(t, non_blocking=True)
+            return tokens_per_step(wl, self.cfg)
         y, S, _ = la.chunk_forward(q, k, v, self.kind, lg, wl.normalize, self.S0, self.z0,
                                    out=self.out, final_state=self.S, final_z=self.z,
                                    reverse=self.direction == "reverse")
@@ -279,6 +312,15 @@ class Job:
         p["log_g"] = self.host["log_g"].pin_memory() if self.host["log_g"] is not None else None
         p["y"] = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         p["S"] = torch.empty(self.S.shape, dtype=torch.float32).pin_memory()
+        if self.direction == "backward":
+            p["dy"] = self.dy.cpu().pin_memory()
+            for n, t in zip(("dq", "dk", "dv", "dlog"), self.grads[:4]):
+                if t is not None:
+                    p[n] = torch.empty(t.shape, dtype=t.dtype).pin_memory()
+            h2d = sum(p[n].numel() * p[n].element_size() for n in ("q", "k", "v", "log_g", "dy")
+                      if p[n] is not None)
+            d2h = sum(p[n].numel() * p[n].element_size() for n in ("dq", "dk", "dv", "dlog") if n in p)
+            return p, h2d, d2h
         h2d = sum(p[n].numel() * p[n].element_size() for n in ("q", "k", "v", "log_g") if p[n] is not None)
         d2h = p["y"].numel() * p["y"].element_size()
         if self.direction != "bidirectional":
@@ -358,6 +400,8 @@ def cpu_baseline(cfg, budget_s=15.0, direction="forward"):
     per_head_s = 4.0 * wl.Dk * wl.Dv * (wl.T + wl.prefix_T) / 1e9
     if direction == "bidirectional":
         per_head_s *= 2
+    if direction == "backward":
+        per_head_s *= 4  # a checkpointed forward sweep and the backward sweep
     nh = max(1, min(total, int(budget_s * cores / max(per_head_s, 1e-9))))
     nh = min(nh, total)
     heads = list(range(nh))
@@ -369,8 +413,14 @@ def cpu_baseline(cfg, budget_s=15.0, direction="forward"):
         _, S0, z0 = oracle.forward(pre["q"], pre["k"], pre["v"], 0, None, True, nthreads=threads)
         init = dict(init_state=S0, init_z=z0)
     fn = {"forward": oracle.forward, "reverse": oracle.reverse}.get(direction)
+    if direction == "backward":
+        g = torch.Generator().manual_seed(wl.seed + 500)
+        dy = torch.randn(nh, wl.T, wl.Dv, generator=g).reshape(1, nh, wl.T, wl.Dv).to(wl.torch_dtype)
+        dy = dy.reshape(inp["q"].shape[:3] + (wl.Dv,))
     t0 = time.perf_counter()
-    if fn is None:
+    if direction == "backward":
+        oracle.backward(inp["q"], inp["k"], inp["v"], dy, inp["decay_kind"], inp["log_g"], False, nthreads=threads)
+    elif fn is None:
         oracle.bidirectional(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize,
                              nthreads=threads)
     else:
@@ -433,9 +483,11 @@ def run_ours(args, rank, world, dist_on, device):
                 "peak_source": pk_kind,
                 "kernel": "la_decode (decode_vec_kernel)" if cfg == 5 else
                 ("la_fwd_f32 (fwd_f32_kernel)" if wl.dtype == "f32" else
-                 ({1: "fwd_ws_kernel", 2: "fwd_ws_kernel (state pass + output pass)"
-                  if args.direction != "bidirectional" else "fwd_ws_kernel (forward + reverse scan)",
-                  4: "fwd_ws_kernel (state + output pass, forward and reverse)"}[job.fwd_launches])),
+                 ("fwd_ws_kernel (three scans) and the backward's small kernels"
+                  if args.direction == "backward" else
+                  {1: "fwd_ws_kernel", 2: "fwd_ws_kernel (state pass + output pass)"
+                   if args.direction != "bidirectional" else "fwd_ws_kernel (forward + reverse scan)",
+                   4: "fwd_ws_kernel (state + output pass, forward and reverse)"}[job.fwd_launches])),
                 "algorithmic_bytes_per_launch": bytes_launch,
                 "tensor_frac": round(algorithmic_flops(wl, cfg, args.direction) / (launch_ms / 1e3) / 1e12 / pk.get("bf16_tflops", 1590.0), 4)}
 
@@ -519,10 +571,12 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
-    ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional"])
+    ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional", "backward"])
     args = ap.parse_args()
     if args.config == 5 and args.direction != "forward":
         ap.error("--direction applies to the whole-sequence configs 1-4")
+    if args.direction == "backward" and W.WORKLOADS[args.config].normalize:
+        ap.error("--direction backward: the library's backward covers the unnormalised forward (configs 1, 2, 4)")
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3

@@ -234,6 +234,69 @@ LA_API la_status la_chunk_bidirectional_ws(const void* q, const void* k, const v
                                     la_stream_t stream);
 
 /*
+ * la_chunk_backward_workspace_size - scratch bytes that la_chunk_backward_ws
+ * needs for these sizes (always > 0 for B*H > 0 and T > 0).
+ */
+LA_API size_t la_chunk_backward_workspace_size(int B, int H, int T, int Dk, int Dv,
+                                               la_dtype dtype, int decay_kind);
+
+/*
+ * la_chunk_backward_ws - gradients of the unnormalised forward pass.
+ *
+ * For L = sum_t dy_t . y_t + <d_final_state, S_T> through la_chunk_forward
+ * (normalize = 0), with dS_t = dL/dS_t (every later use of S_t included):
+ *
+ *   dS_t = q_t dy_t^T + g_{t+1} dS_{t+1},   dS_T = q_T dy_T^T + d_final_state
+ *   dq_t = S_t dy_t        dk_t = dS_t v_t        dv_t = dS_t^T k_t
+ *   d_init_state = g_1 dS_1
+ *   d log g_t = g_t <dS_t, S_{t-1}>  =  sum_{s >= t} (q_s . dq_s - k_s . dk_s)
+ *               + <d_final_state, S_T>
+ *
+ * The gradients of the scan are scans again (BlinkDL/RWKV-LM discussion 189,
+ * fourth bullet: the gradient is computed with cumulative sums as well), and
+ * the library runs them on its forward and reverse scan kernels:
+ *   dq = forward scan of (q', k', v') = (dy, v, k) from S_0^T  (its state is S_t^T);
+ *   dk = reverse scan of (v, dy, q) from d_final_state^T        (state dS_t^T);
+ *   dv = reverse scan of (k, q, dy) from d_final_state          (state dS_t);
+ * the reverse scans take the decay one token later (g_{t+1}, and 1 for the
+ * last token).  The decay gradient is the suffix sum on the second line
+ * (the identity <dS_t,S_t> - g_t <dS_t,S_{t-1}> = k_t . dk_t, summed from
+ * the end).  Its bf16 error grows with the square root of the number of
+ * summed tokens: each q . dq and k . dk carries the rounding of the bf16 dq
+ * and dk it is formed from.
+ *
+ *   q, k, v, decay, init_state, B, H, T, Dk, Dv, dtype   as the forward call
+ *                  (init_state NULL: zeros).
+ *   dy             [B,H,T,Dv] `dtype`: dL/dy.  Required (for T > 0).
+ *   d_final_state  NULL (zeros) or [B,H,Dk,Dv] fp32: dL/dS_T.
+ *   dq, dk         [B,H,T,Dk] `dtype`; dv [B,H,T,Dv] `dtype`.  Required.
+ *   d_log_g        NULL (not computed) or fp32 with the shape of decay->log_g:
+ *                  [H] for a per-head decay (summed over b and t), [B,H,T]
+ *                  for a per-step decay.  Must be NULL without a decay.
+ *   d_init_state   NULL (not written) or [B,H,Dk,Dv] fp32: dL/dS_0.
+ *   workspace      device memory of at least
+ *                  la_chunk_backward_workspace_size(...) bytes, 16-byte
+ *                  aligned, used on `stream` only.  Required (for T > 0).
+ *
+ * Several launches on `stream`: three scans (each possibly a state pass and
+ * an output pass) and small kernels for the transposed carried states, the
+ * shifted decay, d_init_state and d_log_g.  Outputs must not overlap inputs
+ * or each other.
+ *
+ * Errors: as la_chunk_forward_ws, plus LA_ERR_INVALID_ARG for a NULL
+ * required pointer (dy, dq, dk, dv, workspace), a workspace smaller than
+ * la_chunk_backward_workspace_size or misaligned, or d_log_g given without a
+ * decay.  The normalised forward has no backward here (the function has no
+ * normalize argument).
+ */
+LA_API la_status la_chunk_backward_ws(const void* q, const void* k, const void* v,
+                               const la_decay* decay, const float* init_state,
+                               const void* dy, const float* d_final_state,
+                               void* dq, void* dk, void* dv, float* d_log_g, float* d_init_state,
+                               int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                               void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
  * device array inside this library (la_chunk_forward_noalloc_capacity()
  * bytes, 16 MiB, one per device, reserved when the library's device code is

@@ -13,7 +13,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "bidirectional", "workspace_size", "decode_step", "device_error", "LAError", "lib", "library_path",
+__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "workspace_size", "backward_workspace_size",
+           "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -23,6 +24,7 @@ DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
 LA_F32, LA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
                     "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
+                    "la_chunk_backward_ws", "la_chunk_backward_workspace_size",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -61,6 +63,11 @@ def lib():
         L.la_chunk_bidirectional_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp,
                                                 i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
         L.la_chunk_bidirectional_ws.restype = i
+        L.la_chunk_backward_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), vp, vp, vp, vp, vp, vp, vp, vp,
+                                           i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_chunk_backward_ws.restype = i
+        L.la_chunk_backward_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
         L.la_chunk_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_forward_workspace_size.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
@@ -217,6 +224,70 @@ def bidirectional(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False, o
             _ptr(out), B, H, T, Dk, Dv, code, _ptr(workspace), 0 if workspace is None else workspace.numel(),
             _stream(stream, dev)))
     return out
+
+
+def backward_workspace_size(B, H, T, Dk, Dv, dtype=torch.bfloat16, decay_kind=DECAY_NONE):
+    """Scratch bytes chunk_backward needs (la_chunk_backward_workspace_size)."""
+    return int(lib().la_chunk_backward_workspace_size(B, H, T, Dk, Dv, _dtype_code(dtype), int(decay_kind)))
+
+
+def chunk_backward(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=None, d_final_state=None,
+                   need_log_g=True, need_init_state=True, stream=None, workspace=None, out=None):
+    """Gradients of the unnormalised forward (la_chunk_backward_ws) for the
+    loss sum(dy * y) + sum(d_final_state * final_state).
+
+    q, k: [B,H,T,Dk]; v, dy: [B,H,T,Dv] (float32 or bfloat16, all one dtype);
+    decay_kind / log_g as chunk_forward; init_state [B,H,Dk,Dv] fp32 or None;
+    d_final_state [B,H,Dk,Dv] fp32 or None.  Returns (dq, dk, dv, d_log_g,
+    d_init_state): dq, dk, dv in the input dtype; d_log_g fp32 with log_g's
+    shape (None without a decay or need_log_g=False); d_init_state fp32 (None
+    with need_init_state=False).  workspace: None allocates it with torch on
+    the call's stream, or a CUDA uint8 tensor of at least
+    backward_workspace_size(...) bytes.  out: None, or a tuple (dq, dk, dv,
+    d_log_g, d_init_state) of preallocated outputs (entries may be None to
+    skip d_log_g / d_init_state).
+    """
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q.dtype)
+    _need(k, "k", (B, H, T, Dk), q.dtype, dev)
+    _need(v, "v", (B, H, T, Dv), q.dtype, dev)
+    _need(dy, "dy", (B, H, T, Dv), q.dtype, dev)
+    _need(q, "q", (B, H, T, Dk), q.dtype, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H, T), torch.float32, dev)
+    _need(init_state, "init_state", (B, H, Dk, Dv), torch.float32, dev)
+    _need(d_final_state, "d_final_state", (B, H, Dk, Dv), torch.float32, dev)
+    if out is None:
+        dq, dk = torch.empty_like(q), torch.empty_like(k)
+        dv = torch.empty_like(v)
+        d_log_g = torch.empty_like(log_g) if (decay_kind != DECAY_NONE and need_log_g) else None
+        d_init = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev) if need_init_state else None
+    else:
+        dq, dk, dv, d_log_g, d_init = out
+        _need(dq, "dq", (B, H, T, Dk), q.dtype, dev)
+        _need(dk, "dk", (B, H, T, Dk), q.dtype, dev)
+        _need(dv, "dv", (B, H, T, Dv), q.dtype, dev)
+        if d_log_g is not None:
+            _need(d_log_g, "d_log_g", tuple(log_g.shape), torch.float32, dev)
+        _need(d_init, "d_init_state", (B, H, Dk, Dv), torch.float32, dev)
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        nbytes = backward_workspace_size(B, H, T, Dk, Dv, q.dtype, decay_kind)
+        if workspace is None:
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+            if stream is not None:
+                workspace.record_stream(stream)
+        elif workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
+        _check(lib().la_chunk_backward_ws(
+            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, _ptr(init_state), _ptr(dy),
+            _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_log_g), _ptr(d_init),
+            B, H, T, Dk, Dv, code, _ptr(workspace), workspace.numel(), _stream(stream, dev)))
+    return dq, dk, dv, d_log_g, d_init
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,

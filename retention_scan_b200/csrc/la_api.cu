@@ -134,6 +134,38 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
     return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+// Scratch of the backward pass, in 256-byte aligned regions (every optional
+// region is reserved, so that the size depends on the sizes only):
+//   S_0^T, d_final_state^T, S_T^T   [B,H,Dv,Dk] fp32 each
+//   shifted log decay               [B,H,T] fp32 (with a decay)
+//   decay-gradient scratch          la::dlog_scratch_doubles doubles
+//   T-segment workspace of the scans (the larger of the two key/value widths' orders)
+struct BwdLayout {
+    size_t s0t, dsft, st, lsh, dlog, scan, scan_bytes, total;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind) {
+    const size_t BH = static_cast<size_t>(B) * H;
+    const size_t state = round256(sizeof(float) * BH * Dk * Dv);
+    BwdLayout L{};
+    L.s0t = 0;
+    L.dsft = L.s0t + state;
+    L.st = L.dsft + state;
+    L.lsh = L.st + state;
+    L.dlog = L.lsh + (kind != LA_DECAY_NONE ? round256(sizeof(float) * BH * T) : 0);
+    L.scan = L.dlog + round256(sizeof(double) * la::dlog_scratch_doubles(B, H, T));
+    L.scan_bytes = 0;
+    if (dtype == LA_BF16) {
+        const size_t a = la::fwd_tc_workspace_bytes(B, H, T, Dv, Dk, false);  // dq, dk scans
+        const size_t b = la::fwd_tc_workspace_bytes(B, H, T, Dk, Dv, false);  // dv scan
+        L.scan_bytes = round256(a > b ? a : b);
+    }
+    L.total = L.scan + L.scan_bytes;
+    return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -190,6 +222,111 @@ la_status la_chunk_bidirectional_ws(const void* q, const void* k, const void* v,
     if (st != LA_OK) return st;
     return scan(q, k, v, decay, normalize, nullptr, nullptr, out, nullptr, nullptr, B, H, T, Dk, Dv, dtype,
                 workspace, workspace_bytes, stream, 1, 1);
+}
+
+size_t la_chunk_backward_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int decay_kind) {
+    if ((dtype != LA_F32 && dtype != LA_BF16) || B < 1 || H < 1 || T < 1 || Dk < 1 || Dv < 1) return 0;
+    if (decay_kind < LA_DECAY_NONE || decay_kind > LA_DECAY_PER_STEP) return 0;
+    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
+    return bwd_layout(B, H, T, Dk, Dv, dtype, decay_kind).total;
+}
+
+// dq, dk, dv by three scans on the forward and reverse scan kernels (the
+// header explains the permutations), then d_init_state and d_log_g.
+la_status la_chunk_backward_ws(const void* q, const void* k, const void* v, const la_decay* decay,
+                               const float* init_state, const void* dy, const float* d_final_state, void* dq,
+                               void* dk, void* dv, float* d_log_g, float* d_init_state, int B, int H, int T, int Dk,
+                               int Dv, la_dtype dtype, void* workspace, size_t workspace_bytes,
+                               la_stream_t stream) {
+    if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    int kind;
+    const float* log_g;
+    if (check_decay(decay, &kind, &log_g) != LA_OK) return LA_ERR_INVALID_ARG;
+    if (d_log_g && (kind == LA_DECAY_NONE || !aligned4(d_log_g))) return LA_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH * 8) || BH > 65535) return BH > 65535 ? LA_ERR_UNSUPPORTED : LA_ERR_INVALID_ARG;
+    for (const void* p : {static_cast<const void*>(init_state), static_cast<const void*>(d_final_state),
+                          static_cast<const void*>(d_init_state)})
+        if (p && !aligned16(p)) return LA_ERR_INVALID_ARG;
+    const bool work = BH > 0 && T > 0;
+    if (work) {
+        for (const void* p : {q, k, v, dy, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                              static_cast<const void*>(dv), static_cast<const void*>(workspace)})
+            if (!p || !aligned16(p)) return LA_ERR_INVALID_ARG;
+    }
+    if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
+    if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
+    if (work && (T + 255) / 256 > 65535) return LA_ERR_UNSUPPORTED;
+    const BwdLayout L = work ? bwd_layout(B, H, T, Dk, Dv, dtype, kind) : BwdLayout{};
+    if (work && workspace_bytes < L.total) return LA_ERR_INVALID_ARG;
+    if (BH == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t sbytes = sizeof(float) * static_cast<size_t>(BH) * Dk * Dv;
+
+    if (T == 0) {  // S_T = S_0: the state gradient passes through; no decay was applied
+        cudaError_t e = cudaSuccess;
+        if (d_init_state)
+            e = d_final_state ? cudaMemcpyAsync(d_init_state, d_final_state, sbytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(d_init_state, 0, sbytes, s);
+        if (e == cudaSuccess && d_log_g && kind == LA_DECAY_PER_HEAD)
+            e = cudaMemsetAsync(d_log_g, 0, sizeof(float) * H, s);
+        return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    }
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* s0t = init_state ? reinterpret_cast<float*>(ws + L.s0t) : nullptr;
+    float* dsft = d_final_state ? reinterpret_cast<float*>(ws + L.dsft) : nullptr;
+    const bool need_st = d_log_g && d_final_state;  // <d_final_state, S_T> enters d_log_g
+    float* st = need_st ? reinterpret_cast<float*>(ws + L.st) : nullptr;
+    float* lsh = kind != LA_DECAY_NONE ? reinterpret_cast<float*>(ws + L.lsh) : nullptr;
+    void* scan_ws = L.scan_bytes ? ws + L.scan : nullptr;
+    const int bh = static_cast<int>(BH);
+    auto cuda_ok = [](cudaError_t e) { return e == cudaSuccess; };
+
+    if (s0t && !cuda_ok(la::launch_transpose(init_state, s0t, bh, Dk, Dv, s))) return LA_ERR_CUDA;
+    if (dsft && !cuda_ok(la::launch_transpose(d_final_state, dsft, bh, Dk, Dv, s))) return LA_ERR_CUDA;
+    if (lsh && !cuda_ok(la::launch_shift_decay(log_g, kind, lsh, B, H, T, s))) return LA_ERR_CUDA;
+    const la_decay shifted{LA_DECAY_PER_STEP, lsh};
+    const la_decay* rdecay = lsh ? &shifted : nullptr;
+
+    // dq = forward scan of (dy, v, k) from S_0^T; its final state is S_T^T
+    la_status r = scan(dy, v, k, decay, 0, s0t, nullptr, dq, st, nullptr, B, H, T, Dv, Dk, dtype, scan_ws,
+                       L.scan_bytes, stream, 0, 0);
+    if (r != LA_OK) return r;
+    // dk = reverse scan of (v, dy, q) from d_final_state^T, decay one token later
+    r = scan(v, dy, q, rdecay, 0, dsft, nullptr, dk, nullptr, nullptr, B, H, T, Dv, Dk, dtype, scan_ws,
+             L.scan_bytes, stream, 1, 0);
+    if (r != LA_OK) return r;
+    // dv = reverse scan of (k, q, dy) from d_final_state; its final state is dS_1
+    r = scan(k, q, dy, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype,
+             scan_ws, L.scan_bytes, stream, 1, 0);
+    if (r != LA_OK) return r;
+    if (d_init_state && kind != LA_DECAY_NONE &&
+        !cuda_ok(la::launch_scale_by_first_decay(d_init_state, log_g, kind, B, H, T, Dk * Dv, s)))
+        return LA_ERR_CUDA;
+    if (d_log_g) {
+        la::DlogArgs a{};
+        a.q = q;
+        a.k = k;
+        a.dq = dq;
+        a.dk = dk;
+        a.d_final_state = d_final_state;
+        a.final_state_t = st;
+        a.d_log_g = d_log_g;
+        a.kind = kind;
+        a.B = B;
+        a.H = H;
+        a.T = T;
+        a.Dk = Dk;
+        a.Dv = Dv;
+        a.dtype = dtype;
+        a.scratch = reinterpret_cast<double*>(ws + L.dlog);
+        a.stream = s;
+        if (!cuda_ok(la::launch_dlog(a))) return LA_ERR_CUDA;
+    }
+    return LA_OK;
 }
 
 la_status la_decode_step(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,

@@ -65,4 +65,34 @@ size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm);
 // Decode step (la_decode.cu).
 cudaError_t launch_decode(const DecodeArgs& a, la_dtype dtype);
 
+// Small kernels of the backward pass (la_bwd.cu).  All asynchronous on
+// `stream`; each returns the launch status.
+//   out[bh] = in[bh]^T for BH matrices of R x C fp32 values.
+cudaError_t launch_transpose(const float* in, float* out, int BH, int R, int C, cudaStream_t stream);
+//   out[b,h,t] = decay of token t + 1 (log, per step; 0 for the last token),
+//   from a per-head ([H]) or per-step ([B,H,T]) log decay.
+cudaError_t launch_shift_decay(const float* log_g, int kind, float* out, int B, int H, int T, cudaStream_t stream);
+//   s[b,h] *= g_1 (the decay of each sequence's first token), [B,H,n] fp32.
+cudaError_t launch_scale_by_first_decay(float* s, const float* log_g, int kind, int B, int H, int T, int n,
+                                        cudaStream_t stream);
+// Gradient of the log decay: d[b,h,t] = sum_{s >= t} (q_s . dq_s - k_s . dk_s)
+// + <dSf[b,h], S_T[b,h]> (S_T given transposed, [Dv, Dk]); per step it is
+// written to d_log_g [B,H,T], per head summed into d_log_g [H].
+struct DlogArgs {
+    const void* q;
+    const void* k;
+    const void* dq;
+    const void* dk;
+    const float* d_final_state;   // may be null
+    const float* final_state_t;   // S_T^T [B,H,Dv,Dk]; read when d_final_state is given
+    float* d_log_g;
+    int kind;                     // LA_DECAY_PER_HEAD or LA_DECAY_PER_STEP
+    int B, H, T, Dk, Dv;
+    la_dtype dtype;
+    double* scratch;              // dlog_scratch_doubles(B, H, T) doubles
+    cudaStream_t stream;
+};
+size_t dlog_scratch_doubles(int B, int H, int T);
+cudaError_t launch_dlog(const DlogArgs& a);
+
 }  // namespace la

@@ -207,3 +207,74 @@ print(r, r2)
     env = dict(os.environ, LA_FAULT_INJECT="launch")
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
     assert out.stdout.split() == ["3", "3"]
+
+
+def _bwd(L, **over):
+    """la_chunk_backward_ws with fake (never dereferenced) aligned addresses."""
+    vp = ctypes.c_void_p
+    a = dict(q=16, k=16, v=16, decay=None, init_state=None, dy=16, dSf=None, dq=16, dk=16, dv=16,
+             dlog=None, dS0=None, B=1, H=1, T=4, Dk=16, Dv=16, dtype=1, ws=256, ws_bytes=None)
+    a.update(over)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = L.la_chunk_backward_workspace_size(a["B"], a["H"], max(a["T"], 1), a["Dk"], a["Dv"],
+                                                           a["dtype"] if a["dtype"] in (0, 1) else 1,
+                                                           a["decay"].kind if a["decay"] is not None else 0)
+    dec = a["decay"]
+    return L.la_chunk_backward_ws(vp(a["q"]), vp(a["k"]), vp(a["v"]), ctypes.byref(dec) if dec is not None else None,
+                                  vp(a["init_state"]), vp(a["dy"]), vp(a["dSf"]), vp(a["dq"]), vp(a["dk"]),
+                                  vp(a["dv"]), vp(a["dlog"]), vp(a["dS0"]), a["B"], a["H"], a["T"], a["Dk"],
+                                  a["Dv"], a["dtype"], vp(a["ws"]), a["ws_bytes"], None)
+
+
+# None of these reach CUDA: the backward validates before it launches.
+@pytest.mark.parametrize("over,status", [
+    (dict(dy=None), 1),
+    (dict(dq=None), 1),
+    (dict(dv=8), 1),                          # not 16-byte aligned
+    (dict(ws=None), 1),                       # the backward needs its workspace
+    (dict(ws=264), 1),                        # misaligned workspace
+    (dict(ws_bytes=64), 1),                   # workspace too small
+    (dict(dlog=64), 1),                       # a decay gradient without a decay
+    (dict(decay=la._Decay(1, 64), dlog=2), 1),  # d_log_g misaligned
+    (dict(dS0=8), 1),
+    (dict(T=-1), 1),
+    (dict(dtype=5), 1),
+    (dict(Dk=48), 2),
+    (dict(dtype=0, Dv=130), 2),
+    (dict(B=0), 0),                           # empty batch: a no-op
+], ids=str)
+def test_backward_validation(L, over, status):
+    assert _bwd(L, **over) == status
+
+
+def test_backward_workspace_size(L):
+    # S_0^T, d_final_state^T, S_T^T, the shifted decay, the decay-gradient
+    # scratch and the scans' T-segment workspace, each rounded to 256 bytes
+    def r(x):
+        return (x + 255) // 256 * 256
+    B, H, T, D = 1, 8, 8192, 64
+    state = r(4 * B * H * D * D)
+    nblk = (T + 255) // 256
+    scan = L.la_chunk_forward_workspace_size(B, H, T, D, D, 1, 0)
+    want = 3 * state + r(4 * B * H * T) + r(8 * (B * H + 2 * B * H * nblk)) + r(scan)
+    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 2) == want
+    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 0) == want - r(4 * B * H * T)
+    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 0, 2) == want - r(scan)  # fp32: no segments
+    assert L.la_chunk_backward_workspace_size(0, H, T, D, D, 1, 0) == 0
+    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 3) == 0
+
+
+def test_injected_launch_failure_backward():
+    code = r'''
+import ctypes, sys
+sys.path.insert(0, %r)
+import retention_scan_b200 as la
+L = la.lib()
+vp = ctypes.c_void_p
+n = L.la_chunk_backward_workspace_size(1, 1, 4, 16, 16, 1, 0)
+print(L.la_chunk_backward_ws(vp(16), vp(16), vp(16), None, None, vp(16), None, vp(16), vp(16), vp(16),
+                             None, None, 1, 1, 4, 16, 16, 1, vp(256), n, None))
+''' % ROOT
+    env = dict(os.environ, LA_FAULT_INJECT="launch")
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
+    assert out.stdout.split() == ["3"]
