@@ -11,6 +11,9 @@ cpu_baseline / reference legs may import this package.  The CUDA library
   decode_step(...)       one token of the same recurrence, in place
   backward(...)          gradients of a loss through the forward recurrence,
                          by the chain rule token by token (la_ref.c)
+  wkv4(...)              the RWKV-4 WKV recurrence: the att_seq loop of
+                         BlinkDL/RWKV-LM issue 167, max-shifted (wkv4_ref.c)
+  wkv4_direct(...)       the same output from its definition, O(T^2), numpy
   parallel_forward(...)  brute-force O(T^2) parallel form, numpy (parallel.py)
   parallel_reverse(...)  brute-force O(T^2) anti-causal form, numpy (parallel.py)
 
@@ -27,6 +30,7 @@ from .parallel import parallel_forward, parallel_reverse  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "la_ref.c")
+_SRCS = (_SRC, os.path.join(_HERE, "wkv4_ref.c"))
 _LIB_PATH = os.path.join(_HERE, "liblaref.so")
 _libs = {}
 
@@ -34,12 +38,13 @@ DECAY_KINDS = {None: 0, "none": 0, "per_head": 1, "per_step": 2}
 
 
 def build(force=False):
-    """Compile la_ref.c into liblaref.so beside it (gcc -O2, pthreads)."""
+    """Compile la_ref.c and wkv4_ref.c into liblaref.so beside them (gcc -O2,
+    pthreads)."""
     if force or not os.path.exists(_LIB_PATH) or \
-            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+            os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(p) for p in _SRCS):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread",
-                        "-o", tmp, _SRC, "-lm"], check=True)
+                        "-o", tmp, *_SRCS, "-lm"], check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -59,6 +64,9 @@ def load_library(path=None):
         lib.la_ref_backward.argtypes = [d, d, d, i, d, i, d, d, d, d, d, d, d, d, d, d, d,
                                         i, i, i, i, i, i]
         lib.la_ref_backward.restype = i
+        if hasattr(lib, "la_ref_wkv4"):
+            lib.la_ref_wkv4.argtypes = [d, d, d, d, d, d, d, i, i, i]
+            lib.la_ref_wkv4.restype = i
         _libs[path] = lib
     return _libs[path]
 
@@ -138,6 +146,50 @@ def backward(q, k, v, dy, decay_kind=0, log_g=None, normalize=False, init_state=
     elif kind == 2:
         dlog_g = dlog
     return dq, dk, dv, dlog_g, dS0, (dz0 if normalize else None)
+
+
+WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)
+
+
+def wkv4(k, v, w, u, init_state=None, lib=None):
+    """RWKV-4 WKV recurrence, float64 (wkv4_ref.c: the att_seq loop of
+    BlinkDL/RWKV-LM issue 167).  k, v [B,T,C]; w (log decay, <= 0), u (bonus)
+    [C]; init_state [B,3,C] (planes aa, bb, pp) or None for an empty state.
+    Returns (out [B,T,C], final_state [B,3,C])."""
+    k, v, w, u, init_state = _f64(k), _f64(v), _f64(w), _f64(u), _f64(init_state)
+    B, T, C = k.shape
+    out = np.zeros((B, T, C))
+    fin = np.zeros((B, 3, C))
+    rc = (lib or load_library()).la_ref_wkv4(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(init_state), _ptr(out),
+                                             _ptr(fin), B, T, C)
+    if rc != 0:
+        raise ValueError("la_ref_wkv4 rejected its arguments")
+    return out, fin
+
+
+def wkv4_direct(k, v, w, u, init_state=None):
+    """The RWKV-4 WKV output written out as its definition, float64 numpy,
+    O(T^2 C): wkv_t = (e^{t w + pp0} aa0 + sum_{i<t} e^{(t-1-i) w + k_i} v_i
+    + e^{u + k_t} v_t) / (e^{t w + pp0} bb0 + sum_{i<t} e^{(t-1-i) w + k_i}
+    + e^{u + k_t}) with 0-based t (BlinkDL/RWKV-LM issue 167's formula 14 as
+    the loop computes it).  Forms the exponentials directly: callers keep the
+    exponents moderate (or shift k, which the ratio ignores)."""
+    k, v, w, u = _f64(k), _f64(v), _f64(w), _f64(u)
+    B, T, C = k.shape
+    out = np.zeros((B, T, C))
+    for t in range(T):
+        lag = (t - 1 - np.arange(t))[None, :, None] * w[None, None, :]   # [1, t, C]
+        wt = np.exp(lag + k[:, :t])                                      # [B, t, C]
+        cur = np.exp(u[None, :] + k[:, t])                               # [B, C]
+        num = (wt * v[:, :t]).sum(axis=1) + cur * v[:, t]
+        den = wt.sum(axis=1) + cur
+        if init_state is not None:
+            s = _f64(init_state)
+            g = np.exp(t * w[None, :] + s[:, 2])
+            num = num + g * s[:, 0]
+            den = den + g * s[:, 1]
+        out[:, t] = num / den
+    return out
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=0, log_g=None, normalize=False, lib=None):

@@ -477,3 +477,96 @@ def backward_parallel_form(bwd, fwd):
             elif kind == 2:
                 _close(dlg, dA_all, 1e-9, "parallel dlog g " + tag)
 
+
+
+# -- RWKV-4 WKV (BlinkDL/RWKV-LM issue 167, the att_seq loop) ----------------
+#
+#   wkv4_direct_form   the loop against its definition written out (O(T^2),
+#                      numpy exponentials), with and without a carried state
+#   wkv4_t1_t2         T = 1: out = v; T = 2 expanded by hand
+#   wkv4_invariants    constant v gives constant out; adding s to every key
+#                      leaves out and (aa, bb) unchanged and moves pp by s
+#   wkv4_split_carry   run(T) == run(T1) -> carry (aa, bb, pp) -> run(T - T1)
+#   wkv4_large_keys    keys near 300 (e^300 overflows fp32) and near -800
+#                      (e^-800 underflows f64): the loop stays finite and
+#                      exact, equal to the definition on the keys shifted
+#                      back (the ratio ignores the shift)
+#   wkv4_no_bonus      u = -1e30: out_t (t >= 1) is the decayed average of the
+#                      earlier values only
+
+def _wkv4_inputs(rng, B, T, C, init=False, kshift=0.0):
+    k = rng.standard_normal((B, T, C)) + kshift
+    v = rng.standard_normal((B, T, C))
+    w = -np.exp(rng.standard_normal(C) - 0.5)
+    u = rng.standard_normal(C) - 0.5
+    S0 = None
+    if init:
+        S0 = np.stack([rng.standard_normal((B, C)), np.abs(rng.standard_normal((B, C))) + 0.1,
+                       rng.standard_normal((B, C)) + kshift], axis=1)
+    return k, v, w, u, S0
+
+
+def wkv4_direct_form(wkv, direct):
+    rng = np.random.default_rng(51)
+    for init in (False, True):
+        for T in (1, 2, 3, 17, 40):
+            k, v, w, u, S0 = _wkv4_inputs(rng, 2, T, 5, init)
+            out, _ = wkv(k, v, w, u, S0)
+            _close(out, direct(k, v, w, u, S0), 1e-12, f"direct form T={T} init={init}")
+
+
+def wkv4_t1_t2(wkv, direct):
+    rng = np.random.default_rng(52)
+    k, v, w, u, _ = _wkv4_inputs(rng, 1, 2, 3)
+    out, fin = wkv(k[:, :1], v[:, :1], w, u)
+    _close(out, v[:, :1], 1e-15, "T=1 out = v")
+    _close(fin[:, 0] * np.exp(fin[:, 2]), np.exp(k[:, 0]) * v[:, 0], 1e-12, "T=1 state numerator")
+    _close(fin[:, 1] * np.exp(fin[:, 2]), np.exp(k[:, 0]), 1e-12, "T=1 state denominator")
+    out, _ = wkv(k, v, w, u)
+    a, b = np.exp(k[0, 0]), np.exp(u + k[0, 1])
+    _close(out[0, 1], (a * v[0, 0] + b * v[0, 1]) / (a + b), 1e-12, "T=2 by hand")
+
+
+def wkv4_invariants(wkv, direct):
+    rng = np.random.default_rng(53)
+    k, v, w, u, _ = _wkv4_inputs(rng, 2, 30, 4)
+    out, _ = wkv(k, np.full_like(v, 1.75), w, u)
+    _close(out, np.full_like(v, 1.75), 1e-13, "constant v")
+    o1, f1 = wkv(k, v, w, u)
+    o2, f2 = wkv(k + 3.25, v, w, u)
+    _close(o2, o1, 1e-12, "key shift: out")
+    _close(f2[:, :2], f1[:, :2], 1e-12, "key shift: aa, bb")
+    _close(f2[:, 2], f1[:, 2] + 3.25, 1e-12, "key shift: pp")
+
+
+def wkv4_split_carry(wkv, direct):
+    rng = np.random.default_rng(54)
+    k, v, w, u, S0 = _wkv4_inputs(rng, 2, 33, 6, init=True)
+    full, ffin = wkv(k, v, w, u, S0)
+    for T1 in (1, 10, 32):
+        a, fa = wkv(k[:, :T1], v[:, :T1], w, u, S0)
+        b, fb = wkv(k[:, T1:], v[:, T1:], w, u, fa)
+        _close(np.concatenate([a, b], axis=1), full, 1e-12, f"split at {T1}: out")
+        _close(fb, ffin, 1e-12, f"split at {T1}: state")
+
+
+def wkv4_large_keys(wkv, direct):
+    rng = np.random.default_rng(55)
+    for shift in (300.0, -800.0):
+        k, v, w, u, _ = _wkv4_inputs(rng, 2, 25, 4, kshift=shift)
+        out, fin = wkv(k, v, w, u)
+        assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin)), f"keys near {shift}: non-finite values"
+        _close(out, direct(k - shift, v, w, u), 1e-12, f"keys near {shift}")
+
+
+def wkv4_no_bonus(wkv, direct):
+    rng = np.random.default_rng(56)
+    k, v, w, u, _ = _wkv4_inputs(rng, 1, 12, 3)
+    u = np.full_like(u, -1e30)
+    out, _ = wkv(k, v, w, u)
+    for t in range(1, 12):
+        wt = np.exp((t - 1 - np.arange(t))[:, None] * w[None, :] + k[0, :t])
+        _close(out[0, t], (wt * v[0, :t]).sum(0) / wt.sum(0), 1e-12, f"no bonus t={t}")
+
+
+WKV4 = [wkv4_direct_form, wkv4_t1_t2, wkv4_invariants, wkv4_split_carry, wkv4_large_keys, wkv4_no_bonus]

@@ -82,6 +82,58 @@ def _run_all_pins(lib):
     return failed
 
 
+WKV4_SRC = os.path.join(os.path.dirname(oracle.__file__), "wkv4_ref.c")
+
+# (name, text in wkv4_ref.c, replacement)
+WKV4_MUTANTS = [
+    ("bonus left out of the read-out", "shifted_pair(pp, u[c] + kt, &fs, &fx);", "shifted_pair(pp, kt, &fs, &fx);"),
+    ("state not decayed", "shifted_pair(w[c] + pp, kt, &fs, &fx);", "shifted_pair(pp, kt, &fs, &fx);"),
+    ("bonus used in the update", "shifted_pair(w[c] + pp, kt, &fs, &fx);",
+     "shifted_pair(w[c] + pp, u[c] + kt, &fs, &fx);"),
+    ("denominator without the state", "out[i] = (fs * aa + fx * vt) / (fs * bb + fx);",
+     "out[i] = (fs * aa + fx * vt) / (fs + fx);"),
+    ("scale not carried", "        pp = m;\n", "        pp = 0.0 * m;\n"),
+    ("empty state at scale 0", "init_state[s + 2 * C] : WKV4_EMPTY_SCALE;", "init_state[s + 2 * C] : 0.0;"),
+    ("shift by the smaller log weight", "const double m = la > lb ? la : lb;", "const double m = la < lb ? la : lb;"),
+    ("decay applied twice", "aa = fs * aa + fx * vt;", "aa = fs * fs * aa + fx * vt;"),
+]
+
+
+def _run_wkv4_pins(lib):
+    wkv = lambda *a: oracle.wkv4(*a, lib=lib)  # noqa: E731
+    failed = []
+    for check in pins.WKV4:
+        try:
+            check(wkv, oracle.wkv4_direct)
+        except AssertionError:
+            failed.append(check.__name__)
+    return failed
+
+
+def _build_copy(tmp_path, wkv4_text=None):
+    paths = []
+    for src in (SRC, WKV4_SRC):
+        p = tmp_path / os.path.basename(src)
+        p.write_text(wkv4_text if (src == WKV4_SRC and wkv4_text is not None) else open(src).read())
+        paths.append(str(p))
+    so = tmp_path / "liblaref_copy.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread", "-o", str(so), *paths, "-lm"],
+                   check=True)
+    return oracle.load_library(str(so))
+
+
+@pytest.mark.parametrize("name,old,new", WKV4_MUTANTS, ids=[m[0] for m in WKV4_MUTANTS])
+def test_wkv4_mutant_is_caught(tmp_path, name, old, new):
+    src = open(WKV4_SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique: {name}"
+    failed = _run_wkv4_pins(_build_copy(tmp_path, src.replace(old, new)))
+    assert failed, f"no pin catches the mutant '{name}'"
+
+
+def test_wkv4_unmutated_copy_passes(tmp_path):
+    assert _run_wkv4_pins(_build_copy(tmp_path)) == []
+
+
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_mutant_is_caught(tmp_path, name, old, new):
     src = open(SRC).read()

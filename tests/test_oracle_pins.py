@@ -115,3 +115,32 @@ def test_backward_empty_sequence(oracle_lib):
     dq, dk, dv, dlg, dS0, _ = oracle.backward(q, q, v, v, 2, np.zeros((1, 2, 0)), False, None, None, dST)
     assert dq.shape == (1, 2, 0, 3) and dv.shape == (1, 2, 0, 4) and dlg.shape == (1, 2, 0)
     assert np.array_equal(dS0, dST)
+
+
+@pytest.mark.parametrize("check", pins.WKV4, ids=lambda f: f.__name__)
+def test_wkv4_oracle(oracle_lib, check):
+    check(oracle.wkv4, oracle.wkv4_direct)
+
+
+def test_wkv4_direct_form_by_brute_force():
+    """The numpy definition itself, against a scalar loop over (t, i)."""
+    import math
+    rng = np.random.default_rng(57)
+    B, T, C = 1, 6, 2
+    k, v = rng.standard_normal((B, T, C)), rng.standard_normal((B, T, C))
+    w, u = -np.exp(rng.standard_normal(C)), rng.standard_normal(C)
+    d = oracle.wkv4_direct(k, v, w, u)
+    for c in range(C):
+        for t in range(T):
+            num = math.exp(u[c] + k[0, t, c]) * v[0, t, c]
+            den = math.exp(u[c] + k[0, t, c])
+            for i in range(t):
+                e = math.exp((t - 1 - i) * w[c] + k[0, i, c])
+                num += e * v[0, i, c]
+                den += e
+            assert abs(d[0, t, c] - num / den) <= 1e-13 * max(1.0, abs(num / den))
+
+
+def test_wkv4_rejects_bad_arguments(oracle_lib):
+    lib = oracle.load_library()
+    assert lib.la_ref_wkv4(None, None, None, None, None, None, None, 1, 1, 1) == -1
