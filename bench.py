@@ -11,6 +11,8 @@ One step is one pass of the hot path over one batch of the workload:
   config 3: normalised, elu+1 feature map, carried state, B=8, H=16, T=4096, D=128
   config 4: gated per-step decay, B=1, H=32, T=65536, D=128
   config 5: decode, B=256, H=32, D=128, normalised, 1024 la_decode_step calls
+  config 6: the RWKV-4 WKV recurrence, B=8, T=4096, C=2048, bf16 -> one
+      la_wkv4_forward call (tokens = B*T; a different recurrence)
 
 --direction reverse times the anti-causal scan (la_chunk_reverse_ws) on the
 same inputs; --direction bidirectional the encoder form (forward scan, then
@@ -533,10 +535,136 @@ def run_ours(args, rank, world, dist_on, device):
     return line
 
 
+# ---------------------------------------------------------------- RWKV-4 WKV (config 6)
+
+WKV4_METRIC = "rwkv4-wkv forward tokens/s (B·T/s) and % of roofline (HBM GB/s)"
+
+
+def wkv4_bytes(wl):
+    """Bytes one la_wkv4_forward call must move: k, v read and out written
+    once, w and u read, the fp32 final state written."""
+    es = 2 if wl.dtype == "bf16" else 4
+    return wl.B * wl.T * wl.C * 3 * es + 2 * wl.C * 4 + wl.B * 3 * wl.C * 4
+
+
+class Wkv4Job:
+    def __init__(self, device, wl, rank=0):
+        import retention_scan_b200 as la
+        self.la, self.wl, self.dev = la, wl, device
+        self.host = W.wkv4_inputs(wl.with_sizes(seed=wl.seed + 7919 * rank))
+        self.k, self.v, self.w, self.u = (self.host[n].to(device) for n in ("k", "v", "w", "u"))
+        self.out = torch.empty(wl.B, wl.T, wl.C, dtype=wl.torch_dtype, device=device)
+        self.fin = torch.empty(wl.B, 3, wl.C, dtype=torch.float32, device=device)
+
+    def step(self):
+        self.la.wkv4_forward(self.k, self.v, self.w, self.u, out=self.out, final_state=self.fin)
+        return 1
+
+    def e2e(self, steps, dist_on):
+        p = {n: self.host[n].pin_memory() for n in ("k", "v", "w", "u")}
+        y = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        stream = torch.cuda.current_stream(self.dev)
+
+        def one():
+            k, v, w, u = (p[n].to(self.dev, non_blocking=True) for n in ("k", "v", "w", "u"))
+            o, _ = self.la.wkv4_forward(k, v, w, u, out=self.out, final_state=self.fin)
+            y.copy_(o, non_blocking=True)
+        for _ in range(2):
+            one()
+        barrier(dist_on)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            one()
+        ev1.record(stream)
+        barrier(dist_on)
+        h2d = sum(p[n].numel() * p[n].element_size() for n in p)
+        return ev0.elapsed_time(ev1) / steps, h2d, y.numel() * y.element_size()
+
+
+def cpu_baseline_wkv4(wl, budget_s=15.0):
+    """The float64 oracle (single-threaded C loop) on whole batch rows of the
+    workload until about budget_s of work."""
+    import oracle
+    oracle.build()
+    per_row_s = wl.T * wl.C * 40 / 1e9  # rough: ~40 f64 operations per channel step
+    nb = max(1, min(wl.B, int(budget_s / max(per_row_s, 1e-9))))
+    inp = W.wkv4_inputs(wl, batches=range(nb))
+    t0 = time.perf_counter()
+    oracle.wkv4(inp["k"], inp["v"], inp["w"], inp["u"])
+    dt = time.perf_counter() - t0
+    return {"value": nb * wl.T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{nb} of {wl.B} batch rows, all {wl.T} tokens x {wl.C} channels, single thread"}
+
+
+def run_wkv4(args, rank, world, dist_on, device):
+    wl = W.WKV4
+    if args.tokens:
+        wl = wl.with_sizes(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
+    if args.batch:
+        wl = wl.with_sizes(B=args.batch, name=f"{wl.name}_B{args.batch}")
+    job = Wkv4Job(device, wl, rank)
+    nbytes = wkv4_bytes(wl)
+    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device) if nbytes < 2 * L2_BYTES else None
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.add_(1)
+        job.step()
+    torch.cuda.synchronize()
+    assert job.la.device_error(device) == 0
+    sampler = ClockSampler(bus_id_of(device)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    per, launches, w0, w1 = time_steps(job, args.steps, flush, dist_on, device)
+    if sampler:
+        time.sleep(0.3)
+        sampler.stop()
+    assert job.la.device_error(device) == 0
+    ms = max_over_ranks(sum(per), dist_on, device) / args.steps
+    pk, pk_kind = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    e2e = None
+    if not args.skip_e2e:
+        e_ms, h2d, d2h = job.e2e(max(1, min(args.steps, 20)), dist_on)
+        e_ms = max_over_ranks(e_ms, dist_on, device)
+        e2e = {"value": wl.B * wl.T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
+    return {
+        "metric": WKV4_METRIC, "value": wl.B * wl.T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+                   "l2": "flushed before every step (512 MB write)" if flush is not None
+                   else "inputs larger than L2",
+                   "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels)"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
+                     "peak_source": pk_kind, "kernel": "la_wkv4 (wkv4_kernel)",
+                     "algorithmic_bytes_per_launch": nbytes},
+        "e2e": e2e, "clocks": sampler.summary(w0, w1) if sampler else None, "gpu_launches": launches,
+    }
+
+
 # ---------------------------------------------------------------- reference arm (the oracle)
 
 def run_reference(args):
     cfg = args.config
+    if cfg == 6:
+        wl = W.WKV4
+        for _ in range(args.warmup):
+            cpu_baseline_wkv4(wl, budget_s=2.0)
+        vals = [cpu_baseline_wkv4(wl, budget_s=8.0) for _ in range(args.steps)]
+        v = statistics.median(x["value"] for x in vals)
+        cb = dict(vals[-1])
+        cb["value"] = v
+        return {"impl": "reference", "metric": WKV4_METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.B * wl.T / v * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C},
+                "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                "gpu_launches": 0}
     wl = W.WORKLOADS[cfg]
     for _ in range(args.warmup):
         cpu_baseline(cfg, budget_s=2.0, direction=args.direction)
@@ -565,7 +693,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -573,11 +701,11 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
     ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional", "backward"])
     args = ap.parse_args()
-    if args.config == 5 and args.direction != "forward":
+    if args.config in (5, 6) and args.direction != "forward":
         ap.error("--direction applies to the whole-sequence configs 1-4")
-    if args.direction == "backward" and W.WORKLOADS[args.config].normalize:
+    if args.direction == "backward" and args.config != 6 and W.WORKLOADS[args.config].normalize:
         ap.error("--direction backward: the library's backward covers the unnormalised forward (configs 1, 2, 4)")
-    default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3}
+    default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
     if args.warmup is None:
@@ -601,10 +729,11 @@ def main():
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
     try:
-        line = run_ours(args, rank, world, dist_on, device)
+        line = (run_wkv4 if args.config == 6 else run_ours)(args, rank, world, dist_on, device)
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(args.config, direction=args.direction)
+                line["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4) if args.config == 6 else
+                                        cpu_baseline(args.config, direction=args.direction))
             print(json.dumps(line), flush=True)
     finally:
         if dist_on:

@@ -297,6 +297,51 @@ LA_API la_status la_chunk_backward_ws(const void* q, const void* k, const void* 
                                void* workspace, size_t workspace_bytes, la_stream_t stream);
 
 /*
+ * la_wkv4_forward - the RWKV-4 WKV recurrence (a different recurrence from
+ * the one above: per channel, exponential key weights, a bonus for the
+ * current token, no query).
+ *
+ * Source: BlinkDL/RWKV-LM issue 167, "Questions about formula 14 and code
+ * implementation in the paper", the att_seq time loop in the opening
+ * comment.  Per batch b and channel c, with time decay w[c] (natural log of
+ * the per-step factor) and bonus u[c]:
+ *
+ *   wkv_t = ( sum_{i<t} e^{(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{(t-1-i) w + k_i}     + e^{u + k_t}     )
+ *
+ * (tokens counted from 0, plus the carried state's share).  The state is
+ * the loop's (aa, bb, pp): the two sums are e^pp aa and e^pp bb, pp a running
+ * log scale, so that only differences <= 0 are exponentiated and no large
+ * key overflows.  Per token the loop first reads out (the state against the
+ * current token at log weight u + k_t), then updates (the state decayed to
+ * w + pp against the token at k_t, the larger log weight the new pp).
+ * Computed in fp32 whatever the input type.
+ *
+ *   k, v, out      [B, T, C], `dtype` (LA_F32 or LA_BF16).  Required (T > 0).
+ *   w, u           [C] fp32, finite.  Required.
+ *   init_state     NULL (the empty state: aa = bb = 0, pp = -1e38) or
+ *                  [B, 3, C] fp32, the planes aa, bb, pp.
+ *   final_state    NULL (not written) or [B, 3, C] fp32; may be the same
+ *                  buffer as init_state (each channel reads its state before
+ *                  it writes it).
+ *   B, T, C        batch, tokens, channels: B, T >= 0, C >= 1; B == 0 is a
+ *                  no-op, T == 0 copies init_state (or the empty state) to
+ *                  final_state.
+ *
+ * Layout note: channels are the fastest index, as in the page's
+ * [T, C]-shaped k[t] and v[t] rows; each channel is an independent scan.
+ *
+ * Errors (synchronous, nothing enqueued): LA_ERR_INVALID_ARG for a NULL
+ * required pointer, negative sizes, C < 1, k, v or out not 16-byte aligned,
+ * w, u or a state not 4-byte aligned, a bad dtype; LA_ERR_UNSUPPORTED for C
+ * not a multiple of 8 (bf16) or 4 (fp32) (the rows are moved as TMA tiles),
+ * or B > 65535; LA_ERR_CUDA if a launch fails.
+ */
+LA_API la_status la_wkv4_forward(const void* k, const void* v, const float* w, const float* u,
+                                 const float* init_state, void* out, float* final_state,
+                                 int B, int T, int C, la_dtype dtype, la_stream_t stream);
+
+/*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
  * device array inside this library (la_chunk_forward_noalloc_capacity()
  * bytes, 16 MiB, one per device, reserved when the library's device code is

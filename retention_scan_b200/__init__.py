@@ -13,7 +13,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "workspace_size", "backward_workspace_size",
+__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "wkv4_forward", "workspace_size",
+           "backward_workspace_size",
            "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
 
@@ -24,7 +25,7 @@ DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
 LA_F32, LA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
                     "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
-                    "la_chunk_backward_ws", "la_chunk_backward_workspace_size",
+                    "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -68,6 +69,8 @@ def lib():
         L.la_chunk_backward_ws.restype = i
         L.la_chunk_backward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
+        L.la_wkv4_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
+        L.la_wkv4_forward.restype = i
         L.la_chunk_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_forward_workspace_size.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
@@ -288,6 +291,35 @@ def chunk_backward(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=No
             _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_log_g), _ptr(d_init),
             B, H, T, Dk, Dv, code, _ptr(workspace), workspace.numel(), _stream(stream, dev)))
     return dq, dk, dv, d_log_g, d_init
+
+
+WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)
+
+
+def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return_final=True, stream=None):
+    """RWKV-4 WKV recurrence (la_wkv4_forward).  k, v: [B,T,C] float32 or
+    bfloat16 CUDA tensors (C a multiple of 8 for bf16, 4 for fp32); w (log
+    of the per-step decay) and u (bonus): [C] fp32; init_state: [B,3,C] fp32
+    (planes aa, bb, pp) or None for the empty state.  Returns (out [B,T,C],
+    final_state [B,3,C] or None).  final_state may be init_state itself."""
+    B, T, C = k.shape
+    dev = k.device
+    code = _dtype_code(k.dtype)
+    _need(v, "v", (B, T, C), k.dtype, dev)
+    _need(k, "k", (B, T, C), k.dtype, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(u, "u", (C,), torch.float32, dev)
+    _need(init_state, "init_state", (B, 3, C), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    _need(out, "out", (B, T, C), k.dtype, dev)
+    if final_state is None and return_final:
+        final_state = torch.empty((B, 3, C), dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (B, 3, C), torch.float32, dev)
+    with torch.cuda.device(dev):
+        _check(lib().la_wkv4_forward(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(init_state), _ptr(out),
+                                     _ptr(final_state), B, T, C, code, _stream(stream, dev)))
+    return out, final_state
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,

@@ -26,12 +26,6 @@ LA_WS_DECL(128)
 #undef LA_WS_DECL
 }  // namespace ws
 
-namespace {
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 EncodeTiledFn encode_tiled() {
     static std::atomic<EncodeTiledFn> fn{nullptr};
     EncodeTiledFn f = fn.load();
@@ -46,6 +40,8 @@ EncodeTiledFn encode_tiled() {
     }
     return f;
 }
+
+namespace {
 
 bool width_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 

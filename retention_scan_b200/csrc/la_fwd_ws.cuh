@@ -240,10 +240,6 @@ struct Ctx {
     int seg, c0, n;  // segment, its first chunk and its number of chunks
 };
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ void fail(const Params& p, volatile int* abort, int code) {
     *abort = 1;
     if (p.err) atomicCAS(p.err, 0, code);

@@ -1,11 +1,19 @@
 // la_internal.h - launcher interface between the C ABI (la_api.cu) and the
 // kernel files.  Not installed; the public interface is include/la.h.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "la.h"
 
 namespace la {
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (so that
+// libcuda is not linked); null if the driver does not provide it.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
 
 // Device error codes written by kernels that give up waiting on a barrier.
 enum DeviceError : int {
@@ -94,5 +102,21 @@ struct DlogArgs {
 };
 size_t dlog_scratch_doubles(int B, int H, int T);
 cudaError_t launch_dlog(const DlogArgs& a);
+
+// RWKV-4 WKV recurrence (la_wkv4.cu).
+struct Wkv4Args {
+    const void* k;
+    const void* v;
+    const float* w;
+    const float* u;
+    const float* init_state;  // [B,3,C] or null (empty state)
+    void* out;
+    float* final_state;       // [B,3,C] or null
+    int B, T, C;
+    la_dtype dtype;
+    int* err_word;
+    cudaStream_t stream;
+};
+cudaError_t launch_wkv4(const Wkv4Args& a);
 
 }  // namespace la

@@ -22,7 +22,7 @@ def L():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "la.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(la_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(la_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_entry_points():
@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
 def test_library_exports_every_declared_symbol(L):
     out = subprocess.run(["nm", "-D", "--defined-only", la.library_path], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (la_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (la_[a-z0-9_]+)\b", out))
     missing = [n for n in declared_functions() if n not in exported]
     assert not missing, f"declared in la.h but not exported: {missing}"
     assert set(la.EXPORTED_SYMBOLS) <= exported
@@ -278,3 +278,31 @@ print(L.la_chunk_backward_ws(vp(16), vp(16), vp(16), None, None, vp(16), None, v
     env = dict(os.environ, LA_FAULT_INJECT="launch")
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
     assert out.stdout.split() == ["3"]
+
+
+def _wkv(L, **over):
+    vp = ctypes.c_void_p
+    a = dict(k=16, v=16, w=4, u=4, S0=None, out=16, Sf=None, B=1, T=4, C=8, dtype=1)
+    a.update(over)
+    return L.la_wkv4_forward(vp(a["k"]), vp(a["v"]), vp(a["w"]), vp(a["u"]), vp(a["S0"]), vp(a["out"]),
+                             vp(a["Sf"]), a["B"], a["T"], a["C"], a["dtype"], None)
+
+
+# None of these reach CUDA.
+@pytest.mark.parametrize("over,status", [
+    (dict(k=None), 1),
+    (dict(out=None), 1),
+    (dict(w=None), 1),
+    (dict(u=2), 1),                      # not 4-byte aligned
+    (dict(v=8), 1),                      # not 16-byte aligned
+    (dict(S0=6), 1),
+    (dict(B=-1), 1),
+    (dict(C=0), 1),
+    (dict(dtype=3), 1),
+    (dict(C=12), 2),                     # bf16 rows: C a multiple of 8
+    (dict(C=6, dtype=0), 2),             # fp32 rows: C a multiple of 4
+    (dict(B=70000), 2),
+    (dict(B=0), 0),
+], ids=str)
+def test_wkv4_validation(L, over, status):
+    assert _wkv(L, **over) == status

@@ -26,6 +26,11 @@ run the same recipe at smaller sizes):
   decode     one token per call, per-head gamma_h, normalised with elu(x)+1 on
              q and k, fp32 state ~ N(0, 0.01^2), key sum |N(0, 0.01^2)|
              (B=256, H=32, Dk=Dv=128, 1024 steps, seed 5)
+  wkv4       the RWKV-4 WKV recurrence: k, v ~ N(0,1) bf16 [B,T,C]; per
+             channel w = -exp(d), d ~ N(-1, 1.5^2) (decay factors from about
+             0.99 to near 0) and bonus u ~ N(-0.6, 0.4^2), fp32; empty start
+             (B=8, T=4096, C=2048, seed 6).  The page gives no sizes or
+             values: these are a mid-sized RWKV-4 layer's shapes.
 """
 import math
 from dataclasses import dataclass, field, replace
@@ -204,3 +209,39 @@ def decode_pool_device(wl, steps, device, seed_offset=0):
     q = _prep_qk(q, wl, Q).to(wl.torch_dtype)
     k = _prep_qk(k, wl, K).to(wl.torch_dtype)
     return q, k, v.to(wl.torch_dtype)
+
+
+# ---------------------------------------------------------------- RWKV-4 WKV
+
+@dataclass(frozen=True)
+class Wkv4Workload:
+    name: str
+    B: int
+    T: int
+    C: int
+    dtype: str   # "bf16" or "f32": k, v, out
+    seed: int
+
+    def with_sizes(self, **kw):
+        return replace(self, **kw)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+WKV4 = Wkv4Workload("wkv4_b8t4096c2048_bf16", B=8, T=4096, C=2048, dtype="bf16", seed=6)
+
+
+def wkv4_inputs(wl, batches=None):
+    """k, v [b, T, C] for the listed batch rows (all by default), each row
+    from its own generators; w, u [C] fp32 from the workload seed."""
+    rows = list(range(wl.B)) if batches is None else list(batches)
+    k = torch.stack([_normal((wl.T, wl.C), wl.seed, Q, b) for b in rows]) if rows else \
+        torch.zeros(0, wl.T, wl.C)
+    v = torch.stack([_normal((wl.T, wl.C), wl.seed, V, b) for b in rows]) if rows else \
+        torch.zeros(0, wl.T, wl.C)
+    d = _normal((wl.C,), wl.seed, A, 0, mean=-1.0, std=1.5)
+    w = -torch.exp(d)
+    u = _normal((wl.C,), wl.seed, S0, 0, mean=-0.6, std=0.4)
+    return dict(k=k.to(wl.torch_dtype), v=v.to(wl.torch_dtype), w=w.float(), u=u.float())
