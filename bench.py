@@ -555,10 +555,13 @@ class Wkv4Job:
         self.k, self.v, self.w, self.u = (self.host[n].to(device) for n in ("k", "v", "w", "u"))
         self.out = torch.empty(wl.B, wl.T, wl.C, dtype=wl.torch_dtype, device=device)
         self.fin = torch.empty(wl.B, 3, wl.C, dtype=torch.float32, device=device)
+        nb = la.wkv4_workspace_size(wl.B, wl.T, wl.C, wl.torch_dtype)
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=device) if nb else False
+        self.launches = 2 if nb else 1  # a state pass before the output pass when segmented
 
     def step(self):
-        self.la.wkv4_forward(self.k, self.v, self.w, self.u, out=self.out, final_state=self.fin)
-        return 1
+        self.la.wkv4_forward(self.k, self.v, self.w, self.u, out=self.out, final_state=self.fin, workspace=self.ws)
+        return self.launches
 
     def e2e(self, steps, dist_on):
         p = {n: self.host[n].pin_memory() for n in ("k", "v", "w", "u")}
@@ -567,7 +570,7 @@ class Wkv4Job:
 
         def one():
             k, v, w, u = (p[n].to(self.dev, non_blocking=True) for n in ("k", "v", "w", "u"))
-            o, _ = self.la.wkv4_forward(k, v, w, u, out=self.out, final_state=self.fin)
+            o, _ = self.la.wkv4_forward(k, v, w, u, out=self.out, final_state=self.fin, workspace=self.ws)
             y.copy_(o, non_blocking=True)
         for _ in range(2):
             one()
@@ -637,10 +640,12 @@ def run_wkv4(args, rank, world, dist_on, device):
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
                    "l2": "flushed before every step (512 MB write)" if flush is not None
                    else "inputs larger than L2",
-                   "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels)"},
+                   "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels"
+                   + (", T-segment)" if job.launches == 2 else ")")},
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
-                     "peak_source": pk_kind, "kernel": "la_wkv4 (wkv4_kernel)",
+                     "peak_source": pk_kind,
+                     "kernel": "wkv4_kernel (state pass + output pass)" if job.launches == 2 else "wkv4_kernel",
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": e2e, "clocks": sampler.summary(w0, w1) if sampler else None, "gpu_launches": launches,
     }

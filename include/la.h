@@ -342,6 +342,31 @@ LA_API la_status la_wkv4_forward(const void* k, const void* v, const float* w, c
                                  int B, int T, int C, la_dtype dtype, la_stream_t stream);
 
 /*
+ * la_wkv4_workspace_size - scratch bytes la_wkv4_forward_ws can use for these
+ * sizes (0 when the sequences would run as one segment).
+ *
+ * la_wkv4_forward_ws - la_wkv4_forward with caller-owned scratch.  Each
+ * channel's loop is sequential in t, so B x C channels alone can leave the
+ * GPU underused; with a workspace of at least la_wkv4_workspace_size bytes
+ * the sequence is cut into T-segments: a first launch computes each earlier
+ * segment's own (aa, bb, pp) from the empty state, the second starts every
+ * segment from the initial state combined with them in order (decayed over
+ * each segment's tokens, then added with the loop's own max-shifted
+ * weighting).  Results equal the single pass up to fp32 rounding.
+ *   workspace   NULL (one segment) or device memory, 16-byte aligned, used on
+ *               `stream` only; a smaller size than la_wkv4_workspace_size
+ *               runs one segment.  In place (final_state == init_state)
+ *               stays allowed.
+ * Other arguments and errors as la_wkv4_forward, plus LA_ERR_INVALID_ARG for
+ * a misaligned workspace.
+ */
+LA_API size_t la_wkv4_workspace_size(int B, int T, int C, la_dtype dtype);
+LA_API la_status la_wkv4_forward_ws(const void* k, const void* v, const float* w, const float* u,
+                                    const float* init_state, void* out, float* final_state,
+                                    int B, int T, int C, la_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, la_stream_t stream);
+
+/*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
  * device array inside this library (la_chunk_forward_noalloc_capacity()
  * bytes, 16 MiB, one per device, reserved when the library's device code is

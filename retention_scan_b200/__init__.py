@@ -26,6 +26,7 @@ LA_F32, LA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
                     "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
                     "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
+                    "la_wkv4_forward_ws", "la_wkv4_workspace_size",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -71,6 +72,10 @@ def lib():
         L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
         L.la_wkv4_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
         L.la_wkv4_forward.restype = i
+        L.la_wkv4_forward_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_wkv4_forward_ws.restype = i
+        L.la_wkv4_workspace_size.argtypes = [i, i, i, i]
+        L.la_wkv4_workspace_size.restype = ctypes.c_size_t
         L.la_chunk_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_forward_workspace_size.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp,
@@ -296,12 +301,20 @@ def chunk_backward(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=No
 WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)
 
 
-def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return_final=True, stream=None):
-    """RWKV-4 WKV recurrence (la_wkv4_forward).  k, v: [B,T,C] float32 or
+def wkv4_workspace_size(B, T, C, dtype=torch.bfloat16):
+    """Scratch bytes wkv4_forward can use (la_wkv4_workspace_size)."""
+    return int(lib().la_wkv4_workspace_size(B, T, C, _dtype_code(dtype)))
+
+
+def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return_final=True, stream=None,
+                 workspace=True):
+    """RWKV-4 WKV recurrence (la_wkv4_forward_ws).  k, v: [B,T,C] float32 or
     bfloat16 CUDA tensors (C a multiple of 8 for bf16, 4 for fp32); w (log
     of the per-step decay) and u (bonus): [C] fp32; init_state: [B,3,C] fp32
     (planes aa, bb, pp) or None for the empty state.  Returns (out [B,T,C],
-    final_state [B,3,C] or None).  final_state may be init_state itself."""
+    final_state [B,3,C] or None).  final_state may be init_state itself.
+    workspace: True allocates the T-segment scratch with torch on the call's
+    stream, None/False runs one segment, or a CUDA uint8 tensor to use."""
     B, T, C = k.shape
     dev = k.device
     code = _dtype_code(k.dtype)
@@ -317,8 +330,16 @@ def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return
         final_state = torch.empty((B, 3, C), dtype=torch.float32, device=dev)
     _need(final_state, "final_state", (B, 3, C), torch.float32, dev)
     with torch.cuda.device(dev):
-        _check(lib().la_wkv4_forward(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(init_state), _ptr(out),
-                                     _ptr(final_state), B, T, C, code, _stream(stream, dev)))
+        if workspace is True:
+            nbytes = wkv4_workspace_size(B, T, C, k.dtype)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+            if workspace is not None and stream is not None:
+                workspace.record_stream(stream)
+        elif workspace is False:
+            workspace = None
+        _check(lib().la_wkv4_forward_ws(_ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(init_state), _ptr(out),
+                                        _ptr(final_state), B, T, C, code, _ptr(workspace),
+                                        0 if workspace is None else workspace.numel(), _stream(stream, dev)))
     return out, final_state
 
 

@@ -329,9 +329,22 @@ la_status la_chunk_backward_ws(const void* q, const void* k, const void* v, cons
     return LA_OK;
 }
 
+size_t la_wkv4_workspace_size(int B, int T, int C, la_dtype dtype) {
+    if ((dtype != LA_F32 && dtype != LA_BF16) || B < 1 || T < 1 || C < 1 || B > 65535) return 0;
+    if (!fits_int(static_cast<long long>(T) * C) || !fits_int(3LL * B * C)) return 0;
+    return la::wkv4_workspace_bytes(B, T, C, dtype);
+}
+
 la_status la_wkv4_forward(const void* k, const void* v, const float* w, const float* u, const float* init_state,
                           void* out, float* final_state, int B, int T, int C, la_dtype dtype, la_stream_t stream) {
+    return la_wkv4_forward_ws(k, v, w, u, init_state, out, final_state, B, T, C, dtype, nullptr, 0, stream);
+}
+
+la_status la_wkv4_forward_ws(const void* k, const void* v, const float* w, const float* u, const float* init_state,
+                             void* out, float* final_state, int B, int T, int C, la_dtype dtype, void* workspace,
+                             size_t workspace_bytes, la_stream_t stream) {
     if (B < 0 || T < 0 || C < 1) return LA_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (!w || !u || !aligned4(w) || !aligned4(u)) return LA_ERR_INVALID_ARG;
     if ((init_state && !aligned4(init_state)) || (final_state && !aligned4(final_state))) return LA_ERR_INVALID_ARG;
@@ -359,6 +372,8 @@ la_status la_wkv4_forward(const void* k, const void* v, const float* w, const fl
     a.C = C;
     a.dtype = dtype;
     a.err_word = err_word_for_current_device();
+    a.workspace = workspace;
+    a.workspace_bytes = workspace ? workspace_bytes : 0;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     return la::launch_wkv4(a) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }

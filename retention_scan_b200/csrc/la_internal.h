@@ -115,8 +115,11 @@ struct Wkv4Args {
     int B, T, C;
     la_dtype dtype;
     int* err_word;
+    void* workspace;          // T-segment states (may be null: one segment)
+    size_t workspace_bytes;
     cudaStream_t stream;
 };
 cudaError_t launch_wkv4(const Wkv4Args& a);
+size_t wkv4_workspace_bytes(int B, int T, int C, la_dtype dtype);
 
 }  // namespace la

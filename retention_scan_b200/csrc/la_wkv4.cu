@@ -11,12 +11,22 @@
 // exponentiated, so no key can overflow.  The kernel runs the loop in fp32
 // in log2 units (every log value times log2 e, exponentials by ex2).
 //
-// Data movement: a CTA owns one batch row and kCW consecutive channels.  One
-// producer thread streams [kTT tokens x kCW channels] tiles of k and v into
-// a ring of kStages shared-memory stages with TMA (about 96 KB in flight per
-// CTA, two CTAs per SM), so the HBM latency is hidden behind the sequential
-// per-token work; each consumer thread reads its channel's column of the
-// tile and writes its output directly (a warp writes 32 consecutive values).
+// Data movement: a CTA owns one batch row, kCW consecutive channels and one
+// T-segment.  One producer thread streams [TT tokens x kCW channels] tiles
+// of k and v into a ring of kStages shared-memory stages with TMA (four CTAs
+// per SM, about 190 KB in flight per SM), so the HBM latency is hidden
+// behind the sequential per-token work; each consumer thread reads its
+// channel's column of the tile and writes its output directly (a warp writes
+// 32 consecutive values).
+//
+// Parallelism: a channel's recurrence is sequential in t, and B x C channels
+// alone leave each scheduler about one warp.  With a workspace, each sequence
+// is cut into T-segments: a state pass computes every earlier segment's own
+// (aa, bb, pp) from an empty state, and the output pass starts segment s
+// from the initial state combined with them in order (decay the running
+// state over a segment's tokens, then add that segment's state with the same
+// max-shifted weighting the loop uses), which multiplies the independent
+// chains per SM.
 // Every barrier wait gives up after kWaitLimitNs, sets the device error word
 // and unwinds.
 #include <cuda.h>
@@ -30,9 +40,11 @@ namespace la {
 namespace {
 
 constexpr int kCW = 64;                 // channels per CTA (one per consumer thread)
-constexpr int kStages = 6;
+constexpr int kStages = 3;              // 3 x 16 KB: four CTAs per SM
 constexpr int kConsumerWarps = kCW / 32;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one producer warp
+constexpr int kCtasPerSm = 4;
+constexpr int kMinSegTokens = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kEmptyScale = -1e38f;   // pp of an empty state (aa = bb = 0)
@@ -43,6 +55,22 @@ struct Tile {
     static constexpr int BYTES = TT * kCW * static_cast<int>(sizeof(E));  // one array's tile
     static constexpr int STAGE = 2 * BYTES;                        // k tile, then v tile
     static constexpr int SMEM = kStages * STAGE + 256;             // + barriers
+};
+
+// T-segments: segment s covers tokens [s * seg_len, min(T, (s + 1) * seg_len)).
+// The state pass (state_pass = 1, segments 0 .. nseg - 2) writes each
+// segment's own state, from an empty one, to ws slot s + 1, and its segment-0
+// CTAs copy the initial state to slot 0; the output pass starts segment s
+// from slot 0 combined with slots 1 .. s.  ws is [B][nseg][3][C] fp32.
+struct WkvParams {
+    const float* w;
+    const float* u;
+    const float* init_state;
+    void* out;
+    float* final_state;
+    float* ws;
+    int T, C, seg_len, nseg, state_pass;
+    int* err;
 };
 
 // Weights of two terms with log2 weights a and b against the larger one:
@@ -62,9 +90,7 @@ __device__ __forceinline__ void store_e(__nv_bfloat16* p, float x) { *p = __floa
 template <typename E>
 __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ CUtensorMap tmk,
                                                         const __grid_constant__ CUtensorMap tmv,
-                                                        const float* __restrict__ w, const float* __restrict__ u,
-                                                        const float* init_state, E* __restrict__ out,
-                                                        float* final_state, int T, int C, int* err) {
+                                                        const __grid_constant__ WkvParams p) {
     using G = Tile<E>;
     // used as declared (not realigned through an integer), so that the
     // compiler keeps the shared address space and reads tiles with LDS;
@@ -74,8 +100,10 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
     uint64_t* empty = full + kStages;
     volatile int* abort = reinterpret_cast<volatile int*>(empty + kStages);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int b = blockIdx.y, c0 = blockIdx.x * kCW;
-    const int ntiles = (T + G::TT - 1) / G::TT;
+    const int b = blockIdx.y, c0 = blockIdx.x * kCW, seg = blockIdx.z;
+    const int T = p.T, C = p.C;
+    const int t0 = seg * p.seg_len, t1 = min(T, t0 + p.seg_len);
+    const int j0 = t0 / G::TT, ntiles = (t1 - t0 + G::TT - 1) / G::TT;  // seg_len is a multiple of TT
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmk);
@@ -97,14 +125,14 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
                 const int s = j % kStages;
                 if (j >= kStages && !mbar_wait_bounded(&empty[s], ((j / kStages) - 1) & 1, kWaitLimitNs)) {
                     *abort = 1;
-                    if (err) atomicCAS(err, 0, kErrTmaWait);
+                    if (p.err) atomicCAS(p.err, 0, kErrTmaWait);
                     break;
                 }
                 if (*abort) break;
                 uint8_t* st = sm + s * G::STAGE;
                 mbar_arrive_expect_tx(&full[s], G::STAGE);
-                tma_load_3d(st, &tmk, &full[s], c0, j * G::TT, b);
-                tma_load_3d(st + G::BYTES, &tmv, &full[s], c0, j * G::TT, b);
+                tma_load_3d(st, &tmk, &full[s], c0, (j0 + j) * G::TT, b);
+                tma_load_3d(st + G::BYTES, &tmv, &full[s], c0, (j0 + j) * G::TT, b);
                 ++issued;
             }
             // copies in flight land before the CTA's shared memory goes away
@@ -117,31 +145,75 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
     // consumer: thread = channel
     const int c = c0 + threadIdx.x;
     const bool live = c < C;
-    const float W = live ? w[c] * kLog2e : 0.f;
-    const float U = live ? u[c] * kLog2e : 0.f;
+    const float W = live ? p.w[c] * kLog2e : 0.f;
+    const float U = live ? p.u[c] * kLog2e : 0.f;
+    const size_t plane = static_cast<size_t>(C);
     float aa = 0.f, bb = 0.f, P = kEmptyScale * kLog2e;
-    if (live && init_state) {
-        const float* s0 = init_state + static_cast<size_t>(b) * 3 * C + c;
-        aa = s0[0];
-        bb = s0[C];
-        P = s0[2 * C] * kLog2e;
+    float* slot0 = p.ws ? p.ws + static_cast<size_t>(b) * p.nseg * 3 * plane + c : nullptr;
+    if (live) {
+        if (p.state_pass) {
+            if (seg == 0) {  // keep the initial state for the output pass
+                const float* s0 = p.init_state ? p.init_state + static_cast<size_t>(b) * 3 * plane + c : nullptr;
+                slot0[0] = s0 ? s0[0] : 0.f;
+                slot0[plane] = s0 ? s0[plane] : 0.f;
+                slot0[2 * plane] = s0 ? s0[2 * plane] : kEmptyScale;
+            }
+        } else if (p.ws) {
+            // the initial state, then each earlier segment: decayed over that
+            // segment's tokens, plus the segment's own state (max-shifted add)
+            aa = slot0[0];
+            bb = slot0[plane];
+            P = slot0[2 * plane] * kLog2e;
+            for (int j = 0; j < seg; ++j) {
+                const float* sj = slot0 + static_cast<size_t>(j + 1) * 3 * plane;
+                const float Pd = P + W * static_cast<float>(p.seg_len);
+                const float Pj = sj[2 * plane] * kLog2e;
+                float fa, fb;
+                shifted_pair(Pd, Pj, fa, fb);
+                aa = fmaf(fa, aa, fb * sj[0]);
+                bb = fmaf(fa, bb, fb * sj[plane]);
+                P = fmaxf(Pd, Pj);
+            }
+        } else if (p.init_state) {
+            const float* s0 = p.init_state + static_cast<size_t>(b) * 3 * plane + c;
+            aa = s0[0];
+            bb = s0[plane];
+            P = s0[2 * plane] * kLog2e;
+        }
     }
-    E* o = out + static_cast<size_t>(b) * T * C + c;
+    E* o = static_cast<E*>(p.out) + (static_cast<size_t>(b) * T + t0) * C + c;
+    // one token: read-out (the state at log weight P, this token at U + K),
+    // then update (the state decayed to W + P, this token at K)
+    auto update = [&](float K, float v) {
+        const float d = W + P;
+        float f1, f2;
+        shifted_pair(d, K, f1, f2);
+        aa = fmaf(f1, aa, f2 * v);
+        bb = fmaf(f1, bb, f2);
+        P = fmaxf(d, K);
+    };
+    auto step = [&](float K, float v) -> float {
+        float e1, e2;
+        shifted_pair(P, U + K, e1, e2);
+        const float y = __fdividef(fmaf(e1, aa, e2 * v), fmaf(e1, bb, e2));
+        update(K, v);
+        return y;
+    };
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j % kStages;
         // whole-warp bounded wait on the tile
         bool got = mbar_try_wait(&full[s], (j / kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) {
-            const uint64_t t0 = global_timer_ns();
+            const uint64_t tw = global_timer_ns();
             while (true) {
                 if (!got) got = mbar_try_wait_sleep(&full[s], (j / kStages) & 1, 20000);
                 if (__all_sync(0xffffffffu, got)) break;
-                bool give_up = *abort != 0 || global_timer_ns() - t0 > kWaitLimitNs;
+                bool give_up = *abort != 0 || global_timer_ns() - tw > kWaitLimitNs;
                 if (__any_sync(0xffffffffu, give_up)) {
                     if (lane == 0) {
                         *abort = 1;
-                        if (err) atomicCAS(err, 0, kErrTmaWait);
+                        if (p.err) atomicCAS(p.err, 0, kErrTmaWait);
                     }
                     ok = false;
                     break;
@@ -151,22 +223,11 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
         }
         const E* tk = reinterpret_cast<const E*>(sm + s * G::STAGE) + threadIdx.x;
         const E* tv = reinterpret_cast<const E*>(sm + s * G::STAGE + G::BYTES) + threadIdx.x;
-        const int n = min(G::TT, T - j * G::TT);
-        // one token: read-out (the state at log weight P, this token at
-        // U + K), then update (the state decayed to W + P, this token at K)
-        auto step = [&](float K, float v) -> float {
-            float e1, e2;
-            shifted_pair(P, U + K, e1, e2);
-            const float y = __fdividef(fmaf(e1, aa, e2 * v), fmaf(e1, bb, e2));
-            const float d = W + P;
-            float f1, f2;
-            shifted_pair(d, K, f1, f2);
-            aa = fmaf(f1, aa, f2 * v);
-            bb = fmaf(f1, bb, f2);
-            P = fmaxf(d, K);
-            return y;
-        };
-        if (live) {
+        const int n = min(G::TT, t1 - (j0 + j) * G::TT);
+        if (live && p.state_pass) {
+#pragma unroll 8
+            for (int i = 0; i < n; ++i) update(load_f(tk + i * kCW) * kLog2e, load_f(tv + i * kCW));
+        } else if (live) {
             // batches of 8 tokens: the next batch's tile reads are issued
             // before this batch's dependent steps, the outputs stored after
             // them, so that memory latency stays off the recurrence's path
@@ -206,11 +267,16 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (ok && live && final_state) {
-        float* s1 = final_state + static_cast<size_t>(b) * 3 * C + c;
-        s1[0] = aa;
-        s1[C] = bb;
-        s1[2 * C] = P * (1.f / kLog2e);
+    if (!ok || !live) return;
+    float* dst = nullptr;
+    if (p.state_pass)
+        dst = slot0 + static_cast<size_t>(seg + 1) * 3 * plane;
+    else if (seg == p.nseg - 1 && p.final_state)
+        dst = p.final_state + static_cast<size_t>(b) * 3 * plane + c;
+    if (dst) {
+        dst[0] = aa;
+        dst[plane] = bb;
+        dst[2 * plane] = P * (1.f / kLog2e);
     }
 }
 
@@ -227,6 +293,33 @@ bool make_wkv_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count_wkv() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || v <= 0)
+        v = 148;
+    return v;
+}
+
+// Segments per sequence: doubled while every segment's CTAs still fit on the
+// GPU at once (kCtasPerSm per SM) and segments keep >= kMinSegTokens tokens;
+// the segment length is a whole number of tiles.
+struct WkvLayout {
+    int nseg, seg_len;
+};
+
+WkvLayout wkv_layout(int B, int T, int C, int tt, bool segments) {
+    const long long ctas = static_cast<long long>(B) * ((C + kCW - 1) / kCW);
+    const long long resident = static_cast<long long>(sm_count_wkv()) * kCtasPerSm;
+    int nseg = 1;
+    if (segments)
+        while (ctas * nseg * 2 <= resident && T / (nseg * 2) >= kMinSegTokens) nseg *= 2;
+    int seg_len = (T + nseg - 1) / nseg;
+    seg_len = (seg_len + tt - 1) / tt * tt;
+    if (seg_len < 1) seg_len = tt;
+    return WkvLayout{(T + seg_len - 1) / seg_len, seg_len};
+}
+
 template <typename E>
 cudaError_t launch_typed(const Wkv4Args& a, CUtensorMapDataType dt) {
     using G = Tile<E>;
@@ -236,9 +329,30 @@ cudaError_t launch_typed(const Wkv4Args& a, CUtensorMapDataType dt) {
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(wkv4_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
     if (e != cudaSuccess) return e;
-    const dim3 grid((a.C + kCW - 1) / kCW, a.B);
-    wkv4_kernel<E><<<grid, kThreads, G::SMEM, a.stream>>>(tmk, tmv, a.w, a.u, a.init_state, static_cast<E*>(a.out),
-                                                          a.final_state, a.T, a.C, a.err_word);
+    WkvLayout L = wkv_layout(a.B, a.T, a.C, G::TT, a.workspace != nullptr);
+    const size_t need = sizeof(float) * static_cast<size_t>(a.B) * L.nseg * 3 * a.C;
+    if (L.nseg > 1 && a.workspace_bytes < need) L = wkv_layout(a.B, a.T, a.C, G::TT, false);
+    WkvParams p{};
+    p.w = a.w;
+    p.u = a.u;
+    p.init_state = a.init_state;
+    p.out = a.out;
+    p.final_state = a.final_state;
+    p.T = a.T;
+    p.C = a.C;
+    p.seg_len = L.seg_len;
+    p.nseg = L.nseg;
+    p.err = a.err_word;
+    const int tiles = (a.C + kCW - 1) / kCW;
+    if (L.nseg > 1) {
+        p.ws = static_cast<float*>(a.workspace);
+        WkvParams ps = p;
+        ps.state_pass = 1;
+        wkv4_kernel<E><<<dim3(tiles, a.B, L.nseg - 1), kThreads, G::SMEM, a.stream>>>(tmk, tmv, ps);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    wkv4_kernel<E><<<dim3(tiles, a.B, L.nseg), kThreads, G::SMEM, a.stream>>>(tmk, tmv, p);
     return cudaGetLastError();
 }
 
@@ -252,6 +366,14 @@ __global__ void wkv4_pass_state_kernel(const float* init_state, float* final_sta
 }
 
 }  // namespace
+
+size_t wkv4_workspace_bytes(int B, int T, int C, la_dtype dtype) {
+    if (B < 1 || T < 1 || C < 1) return 0;
+    const WkvLayout L = wkv_layout(B, T, C, dtype == LA_BF16 ? Tile<__nv_bfloat16>::TT : Tile<float>::TT, true);
+    if (L.nseg < 2) return 0;
+    const size_t b = sizeof(float) * static_cast<size_t>(B) * L.nseg * 3 * C;
+    return (b + 255) / 256 * 256;
+}
 
 cudaError_t launch_wkv4(const Wkv4Args& a) {
     if (a.T == 0) {

@@ -156,3 +156,36 @@ def test_wkv4_workload_sampled_rows():
         ro, rf = oracle.wkv4(inp["k"][b:b + 1], inp["v"][b:b + 1], inp["w"], inp["u"])
         errs = [row_err(out[b:b + 1], ro)] + list(state_errs(fin[b:b + 1], rf).values())
         assert max(errs) <= 2e-2, (b, errs)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("init", [False, True])
+def test_wkv4_t_segments(dtype, init):
+    """One channel tile and a long sequence: the library cuts it into
+    T-segments (a state pass, then the output pass starting each segment from
+    the combined earlier states); ragged last segment."""
+    B, T, C = 1, 4096 + 77, 64
+    assert la().wkv4_workspace_size(B, T, C, dtype) > 0
+    k, v, w, u, S0 = case(B, T, C, dtype, init, seed=4400 + init)
+    check(k, v, w, u, S0)
+    # the same call without a workspace (one segment) agrees to fp32 rounding
+    kd, vd, wd, ud = k.cuda(), v.cuda(), w.cuda(), u.cuda()
+    S0d = None if S0 is None else S0.cuda()
+    a, fa = la().wkv4_forward(kd, vd, wd, ud, S0d)
+    b, fb = la().wkv4_forward(kd, vd, wd, ud, S0d, workspace=False)
+    torch.cuda.synchronize()
+    assert row_err(a, b.cpu().double().numpy()) <= (1e-5 if dtype == torch.float32 else 1e-2)
+    assert max(state_errs(fa, fb.cpu().double().numpy()).values()) <= 1e-5
+
+
+def test_wkv4_t_segments_in_place():
+    """The carried state read and written in place with T-segments."""
+    B, T, C = 2, 3000, 128
+    k, v, w, u, S0 = case(B, T, C, torch.bfloat16, True, seed=4500)
+    assert la().wkv4_workspace_size(B, T, C) > 0
+    ro, rf = oracle.wkv4(k, v, w, u, S0)
+    state = S0.cuda().clone()
+    out, _ = la().wkv4_forward(k.cuda(), v.cuda(), w.cuda(), u.cuda(), state, final_state=state)
+    torch.cuda.synchronize()
+    assert row_err(out, ro) <= 2e-2
+    assert max(state_errs(state, rf).values()) <= 2e-2
