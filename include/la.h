@@ -100,6 +100,22 @@ typedef struct {
     const float* log_g;       /* device pointer, see kind for the shape */
 } la_decay;
 
+/* Input prologue: a feature map on q and k and a scale on q, applied by the
+ * kernels as they read their inputs instead of by a separate pass over
+ * memory.  The normalised linear attention of flash-linear-attention issue
+ * 268 feeds elu(x) + 1 of the queries and keys, and its sequence diagram
+ * passes q * scale; with a prologue the caller hands over the raw q and k.
+ * A NULL prologue, or {LA_FEATURE_NONE, 1.0f}, reads the inputs as they are. */
+typedef enum {
+    LA_FEATURE_NONE = 0,      /* phi(x) = x */
+    LA_FEATURE_ELU1 = 1       /* phi(x) = elu(x) + 1 = (x > 0 ? x + 1 : e^x), in fp32 */
+} la_feature_map;
+
+typedef struct {
+    int feature_map;          /* an la_feature_map value, applied to q and k */
+    float q_scale;            /* q <- q_scale * phi(q); finite */
+} la_prologue;
+
 /*
  * la_chunk_forward - the whole sequence forward pass.
  *
@@ -295,6 +311,44 @@ LA_API la_status la_chunk_backward_ws(const void* q, const void* k, const void* 
                                void* dq, void* dk, void* dv, float* d_log_g, float* d_init_state,
                                int B, int H, int T, int Dk, int Dv, la_dtype dtype,
                                void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * la_chunk_forward_pro_ws - la_chunk_forward_ws on phi(q) * q_scale and
+ * phi(k) (see la_prologue), with the prologue applied inside the kernels.
+ *
+ * The fp32 path applies both as it stages q and k.  The bf16 tensor-core
+ * path applies q_scale in its epilogue (the output is linear in q, and the
+ * normalised output does not depend on the scale of q); it has no feature
+ * map: applying elu(x) + 1 to the Q and K tiles in shared memory would put
+ * one exponential per element (32768 per 128-token chunk at Dk = 128) on
+ * the path from a tile's load to its first MMA, so for bf16 inputs
+ * feature_map must be LA_FEATURE_NONE (else LA_ERR_UNSUPPORTED).
+ *
+ *   prologue        NULL (identity) or a descriptor.
+ *   other arguments as la_chunk_forward_ws.
+ *
+ * Errors as la_chunk_forward_ws, plus LA_ERR_INVALID_ARG for a feature_map
+ * out of range or a q_scale that is not finite.
+ */
+LA_API la_status la_chunk_forward_pro_ws(const void* q, const void* k, const void* v,
+                                  const la_decay* decay, int normalize, const la_prologue* prologue,
+                                  const float* init_state, const float* init_z,
+                                  void* out, float* final_state, float* final_z,
+                                  int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                                  void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * la_decode_step_pro - la_decode_step on phi(q) * q_scale and phi(k) (see
+ * la_prologue), applied as the kernel stages this token's q and k: a
+ * generation loop needs no separate feature-map launch per token.
+ * Arguments and errors as la_decode_step, plus LA_ERR_INVALID_ARG for a
+ * feature_map out of range or a q_scale that is not finite.
+ */
+LA_API la_status la_decode_step_pro(const void* q, const void* k, const void* v,
+                             const la_decay* decay, int normalize, const la_prologue* prologue,
+                             float* state, float* z, void* out,
+                             int B, int H, int Dk, int Dv,
+                             la_dtype dtype, la_stream_t stream);
 
 /*
  * la_wkv4_forward - the RWKV-4 WKV recurrence (a different recurrence from

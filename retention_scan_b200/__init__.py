@@ -16,17 +16,19 @@ import torch
 __all__ = ["chunk_forward", "bidirectional", "chunk_backward", "wkv4_forward", "workspace_size",
            "backward_workspace_size",
            "decode_step", "device_error", "LAError", "lib", "library_path",
-           "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "EXPORTED_SYMBOLS"]
+           "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "FEATURE_NONE", "FEATURE_ELU1", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libla.so")
 
 DECAY_NONE, DECAY_PER_HEAD, DECAY_PER_STEP = 0, 1, 2
+FEATURE_NONE, FEATURE_ELU1 = 0, 1
 LA_F32, LA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward_workspace_size",
                     "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
                     "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
-                    "la_wkv4_forward_ws", "la_wkv4_workspace_size",
+                    "la_wkv4_forward_ws", "la_wkv4_workspace_size", "la_chunk_forward_pro_ws",
+                    "la_decode_step_pro",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -40,6 +42,10 @@ class LAError(RuntimeError):
 
 class _Decay(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("log_g", ctypes.c_void_p)]
+
+
+class _Prologue(ctypes.Structure):
+    _fields_ = [("feature_map", ctypes.c_int), ("q_scale", ctypes.c_float)]
 
 
 _lib = None
@@ -60,6 +66,12 @@ def lib():
         L.la_chunk_forward_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, vp, vp,
                                           i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
         L.la_chunk_forward_ws.restype = i
+        L.la_chunk_forward_pro_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, ctypes.POINTER(_Prologue),
+                                              vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_chunk_forward_pro_ws.restype = i
+        L.la_decode_step_pro.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, ctypes.POINTER(_Prologue), vp, vp,
+                                         vp, i, i, i, i, i, vp]
+        L.la_decode_step_pro.restype = i
         L.la_chunk_reverse_ws.argtypes = L.la_chunk_forward_ws.argtypes
         L.la_chunk_reverse_ws.restype = i
         L.la_chunk_bidirectional_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), i, vp,
@@ -155,7 +167,8 @@ def _workspace(workspace, B, H, T, Dk, Dv, dtype, normalize, stream, dev):
 
 def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
                   init_state=None, init_z=None, out=None, final_state=None, final_z=None,
-                  return_final=True, stream=None, workspace=True, reverse=False):
+                  return_final=True, stream=None, workspace=True, reverse=False,
+                  feature_map=FEATURE_NONE, q_scale=1.0):
     """Whole-sequence forward (la_chunk_forward_ws), or with reverse=True the
     anti-causal scan from the last token back (la_chunk_reverse_ws; the
     carried state then enters after token T and final_* hold the state at
@@ -170,6 +183,9 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     workspace: True allocates the scratch that lets short-on-heads inputs run
     as T-segments (a torch allocation on the call's stream), None/False runs
     without, or a CUDA uint8 tensor to use.
+    feature_map / q_scale: the input prologue (la_chunk_forward_pro_ws): the
+    kernels read phi(q) * q_scale and phi(k), phi = FEATURE_ELU1 (elu + 1,
+    fp32 inputs only) or FEATURE_NONE.  Forward scans only.
     """
     B, H, T, Dk = q.shape
     Dv = v.shape[-1]
@@ -196,12 +212,21 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     d = _decay(decay_kind, log_g)
     with torch.cuda.device(dev):
         workspace = _workspace(workspace, B, H, T, Dk, Dv, q.dtype, normalize, stream, dev)
+        nbytes = 0 if workspace is None else workspace.numel()
+        if feature_map != FEATURE_NONE or q_scale != 1.0:
+            if reverse:
+                raise ValueError("the input prologue applies to the forward scan")
+            pro = _Prologue(int(feature_map), float(q_scale))
+            _check(lib().la_chunk_forward_pro_ws(
+                _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+                ctypes.byref(pro), _ptr(init_state), _ptr(init_z), _ptr(out), _ptr(final_state), _ptr(final_z),
+                B, H, T, Dk, Dv, code, _ptr(workspace), nbytes, _stream(stream, dev)))
+            return out, final_state, (final_z if normalize else None)
         entry = lib().la_chunk_reverse_ws if reverse else lib().la_chunk_forward_ws
         _check(entry(
             _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
             _ptr(init_state), _ptr(init_z), _ptr(out), _ptr(final_state), _ptr(final_z),
-            B, H, T, Dk, Dv, code, _ptr(workspace), 0 if workspace is None else workspace.numel(),
-            _stream(stream, dev)))
+            B, H, T, Dk, Dv, code, _ptr(workspace), nbytes, _stream(stream, dev)))
     return out, final_state, (final_z if normalize else None)
 
 
@@ -344,9 +369,11 @@ def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,
-                out=None, stream=None):
+                out=None, stream=None, feature_map=FEATURE_NONE, q_scale=1.0):
     """One token (la_decode_step); state [B,H,Dk,Dv] and z [B,H,Dk] (fp32) are
-    updated in place.  q, k: [B,H,Dk]; v: [B,H,Dv].  Returns out [B,H,Dv]."""
+    updated in place.  q, k: [B,H,Dk]; v: [B,H,Dv].  Returns out [B,H,Dv].
+    feature_map / q_scale: the input prologue (la_decode_step_pro): the kernel
+    reads phi(q) * q_scale and phi(k)."""
     B, H, Dk = q.shape
     Dv = v.shape[-1]
     dev = q.device
@@ -367,10 +394,17 @@ def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, norma
     _need(out, "out", (B, H, Dv), q.dtype, dev)
     d = _decay(decay_kind, log_g)
     with torch.cuda.device(dev):
-        _check(lib().la_decode_step(
-            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
-            _ptr(state), _ptr(z if normalize else None), _ptr(out), B, H, Dk, Dv, code,
-            _stream(stream, dev)))
+        if feature_map != FEATURE_NONE or q_scale != 1.0:
+            pro = _Prologue(int(feature_map), float(q_scale))
+            _check(lib().la_decode_step_pro(
+                _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+                ctypes.byref(pro), _ptr(state), _ptr(z if normalize else None), _ptr(out), B, H, Dk, Dv, code,
+                _stream(stream, dev)))
+        else:
+            _check(lib().la_decode_step(
+                _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)),
+                _ptr(state), _ptr(z if normalize else None), _ptr(out), B, H, Dk, Dv, code,
+                _stream(stream, dev)))
     return out
 
 

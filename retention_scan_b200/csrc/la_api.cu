@@ -4,6 +4,7 @@
 
 #include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -44,6 +45,17 @@ bool launch_fault_injected() {
 
 bool fits_int(long long x) { return x >= 0 && x <= INT_MAX; }
 
+la_status check_prologue(const la_prologue* pro, int* fmap, float* qscale) {
+    *fmap = LA_FEATURE_NONE;
+    *qscale = 1.f;
+    if (!pro) return LA_OK;
+    if (pro->feature_map < LA_FEATURE_NONE || pro->feature_map > LA_FEATURE_ELU1) return LA_ERR_INVALID_ARG;
+    if (!std::isfinite(pro->q_scale)) return LA_ERR_INVALID_ARG;
+    *fmap = pro->feature_map;
+    *qscale = pro->q_scale;
+    return LA_OK;
+}
+
 la_status check_decay(const la_decay* decay, int* kind, const float** log_g) {
     *kind = LA_DECAY_NONE;
     *log_g = nullptr;
@@ -62,8 +74,11 @@ la_status check_decay(const la_decay* decay, int* kind, const float** log_g) {
 la_status scan(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
                const float* init_state, const float* init_z, void* out, float* final_state, float* final_z,
                int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace, size_t workspace_bytes,
-               la_stream_t stream, int reverse, int accumulate) {
+               la_stream_t stream, int reverse, int accumulate, const la_prologue* pro = nullptr) {
     if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    int fmap;
+    float qscale;
+    if (check_prologue(pro, &fmap, &qscale) != LA_OK) return LA_ERR_INVALID_ARG;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     int kind;
@@ -84,6 +99,7 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
     }
     if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
     if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
+    if (dtype == LA_BF16 && fmap != LA_FEATURE_NONE) return LA_ERR_UNSUPPORTED;  // see la.h
     if (BH == 0) return LA_OK;
     if (launch_fault_injected()) return LA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -122,6 +138,8 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
     a.err_word = err_word_for_current_device();
     a.reverse = reverse;
     a.accumulate = accumulate;
+    a.feature_map = fmap;
+    a.q_scale = qscale;
     cudaError_t e;
     if (dtype == LA_F32) {
         e = la::launch_fwd_f32(a);
@@ -202,6 +220,14 @@ la_status la_chunk_forward_ws(const void* q, const void* k, const void* v, const
                               size_t workspace_bytes, la_stream_t stream) {
     return scan(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T, Dk, Dv, dtype,
                 workspace, workspace_bytes, stream, 0, 0);
+}
+
+la_status la_chunk_forward_pro_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                                  const la_prologue* prologue, const float* init_state, const float* init_z, void* out,
+                                  float* final_state, float* final_z, int B, int H, int T, int Dk, int Dv,
+                                  la_dtype dtype, void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    return scan(q, k, v, decay, normalize, init_state, init_z, out, final_state, final_z, B, H, T, Dk, Dv, dtype,
+                workspace, workspace_bytes, stream, 0, 0, prologue);
 }
 
 la_status la_chunk_reverse_ws(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
@@ -381,6 +407,15 @@ la_status la_wkv4_forward_ws(const void* k, const void* v, const float* w, const
 la_status la_decode_step(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
                          float* state, float* z, void* out, int B, int H, int Dk, int Dv, la_dtype dtype,
                          la_stream_t stream) {
+    return la_decode_step_pro(q, k, v, decay, normalize, nullptr, state, z, out, B, H, Dk, Dv, dtype, stream);
+}
+
+la_status la_decode_step_pro(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
+                             const la_prologue* prologue, float* state, float* z, void* out, int B, int H, int Dk,
+                             int Dv, la_dtype dtype, la_stream_t stream) {
+    int fmap;
+    float qscale;
+    if (check_prologue(prologue, &fmap, &qscale) != LA_OK) return LA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     int kind;
@@ -413,6 +448,8 @@ la_status la_decode_step(const void* q, const void* k, const void* v, const la_d
     a.H = H;
     a.Dk = Dk;
     a.Dv = Dv;
+    a.feature_map = fmap;
+    a.q_scale = qscale;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     return la::launch_decode(a, dtype) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }

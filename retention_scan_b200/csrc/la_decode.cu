@@ -44,6 +44,11 @@ __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float
 __device__ __forceinline__ void from_f(float* p, float x) { *p = x; }
 __device__ __forceinline__ void from_f(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
+// The prologue's feature map: elu(x) + 1 = (x > 0 ? x + 1 : e^x).
+__device__ __forceinline__ float feature(float x, int fmap) {
+    return fmap == LA_FEATURE_ELU1 ? (x > 0.f ? x + 1.f : expf(x)) : x;
+}
+
 __device__ __forceinline__ float decay_of(int kind, const float* log_g, int bh, int h) {
     if (kind == LA_DECAY_PER_HEAD) return expf(log_g[h]);
     if (kind == LA_DECAY_PER_STEP) return expf(log_g[bh]);
@@ -67,7 +72,7 @@ template <typename TIn, int C4>
 __global__ void __launch_bounds__(kThreads) decode_vec_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v, int decay_kind,
     const float* __restrict__ log_g, int normalize, float* __restrict__ state, float* __restrict__ z,
-    TIn* __restrict__ out, int H, int Dk) {
+    TIn* __restrict__ out, int H, int Dk, int fmap, float qscale) {
     constexpr int Dv = 4 * C4;
     constexpr int R = kThreads / C4;
     __shared__ float qs[128], ks[128];
@@ -77,8 +82,8 @@ __global__ void __launch_bounds__(kThreads) decode_vec_kernel(
     const int bh = blockIdx.x, tid = threadIdx.x;
     const float g = decay_of(decay_kind, log_g, bh, bh % H);
     if (tid < Dk) {
-        qs[tid] = to_f(q[static_cast<size_t>(bh) * Dk + tid]);
-        ks[tid] = to_f(k[static_cast<size_t>(bh) * Dk + tid]);
+        qs[tid] = qscale * feature(to_f(q[static_cast<size_t>(bh) * Dk + tid]), fmap);
+        ks[tid] = feature(to_f(k[static_cast<size_t>(bh) * Dk + tid]), fmap);
     }
     const int c4 = tid % C4, r0 = tid / C4;
     const float4 vv = load4(v + static_cast<size_t>(bh) * Dv + 4 * c4);
@@ -142,14 +147,14 @@ template <typename TIn>
 __global__ void __launch_bounds__(128) decode_generic_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v, int decay_kind,
     const float* __restrict__ log_g, int normalize, float* __restrict__ state, float* __restrict__ z,
-    TIn* __restrict__ out, int H, int Dk, int Dv) {
+    TIn* __restrict__ out, int H, int Dk, int Dv, int fmap, float qscale) {
     __shared__ float qs[128], ks[128];
     __shared__ float red[4];
     const int bh = blockIdx.x, tid = threadIdx.x;
     const float g = decay_of(decay_kind, log_g, bh, bh % H);
     if (tid < Dk) {
-        qs[tid] = to_f(q[static_cast<size_t>(bh) * Dk + tid]);
-        ks[tid] = to_f(k[static_cast<size_t>(bh) * Dk + tid]);
+        qs[tid] = qscale * feature(to_f(q[static_cast<size_t>(bh) * Dk + tid]), fmap);
+        ks[tid] = feature(to_f(k[static_cast<size_t>(bh) * Dk + tid]), fmap);
     }
     __syncthreads();
     float num = 0.f;
@@ -186,7 +191,7 @@ cudaError_t launch_typed(const DecodeArgs& a) {
 #define LA_DECODE_VEC(C4)                                                                            \
     decode_vec_kernel<TIn, C4><<<grid, kThreads, 0, a.stream>>>(q, k, v, a.decay_kind, a.log_g,     \
                                                                  a.normalize, a.state, a.z, out, a.H, \
-                                                                 a.Dk)
+                                                                 a.Dk, a.feature_map, a.q_scale)
     switch (a.Dv) {
         case 4: LA_DECODE_VEC(1); break;
         case 8: LA_DECODE_VEC(2); break;
@@ -197,7 +202,7 @@ cudaError_t launch_typed(const DecodeArgs& a) {
         default:
             decode_generic_kernel<TIn><<<grid, 128, 0, a.stream>>>(q, k, v, a.decay_kind, a.log_g,
                                                                    a.normalize, a.state, a.z, out, a.H,
-                                                                   a.Dk, a.Dv);
+                                                                   a.Dk, a.Dv, a.feature_map, a.q_scale);
     }
 #undef LA_DECODE_VEC
     return cudaGetLastError();

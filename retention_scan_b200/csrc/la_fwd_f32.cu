@@ -23,12 +23,17 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kTile = 32;
 
+// The prologue's feature map: elu(x) + 1 = (x > 0 ? x + 1 : e^x).
+__device__ __forceinline__ float feature(float x, int fmap) {
+    return fmap == LA_FEATURE_ELU1 ? (x > 0.f ? x + 1.f : expf(x)) : x;
+}
+
 __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     int decay_kind, const float* __restrict__ log_g, int normalize,
     const float* __restrict__ init_state, const float* __restrict__ init_z,
     float* __restrict__ out, float* __restrict__ final_state, float* __restrict__ final_z,
-    int H, int T, int Dk, int Dv, int reverse, int accumulate) {
+    int H, int T, int Dk, int Dv, int reverse, int accumulate, int fmap, float qscale) {
     extern __shared__ float smem[];
     float* S = smem;                    // [Dk][Dv]
     float* qs = S + Dk * Dv;            // [kTile][Dk]
@@ -56,8 +61,8 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
         const int t0 = tile * kTile, nt = min(kTile, T - t0);
         __syncthreads();  // the previous tile's readers are done
         for (int e = tid; e < nt * Dk; e += kThreads) {
-            qs[e] = q[sq + static_cast<size_t>(t0) * Dk + e];
-            ks[e] = k[sq + static_cast<size_t>(t0) * Dk + e];
+            qs[e] = qscale * feature(q[sq + static_cast<size_t>(t0) * Dk + e], fmap);
+            ks[e] = feature(k[sq + static_cast<size_t>(t0) * Dk + e], fmap);
         }
         for (int e = tid; e < nt * Dv; e += kThreads) vs[e] = v[sv + static_cast<size_t>(t0) * Dv + e];
         for (int j = tid; j < nt; j += kThreads)
@@ -115,7 +120,7 @@ cudaError_t launch_fwd_f32(const FwdArgs& a) {
     fwd_f32_kernel<<<a.B * a.H, kThreads, smem, a.stream>>>(
         static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
         a.decay_kind, a.log_g, a.normalize, a.init_state, a.init_z, static_cast<float*>(a.out),
-        a.final_state, a.final_z, a.H, a.T, a.Dk, a.Dv, a.reverse, a.accumulate);
+        a.final_state, a.final_z, a.H, a.T, a.Dk, a.Dv, a.reverse, a.accumulate, a.feature_map, a.q_scale);
     return cudaGetLastError();
 }
 

@@ -236,6 +236,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     p.err = a.err_word;
     p.reverse = a.reverse;
     p.accumulate = a.accumulate;
+    p.q_scale = a.q_scale;
     p.pdl = kPdlFirst;
     if (L.nS > 0) {
         float* base = static_cast<float*>(a.workspace);

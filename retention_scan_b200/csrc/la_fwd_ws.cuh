@@ -228,6 +228,8 @@ struct Params {
     // instances carry no reverse-scan code); this field selects the instance.
     int reverse;
     int accumulate;      // reverse instances only: add y to the values already in out (fp32 add)
+    float q_scale;       // the output of an unnormalised scan is linear in q: y *= q_scale
+                         // (the normalised output does not depend on the scale of q)
     int pdl;             // (host) launch with programmatic stream serialisation
 };
 
@@ -883,7 +885,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             tmem_wait_ld();
             inv = 1.f / (dd[0] + dd[1]);
         } else {
-            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
+            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] * p.q_scale;
         }
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
@@ -1051,7 +1053,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             tmem_wait_ld();
             inv = 1.f / (dd[0] + dd[1]);
         } else {
-            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t];
+            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] * p.q_scale;
         }
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed

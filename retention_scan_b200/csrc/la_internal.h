@@ -41,6 +41,8 @@ struct FwdArgs {
     size_t workspace_bytes;
     int reverse;              // 1: anti-causal scan, t = T-1 down to 0
     int accumulate;           // 1: add y to the values already in out
+    int feature_map;          // la_feature_map on q and k (fp32 path only)
+    float q_scale;            // q <- q_scale * phi(q)
 };
 
 struct DecodeArgs {
@@ -54,6 +56,8 @@ struct DecodeArgs {
     float* z;
     void* out;
     int B, H, Dk, Dv;
+    int feature_map;          // la_feature_map on q and k
+    float q_scale;            // q <- q_scale * phi(q)
     cudaStream_t stream;
 };
 

@@ -320,3 +320,25 @@ def test_wkv4_workspace_size(L):
     vp = ctypes.c_void_p
     assert L.la_wkv4_forward_ws(vp(16), vp(16), vp(4), vp(4), None, vp(16), None, 1, 4, 8, 1, vp(24), 64,
                                 None) == 1  # misaligned workspace
+
+
+def test_prologue_validation(L):
+    vp = ctypes.c_void_p
+
+    def fwd(pro, dtype=1):
+        return L.la_chunk_forward_pro_ws(vp(16), vp(16), vp(16), None, 0, ctypes.byref(pro) if pro else None,
+                                         None, None, vp(16), None, None, 1, 1, 4, 16, 16, dtype, None, 0, None)
+
+    def dec(pro):
+        return L.la_decode_step_pro(vp(16), vp(16), vp(16), None, 0, ctypes.byref(pro), vp(16), None, vp(16),
+                                    1, 1, 16, 16, 1, None)
+    P = la._Prologue
+    assert fwd(P(2, 1.0)) == 1                   # feature map out of range
+    assert fwd(P(0, float("inf"))) == 1          # q scale not finite
+    assert fwd(P(0, float("nan"))) == 1
+    assert fwd(P(1, 1.0)) == 2                   # bf16 tensor-core path: no feature map
+    assert dec(P(-1, 1.0)) == 1
+    assert dec(P(0, float("inf"))) == 1
+    # B = 0 with valid prologues: no-ops (the fp32 path takes the feature map)
+    assert L.la_chunk_forward_pro_ws(None, None, None, None, 0, ctypes.byref(P(1, 0.5)), None, None, None, None,
+                                     None, 0, 1, 4, 16, 16, 0, None, 0, None) == 0
