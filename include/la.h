@@ -302,8 +302,7 @@ LA_API size_t la_chunk_backward_workspace_size(int B, int H, int T, int Dk, int 
  * Errors: as la_chunk_forward_ws, plus LA_ERR_INVALID_ARG for a NULL
  * required pointer (dy, dq, dk, dv, workspace), a workspace smaller than
  * la_chunk_backward_workspace_size or misaligned, or d_log_g given without a
- * decay.  The normalised forward has no backward here (the function has no
- * normalize argument).
+ * decay.  The normalised forward's backward is la_chunk_backward_norm_ws.
  */
 LA_API la_status la_chunk_backward_ws(const void* q, const void* k, const void* v,
                                const la_decay* decay, const float* init_state,
@@ -419,6 +418,49 @@ LA_API la_status la_wkv4_forward_ws(const void* k, const void* v, const float* w
                                     const float* init_state, void* out, float* final_state,
                                     int B, int T, int C, la_dtype dtype, void* workspace,
                                     size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * la_chunk_backward_norm_workspace_size - scratch bytes that
+ * la_chunk_backward_norm_ws needs (always > 0 for B*H > 0 and T > 0).
+ */
+LA_API size_t la_chunk_backward_norm_workspace_size(int B, int H, int T, int Dk, int Dv,
+                                                    la_dtype dtype, int decay_kind);
+
+/*
+ * la_chunk_backward_norm_ws - gradients of the normalised forward pass
+ * (normalize = 1): y_t = n_t / den_t with n_t = S_t^T q_t, den_t = q_t . z_t,
+ * for L = sum_t dy_t . y_t + <d_final_state, S_T> + <d_final_z, z_T>.
+ *
+ * With dn_t = dy_t / den_t and dden_t = -(dy_t . n_t) / den_t^2:
+ *   dq_t = S_t dn_t + dden_t z_t
+ *   dS_t = q_t dn_t^T + g_{t+1} dS_{t+1}     dz_t = dden_t q_t + g_{t+1} dz_{t+1}
+ *   dk_t = dS_t v_t + dz_t                   dv_t = dS_t^T k_t
+ *   d_init_state = g_1 dS_1,  d_init_z = g_1 dz_1
+ *   d log g_t = sum_{s >= t} (q_s . dq_s - k_s . dk_s) + <d_final_state, S_T>
+ *               + <d_final_z, z_T>
+ * All of it runs on the scan kernels, as in la_chunk_backward_ws: the
+ * numerator and the denominator are recomputed by two forward scans (the
+ * denominator as the scan of a 16-wide value panel whose first column is 1,
+ * so that its state's first column is z_t), dn and dden by a small kernel,
+ * and the key-sum terms dden_t z_t and dz_t by scans of 16-wide panels (the
+ * second adds into dk); dq's two parts are added by a small kernel.
+ *
+ *   init_z         NULL (zeros) or z_0 [B,H,Dk] fp32; required with init_state.
+ *   d_final_z      NULL (zeros) or dL/dz_T [B,H,Dk] fp32.
+ *   d_init_z       NULL (not written) or [B,H,Dk] fp32: dL/dz_0.
+ *   workspace      at least la_chunk_backward_norm_workspace_size(...) bytes.
+ *   other arguments as la_chunk_backward_ws.
+ *
+ * Errors as la_chunk_backward_ws, plus LA_ERR_INVALID_ARG for init_state
+ * without init_z.
+ */
+LA_API la_status la_chunk_backward_norm_ws(const void* q, const void* k, const void* v,
+                                    const la_decay* decay, const float* init_state, const float* init_z,
+                                    const void* dy, const float* d_final_state, const float* d_final_z,
+                                    void* dq, void* dk, void* dv, float* d_log_g,
+                                    float* d_init_state, float* d_init_z,
+                                    int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                                    void* workspace, size_t workspace_bytes, la_stream_t stream);
 
 /*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed

@@ -13,7 +13,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "wkv4_forward", "workspace_size",
+__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "chunk_backward_normalized", "wkv4_forward",
+           "workspace_size",
            "backward_workspace_size",
            "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "FEATURE_NONE", "FEATURE_ELU1", "EXPORTED_SYMBOLS"]
@@ -28,7 +29,7 @@ EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward
                     "la_chunk_reverse_ws", "la_chunk_bidirectional_ws",
                     "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
                     "la_wkv4_forward_ws", "la_wkv4_workspace_size", "la_chunk_forward_pro_ws",
-                    "la_decode_step_pro",
+                    "la_decode_step_pro", "la_chunk_backward_norm_ws", "la_chunk_backward_norm_workspace_size",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -80,6 +81,11 @@ def lib():
         L.la_chunk_backward_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), vp, vp, vp, vp, vp, vp, vp, vp,
                                            i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
         L.la_chunk_backward_ws.restype = i
+        L.la_chunk_backward_norm_ws.argtypes = [vp, vp, vp, ctypes.POINTER(_Decay), vp, vp, vp, vp, vp, vp, vp, vp,
+                                                vp, vp, vp, i, i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        L.la_chunk_backward_norm_ws.restype = i
+        L.la_chunk_backward_norm_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        L.la_chunk_backward_norm_workspace_size.restype = ctypes.c_size_t
         L.la_chunk_backward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
         L.la_wkv4_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -366,6 +372,51 @@ def wkv4_forward(k, v, w, u, init_state=None, out=None, final_state=None, return
                                         _ptr(final_state), B, T, C, code, _ptr(workspace),
                                         0 if workspace is None else workspace.numel(), _stream(stream, dev)))
     return out, final_state
+
+
+def chunk_backward_normalized(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=None, init_z=None,
+                              d_final_state=None, d_final_z=None, need_log_g=True, need_init_state=True,
+                              stream=None, workspace=None):
+    """Gradients of the normalised forward (la_chunk_backward_norm_ws) for the
+    loss sum(dy * y) + sum(d_final_state * final_state) + sum(d_final_z *
+    final_z).  Arguments as chunk_backward, plus init_z / d_final_z [B,H,Dk]
+    fp32 (init_z is required with init_state).  Returns (dq, dk, dv,
+    d_log_g, d_init_state, d_init_z)."""
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q.dtype)
+    _need(k, "k", (B, H, T, Dk), q.dtype, dev)
+    _need(v, "v", (B, H, T, Dv), q.dtype, dev)
+    _need(dy, "dy", (B, H, T, Dv), q.dtype, dev)
+    _need(q, "q", (B, H, T, Dk), q.dtype, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H, T), torch.float32, dev)
+    _need(init_state, "init_state", (B, H, Dk, Dv), torch.float32, dev)
+    _need(init_z, "init_z", (B, H, Dk), torch.float32, dev)
+    _need(d_final_state, "d_final_state", (B, H, Dk, Dv), torch.float32, dev)
+    _need(d_final_z, "d_final_z", (B, H, Dk), torch.float32, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    d_log_g = torch.empty_like(log_g) if (decay_kind != DECAY_NONE and need_log_g) else None
+    d_init = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev) if need_init_state else None
+    d_init_z = torch.empty((B, H, Dk), dtype=torch.float32, device=dev) if need_init_state else None
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        nbytes = int(lib().la_chunk_backward_norm_workspace_size(B, H, T, Dk, Dv, code, int(decay_kind)))
+        if workspace is None:
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+            if stream is not None:
+                workspace.record_stream(stream)
+        elif workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise ValueError("workspace: expected a contiguous uint8 tensor on the inputs' device")
+        _check(lib().la_chunk_backward_norm_ws(
+            _ptr(q), _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, _ptr(init_state), _ptr(init_z),
+            _ptr(dy), _ptr(d_final_state), _ptr(d_final_z), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_log_g),
+            _ptr(d_init), _ptr(d_init_z), B, H, T, Dk, Dv, code, _ptr(workspace), workspace.numel(),
+            _stream(stream, dev)))
+    return dq, dk, dv, d_log_g, d_init, d_init_z
 
 
 def decode_step(q, k, v, state, z=None, decay_kind=DECAY_NONE, log_g=None, normalize=False,

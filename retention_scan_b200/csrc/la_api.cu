@@ -184,6 +184,101 @@ BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int ki
     return L;
 }
 
+// Scratch of the normalised backward: the unnormalised backward's regions,
+// then the key-sum panels (fp32: z_0 as a [Dk][16] and a [16][Dk] panel,
+// d_final_z as [16][Dk], the recomputed z_T as [Dk][16], dz_1 as [16][Dk])
+// and the per-token arrays (`dtype`): the ones panel, the denominator panel,
+// the numerator n, dn, the dden panel and the key-sum part of dq.
+struct NormLayout {
+    BwdLayout base;
+    size_t z0p, z0t, dzft, ztp, dz1p, ones, denp, num, dn, ddp, dq2, scan, scan_bytes, total;
+};
+
+NormLayout norm_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind) {
+    NormLayout L{};
+    L.base = bwd_layout(B, H, T, Dk, Dv, dtype, kind);
+    const size_t BH = static_cast<size_t>(B) * H, es = dtype == LA_BF16 ? 2 : 4;
+    const size_t panel = round256(sizeof(float) * BH * Dk * 16);
+    const size_t tok16 = round256(es * BH * T * 16);
+    L.z0p = L.base.scan;  // after the unnormalised regions (whose own scan area moves to the end)
+    L.z0t = L.z0p + panel;
+    L.dzft = L.z0t + panel;
+    L.ztp = L.dzft + panel;
+    L.dz1p = L.ztp + panel;
+    L.ones = L.dz1p + panel;
+    L.denp = L.ones + tok16;
+    L.num = L.denp + tok16;
+    L.dn = L.num + round256(es * BH * T * Dv);
+    L.ddp = L.dn + round256(es * BH * T * Dv);
+    L.dq2 = L.ddp + tok16;
+    L.scan = L.dq2 + round256(es * BH * T * Dk);
+    L.scan_bytes = 0;
+    if (dtype == LA_BF16) {
+        const int dims[6][2] = {{Dk, Dv}, {Dk, 16}, {Dv, Dk}, {16, Dk}, {Dk, Dv}, {Dv, Dk}};
+        for (const auto& d : dims) {
+            const size_t b = la::fwd_tc_workspace_bytes(B, H, T, d[0], d[1], false);
+            if (b > L.scan_bytes) L.scan_bytes = b;
+        }
+        L.scan_bytes = round256(L.scan_bytes);
+    }
+    L.total = L.scan + L.scan_bytes;
+    return L;
+}
+
+// The normalised backward with the value panel [v | 1 | 0] (W = a supported
+// width > Dv): one scan gives [n | den], and dq, dk each come from one scan
+// of [dn | dden | 0] against it, so that the cancellation between the
+// numerator's and the denominator's terms happens inside the scores (fp32)
+// instead of between two rounded outputs.  Regions (256-aligned): the
+// unnormalised layout's shifted decay and decay-gradient scratch, then fp32
+// state panels [S_0 | z_0], its transpose, [dSf | dzf], its transpose, the
+// final state of the first scan and of the dk scan, then per-token arrays
+// (`dtype`): the value panel, [n | den], [dn | dden], dn, and the scans'
+// T-segment workspace.
+int panel_width(int Dv, la_dtype dtype) {
+    if (dtype == LA_F32) return Dv + 1 <= 128 ? Dv + 1 : 0;
+    for (int w : {32, 64, 128})
+        if (w > Dv) return w;
+    return 0;
+}
+
+struct PanelLayout {
+    BwdLayout base;
+    int W;
+    size_t ainit, binit, dpan, cinit, f1, f4, pk, nd, pq, dn, scan, scan_bytes, total;
+};
+
+PanelLayout panel_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind) {
+    PanelLayout L{};
+    L.base = bwd_layout(B, H, T, Dk, Dv, dtype, kind);
+    L.W = panel_width(Dv, dtype);
+    const size_t BH = static_cast<size_t>(B) * H, es = dtype == LA_BF16 ? 2 : 4, W = L.W;
+    const size_t sp = round256(sizeof(float) * BH * Dk * W);
+    const size_t tw = round256(es * BH * T * W);
+    L.ainit = L.base.scan;
+    L.binit = L.ainit + sp;
+    L.dpan = L.binit + sp;
+    L.cinit = L.dpan + sp;
+    L.f1 = L.cinit + sp;
+    L.f4 = L.f1 + sp;
+    L.pk = L.f4 + sp;
+    L.nd = L.pk + tw;
+    L.pq = L.nd + tw;
+    L.dn = L.pq + tw;
+    L.scan = L.dn + round256(es * BH * T * Dv);
+    L.scan_bytes = 0;
+    if (dtype == LA_BF16) {
+        const int dims[4][2] = {{Dk, L.W}, {L.W, Dk}, {Dk, Dv}, {Dv, Dk}};
+        for (const auto& d : dims) {
+            const size_t b = la::fwd_tc_workspace_bytes(B, H, T, d[0], d[1], false);
+            if (b > L.scan_bytes) L.scan_bytes = b;
+        }
+        L.scan_bytes = round256(L.scan_bytes);
+    }
+    L.total = L.scan + L.scan_bytes;
+    return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -339,7 +434,10 @@ la_status la_chunk_backward_ws(const void* q, const void* k, const void* v, cons
         a.dq = dq;
         a.dk = dk;
         a.d_final_state = d_final_state;
-        a.final_state_t = st;
+        a.st = st;  // S_T^T [Dv][Dk]
+        a.st_bh = static_cast<long long>(Dk) * Dv;
+        a.st_i = 1;
+        a.st_j = Dk;
         a.d_log_g = d_log_g;
         a.kind = kind;
         a.B = B;
@@ -359,6 +457,234 @@ size_t la_wkv4_workspace_size(int B, int T, int C, la_dtype dtype) {
     if ((dtype != LA_F32 && dtype != LA_BF16) || B < 1 || T < 1 || C < 1 || B > 65535) return 0;
     if (!fits_int(static_cast<long long>(T) * C) || !fits_int(3LL * B * C)) return 0;
     return la::wkv4_workspace_bytes(B, T, C, dtype);
+}
+
+size_t la_chunk_backward_norm_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int decay_kind) {
+    if ((dtype != LA_F32 && dtype != LA_BF16) || B < 1 || H < 1 || T < 1 || Dk < 1 || Dv < 1) return 0;
+    if (decay_kind < LA_DECAY_NONE || decay_kind > LA_DECAY_PER_STEP) return 0;
+    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
+    if (panel_width(Dv, dtype)) return panel_layout(B, H, T, Dk, Dv, dtype, decay_kind).total;
+    return norm_layout(B, H, T, Dk, Dv, dtype, decay_kind).total;
+}
+
+// The normalised forward's gradients by scans: n and the denominator are
+// recomputed (the denominator as the scan of a ones value panel), then
+// dn = dy / den and dden = -(dy . n) / den^2 feed the scans of the
+// unnormalised backward plus two 16-wide panel scans for the key-sum path.
+la_status la_chunk_backward_norm_ws(const void* q, const void* k, const void* v, const la_decay* decay,
+                                    const float* init_state, const float* init_z, const void* dy,
+                                    const float* d_final_state, const float* d_final_z, void* dq, void* dk, void* dv,
+                                    float* d_log_g, float* d_init_state, float* d_init_z, int B, int H, int T, int Dk,
+                                    int Dv, la_dtype dtype, void* workspace, size_t workspace_bytes,
+                                    la_stream_t stream) {
+    if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    int kind;
+    const float* log_g;
+    if (check_decay(decay, &kind, &log_g) != LA_OK) return LA_ERR_INVALID_ARG;
+    if (d_log_g && (kind == LA_DECAY_NONE || !aligned4(d_log_g))) return LA_ERR_INVALID_ARG;
+    if (init_state && !init_z) return LA_ERR_INVALID_ARG;  // a carried state needs its key sum
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH * 8) || BH > 65535) return BH > 65535 ? LA_ERR_UNSUPPORTED : LA_ERR_INVALID_ARG;
+    for (const void* p : {static_cast<const void*>(init_state), static_cast<const void*>(init_z),
+                          static_cast<const void*>(d_final_state), static_cast<const void*>(d_final_z),
+                          static_cast<const void*>(d_init_state), static_cast<const void*>(d_init_z)})
+        if (p && !aligned16(p)) return LA_ERR_INVALID_ARG;
+    const bool work = BH > 0 && T > 0;
+    if (work) {
+        for (const void* p : {q, k, v, dy, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                              static_cast<const void*>(dv), static_cast<const void*>(workspace)})
+            if (!p || !aligned16(p)) return LA_ERR_INVALID_ARG;
+    }
+    if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
+    if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
+    if (work && (T + 255) / 256 > 65535) return LA_ERR_UNSUPPORTED;
+    const int W = panel_width(Dv, dtype);
+    const NormLayout L = work && !W ? norm_layout(B, H, T, Dk, Dv, dtype, kind) : NormLayout{};
+    const PanelLayout LP = work && W ? panel_layout(B, H, T, Dk, Dv, dtype, kind) : PanelLayout{};
+    if (work && workspace_bytes < (W ? LP.total : L.total)) return LA_ERR_INVALID_ARG;
+    if (BH == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t sbytes = sizeof(float) * static_cast<size_t>(BH) * Dk * Dv;
+    const size_t zbytes = sizeof(float) * static_cast<size_t>(BH) * Dk;
+
+    if (T == 0) {  // the state and key-sum gradients pass through
+        cudaError_t e = cudaSuccess;
+        if (d_init_state)
+            e = d_final_state ? cudaMemcpyAsync(d_init_state, d_final_state, sbytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(d_init_state, 0, sbytes, s);
+        if (e == cudaSuccess && d_init_z)
+            e = d_final_z ? cudaMemcpyAsync(d_init_z, d_final_z, zbytes, cudaMemcpyDeviceToDevice, s)
+                          : cudaMemsetAsync(d_init_z, 0, zbytes, s);
+        if (e == cudaSuccess && d_log_g && kind == LA_DECAY_PER_HEAD)
+            e = cudaMemsetAsync(d_log_g, 0, sizeof(float) * H, s);
+        return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    }
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto at = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    const int bh = static_cast<int>(BH);
+    const long long ntok = BH * T;
+    la_status r;
+#define LA_SCAN(...)                      \
+    do {                                  \
+        r = scan(__VA_ARGS__);            \
+        if (r != LA_OK) return r;         \
+    } while (0)
+    if (W) {
+        float* lsh = kind != LA_DECAY_NONE ? at(LP.base.lsh) : nullptr;
+        const bool has_init = init_state || init_z, has_final = d_final_state || d_final_z;
+        float* ainit = has_init ? at(LP.ainit) : nullptr;
+        float* binit = has_init ? at(LP.binit) : nullptr;
+        float* cinit = has_final ? at(LP.cinit) : nullptr;
+        float* f1 = (d_log_g && has_final) ? at(LP.f1) : nullptr;
+        float* f4 = d_init_z ? at(LP.f4) : nullptr;
+        void* pk = ws + LP.pk;
+        void* nd = ws + LP.nd;
+        void* pq = ws + LP.pq;
+        void* dn = ws + LP.dn;
+        void* scan_ws = LP.scan_bytes ? ws + LP.scan : nullptr;
+        const size_t sw = LP.scan_bytes;
+        if (lsh && !ok(la::launch_shift_decay(log_g, kind, lsh, B, H, T, s))) return LA_ERR_CUDA;
+        if (ainit && (!ok(la::launch_pack_state_panel(init_state, init_z, ainit, bh, Dk, Dv, W, s)) ||
+                      !ok(la::launch_transpose(ainit, binit, bh, Dk, W, s))))
+            return LA_ERR_CUDA;
+        if (cinit && (!ok(la::launch_pack_state_panel(d_final_state, d_final_z, at(LP.dpan), bh, Dk, Dv, W, s)) ||
+                      !ok(la::launch_transpose(at(LP.dpan), cinit, bh, Dk, W, s))))
+            return LA_ERR_CUDA;
+        if (!ok(la::launch_pack_value_panel(v, pk, Dv, W, ntok, dtype, s))) return LA_ERR_CUDA;
+        const la_decay shifted{LA_DECAY_PER_STEP, lsh};
+        const la_decay* rdecay = lsh ? &shifted : nullptr;
+        // [n | den] = q^T [S | z] by one scan of the value panel [v | 1]
+        LA_SCAN(q, k, pk, decay, 0, ainit, nullptr, nd, f1, nullptr, B, H, T, Dk, W, dtype, scan_ws, sw, stream, 0,
+                0);
+        if (!ok(la::launch_norm_grad_panel(dy, nd, pq, dn, Dv, W, ntok, dtype, s))) return LA_ERR_CUDA;
+        // dq_t = [S_t | z_t] [dn_t; dden_t]: scores [dn | dden] . [v | 1]
+        LA_SCAN(pq, pk, k, decay, 0, binit, nullptr, dq, nullptr, nullptr, B, H, T, W, Dk, dtype, scan_ws, sw,
+                stream, 0, 0);
+        // dk_t = [dS_t^T; dz_t^T]^T [v_t; 1]: the reverse scan of ([v | 1], [dn | dden], q)
+        LA_SCAN(pk, pq, q, rdecay, 0, cinit, nullptr, dk, f4, nullptr, B, H, T, W, Dk, dtype, scan_ws, sw, stream,
+                1, 0);
+        LA_SCAN(k, q, dn, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype,
+                scan_ws, sw, stream, 1, 0);
+        if (d_init_state && kind != LA_DECAY_NONE &&
+            !ok(la::launch_scale_by_first_decay(d_init_state, log_g, kind, B, H, T, Dk * Dv, s)))
+            return LA_ERR_CUDA;
+        if (f4 && !ok(la::launch_panel_row_scaled(f4, d_init_z, log_g, kind, B, H, T, Dk, W, Dv, s)))
+            return LA_ERR_CUDA;
+        if (d_log_g) {
+            la::DlogArgs a{};
+            a.q = q;
+            a.k = k;
+            a.dq = dq;
+            a.dk = dk;
+            a.d_final_state = d_final_state;
+            a.st = f1;  // [S_T | z_T | 0] as [Dk][W]
+            a.st_bh = static_cast<long long>(Dk) * W;
+            a.st_i = W;
+            a.st_j = 1;
+            a.d_final_z = d_final_z;
+            a.zt = f1 ? f1 + Dv : nullptr;
+            a.zt_bh = static_cast<long long>(Dk) * W;
+            a.zt_i = W;
+            a.d_log_g = d_log_g;
+            a.kind = kind;
+            a.B = B;
+            a.H = H;
+            a.T = T;
+            a.Dk = Dk;
+            a.Dv = Dv;
+            a.dtype = dtype;
+            a.scratch = reinterpret_cast<double*>(ws + LP.base.dlog);
+            a.stream = s;
+            if (!ok(la::launch_dlog(a))) return LA_ERR_CUDA;
+        }
+        return LA_OK;
+    }
+    // Dv + 1 above the widest panel: the numerator's and the denominator's
+    // terms of dq and dk come from separate scans and are added
+    float* s0t = init_state ? at(L.base.s0t) : nullptr;
+    float* dsft = d_final_state ? at(L.base.dsft) : nullptr;
+    const bool need_st = d_log_g && d_final_state;
+    float* st = need_st ? at(L.base.st) : nullptr;
+    float* lsh = kind != LA_DECAY_NONE ? at(L.base.lsh) : nullptr;
+    float* z0p = init_z ? at(L.z0p) : nullptr;
+    float* z0t = init_z ? at(L.z0t) : nullptr;
+    float* dzft = d_final_z ? at(L.dzft) : nullptr;
+    float* ztp = (d_log_g && d_final_z) ? at(L.ztp) : nullptr;
+    float* dz1p = d_init_z ? at(L.dz1p) : nullptr;
+    void* ones = ws + L.ones;
+    void* denp = ws + L.denp;
+    void* num = ws + L.num;
+    void* dn = ws + L.dn;
+    void* ddp = ws + L.ddp;
+    void* dq2 = ws + L.dq2;
+    void* scan_ws = L.scan_bytes ? ws + L.scan : nullptr;
+    const size_t sw = L.scan_bytes;
+
+    if (s0t && !ok(la::launch_transpose(init_state, s0t, bh, Dk, Dv, s))) return LA_ERR_CUDA;
+    if (dsft && !ok(la::launch_transpose(d_final_state, dsft, bh, Dk, Dv, s))) return LA_ERR_CUDA;
+    if (lsh && !ok(la::launch_shift_decay(log_g, kind, lsh, B, H, T, s))) return LA_ERR_CUDA;
+    if (z0p && !ok(la::launch_vec_panel(init_z, z0p, bh, Dk, true, s))) return LA_ERR_CUDA;
+    if (z0t && !ok(la::launch_vec_panel(init_z, z0t, bh, Dk, false, s))) return LA_ERR_CUDA;
+    if (dzft && !ok(la::launch_vec_panel(d_final_z, dzft, bh, Dk, false, s))) return LA_ERR_CUDA;
+    if (!ok(la::launch_ones_panel(ones, ntok, dtype, s))) return LA_ERR_CUDA;
+    const la_decay shifted{LA_DECAY_PER_STEP, lsh};
+    const la_decay* rdecay = lsh ? &shifted : nullptr;
+    // numerator n_t = q_t^T S_t and denominator q_t . z_t (ones value panel, column 0)
+    LA_SCAN(q, k, v, decay, 0, init_state, nullptr, num, nullptr, nullptr, B, H, T, Dk, Dv, dtype, scan_ws, sw,
+            stream, 0, 0);
+    LA_SCAN(q, k, ones, decay, 0, z0p, nullptr, denp, ztp, nullptr, B, H, T, Dk, 16, dtype, scan_ws, sw, stream, 0,
+            0);
+    if (!ok(la::launch_norm_grad(dy, num, denp, dn, ddp, Dv, ntok, dtype, s))) return LA_ERR_CUDA;
+    // dq = S_t dn_t + dden_t z_t
+    LA_SCAN(dn, v, k, decay, 0, s0t, nullptr, dq, st, nullptr, B, H, T, Dv, Dk, dtype, scan_ws, sw, stream, 0, 0);
+    LA_SCAN(ddp, ones, k, decay, 0, z0t, nullptr, dq2, nullptr, nullptr, B, H, T, 16, Dk, dtype, scan_ws, sw,
+            stream, 0, 0);
+    if (!ok(la::launch_add_into(dq, dq2, ntok * Dk, dtype, s))) return LA_ERR_CUDA;
+    // dk = dS_t v_t + dz_t (the second scan adds into dk), dv = dS_t^T k_t
+    LA_SCAN(v, dn, q, rdecay, 0, dsft, nullptr, dk, nullptr, nullptr, B, H, T, Dv, Dk, dtype, scan_ws, sw, stream,
+            1, 0);
+    LA_SCAN(ones, ddp, q, rdecay, 0, dzft, nullptr, dk, dz1p, nullptr, B, H, T, 16, Dk, dtype, scan_ws, sw, stream,
+            1, 1);
+    LA_SCAN(k, q, dn, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype, scan_ws,
+            sw, stream, 1, 0);
+#undef LA_SCAN
+    if (d_init_state && kind != LA_DECAY_NONE &&
+        !ok(la::launch_scale_by_first_decay(d_init_state, log_g, kind, B, H, T, Dk * Dv, s)))
+        return LA_ERR_CUDA;
+    if (dz1p && !ok(la::launch_panel_row_scaled(dz1p, d_init_z, log_g, kind, B, H, T, Dk, 16, 0, s)))
+        return LA_ERR_CUDA;
+    if (d_log_g) {
+        la::DlogArgs a{};
+        a.q = q;
+        a.k = k;
+        a.dq = dq;
+        a.dk = dk;
+        a.d_final_state = d_final_state;
+        a.st = st;  // S_T^T [Dv][Dk]
+        a.st_bh = static_cast<long long>(Dk) * Dv;
+        a.st_i = 1;
+        a.st_j = Dk;
+        a.d_final_z = d_final_z;
+        a.zt = ztp;  // column 0 of [Dk][16]
+        a.zt_bh = 16LL * Dk;
+        a.zt_i = 16;
+        a.d_log_g = d_log_g;
+        a.kind = kind;
+        a.B = B;
+        a.H = H;
+        a.T = T;
+        a.Dk = Dk;
+        a.Dv = Dv;
+        a.dtype = dtype;
+        a.scratch = reinterpret_cast<double*>(ws + L.base.dlog);
+        a.stream = s;
+        if (!ok(la::launch_dlog(a))) return LA_ERR_CUDA;
+    }
+    return LA_OK;
 }
 
 la_status la_wkv4_forward(const void* k, const void* v, const float* w, const float* u, const float* init_state,

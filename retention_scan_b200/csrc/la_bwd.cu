@@ -72,16 +72,24 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
     return __bfloat162float(x);
 }
 
-// <dSf, S_T> per (b, h), with S_T given transposed; one block per (b, h).
-__global__ void terminal_kernel(const float* __restrict__ dsf, const float* __restrict__ st_t, double* __restrict__ out,
-                                int Dk, int Dv) {
+// <dSf, S_T> (+ <dzf, z_T>) per (b, h); S_T[i][j] at st[bh * st_bh + i * st_i
+// + j * st_j], z_T[i] at zt[bh * zt_bh + i * zt_i]; one block per (b, h).
+__global__ void terminal_kernel(const float* __restrict__ dsf, const float* __restrict__ st, long long st_bh,
+                                int st_i, int st_j, const float* __restrict__ dzf, const float* __restrict__ zt,
+                                long long zt_bh, int zt_i, double* __restrict__ out, int Dk, int Dv) {
     const int bh = blockIdx.x;
     const size_t base = static_cast<size_t>(bh) * Dk * Dv;
     double acc = 0.0;
-    for (int e = threadIdx.x; e < Dk * Dv; e += blockDim.x) {
-        const int i = e / Dv, j = e % Dv;
-        acc += static_cast<double>(dsf[base + e]) * st_t[base + static_cast<size_t>(j) * Dk + i];
-    }
+    if (dsf)
+        for (int e = threadIdx.x; e < Dk * Dv; e += blockDim.x) {
+            const int i = e / Dv, j = e % Dv;
+            acc += static_cast<double>(dsf[base + e]) *
+                   st[bh * st_bh + static_cast<long long>(i) * st_i + static_cast<long long>(j) * st_j];
+        }
+    if (dzf)
+        for (int i = threadIdx.x; i < Dk; i += blockDim.x)
+            acc += static_cast<double>(dzf[static_cast<size_t>(bh) * Dk + i]) *
+                   zt[bh * zt_bh + static_cast<long long>(i) * zt_i];
     __shared__ double red[256];
     red[threadIdx.x] = acc;
     __syncthreads();
@@ -193,7 +201,212 @@ __global__ void dlog_head_kernel(float* __restrict__ out, int B, int H, int nblk
     if (threadIdx.x == 0) out[h] = static_cast<float>(red[0]);
 }
 
+// [n][16] panel with column 0 = 1 and the rest 0 (the value panel whose scan
+// gives the key sum: S = sum k 1^T, so q^T S = q . z in column 0).
+template <typename E>
+__global__ void ones_panel_kernel(E* __restrict__ out, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n * 16;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        out[i] = static_cast<E>((i & 15) == 0 ? 1.f : 0.f);
+}
+
+// Per (b, h): the Dk vector x into column 0 of a [Dk][16] panel (rows) or
+// row 0 of a [16][Dk] panel (cols), zeros elsewhere, fp32.
+__global__ void vec_panel_kernel(const float* __restrict__ x, float* __restrict__ out, int Dk, int rows,
+                                 long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long bh = i / (16LL * Dk);
+        const int e = static_cast<int>(i - bh * 16LL * Dk);
+        float val = 0.f;
+        if (x) {
+            if (rows && (e & 15) == 0) val = x[bh * Dk + e / 16];
+            if (!rows && e < Dk) val = x[bh * Dk + e];
+        }
+        out[i] = val;
+    }
+}
+
+// Normalised output y = n / den: per token, dn = dy / den and
+// dden = -(dy . n) / den^2 (the latter as column 0 of a 16-wide panel).
+// One warp per token.
+template <typename E>
+__global__ void norm_grad_kernel(const E* __restrict__ dy, const E* __restrict__ num,
+                                 const E* __restrict__ den_panel, E* __restrict__ dn, E* __restrict__ dden_panel,
+                                 int Dv, long long ntok) {
+    const int lane = threadIdx.x % 32;
+    const long long w0 = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
+    const long long nw = static_cast<long long>(gridDim.x) * blockDim.x / 32;
+    for (long long t = w0; t < ntok; t += nw) {
+        const float den = to_f(den_panel[t * 16]);
+        const float inv = 1.f / den;
+        const size_t row = static_cast<size_t>(t) * Dv;
+        float dot = 0.f;
+        for (int c = lane; c < Dv; c += 32) {
+            const float g = to_f(dy[row + c]);
+            dot = fmaf(g, to_f(num[row + c]), dot);
+            dn[row + c] = static_cast<E>(g * inv);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane < 16) dden_panel[t * 16 + lane] = static_cast<E>(lane == 0 ? -dot * inv * inv : 0.f);
+    }
+}
+
+// PK[t] = [v_t | 1 | 0 ...], W wide (W > Dv).
+template <typename E>
+__global__ void pack_value_panel_kernel(const E* __restrict__ v, E* __restrict__ pk, int Dv, int W, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n * W;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long t = i / W;
+        const int c = static_cast<int>(i - t * W);
+        pk[i] = c < Dv ? v[t * Dv + c] : static_cast<E>(c == Dv ? 1.f : 0.f);
+    }
+}
+
+// [S | z | 0] as [Dk][W] fp32 per (b, h) (S [Dk][Dv], z [Dk]; null: zeros).
+__global__ void pack_state_panel_kernel(const float* __restrict__ S, const float* __restrict__ z,
+                                        float* __restrict__ out, int Dk, int Dv, int W, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long bhi = i / W;  // bh * Dk + row
+        const int c = static_cast<int>(i - bhi * W);
+        float x = 0.f;
+        if (c < Dv && S) x = S[bhi * Dv + c];
+        if (c == Dv && z) x = z[bhi];
+        out[i] = x;
+    }
+}
+
+// From [n | den | ..] (W wide): PQ[t] = [dn_t | dden_t | 0 ...] (W wide) and
+// dn [t] (Dv wide); dn = dy / den, dden = -(dy . n) / den^2.  One warp per token.
+template <typename E>
+__global__ void norm_grad_panel_kernel(const E* __restrict__ dy, const E* __restrict__ nd, E* __restrict__ pq,
+                                       E* __restrict__ dn, int Dv, int W, long long ntok) {
+    const int lane = threadIdx.x % 32;
+    const long long w0 = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
+    const long long nw = static_cast<long long>(gridDim.x) * blockDim.x / 32;
+    for (long long t = w0; t < ntok; t += nw) {
+        const size_t rw = static_cast<size_t>(t) * W, rv = static_cast<size_t>(t) * Dv;
+        const float inv = 1.f / to_f(nd[rw + Dv]);
+        float dot = 0.f;
+        for (int c = lane; c < Dv; c += 32) {
+            const float g = to_f(dy[rv + c]);
+            dot = fmaf(g, to_f(nd[rw + c]), dot);
+            const E x = static_cast<E>(g * inv);
+            dn[rv + c] = x;
+            pq[rw + c] = x;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        for (int c = Dv + lane; c < W; c += 32) pq[rw + c] = static_cast<E>(c == Dv ? -dot * inv * inv : 0.f);
+    }
+}
+
+template <typename E>
+__global__ void add_into_kernel(E* __restrict__ a, const E* __restrict__ b, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        a[i] = static_cast<E>(to_f(a[i]) + to_f(b[i]));
+}
+
+// out[bh][i] = g_1 * panel[bh * rows * Dk + row * Dk + i] (one row of a
+// [rows][Dk] state panel), g_1 the decay of the sequence's first token (1
+// without a decay).
+__global__ void panel_row_scaled_kernel(const float* __restrict__ panel, float* __restrict__ out,
+                                        const float* __restrict__ lg, int kind, int H, int T, int Dk, int rows,
+                                        int row, long long n) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long bh = i / Dk;
+        const int e = static_cast<int>(i - bh * Dk);
+        float g = 1.f;
+        if (kind == LA_DECAY_PER_STEP) g = expf(lg[bh * T]);
+        if (kind == LA_DECAY_PER_HEAD) g = expf(lg[bh % H]);
+        out[i] = g * panel[(bh * rows + row) * static_cast<long long>(Dk) + e];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_ones_panel(void* out, long long n, la_dtype dtype, cudaStream_t stream) {
+    if (dtype == LA_BF16)
+        ones_panel_kernel<__nv_bfloat16><<<grid_for(n * 16, 256), 256, 0, stream>>>(static_cast<__nv_bfloat16*>(out), n);
+    else
+        ones_panel_kernel<float><<<grid_for(n * 16, 256), 256, 0, stream>>>(static_cast<float*>(out), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_vec_panel(const float* x, float* out, int BH, int Dk, bool rows, cudaStream_t stream) {
+    const long long n = 16LL * BH * Dk;
+    vec_panel_kernel<<<grid_for(n, 256), 256, 0, stream>>>(x, out, Dk, rows ? 1 : 0, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_grad(const void* dy, const void* num, const void* den_panel, void* dn, void* dden_panel,
+                             int Dv, long long ntok, la_dtype dtype, cudaStream_t stream) {
+    const int grid = grid_for(ntok * 32, 256);
+    if (dtype == LA_BF16)
+        norm_grad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(num),
+            static_cast<const __nv_bfloat16*>(den_panel), static_cast<__nv_bfloat16*>(dn),
+            static_cast<__nv_bfloat16*>(dden_panel), Dv, ntok);
+    else
+        norm_grad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dy), static_cast<const float*>(num),
+                                                         static_cast<const float*>(den_panel), static_cast<float*>(dn),
+                                                         static_cast<float*>(dden_panel), Dv, ntok);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_value_panel(const void* v, void* pk, int Dv, int W, long long ntok, la_dtype dtype,
+                                   cudaStream_t stream) {
+    const int grid = grid_for(ntok * W, 256);
+    if (dtype == LA_BF16)
+        pack_value_panel_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v),
+                                                                         static_cast<__nv_bfloat16*>(pk), Dv, W, ntok);
+    else
+        pack_value_panel_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(v), static_cast<float*>(pk),
+                                                                 Dv, W, ntok);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_state_panel(const float* S, const float* z, float* out, int BH, int Dk, int Dv, int W,
+                                    cudaStream_t stream) {
+    const long long n = static_cast<long long>(BH) * Dk * W;
+    pack_state_panel_kernel<<<grid_for(n, 256), 256, 0, stream>>>(S, z, out, Dk, Dv, W, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_grad_panel(const void* dy, const void* nd, void* pq, void* dn, int Dv, int W, long long ntok,
+                                   la_dtype dtype, cudaStream_t stream) {
+    const int grid = grid_for(ntok * 32, 256);
+    if (dtype == LA_BF16)
+        norm_grad_panel_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(nd),
+            static_cast<__nv_bfloat16*>(pq), static_cast<__nv_bfloat16*>(dn), Dv, W, ntok);
+    else
+        norm_grad_panel_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dy),
+                                                               static_cast<const float*>(nd), static_cast<float*>(pq),
+                                                               static_cast<float*>(dn), Dv, W, ntok);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_add_into(void* a, const void* b, long long n, la_dtype dtype, cudaStream_t stream) {
+    if (dtype == LA_BF16)
+        add_into_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), n);
+    else
+        add_into_kernel<float><<<grid_for(n, 256), 256, 0, stream>>>(static_cast<float*>(a),
+                                                                    static_cast<const float*>(b), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_panel_row_scaled(const float* panel, float* out, const float* log_g, int kind, int B, int H,
+                                    int T, int Dk, int rows, int row, cudaStream_t stream) {
+    const long long n = static_cast<long long>(B) * H * Dk;
+    panel_row_scaled_kernel<<<grid_for(n, 256), 256, 0, stream>>>(panel, out, log_g, kind, H, T, Dk, rows, row, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_transpose(const float* in, float* out, int BH, int R, int C, cudaStream_t stream) {
     const dim3 grid((C + 31) / 32, (R + 31) / 32, std::min(BH, 65535));
@@ -224,11 +437,12 @@ cudaError_t launch_dlog(const DlogArgs& a) {
     const int BH = a.B * a.H;
     const int nblk = (a.T + kDlogTokens - 1) / kDlogTokens;
     if (nblk > 65535 || BH > 65535) return cudaErrorInvalidValue;
-    double* terminal = a.d_final_state ? a.scratch : nullptr;
+    double* terminal = (a.d_final_state || a.d_final_z) ? a.scratch : nullptr;
     double* blk_a = a.scratch + BH;
     double* blk_x = blk_a + static_cast<size_t>(BH) * nblk;
     if (terminal) {
-        terminal_kernel<<<BH, 256, 0, a.stream>>>(a.d_final_state, a.final_state_t, terminal, a.Dk, a.Dv);
+        terminal_kernel<<<BH, 256, 0, a.stream>>>(a.d_final_state, a.st, a.st_bh, a.st_i, a.st_j, a.d_final_z, a.zt,
+                                                  a.zt_bh, a.zt_i, terminal, a.Dk, a.Dv);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -96,7 +96,13 @@ struct DlogArgs {
     const void* dq;
     const void* dk;
     const float* d_final_state;   // may be null
-    const float* final_state_t;   // S_T^T [B,H,Dv,Dk]; read when d_final_state is given
+    const float* st;              // S_T[i][j] at st[bh * st_bh + i * st_i + j * st_j] (when d_final_state)
+    long long st_bh;
+    int st_i, st_j;
+    const float* d_final_z;       // may be null (normalised forward only)
+    const float* zt;              // z_T[i] at zt[bh * zt_bh + i * zt_i] (when d_final_z)
+    long long zt_bh;
+    int zt_i;
     float* d_log_g;
     int kind;                     // LA_DECAY_PER_HEAD or LA_DECAY_PER_STEP
     int B, H, T, Dk, Dv;
@@ -106,6 +112,29 @@ struct DlogArgs {
 };
 size_t dlog_scratch_doubles(int B, int H, int T);
 cudaError_t launch_dlog(const DlogArgs& a);
+// Normalised backward helpers (la_bwd.cu):
+//   [n][16] panel, column 0 = 1, the rest 0 (`dtype`)
+cudaError_t launch_ones_panel(void* out, long long n, la_dtype dtype, cudaStream_t stream);
+//   per (b, h) the Dk vector x (null: zeros) into column 0 of [Dk][16]
+//   (rows = true) or row 0 of [16][Dk] (rows = false), fp32
+cudaError_t launch_vec_panel(const float* x, float* out, int BH, int Dk, bool rows, cudaStream_t stream);
+//   dn = dy / den, dden panel column 0 = -(dy . n) / den^2, per token
+cudaError_t launch_norm_grad(const void* dy, const void* num, const void* den_panel, void* dn, void* dden_panel,
+                             int Dv, long long ntok, la_dtype dtype, cudaStream_t stream);
+//   a += b elementwise (`dtype`)
+cudaError_t launch_add_into(void* a, const void* b, long long n, la_dtype dtype, cudaStream_t stream);
+//   out[b,h,:] = g_1 * row `row` of panel [B,H,rows,Dk]
+cudaError_t launch_panel_row_scaled(const float* panel, float* out, const float* log_g, int kind, int B, int H,
+                                    int T, int Dk, int rows, int row, cudaStream_t stream);
+//   PK[t] = [v_t | 1 | 0 ...], W wide (`dtype`)
+cudaError_t launch_pack_value_panel(const void* v, void* pk, int Dv, int W, long long ntok, la_dtype dtype,
+                                    cudaStream_t stream);
+//   [S | z | 0] as [Dk][W] fp32 per (b, h); S, z may be null (zeros)
+cudaError_t launch_pack_state_panel(const float* S, const float* z, float* out, int BH, int Dk, int Dv, int W,
+                                    cudaStream_t stream);
+//   from [n | den | ..] (W wide): PQ = [dn | dden | 0 ..] (W wide) and dn (Dv wide)
+cudaError_t launch_norm_grad_panel(const void* dy, const void* nd, void* pq, void* dn, int Dv, int W, long long ntok,
+                                   la_dtype dtype, cudaStream_t stream);
 
 // RWKV-4 WKV recurrence (la_wkv4.cu).
 struct Wkv4Args {

@@ -342,3 +342,23 @@ def test_prologue_validation(L):
     # B = 0 with valid prologues: no-ops (the fp32 path takes the feature map)
     assert L.la_chunk_forward_pro_ws(None, None, None, None, 0, ctypes.byref(P(1, 0.5)), None, None, None, None,
                                      None, 0, 1, 4, 16, 16, 0, None, 0, None) == 0
+
+
+def test_backward_norm_validation(L):
+    vp = ctypes.c_void_p
+
+    def bn(**over):
+        a = dict(q=16, k=16, v=16, init_state=None, init_z=None, dy=16, dq=16, dk=16, dv=16, ws=256, B=1, T=4)
+        a.update(over)
+        n = L.la_chunk_backward_norm_workspace_size(1, 1, max(a["T"], 1), 16, 16, 1, 0)
+        return L.la_chunk_backward_norm_ws(vp(a["q"]), vp(a["k"]), vp(a["v"]), None, vp(a["init_state"]),
+                                           vp(a["init_z"]), vp(a["dy"]), None, None, vp(a["dq"]), vp(a["dk"]),
+                                           vp(a["dv"]), None, None, None, a["B"], 1, a["T"], 16, 16, 1,
+                                           vp(a["ws"]), n, None)
+    assert bn(init_state=32, init_z=None) == 1   # a carried state without its key sum
+    assert bn(dy=None) == 1
+    assert bn(ws=None) == 1
+    assert bn(dk=8) == 1
+    assert bn(B=0) == 0
+    assert L.la_chunk_backward_norm_workspace_size(1, 8, 8192, 64, 64, 1, 2) > \
+        L.la_chunk_backward_workspace_size(1, 8, 8192, 64, 64, 1, 2)
