@@ -17,9 +17,10 @@ One step is one pass of the hot path over one batch of the workload:
 --direction reverse times the anti-causal scan (la_chunk_reverse_ws) on the
 same inputs; --direction bidirectional the encoder form (forward scan, then
 the reverse scan adding to its output; no carried state); --direction
-backward the gradients of the unnormalised forward (la_chunk_backward_ws:
-dq, dk, dv, the log-decay gradient and, with a carried state, the initial
-state's) for a seeded upstream gradient dy.  Configs 1-4 (backward: 1, 2, 4).
+backward the gradients of the forward (la_chunk_backward_ws, or
+la_chunk_backward_norm_ws for the normalised workload: dq, dk, dv, the
+log-decay gradient and, with a carried state, the initial state's and key
+sum's) for a seeded upstream gradient dy.  Configs 1-4.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
@@ -235,13 +236,13 @@ class Job:
             self.grads = (torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v),
                           torch.empty_like(self.log_g) if self.log_g is not None else None,
                           torch.empty(wl.B, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=device))
-            self.bws = torch.empty(la.backward_workspace_size(wl.B, wl.H, wl.T, wl.Dk, wl.Dv, wl.torch_dtype,
-                                                              self.kind), dtype=torch.uint8, device=device)
-            # three scans (each a state pass and an output pass when segmented),
-            # the state transpose, the shifted decay, and the decay-gradient kernels
-            scans = 3 * (2 if (wl.dtype != "f32" and la.workspace_size(
-                wl.B, wl.H, wl.T, wl.Dv, wl.Dk, wl.torch_dtype, False) > 0) else 1)
-            self.fwd_launches = scans + (0 if self.kind == 0 else (1 + 1 + 2 + (1 if self.kind == 1 else 0)))
+            if wl.normalize:
+                nb = int(la.lib().la_chunk_backward_norm_workspace_size(wl.B, wl.H, wl.T, wl.Dk, wl.Dv, 1,
+                                                                         self.kind))
+            else:
+                nb = la.backward_workspace_size(wl.B, wl.H, wl.T, wl.Dk, wl.Dv, wl.torch_dtype, self.kind)
+            self.bws = torch.empty(nb, dtype=torch.uint8, device=device)
+            self.fwd_launches = backward_launches(la, wl, self.kind, wl.prefix_T > 0)
         if wl.prefix_T and direction != "bidirectional":
             # carried state of the workload: the library's own forward over the seeded prefix
             pre = W.prefix_inputs(wl)
@@ -257,6 +258,9 @@ class Job:
             return wl.steps
         if self.direction == "bidirectional":
             la.bidirectional(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, out=self.out)
+        elif self.direction == "backward" and wl.normalize:
+            la.chunk_backward_normalized(self.q, self.k, self.v, self.dy, self.kind, self.log_g, self.S0, self.z0,
+                                         workspace=self.bws)
         elif self.direction == "backward":
             la.chunk_backward(self.q, self.k, self.v, self.dy, self.kind, self.log_g, self.S0, None,
                               workspace=self.bws, out=self.grads)
@@ -288,8 +292,12 @@ class Job:
             return tokens_per_step(wl, self.cfg)
         if self.direction == "backward":
             dy = pinned["dy"].to(self.dev, non_blocking=True)
-            dq, dk, dv, dlg, _ = la.chunk_backward(q, k, v, dy, self.kind, lg, self.S0, None, workspace=self.bws,
-                                                   out=self.grads)
+            if wl.normalize:
+                dq, dk, dv, dlg, _, _ = la.chunk_backward_normalized(q, k, v, dy, self.kind, lg, self.S0, self.z0,
+                                                                     workspace=self.bws)
+            else:
+                dq, dk, dv, dlg, _ = la.chunk_backward(q, k, v, dy, self.kind, lg, self.S0, None,
+                                                       workspace=self.bws, out=self.grads)
             for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("dlog", dlg)):
                 if t is not None:
                     pinned[n].copy_(t, non_blocking=True)
@@ -328,6 +336,25 @@ class Job:
         if self.direction != "bidirectional":
             d2h += p["S"].numel() * 4
         return p, h2d, d2h
+
+
+def backward_launches(la, wl, kind, carried):
+    """Kernel launches of one backward call, as the library issues them: its
+    scans (two launches each when T-segmented) and its small kernels."""
+    def scan(dk, dv):
+        return 2 if (wl.dtype != "f32" and la.workspace_size(wl.B, wl.H, wl.T, dk, dv, wl.torch_dtype, False) > 0) \
+            else 1
+    decay = kind != 0
+    dlog = (2 + (1 if kind == 1 else 0)) if decay else 0  # block scan, offsets, per-head sum (no final-state term)
+    n = (1 if decay else 0) * 2 + dlog                    # shifted decay, d_init_state scaled by g_1
+    if not wl.normalize:
+        return n + (1 if carried else 0) + 2 * scan(wl.Dv, wl.Dk) + scan(wl.Dk, wl.Dv)
+    if wl.Dv + 1 > 128:  # numerator and denominator terms from separate scans
+        return (n + (1 if carried else 0) + (2 if carried else 0) + 1 + scan(wl.Dk, wl.Dv) + scan(wl.Dk, 16) + 1
+                + scan(wl.Dv, wl.Dk) + scan(16, wl.Dk) + 1 + scan(wl.Dv, wl.Dk) + scan(16, wl.Dk)
+                + scan(wl.Dk, wl.Dv) + 1)
+    W = next(w for w in (32, 64, 128) if w > wl.Dv) if wl.dtype != "f32" else wl.Dv + 1
+    return (n + (2 if carried else 0) + 1 + scan(wl.Dk, W) + 1 + 2 * scan(W, wl.Dk) + scan(wl.Dk, wl.Dv) + 1)
 
 
 def barrier(dist_on):
@@ -421,7 +448,8 @@ def cpu_baseline(cfg, budget_s=15.0, direction="forward"):
         dy = dy.reshape(inp["q"].shape[:3] + (wl.Dv,))
     t0 = time.perf_counter()
     if direction == "backward":
-        oracle.backward(inp["q"], inp["k"], inp["v"], dy, inp["decay_kind"], inp["log_g"], False, nthreads=threads)
+        oracle.backward(inp["q"], inp["k"], inp["v"], dy, inp["decay_kind"], inp["log_g"], wl.normalize,
+                        nthreads=threads, **init)
     elif fn is None:
         oracle.bidirectional(inp["q"], inp["k"], inp["v"], inp["decay_kind"], inp["log_g"], wl.normalize,
                              nthreads=threads)
@@ -708,8 +736,6 @@ def main():
     args = ap.parse_args()
     if args.config in (5, 6) and args.direction != "forward":
         ap.error("--direction applies to the whole-sequence configs 1-4")
-    if args.direction == "backward" and args.config != 6 and W.WORKLOADS[args.config].normalize:
-        ap.error("--direction backward: the library's backward covers the unnormalised forward (configs 1, 2, 4)")
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
