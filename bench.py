@@ -345,7 +345,7 @@ def backward_launches(la, wl, kind, carried):
         return 2 if (wl.dtype != "f32" and la.workspace_size(wl.B, wl.H, wl.T, dk, dv, wl.torch_dtype, False) > 0) \
             else 1
     decay = kind != 0
-    dlog = (2 + (1 if kind == 1 else 0)) if decay else 0  # block scan, offsets, per-head sum (no final-state term)
+    dlog = (3 + (1 if kind == 1 else 0)) if decay else 0  # block scan, block suffixes, offsets, per-head sum
     n = (1 if decay else 0) * 2 + dlog                    # shifted decay, d_init_state scaled by g_1
     if not wl.normalize:
         return n + (1 if carried else 0) + 2 * scan(wl.Dv, wl.Dk) + scan(wl.Dk, wl.Dv)

@@ -116,16 +116,43 @@ __global__ void __launch_bounds__(256) dlog_block_kernel(const E* __restrict__ q
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int t0 = blk * kDlogTokens;
     const int n = min(kDlogTokens, T - t0);
-    for (int i = warp; i < kDlogTokens; i += 8) {
-        float s = 0.f;
-        if (i < n) {
-            const size_t row = (static_cast<size_t>(bh) * T + t0 + i) * Dk;
-            for (int e = lane; e < Dk; e += 32)
-                s += to_f(q[row + e]) * to_f(dq[row + e]) - to_f(k[row + e]) * to_f(dk[row + e]);
+    constexpr int VEC = 16 / sizeof(E);  // elements per 16-byte load
+    const int lpt = Dk / VEC;            // lanes per token with 16-byte loads
+    if (Dk % VEC == 0 && lpt <= 32 && (lpt & (lpt - 1)) == 0) {
+        // groups of lpt lanes each take one token (a row of 16-byte loads),
+        // 32 / lpt tokens per warp at a time
+        const int tpw = 32 / lpt, sub = lane / lpt, l = lane % lpt;
+        for (int i0 = warp * tpw; i0 < kDlogTokens; i0 += 8 * tpw) {
+            const int i = i0 + sub;
+            float s = 0.f;
+            if (i < n) {
+                const size_t row = (static_cast<size_t>(bh) * T + t0 + i) * Dk + static_cast<size_t>(l) * VEC;
+                const uint4 vq = *reinterpret_cast<const uint4*>(q + row);
+                const uint4 vdq = *reinterpret_cast<const uint4*>(dq + row);
+                const uint4 vk = *reinterpret_cast<const uint4*>(k + row);
+                const uint4 vdk = *reinterpret_cast<const uint4*>(dk + row);
+                const E* eq = reinterpret_cast<const E*>(&vq);
+                const E* edq = reinterpret_cast<const E*>(&vdq);
+                const E* ek = reinterpret_cast<const E*>(&vk);
+                const E* edk = reinterpret_cast<const E*>(&vdk);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                for (int e = 0; e < VEC; ++e) s += to_f(eq[e]) * to_f(edq[e]) - to_f(ek[e]) * to_f(edk[e]);
+            }
+            for (int o = lpt / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (l == 0 && i < kDlogTokens) a[i] = s;
         }
-        if (lane == 0) a[i] = s;
+    } else {
+        for (int i = warp; i < kDlogTokens; i += 8) {
+            float s = 0.f;
+            if (i < n) {
+                const size_t row = (static_cast<size_t>(bh) * T + t0 + i) * Dk;
+                for (int e = lane; e < Dk; e += 32)
+                    s += to_f(q[row + e]) * to_f(dq[row + e]) - to_f(k[row + e]) * to_f(dk[row + e]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            }
+            if (lane == 0) a[i] = s;
+        }
     }
     __syncthreads();
     // suffix sums: thread i holds token i; warp-level inclusive suffix scan,
@@ -157,21 +184,36 @@ __global__ void __launch_bounds__(256) dlog_block_kernel(const E* __restrict__ q
     }
 }
 
+// Per (b, h): blk_off[j] = the totals of a over the blocks after j, in
+// chunks of 256 blocks from the end (a fixed summation order).
+__global__ void dlog_suffix_kernel(const double* __restrict__ blk_a, double* __restrict__ blk_off, int nblk) {
+    const int bh = blockIdx.x;
+    __shared__ double sh[256];
+    double carry = 0.0;  // totals of the blocks after the current chunk
+    for (int c1 = nblk; c1 > 0; c1 -= 256) {
+        const int c0 = c1 > 256 ? c1 - 256 : 0, m = c1 - c0;
+        const int j = c0 + threadIdx.x;
+        sh[threadIdx.x] = threadIdx.x < m ? blk_a[static_cast<size_t>(bh) * nblk + j] : 0.0;
+        __syncthreads();
+        double acc = carry;
+        for (int jj = threadIdx.x + 1; jj < m; ++jj) acc += sh[jj];
+        if (threadIdx.x < m) blk_off[static_cast<size_t>(bh) * nblk + j] = acc;
+        double tot = 0.0;
+        for (int jj = 0; jj < m; ++jj) tot += sh[jj];
+        carry += tot;
+        __syncthreads();
+    }
+}
+
 // Block (blk, bh): the offset of block blk is the terminal term plus the
 // totals of a over every later block; per step it is added to the block's
 // tokens, per head the block's contribution (its local sums plus n times the
 // offset) goes to blk_x for the final reduction.
 __global__ void dlog_offset_kernel(float* __restrict__ x, int per_step, int T, int nblk,
-                                   const double* __restrict__ blk_a, double* __restrict__ blk_x,
+                                   const double* __restrict__ blk_off, double* __restrict__ blk_x,
                                    const double* __restrict__ terminal) {
     const int blk = blockIdx.x, bh = blockIdx.y;
-    __shared__ double off;
-    if (threadIdx.x == 0) {
-        double o = terminal ? terminal[bh] : 0.0;
-        for (int j = nblk - 1; j > blk; --j) o += blk_a[static_cast<size_t>(bh) * nblk + j];
-        off = o;
-    }
-    __syncthreads();
+    const double off = (terminal ? terminal[bh] : 0.0) + blk_off[static_cast<size_t>(bh) * nblk + blk];
     const int t0 = blk * kDlogTokens, n = min(kDlogTokens, T - t0);
     if (per_step) {
         if (threadIdx.x < n) {
@@ -430,7 +472,7 @@ cudaError_t launch_scale_by_first_decay(float* s, const float* log_g, int kind, 
 size_t dlog_scratch_doubles(int B, int H, int T) {
     const size_t BH = static_cast<size_t>(B) * H;
     const size_t nblk = (static_cast<size_t>(T) + kDlogTokens - 1) / kDlogTokens;
-    return BH + 2 * BH * nblk;  // terminal terms, block totals of a, block sums of x
+    return BH + 3 * BH * nblk;  // terminal terms, block totals of a, block sums of x, block offsets
 }
 
 cudaError_t launch_dlog(const DlogArgs& a) {
@@ -440,6 +482,7 @@ cudaError_t launch_dlog(const DlogArgs& a) {
     double* terminal = (a.d_final_state || a.d_final_z) ? a.scratch : nullptr;
     double* blk_a = a.scratch + BH;
     double* blk_x = blk_a + static_cast<size_t>(BH) * nblk;
+    double* blk_off = blk_x + static_cast<size_t>(BH) * nblk;
     if (terminal) {
         terminal_kernel<<<BH, 256, 0, a.stream>>>(a.d_final_state, a.st, a.st_bh, a.st_i, a.st_j, a.d_final_z, a.zt,
                                                   a.zt_bh, a.zt_i, terminal, a.Dk, a.Dv);
@@ -459,7 +502,10 @@ cudaError_t launch_dlog(const DlogArgs& a) {
             static_cast<const float*>(a.dk), a.d_log_g, per_step, a.T, a.Dk, nblk, blk_a, blk_x);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    dlog_offset_kernel<<<grid, kDlogTokens, 0, a.stream>>>(a.d_log_g, per_step, a.T, nblk, blk_a, blk_x, terminal);
+    dlog_suffix_kernel<<<BH, 256, 0, a.stream>>>(blk_a, blk_off, nblk);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dlog_offset_kernel<<<grid, kDlogTokens, 0, a.stream>>>(a.d_log_g, per_step, a.T, nblk, blk_off, blk_x, terminal);
     e = cudaGetLastError();
     if (e != cudaSuccess || per_step) return e;
     dlog_head_kernel<<<a.H, 256, 0, a.stream>>>(a.d_log_g, a.B, a.H, nblk, blk_x);

@@ -256,7 +256,7 @@ def test_backward_workspace_size(L):
     state = r(4 * B * H * D * D)
     nblk = (T + 255) // 256
     scan = L.la_chunk_forward_workspace_size(B, H, T, D, D, 1, 0)
-    want = 3 * state + r(4 * B * H * T) + r(8 * (B * H + 2 * B * H * nblk)) + r(scan)
+    want = 3 * state + r(4 * B * H * T) + r(8 * (B * H + 3 * B * H * nblk)) + r(scan)
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 2) == want
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 0) == want - r(4 * B * H * T)
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 0, 2) == want - r(scan)  # fp32: no segments
