@@ -357,6 +357,39 @@ def backward_launches(la, wl, kind, carried):
     return (n + (2 if carried else 0) + 1 + scan(wl.Dk, W) + 1 + 2 * scan(W, wl.Dk) + scan(wl.Dk, wl.Dv) + 1)
 
 
+def decode_graph_timing(job, device, dist_on, reps=3):
+    """The decode workload's 1024 token steps captured once in a CUDA graph
+    and replayed (the launch overhead of the per-token calls removed), timed
+    like the plain steps: CUDA events around each replay, max over ranks."""
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream(device))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        job.step()  # warm the stream before capture
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            job.step()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    ms = []
+    cur = torch.cuda.current_stream(device)
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        g.replay()
+        e1.record(cur)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    barrier(dist_on)
+    assert job.la.device_error(device) == 0
+    per_token = max_over_ranks(statistics.median(ms), dist_on, device) / job.wl.steps
+    del g
+    return {"ms_per_token": round(per_token, 5), "launches_per_replay": job.wl.steps,
+            "tokens_per_s": job.wl.B * job.wl.H / (per_token / 1e3)}
+
+
 def barrier(dist_on):
     if dist_on:
         torch.distributed.barrier()
@@ -501,6 +534,7 @@ def run_ours(args, rank, world, dist_on, device):
     ms_per_step = total_ms / args.steps
     tokens = tokens_per_step(wl, cfg) * world
     value = tokens / (ms_per_step / 1e3)
+    graph = decode_graph_timing(job, device, dist_on) if cfg == 5 and not args.skip_e2e else None
 
     # the path's kernels: one decode call, or one forward (a T-segmented forward
     # is a state pass and an output pass of the same kernel, timed together)
@@ -560,6 +594,8 @@ def run_ours(args, rank, world, dist_on, device):
         "roofline": roofline, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches,
     }
+    if graph:
+        line["decode_graph"] = graph
     return line
 
 
