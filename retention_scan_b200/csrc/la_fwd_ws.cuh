@@ -555,77 +555,105 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             ++pseen;
             moved = true;
         }
-        if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA)) {
-            tc_fence_after_sync();
-            const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
-            const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
-            if (leader) {
+        // Q K^T of chunk m1
+        auto issue_qk = [&]() {
+            if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA)) {
+                tc_fence_after_sync();
+                const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
+                const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem + 128 * (m1 % G::NA), dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4),
-                              G::IDESC_QK, kk > 0);
-                umma_commit(&bar[B_AFULL + m1 % G::NA]);
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16(tmem + 128 * (m1 % G::NA), dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4),
+                                  G::IDESC_QK, kk > 0);
+                    umma_commit(&bar[B_AFULL + m1 % G::NA]);
+                }
+                __syncwarp();
+                ++m1;
+                moved = true;
             }
-            __syncwarp();
-            ++m1;
-            moved = true;
-        }
-        if (kv < m1 && (bits & kPrep) && (!(bits & kDir) || kv < pseen) && (bits & kDse)) {
-            // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
-            // repeats the key panel when Dk < 128
-            tc_fence_after_sync();
-            const int b = kv % G::NDS;
-            const uint64_t dk = make_smem_desc(k_addr(kv), DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
-            const uint64_t dv = make_smem_desc(v_addr(kv), C * G::WV, 8 * G::WV, G::WV);
-            const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
-            if (leader) {
+        };
+        // K^T V' of chunk kv
+        auto issue_kv = [&]() {
+            if (kv < m1 && (bits & kPrep) && (!(bits & kDir) || kv < pseen) && (bits & kDse)) {
+                // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
+                // repeats the key panel when Dk < 128
+                tc_fence_after_sync();
+                const int b = kv % G::NDS;
+                const uint64_t dk = make_smem_desc(k_addr(kv), DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
+                const uint64_t dv = make_smem_desc(v_addr(kv), C * G::WV, 8 * G::WV, G::WV);
+                const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
-                umma_commit(&bar[B_DSFULL + b]);
-                umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
+                    umma_commit(&bar[B_DSFULL + b]);
+                    umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
+                }
+                __syncwarp();
+                ++kv;
+                moved = true;
             }
-            __syncwarp();
-            ++kv;
-            moved = true;
-        }
-        if (qs < kv && (bits & kOe) && (bits & kSb)) {
-            // O = Q S (and den = Q z), opening the accumulator of chunk qs
-            tc_fence_after_sync();
-            const int ro = qs % G::NO, sbb = qs % G::NSB;
-            const uint64_t dq = make_smem_desc(q_addr(qs), 16, 8 * G::WK, G::WK);
-            // B = [S | z] panels of the bf16 state copy
-            const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
-            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
-            if (leader) {
+        };
+        // Q S of chunk qs
+        auto issue_qs = [&]() {
+            if (qs < kv && (bits & kOe) && (bits & kSb)) {
+                // O = Q S (and den = Q z), opening the accumulator of chunk qs
+                tc_fence_after_sync();
+                const int ro = qs % G::NO, sbb = qs % G::NSB;
+                const uint64_t dq = make_smem_desc(q_addr(qs), 16, 8 * G::WK, G::WK);
+                // B = [S | z] panels of the bf16 state copy
+                const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
+                const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
-                umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // Q K^T and Q S of this chunk have run
-                umma_commit(&bar[B_SBEMPTY + sbb]);
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
+                    umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // Q K^T and Q S of this chunk have run
+                    umma_commit(&bar[B_SBEMPTY + sbb]);
+                }
+                __syncwarp();
+                ++qs;
+                moved = true;
             }
-            __syncwarp();
-            ++qs;
-            moved = true;
-        }
-        if (pv < qs && pv < pseen) {
-            // P V (and P W) accumulate into the O that Q S opened
-            tc_fence_after_sync();
-            const int pb = pv % G::NPB, ro = pv % G::NO;
-            const uint64_t dv = make_smem_desc(v_addr(pv), C * G::WV, 8 * G::WV, G::WV);
-            const uint32_t pa = tmem + G::COL_P0 + 64 * pb;
-            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
-            if (leader) {
+        };
+        // P V of chunk pv
+        auto issue_pv = [&]() {
+            if (pv < qs && pv < pseen) {
+                // P V (and P W) accumulate into the O that Q S opened
+                tc_fence_after_sync();
+                const int pb = pv % G::NPB, ro = pv % G::NO;
+                const uint64_t dv = make_smem_desc(v_addr(pv), C * G::WV, 8 * G::WV, G::WV);
+                const uint32_t pa = tmem + G::COL_P0 + 64 * pb;
+                const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
-                umma_commit(&bar[B_OFULL + ro]);
-                umma_commit(&bar[B_PEMPTY + pb]);
-                umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
+                    umma_commit(&bar[B_OFULL + ro]);
+                    umma_commit(&bar[B_PEMPTY + pb]);
+                    umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
+                }
+                __syncwarp();
+                ++pv;
+                moved = true;
             }
-            __syncwarp();
-            ++pv;
-            moved = true;
+        };
+        // Order within a pass: the newest chunks' Q K^T and K^T V' first for
+        // Dk = 128.  With Dk <= 64 the chunk period is set by the Q ring (a
+        // stage is held until the chunk's Q S) and the issuing thread waits
+        // behind the MMAs already queued, so Q S and P V of the older chunks
+        // go first (measured: 3% faster at Dk = 64, slower at Dk = 128).
+        if constexpr (DK <= 64) {
+            issue_qs();
+            issue_pv();
+            issue_qk();
+            issue_kv();
+        } else {
+            issue_qk();
+            issue_kv();
+            issue_qs();
+            issue_pv();
         }
         if (moved) {
             idle_since = 0;
