@@ -14,6 +14,8 @@ cpu_baseline / reference legs may import this package.  The CUDA library
   wkv4(...)              the RWKV-4 WKV recurrence: the att_seq loop of
                          BlinkDL/RWKV-LM issue 167, max-shifted (wkv4_ref.c)
   wkv4_direct(...)       the same output from its definition, O(T^2), numpy
+  ema(...)               the cumulative EMA of RetNet issue 21 (values,
+                         factors, reverse), per channel (ema_ref.c)
   parallel_forward(...)  brute-force O(T^2) parallel form, numpy (parallel.py)
   parallel_reverse(...)  brute-force O(T^2) anti-causal form, numpy (parallel.py)
 
@@ -30,7 +32,7 @@ from .parallel import parallel_forward, parallel_reverse  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "la_ref.c")
-_SRCS = (_SRC, os.path.join(_HERE, "wkv4_ref.c"))
+_SRCS = (_SRC, os.path.join(_HERE, "wkv4_ref.c"), os.path.join(_HERE, "ema_ref.c"))
 _LIB_PATH = os.path.join(_HERE, "liblaref.so")
 _libs = {}
 
@@ -67,6 +69,9 @@ def load_library(path=None):
         if hasattr(lib, "la_ref_wkv4"):
             lib.la_ref_wkv4.argtypes = [d, d, d, d, d, d, d, i, i, i]
             lib.la_ref_wkv4.restype = i
+        if hasattr(lib, "la_ref_ema"):
+            lib.la_ref_ema.argtypes = [d, d, d, d, d, i, i, i, i]
+            lib.la_ref_ema.restype = i
         _libs[path] = lib
     return _libs[path]
 
@@ -146,6 +151,22 @@ def backward(q, k, v, dy, decay_kind=0, log_g=None, normalize=False, init_state=
     elif kind == 2:
         dlog_g = dlog
     return dq, dk, dv, dlog_g, dS0, (dz0 if normalize else None)
+
+
+def ema(x, f, init_state=None, reverse=False, lib=None):
+    """Cumulative EMA along T, float64 (ema_ref.c: RetNet issue 21's
+    cumulative_ema): s <- f_t s + x_t per channel, out_t = s.  x, f
+    [B,T,C]; init_state [B,C] or None (0).  Returns (out [B,T,C], final
+    state [B,C])."""
+    x, f, init_state = _f64(x), _f64(f), _f64(init_state)
+    B, T, C = x.shape
+    out = np.zeros((B, T, C))
+    fin = np.zeros((B, C))
+    rc = (lib or load_library()).la_ref_ema(_ptr(x), _ptr(f), _ptr(init_state), _ptr(out), _ptr(fin), B, T, C,
+                                            int(bool(reverse)))
+    if rc != 0:
+        raise ValueError("la_ref_ema rejected its arguments")
+    return out, fin
 
 
 WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)

@@ -570,3 +570,92 @@ def wkv4_no_bonus(wkv, direct):
 
 
 WKV4 = [wkv4_direct_form, wkv4_t1_t2, wkv4_invariants, wkv4_split_carry, wkv4_large_keys, wkv4_no_bonus]
+
+
+# -- cumulative EMA (RetNet issue 21, cumulative_ema) -------------------------
+#
+#   ema_constant_factor  f = gamma everywhere: out_t = sum_i gamma^(t-i) x_i
+#                        + gamma^(t+1) s0 with integer powers
+#   ema_cumsum           f = 1: numpy cumsum;  f = 0: out = x
+#   ema_operator         segment summaries (state from 0, product of
+#                        factors) folded with (xa, fa) o (xb, fb) =
+#                        (xa fb + xb, fa fb) in random bracketings equal the
+#                        full run's final state
+#   ema_reverse          reverse == flip(forward(flip(x), flip(f)))
+#   ema_split_carry      run(T) == run(T1) -> carry -> run(T - T1)
+
+def _ema_inputs(rng, B, T, C):
+    return rng.standard_normal((B, T, C)), rng.uniform(0.3, 1.0, (B, T, C)), rng.standard_normal((B, C))
+
+
+def ema_constant_factor(ema):
+    rng = np.random.default_rng(71)
+    x, _, s0 = _ema_inputs(rng, 2, 19, 3)
+    g = 0.83
+    out, fin = ema(x, np.full_like(x, g), s0)
+    t = np.arange(19)
+    P = np.tril(g ** (t[:, None] - t[None, :]).clip(min=0)) * (t[:, None] >= t[None, :])
+    want = np.einsum("ts,bsc->btc", P, x) + (g ** (t + 1))[None, :, None] * s0[:, None, :]
+    _close(out, want, 1e-12, "constant factor")
+    _close(fin, want[:, -1], 1e-12, "constant factor final")
+
+
+def ema_cumsum(ema):
+    rng = np.random.default_rng(72)
+    x, _, _ = _ema_inputs(rng, 2, 23, 4)
+    out, _ = ema(x, np.ones_like(x))
+    _close(out, np.cumsum(x, axis=1), 1e-12, "f = 1 is a cumsum")
+    out, _ = ema(x, np.zeros_like(x))
+    _close(out, x, 0.0, "f = 0 is the identity")
+
+
+def ema_operator(ema):
+    rng = np.random.default_rng(73)
+    x, f, _ = _ema_inputs(rng, 1, 40, 2)
+    _, full = ema(x, f)
+    cuts = np.sort(rng.choice(np.arange(1, 40), size=5, replace=False))
+    spans = np.split(np.arange(40), cuts)
+    items = []
+    for sp in spans:
+        _, fin = ema(x[:, sp], f[:, sp])
+        items.append((fin, np.prod(f[:, sp], axis=1)))
+
+    def op(a, b):  # RetNet issue 21's pairing of (value, factor)
+        return a[0] * b[1] + b[0], a[1] * b[1]
+
+    for trial in range(6):
+        seq = list(items)
+        while len(seq) > 1:  # a random bracketing
+            j = rng.integers(0, len(seq) - 1)
+            seq[j:j + 2] = [op(seq[j], seq[j + 1])]
+        _close(seq[0][0], full, 1e-12, f"bracketing {trial}")
+
+
+def ema_reverse(ema):
+    rng = np.random.default_rng(74)
+    x, f, s0 = _ema_inputs(rng, 2, 17, 3)
+    out, fin = ema(x, f, s0, reverse=True)
+    o2, f2 = ema(x[:, ::-1].copy(), f[:, ::-1].copy(), s0)
+    _close(out, o2[:, ::-1], 1e-12, "reverse = flip forward flip")
+    _close(fin, f2, 1e-12, "reverse final state")
+
+
+def ema_split_carry(ema):
+    rng = np.random.default_rng(75)
+    x, f, s0 = _ema_inputs(rng, 2, 31, 3)
+    for rev in (False, True):
+        full, ffin = ema(x, f, s0, reverse=rev)
+        for T1 in (1, 12, 30):
+            if not rev:
+                a, fa = ema(x[:, :T1], f[:, :T1], s0)
+                b, fb = ema(x[:, T1:], f[:, T1:], fa)
+                got = np.concatenate([a, b], axis=1)
+            else:
+                b, fb0 = ema(x[:, T1:], f[:, T1:], s0, reverse=True)
+                a, fb = ema(x[:, :T1], f[:, :T1], fb0, reverse=True)
+                got = np.concatenate([a, b], axis=1)
+            _close(got, full, 1e-12, f"split at {T1} reverse={rev}")
+            _close(fb, ffin, 1e-12, f"split at {T1} reverse={rev}: state")
+
+
+EMA = [ema_constant_factor, ema_cumsum, ema_operator, ema_reverse, ema_split_carry]

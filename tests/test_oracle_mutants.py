@@ -110,11 +110,52 @@ def _run_wkv4_pins(lib):
     return failed
 
 
-def _build_copy(tmp_path, wkv4_text=None):
+EMA_SRC = os.path.join(os.path.dirname(oracle.__file__), "ema_ref.c")
+
+# (name, text in ema_ref.c, replacement)
+EMA_MUTANTS = [
+    ("factor ignored", "s = f[i] * s + x[i];", "s = s + x[i];"),
+    ("decay after the add", "s = f[i] * s + x[i];", "s = f[i] * (s + x[i]);"),
+    ("factor of the previous step", "s = f[i] * s + x[i];",
+     "s = f[i > (size_t)C ? i - C : i] * s + x[i];"),
+    ("reverse runs forward", "const int t = reverse ? T - 1 - step : step;", "const int t = step;"),
+    ("carried state ignored", "double s = init_state ? init_state[(size_t)b * C + c] : 0.0;", "double s = 0.0;"),
+]
+
+
+def _run_ema_pins(lib):
+    fn = lambda *a, **kw: oracle.ema(*a, lib=lib, **kw)  # noqa: E731
+    failed = []
+    for check in pins.EMA:
+        try:
+            check(fn)
+        except AssertionError:
+            failed.append(check.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name,old,new", EMA_MUTANTS, ids=[m[0] for m in EMA_MUTANTS])
+def test_ema_mutant_is_caught(tmp_path, name, old, new):
+    src = open(EMA_SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique: {name}"
+    failed = _run_ema_pins(_build_copy(tmp_path, ema_text=src.replace(old, new)))
+    assert failed, f"no pin catches the mutant '{name}'"
+
+
+def test_ema_unmutated_copy_passes(tmp_path):
+    assert _run_ema_pins(_build_copy(tmp_path)) == []
+
+
+def _build_copy(tmp_path, wkv4_text=None, ema_text=None):
     paths = []
-    for src in (SRC, WKV4_SRC):
+    for src in (SRC, WKV4_SRC, EMA_SRC):
         p = tmp_path / os.path.basename(src)
-        p.write_text(wkv4_text if (src == WKV4_SRC and wkv4_text is not None) else open(src).read())
+        text = open(src).read()
+        if src == WKV4_SRC and wkv4_text is not None:
+            text = wkv4_text
+        if src == EMA_SRC and ema_text is not None:
+            text = ema_text
+        p.write_text(text)
         paths.append(str(p))
     so = tmp_path / "liblaref_copy.so"
     subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread", "-o", str(so), *paths, "-lm"],

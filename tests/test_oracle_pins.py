@@ -144,3 +144,8 @@ def test_wkv4_direct_form_by_brute_force():
 def test_wkv4_rejects_bad_arguments(oracle_lib):
     lib = oracle.load_library()
     assert lib.la_ref_wkv4(None, None, None, None, None, None, None, 1, 1, 1) == -1
+
+
+@pytest.mark.parametrize("check", pins.EMA, ids=lambda f: f.__name__)
+def test_ema_oracle(oracle_lib, check):
+    check(oracle.ema)
