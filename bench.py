@@ -13,6 +13,8 @@ One step is one pass of the hot path over one batch of the workload:
   config 5: decode, B=256, H=32, D=128, normalised, 1024 la_decode_step calls
   config 6: the RWKV-4 WKV recurrence, B=8, T=4096, C=2048, bf16 -> one
       la_wkv4_forward call (tokens = B*T; a different recurrence)
+  config 7: RetNet issue 21's cumulative EMA (values, factors), B=8, T=4096,
+      C=2048, bf16 -> one la_ema_scan call (tokens = B*T)
 
 --direction reverse times the anti-causal scan (la_chunk_reverse_ws) on the
 same inputs; --direction bidirectional the encoder form (forward scan, then
@@ -611,6 +613,66 @@ def wkv4_bytes(wl):
     return wl.B * wl.T * wl.C * 3 * es + 2 * wl.C * 4 + wl.B * 3 * wl.C * 4
 
 
+EMA_METRIC = "cumulative-ema tokens/s (B·T/s) and % of roofline (HBM GB/s)"
+
+
+def ema_bytes(wl):
+    """Bytes one la_ema_scan call must move: x, f read and out written once,
+    the fp32 final state written."""
+    es = 2 if wl.dtype == "bf16" else 4
+    return wl.B * wl.T * wl.C * 3 * es + wl.B * wl.C * 4
+
+
+class EmaJob:
+    def __init__(self, device, wl, rank=0):
+        import retention_scan_b200 as la
+        self.la, self.wl, self.dev = la, wl, device
+        self.host = W.ema_inputs(wl.with_sizes(seed=wl.seed + 7919 * rank))
+        self.x, self.f = (self.host[n].to(device) for n in ("x", "f"))
+        self.out = torch.empty(wl.B, wl.T, wl.C, dtype=wl.torch_dtype, device=device)
+        self.fin = torch.empty(wl.B, wl.C, dtype=torch.float32, device=device)
+        self.launches = 1
+
+    def step(self):
+        self.la.ema_scan(self.x, self.f, out=self.out, final_state=self.fin)
+        return 1
+
+    def e2e(self, steps, dist_on):
+        p = {n: self.host[n].pin_memory() for n in ("x", "f")}
+        y = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        stream = torch.cuda.current_stream(self.dev)
+
+        def one():
+            x, f = (p[n].to(self.dev, non_blocking=True) for n in ("x", "f"))
+            o, _ = self.la.ema_scan(x, f, out=self.out, final_state=self.fin)
+            y.copy_(o, non_blocking=True)
+        for _ in range(2):
+            one()
+        barrier(dist_on)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            one()
+        ev1.record(stream)
+        barrier(dist_on)
+        h2d = sum(p[n].numel() * p[n].element_size() for n in p)
+        return ev0.elapsed_time(ev1) / steps, h2d, y.numel() * y.element_size()
+
+
+def cpu_baseline_ema(wl, budget_s=15.0):
+    """The float64 oracle (single-threaded C loop) on whole batch rows."""
+    import oracle
+    oracle.build()
+    per_row_s = wl.T * wl.C * 6 / 1e9
+    nb = max(1, min(wl.B, int(budget_s / max(per_row_s, 1e-9))))
+    inp = W.ema_inputs(wl, batches=range(nb))
+    t0 = time.perf_counter()
+    oracle.ema(inp["x"], inp["f"])
+    dt = time.perf_counter() - t0
+    return {"value": nb * wl.T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{nb} of {wl.B} batch rows, all {wl.T} tokens x {wl.C} channels, single thread"}
+
+
 class Wkv4Job:
     def __init__(self, device, wl, rank=0):
         import retention_scan_b200 as la
@@ -665,13 +727,16 @@ def cpu_baseline_wkv4(wl, budget_s=15.0):
 
 
 def run_wkv4(args, rank, world, dist_on, device):
-    wl = W.WKV4
+    """The per-channel scans on [B, T, C]: config 6 (RWKV-4 WKV), config 7
+    (cumulative EMA)."""
+    ema = args.config == 7
+    wl = W.EMA if ema else W.WKV4
     if args.tokens:
         wl = wl.with_sizes(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.batch:
         wl = wl.with_sizes(B=args.batch, name=f"{wl.name}_B{args.batch}")
-    job = Wkv4Job(device, wl, rank)
-    nbytes = wkv4_bytes(wl)
+    job = (EmaJob if ema else Wkv4Job)(device, wl, rank)
+    nbytes = (ema_bytes if ema else wkv4_bytes)(wl)
     flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device) if nbytes < 2 * L2_BYTES else None
     for _ in range(args.warmup):
         if flush is not None:
@@ -698,7 +763,8 @@ def run_wkv4(args, rank, world, dist_on, device):
         e2e = {"value": wl.B * wl.T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
     return {
-        "metric": WKV4_METRIC, "value": wl.B * wl.T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "metric": EMA_METRIC if ema else WKV4_METRIC, "value": wl.B * wl.T * world / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
@@ -709,7 +775,8 @@ def run_wkv4(args, rank, world, dist_on, device):
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
                      "peak_source": pk_kind,
-                     "kernel": "wkv4_kernel (state pass + output pass)" if job.launches == 2 else "wkv4_kernel",
+                     "kernel": "ema_kernel" if ema else
+                     ("wkv4_kernel (state pass + output pass)" if job.launches == 2 else "wkv4_kernel"),
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": e2e, "clocks": sampler.summary(w0, w1) if sampler else None, "gpu_launches": launches,
     }
@@ -719,15 +786,17 @@ def run_wkv4(args, rank, world, dist_on, device):
 
 def run_reference(args):
     cfg = args.config
-    if cfg == 6:
-        wl = W.WKV4
+    if cfg in (6, 7):
+        wl = W.WKV4 if cfg == 6 else W.EMA
+        base = cpu_baseline_wkv4 if cfg == 6 else cpu_baseline_ema
         for _ in range(args.warmup):
-            cpu_baseline_wkv4(wl, budget_s=2.0)
-        vals = [cpu_baseline_wkv4(wl, budget_s=8.0) for _ in range(args.steps)]
+            base(wl, budget_s=2.0)
+        vals = [base(wl, budget_s=8.0) for _ in range(args.steps)]
         v = statistics.median(x["value"] for x in vals)
         cb = dict(vals[-1])
         cb["value"] = v
-        return {"impl": "reference", "metric": WKV4_METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        return {"impl": "reference", "metric": WKV4_METRIC if cfg == 6 else EMA_METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": 1,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.B * wl.T / v * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C},
@@ -762,7 +831,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -770,9 +839,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
     ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional", "backward"])
     args = ap.parse_args()
-    if args.config in (5, 6) and args.direction != "forward":
+    if args.config in (5, 6, 7) and args.direction != "forward":
         ap.error("--direction applies to the whole-sequence configs 1-4")
-    default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200}
+    default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200, 7: 200}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
     if args.warmup is None:
@@ -796,10 +865,11 @@ def main():
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
     try:
-        line = (run_wkv4 if args.config == 6 else run_ours)(args, rank, world, dist_on, device)
+        line = (run_wkv4 if args.config in (6, 7) else run_ours)(args, rank, world, dist_on, device)
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
                 line["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4) if args.config == 6 else
+                                        cpu_baseline_ema(W.EMA) if args.config == 7 else
                                         cpu_baseline(args.config, direction=args.direction))
             print(json.dumps(line), flush=True)
     finally:

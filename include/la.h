@@ -463,6 +463,44 @@ LA_API la_status la_chunk_backward_norm_ws(const void* q, const void* k, const v
                                     void* workspace, size_t workspace_bytes, la_stream_t stream);
 
 /*
+ * la_ema_scan - the cumulative exponential moving average: element-wise
+ * values and factors scanned along T per channel.
+ *
+ * Source: Jamie-Stirling/RetNet issue 21, "Proposed improvement/
+ * collaboration: removing the O(T^2) training cost", cumulative_ema(values,
+ * factors, reverse): each output is the previous output times this step's
+ * factor plus this step's value (the listing's pairing operator
+ * (xa, fa) o (xb, fb) = (xa fb + xb, fa fb)); with reverse, the non-reversed
+ * scan of the time-reversed arguments, reversed back.  Per batch b and
+ * channel c, with s the carried state:
+ *
+ *   forward:  s <- f_t s + x_t,  out_t = s,   t = 0 .. T-1
+ *   reverse:  s <- f_t s + x_t,  out_t = s,   t = T-1 .. 0
+ *
+ * The page's retention(Q, K, gamma, V) runs this scan over K (x) V with
+ * factors gamma; la_chunk_forward is the fused form of that path.  Computed
+ * in fp32 whatever the input type.
+ *
+ *   x, f, out      [B, T, C], `dtype` (LA_F32 or LA_BF16), channels fastest.
+ *                  Required (T > 0).
+ *   init_state     NULL (0) or [B, C] fp32: the state before the first scanned step.
+ *   final_state    NULL (not written) or [B, C] fp32: the state after the
+ *                  last scanned step; may be the same buffer as init_state.
+ *   reverse        0 forward, 1 reverse.
+ *   B, T, C        B, T >= 0, C >= 1; B == 0 is a no-op, T == 0 copies
+ *                  init_state (or 0) to final_state.
+ *
+ * Errors (synchronous, nothing enqueued): LA_ERR_INVALID_ARG for a NULL
+ * required pointer, negative sizes, C < 1, x, f or out not 16-byte aligned,
+ * a state not 4-byte aligned, a bad dtype; LA_ERR_UNSUPPORTED for C not a
+ * multiple of 8 (bf16) or 4 (fp32), or B > 65535; LA_ERR_CUDA if a launch
+ * fails.
+ */
+LA_API la_status la_ema_scan(const void* x, const void* f, const float* init_state, void* out,
+                             float* final_state, int B, int T, int C, la_dtype dtype, int reverse,
+                             la_stream_t stream);
+
+/*
  * la_chunk_forward_noalloc - la_chunk_forward_ws whose workspace is a fixed
  * device array inside this library (la_chunk_forward_noalloc_capacity()
  * bytes, 16 MiB, one per device, reserved when the library's device code is

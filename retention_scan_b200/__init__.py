@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "chunk_backward_normalized", "wkv4_forward",
+__all__ = ["chunk_forward", "bidirectional", "chunk_backward", "chunk_backward_normalized", "wkv4_forward", "ema_scan",
            "workspace_size",
            "backward_workspace_size",
            "decode_step", "device_error", "LAError", "lib", "library_path",
@@ -30,6 +30,7 @@ EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward
                     "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
                     "la_wkv4_forward_ws", "la_wkv4_workspace_size", "la_chunk_forward_pro_ws",
                     "la_decode_step_pro", "la_chunk_backward_norm_ws", "la_chunk_backward_norm_workspace_size",
+                    "la_ema_scan",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -88,6 +89,8 @@ def lib():
         L.la_chunk_backward_norm_workspace_size.restype = ctypes.c_size_t
         L.la_chunk_backward_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
+        L.la_ema_scan.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        L.la_ema_scan.restype = i
         L.la_wkv4_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
         L.la_wkv4_forward.restype = i
         L.la_wkv4_forward_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, ctypes.c_size_t, vp]
@@ -327,6 +330,29 @@ def chunk_backward(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=No
             _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_log_g), _ptr(d_init),
             B, H, T, Dk, Dv, code, _ptr(workspace), workspace.numel(), _stream(stream, dev)))
     return dq, dk, dv, d_log_g, d_init
+
+
+def ema_scan(x, f, init_state=None, reverse=False, out=None, final_state=None, return_final=True, stream=None):
+    """Cumulative EMA along T (la_ema_scan): s <- f_t s + x_t per channel,
+    out_t = s, forward or reverse.  x, f: [B,T,C] float32 or bfloat16 CUDA
+    tensors (C a multiple of 8 for bf16, 4 for fp32); init_state [B,C] fp32
+    or None.  Returns (out [B,T,C], final_state [B,C] or None)."""
+    B, T, C = x.shape
+    dev = x.device
+    code = _dtype_code(x.dtype)
+    _need(f, "f", (B, T, C), x.dtype, dev)
+    _need(x, "x", (B, T, C), x.dtype, dev)
+    _need(init_state, "init_state", (B, C), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, T, C), dtype=x.dtype, device=dev)
+    _need(out, "out", (B, T, C), x.dtype, dev)
+    if final_state is None and return_final:
+        final_state = torch.empty((B, C), dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (B, C), torch.float32, dev)
+    with torch.cuda.device(dev):
+        _check(lib().la_ema_scan(_ptr(x), _ptr(f), _ptr(init_state), _ptr(out), _ptr(final_state), B, T, C, code,
+                                 int(bool(reverse)), _stream(stream, dev)))
+    return out, final_state
 
 
 WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)

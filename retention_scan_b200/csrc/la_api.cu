@@ -730,6 +730,37 @@ la_status la_wkv4_forward_ws(const void* k, const void* v, const float* w, const
     return la::launch_wkv4(a) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+la_status la_ema_scan(const void* x, const void* f, const float* init_state, void* out, float* final_state, int B,
+                      int T, int C, la_dtype dtype, int reverse, la_stream_t stream) {
+    if (B < 0 || T < 0 || C < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if ((init_state && !aligned4(init_state)) || (final_state && !aligned4(final_state))) return LA_ERR_INVALID_ARG;
+    if (B > 0 && T > 0) {
+        if (!x || !f || !out) return LA_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(f) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    }
+    // rows of x and f are TMA tiles: their byte stride must be a multiple of 16
+    if (C % (dtype == LA_BF16 ? 8 : 4) != 0) return LA_ERR_UNSUPPORTED;
+    if (B > 65535 || !fits_int(static_cast<long long>(T) * C) || !fits_int(static_cast<long long>(B) * C))
+        return LA_ERR_UNSUPPORTED;
+    if (B == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    la::EmaArgs a{};
+    a.x = x;
+    a.f = f;
+    a.init_state = init_state;
+    a.out = out;
+    a.final_state = final_state;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.dtype = dtype;
+    a.reverse = reverse ? 1 : 0;
+    a.err_word = err_word_for_current_device();
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    return la::launch_ema(a) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 la_status la_decode_step(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
                          float* state, float* z, void* out, int B, int H, int Dk, int Dv, la_dtype dtype,
                          la_stream_t stream) {

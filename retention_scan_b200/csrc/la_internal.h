@@ -153,6 +153,24 @@ struct Wkv4Args {
     cudaStream_t stream;
 };
 cudaError_t launch_wkv4(const Wkv4Args& a);
+// [B, T, C] tensor map (la_wkv4.cu), boxes of [1, box_t, box_c], no swizzle.
+bool make_btc_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int es, int B, int T, int C, int box_c,
+                  int box_t);
+
+// Cumulative EMA along T (la_ema.cu).
+struct EmaArgs {
+    const void* x;            // values [B, T, C]
+    const void* f;            // factors [B, T, C]
+    const float* init_state;  // [B, C] or null (0)
+    void* out;                // [B, T, C]
+    float* final_state;       // [B, C] or null
+    int B, T, C;
+    la_dtype dtype;
+    int reverse;
+    int* err_word;
+    cudaStream_t stream;
+};
+cudaError_t launch_ema(const EmaArgs& a);
 size_t wkv4_workspace_bytes(int B, int T, int C, la_dtype dtype);
 
 }  // namespace la

@@ -280,17 +280,8 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
     }
 }
 
-// [B, T, C] tensor, boxes of [1, TT tokens, kCW channels], no swizzle.
 bool make_wkv_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int es, int B, int T, int C, int TT) {
-    EncodeTiledFn f = encode_tiled();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * es, static_cast<cuuint64_t>(C) * es * T};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kCW), static_cast<cuuint32_t>(TT), 1};
-    const cuuint32_t elem[3] = {1, 1, 1};
-    return f(map, dt, 3, const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return make_btc_map(map, base, dt, es, B, T, C, kCW, TT);
 }
 
 int sm_count_wkv() {
@@ -366,6 +357,20 @@ __global__ void wkv4_pass_state_kernel(const float* init_state, float* final_sta
 }
 
 }  // namespace
+
+// [B, T, C] tensor, boxes of [1, box_t tokens, box_c channels], no swizzle.
+bool make_btc_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int es, int B, int T, int C, int box_c,
+                  int box_t) {
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * es, static_cast<cuuint64_t>(C) * es * T};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_t), 1};
+    const cuuint32_t elem[3] = {1, 1, 1};
+    return f(map, dt, 3, const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t wkv4_workspace_bytes(int B, int T, int C, la_dtype dtype) {
     if (B < 1 || T < 1 || C < 1) return 0;

@@ -362,3 +362,21 @@ def test_backward_norm_validation(L):
     assert bn(B=0) == 0
     assert L.la_chunk_backward_norm_workspace_size(1, 8, 8192, 64, 64, 1, 2) > \
         L.la_chunk_backward_workspace_size(1, 8, 8192, 64, 64, 1, 2)
+
+
+def test_ema_validation(L):
+    vp = ctypes.c_void_p
+
+    def ema(**over):
+        a = dict(x=16, f=16, s0=None, out=16, sf=None, B=1, T=4, C=8, dtype=1, rev=0)
+        a.update(over)
+        return L.la_ema_scan(vp(a["x"]), vp(a["f"]), vp(a["s0"]), vp(a["out"]), vp(a["sf"]), a["B"], a["T"], a["C"],
+                             a["dtype"], a["rev"], None)
+    assert ema(x=None) == 1
+    assert ema(f=8) == 1          # not 16-byte aligned
+    assert ema(s0=2) == 1         # not 4-byte aligned
+    assert ema(C=0) == 1
+    assert ema(dtype=4) == 1
+    assert ema(C=12) == 2         # bf16 rows: C a multiple of 8
+    assert ema(C=6, dtype=0) == 2
+    assert ema(B=0) == 0

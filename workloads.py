@@ -26,6 +26,10 @@ run the same recipe at smaller sizes):
   decode     one token per call, per-head gamma_h, normalised with elu(x)+1 on
              q and k, fp32 state ~ N(0, 0.01^2), key sum |N(0, 0.01^2)|
              (B=256, H=32, Dk=Dv=128, 1024 steps, seed 5)
+  ema        RetNet issue 21's cumulative EMA: values x ~ N(0,1) and factors
+             f = sigmoid(a), a ~ N(3,1) (the page's elementwise EMA uses
+             sigmoid factors), bf16 [B,T,C]; zero start (B=8, T=4096,
+             C=2048, seed 7)
   wkv4       the RWKV-4 WKV recurrence: k, v ~ N(0,1) bf16 [B,T,C]; per
              channel w = -exp(d), d ~ N(-1, 1.5^2) (decay factors from about
              0.99 to near 0) and bonus u ~ N(-0.6, 0.4^2), fp32; empty start
@@ -245,3 +249,18 @@ def wkv4_inputs(wl, batches=None):
     w = -torch.exp(d)
     u = _normal((wl.C,), wl.seed, S0, 0, mean=-0.6, std=0.4)
     return dict(k=k.to(wl.torch_dtype), v=v.to(wl.torch_dtype), w=w.float(), u=u.float())
+
+
+# ---------------------------------------------------------------- cumulative EMA
+
+EMA = Wkv4Workload("ema_b8t4096c2048_bf16", B=8, T=4096, C=2048, dtype="bf16", seed=7)
+
+
+def ema_inputs(wl, batches=None):
+    """x, f [b, T, C] for the listed batch rows (all by default), each row
+    from its own generators: x ~ N(0,1), f = sigmoid(N(3,1))."""
+    rows = list(range(wl.B)) if batches is None else list(batches)
+    x = torch.stack([_normal((wl.T, wl.C), wl.seed, V, b) for b in rows])
+    f = torch.stack([torch.sigmoid(_normal((wl.T, wl.C), wl.seed, A, b, mean=3.0)) for b in rows])
+    return dict(x=x.to(wl.torch_dtype), f=f.to(wl.torch_dtype))
+
