@@ -9,10 +9,10 @@
 // One CTA per (batch row, 64 channels): a producer thread streams
 // [TT tokens x 64 channels] tiles of x and f into a ring of shared-memory
 // stages with TMA (in scan order: from the last tile for the reverse scan),
-// and each consumer thread (one per channel) runs its recurrence in fp32,
-// one FMA per step, reading its column of each tile with shared-memory loads
-// eight tokens ahead of the dependent steps.  The work per step is small, so
-// the kernel is bound by memory traffic: x and f read once, out written once.
+// and each consumer thread runs the recurrences of two adjacent channels in
+// fp32 (one 4- or 8-byte shared-memory load per array and step, one packed
+// store, two independent FMA chains), eight tokens ahead of the dependent
+// steps.  The direction is a template argument.
 // Every barrier wait gives up after kWaitLimitNs, sets the device error word
 // and unwinds.
 #include <cuda.h>
@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kCW = 64;
 constexpr int kStages = 4;
-constexpr int kConsumerWarps = kCW / 32;
+constexpr int kConsumerWarps = kCW / 64;  // two channels per thread
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
@@ -39,16 +39,21 @@ struct EmaTile {
     static constexpr int SMEM = kStages * STAGE + 256;
 };
 
-__device__ __forceinline__ float load_f(const float* p) { return *p; }
-__device__ __forceinline__ float load_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-__device__ __forceinline__ void store_e(float* p, float x) { *p = x; }
-__device__ __forceinline__ void store_e(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+// two adjacent channels
+__device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ void store2(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float2 v) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
 
-template <typename E>
+template <typename E, bool REV>
 __global__ void __launch_bounds__(kThreads) ema_kernel(const __grid_constant__ CUtensorMap tmx,
                                                        const __grid_constant__ CUtensorMap tmf,
                                                        const float* init_state, E* __restrict__ out,
-                                                       float* final_state, int T, int C, int reverse, int* err) {
+                                                       float* final_state, int T, int C, int* err) {
     using G = EmaTile<E>;
     extern __shared__ __align__(128) uint8_t sm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kStages * G::STAGE);
@@ -57,7 +62,7 @@ __global__ void __launch_bounds__(kThreads) ema_kernel(const __grid_constant__ C
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int b = blockIdx.y, c0 = blockIdx.x * kCW;
     const int ntiles = (T + G::TT - 1) / G::TT;
-    auto tile_of = [&](int j) { return reverse ? ntiles - 1 - j : j; };  // memory tile of the j-th scanned tile
+    auto tile_of = [&](int j) { return REV ? ntiles - 1 - j : j; };  // memory tile of the j-th scanned tile
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmx);
@@ -94,9 +99,11 @@ __global__ void __launch_bounds__(kThreads) ema_kernel(const __grid_constant__ C
         return;
     }
 
-    const int c = c0 + threadIdx.x;
+    const int c = c0 + 2 * threadIdx.x;  // channels c, c + 1 (C is even)
     const bool live = c < C;
-    float sv = (live && init_state) ? init_state[static_cast<size_t>(b) * C + c] : 0.f;
+    float2 sv = make_float2(0.f, 0.f);
+    if (live && init_state) sv = make_float2(init_state[static_cast<size_t>(b) * C + c],
+                                             init_state[static_cast<size_t>(b) * C + c + 1]);
     E* ob = out + static_cast<size_t>(b) * T * C + c;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
@@ -119,37 +126,45 @@ __global__ void __launch_bounds__(kThreads) ema_kernel(const __grid_constant__ C
             }
             if (!ok) break;
         }
-        const E* tx = reinterpret_cast<const E*>(sm + s * G::STAGE) + threadIdx.x;
-        const E* tf = reinterpret_cast<const E*>(sm + s * G::STAGE + G::BYTES) + threadIdx.x;
+        const E* tx = reinterpret_cast<const E*>(sm + s * G::STAGE) + 2 * threadIdx.x;
+        const E* tf = reinterpret_cast<const E*>(sm + s * G::STAGE + G::BYTES) + 2 * threadIdx.x;
         const int t0 = tile_of(j) * G::TT;
         const int n = min(G::TT, T - t0);
         if (live) {
-            // row r of the tile in scan order: forward r = i, reverse r = n - 1 - i
-            auto row = [&](int i) { return reverse ? n - 1 - i : i; };
+            // rows in scan order: forward from row 0, reverse from row n - 1
+            const E* px = tx + (REV ? (n - 1) * kCW : 0);
+            const E* pf = tf + (REV ? (n - 1) * kCW : 0);
+            E* po = ob + static_cast<size_t>(t0 + (REV ? n - 1 : 0)) * C;
+            constexpr int dr = REV ? -kCW : kCW;
+            const long long dout = REV ? -static_cast<long long>(C) : static_cast<long long>(C);
             const int nb = n / 8;
-            float xx[8], ff[8];
+            float2 xx[8], ff[8];
             if (nb > 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    xx[e] = load_f(tx + row(e) * kCW);
-                    ff[e] = load_f(tf + row(e) * kCW);
+                    xx[e] = load2(px + e * dr);
+                    ff[e] = load2(pf + e * dr);
                 }
             }
             for (int bi = 0; bi < nb; ++bi) {
-                float xn[8], fn[8], yy[8];
-                const int nxt = bi + 1 < nb ? (bi + 1) * 8 : bi * 8;  // (a harmless re-read at the end)
+                float2 xn[8], fn[8], yy[8];
+                const int nxt = bi + 1 < nb ? 8 : 0;  // (a harmless re-read at the end)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    xn[e] = load_f(tx + row(nxt + e) * kCW);
-                    fn[e] = load_f(tf + row(nxt + e) * kCW);
+                    xn[e] = load2(px + (nxt + e) * dr);
+                    fn[e] = load2(pf + (nxt + e) * dr);
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    sv = fmaf(ff[e], sv, xx[e]);
+                    sv.x = fmaf(ff[e].x, sv.x, xx[e].x);
+                    sv.y = fmaf(ff[e].y, sv.y, xx[e].y);
                     yy[e] = sv;
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) store_e(ob + static_cast<size_t>(t0 + row(bi * 8 + e)) * C, yy[e]);
+                for (int e = 0; e < 8; ++e) store2(po + e * dout, yy[e]);
+                po += 8 * dout;
+                px += 8 * dr;
+                pf += 8 * dr;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     xx[e] = xn[e];
@@ -157,27 +172,36 @@ __global__ void __launch_bounds__(kThreads) ema_kernel(const __grid_constant__ C
                 }
             }
             for (int i = nb * 8; i < n; ++i) {
-                sv = fmaf(load_f(tf + row(i) * kCW), sv, load_f(tx + row(i) * kCW));
-                store_e(ob + static_cast<size_t>(t0 + row(i)) * C, sv);
+                const float2 x2 = load2(px), f2 = load2(pf);
+                sv.x = fmaf(f2.x, sv.x, x2.x);
+                sv.y = fmaf(f2.y, sv.y, x2.y);
+                store2(po, sv);
+                po += dout;
+                px += dr;
+                pf += dr;
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (ok && live && final_state) final_state[static_cast<size_t>(b) * C + c] = sv;
+    if (ok && live && final_state) {
+        final_state[static_cast<size_t>(b) * C + c] = sv.x;
+        final_state[static_cast<size_t>(b) * C + c + 1] = sv.y;
+    }
 }
 
-template <typename E>
+template <typename E, bool REV>
 cudaError_t launch_typed(const EmaArgs& a, CUtensorMapDataType dt) {
     using G = EmaTile<E>;
     CUtensorMap tmx, tmf;
     if (!make_btc_map(&tmx, a.x, dt, sizeof(E), a.B, a.T, a.C, kCW, G::TT) ||
         !make_btc_map(&tmf, a.f, dt, sizeof(E), a.B, a.T, a.C, kCW, G::TT))
         return cudaErrorInvalidValue;
-    const cudaError_t e = cudaFuncSetAttribute(ema_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+    const cudaError_t e =
+        cudaFuncSetAttribute(ema_kernel<E, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
     if (e != cudaSuccess) return e;
-    ema_kernel<E><<<dim3((a.C + kCW - 1) / kCW, a.B), kThreads, G::SMEM, a.stream>>>(
-        tmx, tmf, a.init_state, static_cast<E*>(a.out), a.final_state, a.T, a.C, a.reverse, a.err_word);
+    ema_kernel<E, REV><<<dim3((a.C + kCW - 1) / kCW, a.B), kThreads, G::SMEM, a.stream>>>(
+        tmx, tmf, a.init_state, static_cast<E*>(a.out), a.final_state, a.T, a.C, a.err_word);
     return cudaGetLastError();
 }
 
@@ -190,8 +214,11 @@ cudaError_t launch_ema(const EmaArgs& a) {
         return a.init_state ? cudaMemcpyAsync(a.final_state, a.init_state, bytes, cudaMemcpyDeviceToDevice, a.stream)
                             : cudaMemsetAsync(a.final_state, 0, bytes, a.stream);
     }
-    return a.dtype == LA_BF16 ? launch_typed<__nv_bfloat16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
-                              : launch_typed<float>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    if (a.dtype == LA_BF16)
+        return a.reverse ? launch_typed<__nv_bfloat16, true>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                         : launch_typed<__nv_bfloat16, false>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    return a.reverse ? launch_typed<float, true>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                     : launch_typed<float, false>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
 }
 
 }  // namespace la
