@@ -13,8 +13,8 @@
 //
 // Data movement: a CTA owns one batch row, kCW consecutive channels and one
 // T-segment.  One producer thread streams [TT tokens x kCW channels] tiles
-// of k and v into a ring of kStages shared-memory stages with TMA (four CTAs
-// per SM, about 190 KB in flight per SM), so the HBM latency is hidden
+// of k and v into a ring of kStages shared-memory stages with TMA (eight CTAs
+// per SM, about 200 KB in flight per SM), so the HBM latency is hidden
 // behind the sequential per-token work; each consumer thread reads its
 // channel's column of the tile and writes its output directly (a warp writes
 // 32 consecutive values).
@@ -40,10 +40,10 @@ namespace la {
 namespace {
 
 constexpr int kCW = 64;                 // channels per CTA (one per consumer thread)
-constexpr int kStages = 3;              // 3 x 16 KB: four CTAs per SM
+constexpr int kStages = 3;              // 3 x 8 KB: eight CTAs per SM
 constexpr int kConsumerWarps = kCW / 32;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one producer warp
-constexpr int kCtasPerSm = 4;
+constexpr int kCtasPerSm = 8;
 constexpr int kMinSegTokens = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -51,7 +51,7 @@ constexpr float kEmptyScale = -1e38f;   // pp of an empty state (aa = bb = 0)
 
 template <typename E>
 struct Tile {
-    static constexpr int TT = sizeof(E) == 2 ? 64 : 32;           // tokens per stage
+    static constexpr int TT = sizeof(E) == 2 ? 32 : 16;           // tokens per stage
     static constexpr int BYTES = TT * kCW * static_cast<int>(sizeof(E));  // one array's tile
     static constexpr int STAGE = 2 * BYTES;                        // k tile, then v tile
     static constexpr int SMEM = kStages * STAGE + 256;             // + barriers
@@ -319,6 +319,10 @@ cudaError_t launch_typed(const Wkv4Args& a, CUtensorMapDataType dt) {
         !make_wkv_map(&tmv, a.v, dt, sizeof(E), a.B, a.T, a.C, G::TT))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(wkv4_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+    if (e != cudaSuccess) return e;
+    // all of the SM's shared memory, so that kCtasPerSm CTAs stay resident
+    e = cudaFuncSetAttribute(wkv4_kernel<E>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     WkvLayout L = wkv_layout(a.B, a.T, a.C, G::TT, a.workspace != nullptr);
     const size_t need = sizeof(float) * static_cast<size_t>(a.B) * L.nseg * 3 * a.C;

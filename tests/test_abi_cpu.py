@@ -309,10 +309,10 @@ def test_wkv4_validation(L, over, status):
 
 
 def test_wkv4_workspace_size(L):
-    # 148 SMs (the host default without a device), four CTAs per SM, CTAs of
-    # 64 channels: B8 C2048 (256 CTAs) doubles once to two segments of 2048
+    # 148 SMs (the host default without a device), eight CTAs per SM, CTAs of
+    # 64 channels: B8 C2048 (256 CTAs) doubles twice to four segments of 1024
     # tokens; one CTA and T = 4173 reaches eight segments of at least 512
-    assert L.la_wkv4_workspace_size(8, 4096, 2048, 1) == 8 * 2 * 3 * 2048 * 4
+    assert L.la_wkv4_workspace_size(8, 4096, 2048, 1) == 8 * 4 * 3 * 2048 * 4
     assert L.la_wkv4_workspace_size(1, 4173, 64, 1) == 1 * 8 * 3 * 64 * 4
     assert L.la_wkv4_workspace_size(2, 1000, 192, 1) == 0   # segments would be shorter than 512 tokens
     assert L.la_wkv4_workspace_size(0, 4096, 64, 1) == 0

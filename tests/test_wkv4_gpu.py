@@ -115,6 +115,46 @@ def test_wkv4_large_keys_stay_finite(dtype):
     assert max(errs.values()) <= bar, (errs, bar)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_wkv4_mixed_scales(dtype):
+    """Inputs that take every branch of the kernel's per-token work: key
+    spikes far above and below the running scale in some channels and some
+    tokens (single batches of eight tokens redone token by token), channels
+    with a large bonus or a growing factor (w > 0: their warps always step
+    token by token), an empty start in one batch row and a carried state at
+    a large scale in the other; T and C ragged."""
+    B, T, C = 2, 333, 72
+    g = torch.Generator().manual_seed(4250)
+    k = torch.randn(B, T, C, generator=g)
+    spikes = torch.rand(B, T, C, generator=g)
+    k = torch.where(spikes < 0.01, k + 70.0, k)
+    k = torch.where(spikes > 0.99, k - 120.0, k)
+    v = torch.randn(B, T, C, generator=g)
+    w = -torch.exp(torch.randn(C, generator=g) * 1.5 - 1.0)
+    w[5] = 0.0
+    w[40] = 0.05
+    w[70] = -60.0
+    u = torch.randn(C, generator=g) * 0.4 - 0.6
+    u[33] = 30.0
+    u[66] = -40.0
+    S0 = torch.stack([torch.randn(B, C, generator=g), torch.rand(B, C, generator=g) + 0.1,
+                      torch.randn(B, C, generator=g) + 50.0], dim=1)
+    S0[0, 0] = 0.0
+    S0[0, 1] = 0.0
+    S0[0, 2] = oracle.WKV4_EMPTY_SCALE
+    k, v = k.to(dtype), v.to(dtype)
+    out, fin = la().wkv4_forward(k.cuda(), v.cuda(), w.cuda(), u.cuda(), S0.cuda())
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+    ro, rf = oracle.wkv4(k, v, w, u, S0)
+    assert row_err(out, ro) <= TOL[dtype]
+    # the running scale reaches about 70 (100 in log2 units): the state bar
+    # of the large-key case
+    bar = max(TOL[dtype], 8 * 2.0 ** -16 * T ** 0.5)
+    errs = state_errs(fin, rf)
+    assert max(errs.values()) <= bar, (errs, bar)
+
+
 def test_wkv4_split_and_carry_in_place():
     """Two calls with the state carried in place equal one call."""
     k, v, w, u, S0 = case(3, 257, 128, torch.bfloat16, True, seed=4300)
