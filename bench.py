@@ -1,7 +1,7 @@
 """Benchmark of the causal-linear-attention library on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
-                    [--direction forward|reverse|bidirectional]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..7] [--impl ours|reference]
+                    [--direction forward|reverse|bidirectional|backward]
 
 One step is one pass of the hot path over one batch of the workload:
 
@@ -22,7 +22,8 @@ the reverse scan adding to its output; no carried state); --direction
 backward the gradients of the forward (la_chunk_backward_ws, or
 la_chunk_backward_norm_ws for the normalised workload: dq, dk, dv, the
 log-decay gradient and, with a carried state, the initial state's and key
-sum's) for a seeded upstream gradient dy.  Configs 1-4.
+sum's) for a seeded upstream gradient dy.  Configs 1-4; config 7 takes
+forward or reverse (la_ema_scan's reverse flag).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
@@ -624,9 +625,9 @@ def ema_bytes(wl):
 
 
 class EmaJob:
-    def __init__(self, device, wl, rank=0):
+    def __init__(self, device, wl, rank=0, reverse=False):
         import retention_scan_b200 as la
-        self.la, self.wl, self.dev = la, wl, device
+        self.la, self.wl, self.dev, self.reverse = la, wl, device, reverse
         self.host = W.ema_inputs(wl.with_sizes(seed=wl.seed + 7919 * rank))
         self.x, self.f = (self.host[n].to(device) for n in ("x", "f"))
         self.out = torch.empty(wl.B, wl.T, wl.C, dtype=wl.torch_dtype, device=device)
@@ -634,7 +635,7 @@ class EmaJob:
         self.launches = 1
 
     def step(self):
-        self.la.ema_scan(self.x, self.f, out=self.out, final_state=self.fin)
+        self.la.ema_scan(self.x, self.f, out=self.out, final_state=self.fin, reverse=self.reverse)
         return 1
 
     def e2e(self, steps, dist_on):
@@ -644,7 +645,7 @@ class EmaJob:
 
         def one():
             x, f = (p[n].to(self.dev, non_blocking=True) for n in ("x", "f"))
-            o, _ = self.la.ema_scan(x, f, out=self.out, final_state=self.fin)
+            o, _ = self.la.ema_scan(x, f, out=self.out, final_state=self.fin, reverse=self.reverse)
             y.copy_(o, non_blocking=True)
         for _ in range(2):
             one()
@@ -659,7 +660,7 @@ class EmaJob:
         return ev0.elapsed_time(ev1) / steps, h2d, y.numel() * y.element_size()
 
 
-def cpu_baseline_ema(wl, budget_s=15.0):
+def cpu_baseline_ema(wl, budget_s=15.0, reverse=False):
     """The float64 oracle (single-threaded C loop) on whole batch rows."""
     import oracle
     oracle.build()
@@ -667,7 +668,7 @@ def cpu_baseline_ema(wl, budget_s=15.0):
     nb = max(1, min(wl.B, int(budget_s / max(per_row_s, 1e-9))))
     inp = W.ema_inputs(wl, batches=range(nb))
     t0 = time.perf_counter()
-    oracle.ema(inp["x"], inp["f"])
+    oracle.ema(inp["x"], inp["f"], reverse=reverse)
     dt = time.perf_counter() - t0
     return {"value": nb * wl.T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{nb} of {wl.B} batch rows, all {wl.T} tokens x {wl.C} channels, single thread"}
@@ -735,7 +736,7 @@ def run_wkv4(args, rank, world, dist_on, device):
         wl = wl.with_sizes(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.batch:
         wl = wl.with_sizes(B=args.batch, name=f"{wl.name}_B{args.batch}")
-    job = (EmaJob if ema else Wkv4Job)(device, wl, rank)
+    job = EmaJob(device, wl, rank, reverse=args.direction == "reverse") if ema else Wkv4Job(device, wl, rank)
     nbytes = (ema_bytes if ema else wkv4_bytes)(wl)
     flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device) if nbytes < 2 * L2_BYTES else None
     for _ in range(args.warmup):
@@ -768,6 +769,7 @@ def run_wkv4(args, rank, world, dist_on, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+                   **({"direction": args.direction} if ema else {}),
                    "l2": "flushed before every step (512 MB write)" if flush is not None
                    else "inputs larger than L2",
                    "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels"
@@ -839,8 +841,10 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
     ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional", "backward"])
     args = ap.parse_args()
-    if args.config in (5, 6, 7) and args.direction != "forward":
-        ap.error("--direction applies to the whole-sequence configs 1-4")
+    if args.config in (5, 6) and args.direction != "forward":
+        ap.error("--direction applies to the whole-sequence configs 1-4 and 7")
+    if args.config == 7 and args.direction not in ("forward", "reverse"):
+        ap.error("the cumulative EMA (config 7) scans forward or reverse")
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200, 7: 200}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
@@ -869,7 +873,8 @@ def main():
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
                 line["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4) if args.config == 6 else
-                                        cpu_baseline_ema(W.EMA) if args.config == 7 else
+                                        cpu_baseline_ema(W.EMA, reverse=args.direction == "reverse")
+                                        if args.config == 7 else
                                         cpu_baseline(args.config, direction=args.direction))
             print(json.dumps(line), flush=True)
     finally:
