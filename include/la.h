@@ -226,6 +226,70 @@ LA_API la_status la_chunk_reverse_ws(const void* q, const void* k, const void* v
                               la_stream_t stream);
 
 /*
+ * la_chunk_state_ws - the state a span of the sequence leaves when it starts
+ * from zero, and the span's total log decay (no outputs, no queries).
+ *
+ *   S_0 = 0, z_0 = 0;  S_t = g_t S_{t-1} + k_t v_t^T,  z_t = g_t z_{t-1} + k_t
+ *   state_out = S_T,  z_out = z_T,  log_g_total[b,h] = sum_t log g_t
+ *
+ * With these, the state entering any later span follows from the associative
+ * combination of consecutive spans, RetNet issue 21 (the paragraph on the
+ * associative EMA operator): (S_a, G_a) o (S_b, G_b) = (G_b S_a + S_b, G_a G_b)
+ * with G = exp(log_g_total) (la_state_combine).  This is the first step of a
+ * sequence split along T over GPUs: each span's state, one exchange of them,
+ * then each span's forward from the combined state entering it.
+ *
+ *   k, v, decay, normalize, B, H, T, Dk, Dv, dtype   as la_chunk_forward_ws
+ *   state_out    [B, H, Dk, Dv] fp32, required, 16-byte aligned.
+ *   z_out        [B, H, Dk] fp32, required (16-byte aligned) when normalize,
+ *                else ignored.
+ *   log_g_total  [B, H] fp32 natural log, or NULL (not written).
+ *   workspace    bf16: at least la_chunk_state_workspace_size(...) bytes,
+ *                16-byte aligned, required when T > 0; fp32: unused.
+ *
+ * T == 0 writes zero states and a zero log total.  Errors: as
+ * la_chunk_forward_ws, and LA_ERR_INVALID_ARG for a missing or short bf16
+ * workspace.  bf16 runs the chunked kernel's state pass over pieces of the
+ * span and folds them; fp32 runs the recurrent kernel without its outputs.
+ */
+LA_API size_t la_chunk_state_workspace_size(int B, int H, int T, int Dk, int Dv,
+                                            la_dtype dtype, int normalize);
+LA_API la_status la_chunk_state_ws(const void* k, const void* v, const la_decay* decay,
+                                   int normalize, float* state_out, float* z_out,
+                                   float* log_g_total, int B, int H, int T, int Dk, int Dv,
+                                   la_dtype dtype, void* workspace, size_t workspace_bytes,
+                                   la_stream_t stream);
+
+/*
+ * la_state_combine - the left fold of n consecutive spans' states with the
+ * associative operator above (RetNet issue 21, the associative EMA operator):
+ *
+ *   S <- init_state (or 0),  z <- init_z (or 0)
+ *   for j = 0 .. n-1:  S <- exp(L_j) S + S_j,  z <- exp(L_j) z + z_j
+ *   state_out = S,  z_out = z,  log_g_out = sum_j L_j
+ *
+ * so that state_out is the state after spans 0..n-1 entered with init_state.
+ *   seg_state   span j's [B, H, Dk, Dv] fp32 state at seg_state + j * state_stride
+ *   seg_z       span j's [B, H, Dk] key sum at seg_z + j * z_stride (needed when
+ *               z_out is given and n > 0)
+ *   seg_log_g   span j's [B, H] natural-log total decay at seg_log_g + j * log_stride
+ *               (strides in floats, >= 0)
+ *   init_state, init_z   [B, H, Dk, Dv] / [B, H, Dk] fp32 or NULL (zero)
+ *   state_out   [B, H, Dk, Dv] fp32, required; may be init_state (each element
+ *               is read before it is written)
+ *   z_out, log_g_out     [B, H, Dk] / [B, H] fp32 or NULL (not written)
+ * Every pointer 4-byte aligned.  n == 0 copies the initial state (or zeros).
+ * Errors: LA_ERR_INVALID_ARG for negative sizes or strides, a missing
+ * required pointer or a misaligned one; LA_ERR_CUDA if the launch fails.
+ */
+LA_API la_status la_state_combine(const float* seg_state, const float* seg_z,
+                                  const float* seg_log_g, long long state_stride,
+                                  long long z_stride, long long log_stride, int n,
+                                  const float* init_state, const float* init_z,
+                                  float* state_out, float* z_out, float* log_g_out,
+                                  int B, int H, int Dk, int Dv, la_stream_t stream);
+
+/*
  * la_chunk_bidirectional_ws - the bidirectional (encoder) form:
  * out = y_forward + y_reverse, both scans from zero states.
  *

@@ -14,7 +14,7 @@ import os
 import torch
 
 __all__ = ["chunk_forward", "bidirectional", "chunk_backward", "chunk_backward_normalized", "wkv4_forward", "ema_scan",
-           "workspace_size",
+           "chunk_state", "state_combine", "state_workspace_size", "workspace_size",
            "backward_workspace_size",
            "decode_step", "device_error", "LAError", "lib", "library_path",
            "DECAY_NONE", "DECAY_PER_HEAD", "DECAY_PER_STEP", "FEATURE_NONE", "FEATURE_ELU1", "EXPORTED_SYMBOLS"]
@@ -30,7 +30,7 @@ EXPORTED_SYMBOLS = ("la_chunk_forward", "la_chunk_forward_ws", "la_chunk_forward
                     "la_chunk_backward_ws", "la_chunk_backward_workspace_size", "la_wkv4_forward",
                     "la_wkv4_forward_ws", "la_wkv4_workspace_size", "la_chunk_forward_pro_ws",
                     "la_decode_step_pro", "la_chunk_backward_norm_ws", "la_chunk_backward_norm_workspace_size",
-                    "la_ema_scan",
+                    "la_ema_scan", "la_chunk_state_ws", "la_chunk_state_workspace_size", "la_state_combine",
                     "la_decode_step", "la_status_string", "la_device_error", "la_version")
 
 
@@ -91,6 +91,14 @@ def lib():
         L.la_chunk_backward_workspace_size.restype = ctypes.c_size_t
         L.la_ema_scan.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
         L.la_ema_scan.restype = i
+        L.la_chunk_state_ws.argtypes = [vp, vp, ctypes.POINTER(_Decay), i, vp, vp, vp, i, i, i, i, i, i, vp,
+                                        ctypes.c_size_t, vp]
+        L.la_chunk_state_ws.restype = i
+        L.la_chunk_state_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        L.la_chunk_state_workspace_size.restype = ctypes.c_size_t
+        ll = ctypes.c_longlong
+        L.la_state_combine.argtypes = [vp, vp, vp, ll, ll, ll, i, vp, vp, vp, vp, vp, i, i, i, i, vp]
+        L.la_state_combine.restype = i
         L.la_wkv4_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
         L.la_wkv4_forward.restype = i
         L.la_wkv4_forward_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, ctypes.c_size_t, vp]
@@ -330,6 +338,95 @@ def chunk_backward(q, k, v, dy, decay_kind=DECAY_NONE, log_g=None, init_state=No
             _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_log_g), _ptr(d_init),
             B, H, T, Dk, Dv, code, _ptr(workspace), workspace.numel(), _stream(stream, dev)))
     return dq, dk, dv, d_log_g, d_init
+
+
+def state_workspace_size(B, H, T, Dk, Dv, dtype=torch.bfloat16, normalize=False):
+    """Scratch bytes chunk_state needs for these sizes (la_chunk_state_workspace_size)."""
+    return int(lib().la_chunk_state_workspace_size(B, H, T, Dk, Dv, _dtype_code(dtype), int(bool(normalize))))
+
+
+def chunk_state(k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False, state_out=None, z_out=None,
+                log_g_total=None, stream=None, workspace=True):
+    """A span's own state from zero and its total log decay (la_chunk_state_ws):
+    S_T and z_T of the recurrence started from zero, and sum_t log g_t per
+    (b, h).  k [B,H,T,Dk], v [B,H,T,Dv] float32 or bfloat16; decay as
+    chunk_forward.  Returns (state [B,H,Dk,Dv], z [B,H,Dk] or None,
+    log_g_total [B,H]), fp32.  workspace: True allocates the bf16 scratch, or
+    a CUDA uint8 tensor of at least state_workspace_size bytes."""
+    B, H, T, Dk = k.shape
+    Dv = v.shape[-1]
+    dev = k.device
+    code = _dtype_code(k.dtype)
+    _need(v, "v", (B, H, T, Dv), k.dtype, dev)
+    if decay_kind == DECAY_PER_HEAD:
+        _need(log_g, "log_g", (H,), torch.float32, dev)
+    elif decay_kind == DECAY_PER_STEP:
+        _need(log_g, "log_g", (B, H, T), torch.float32, dev)
+    if state_out is None:
+        state_out = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
+    if z_out is None and normalize:
+        z_out = torch.empty((B, H, Dk), dtype=torch.float32, device=dev)
+    if log_g_total is None:
+        log_g_total = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", (B, H, Dk, Dv), torch.float32, dev)
+    _need(z_out, "z_out", (B, H, Dk), torch.float32, dev)
+    _need(log_g_total, "log_g_total", (B, H), torch.float32, dev)
+    d = _decay(decay_kind, log_g)
+    with torch.cuda.device(dev):
+        if workspace is True:
+            nbytes = state_workspace_size(B, H, T, Dk, Dv, k.dtype, normalize)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+            if workspace is not None and stream is not None:
+                workspace.record_stream(stream)
+        elif workspace is False:
+            workspace = None
+        _check(lib().la_chunk_state_ws(
+            _ptr(k), _ptr(v), ctypes.byref(d) if d is not None else None, int(bool(normalize)), _ptr(state_out),
+            _ptr(z_out if normalize else None), _ptr(log_g_total), B, H, T, Dk, Dv, code, _ptr(workspace),
+            0 if workspace is None else workspace.numel(), _stream(stream, dev)))
+    return state_out, (z_out if normalize else None), log_g_total
+
+
+def _span_rows(t, name, inner):
+    """t: [n, *inner] fp32 whose spans (dim 0) are each contiguous; its
+    stride along dim 0 in floats."""
+    if tuple(t.shape[1:]) != tuple(inner):
+        raise ValueError(f"{name}: expected shape [n, {', '.join(map(str, inner))}], got {tuple(t.shape)}")
+    if t.dtype != torch.float32:
+        raise TypeError(f"{name}: expected float32, got {t.dtype}")
+    if t.shape[0] > 0 and not t[0].is_contiguous():
+        raise ValueError(f"{name}: each span must be contiguous")
+    return t.stride(0)
+
+
+def state_combine(seg_state, seg_log_g, seg_z=None, init_state=None, init_z=None, state_out=None, z_out=None,
+                  log_g_out=None, stream=None):
+    """The left fold of n consecutive spans' states (la_state_combine):
+    S <- init_state (or 0); for each span j: S <- exp(L_j) S + S_j (z
+    likewise); returns (state, z or None, total log decay).  seg_state
+    [n,B,H,Dk,Dv], seg_log_g [n,B,H], seg_z [n,B,H,Dk] (needed for z) -
+    fp32 CUDA tensors whose spans may be strided views of one buffer."""
+    n, B, H, Dk, Dv = seg_state.shape
+    dev = seg_state.device
+    ss = _span_rows(seg_state, "seg_state", (B, H, Dk, Dv))
+    ls = _span_rows(seg_log_g, "seg_log_g", (B, H))
+    zs = _span_rows(seg_z, "seg_z", (B, H, Dk)) if seg_z is not None else 0
+    if state_out is None:
+        state_out = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
+    if z_out is None and seg_z is not None:
+        z_out = torch.empty((B, H, Dk), dtype=torch.float32, device=dev)
+    if log_g_out is None:
+        log_g_out = torch.empty((B, H), dtype=torch.float32, device=dev)
+    for t, name, shape in ((init_state, "init_state", (B, H, Dk, Dv)), (init_z, "init_z", (B, H, Dk)),
+                           (state_out, "state_out", (B, H, Dk, Dv)), (z_out, "z_out", (B, H, Dk)),
+                           (log_g_out, "log_g_out", (B, H))):
+        _need(t, name, shape, torch.float32, dev)
+    with torch.cuda.device(dev):
+        _check(lib().la_state_combine(
+            _ptr(seg_state) if n else None, _ptr(seg_z) if n and seg_z is not None else None,
+            _ptr(seg_log_g) if n else None, ss, zs, ls, n, _ptr(init_state), _ptr(init_z), _ptr(state_out),
+            _ptr(z_out), _ptr(log_g_out), B, H, Dk, Dv, _stream(stream, dev)))
+    return state_out, z_out, log_g_out
 
 
 def ema_scan(x, f, init_state=None, reverse=False, out=None, final_state=None, return_final=True, stream=None):

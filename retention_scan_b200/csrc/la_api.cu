@@ -333,6 +333,143 @@ la_status la_chunk_reverse_ws(const void* q, const void* k, const void* v, const
                 workspace, workspace_bytes, stream, 1, 0);
 }
 
+size_t la_chunk_state_workspace_size(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int normalize) {
+    if (dtype != LA_BF16 || B < 1 || H < 1 || T < 1) return 0;
+    if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
+    return la::fwd_state_workspace_bytes(B, H, T, Dk, Dv, normalize != 0);
+}
+
+la_status la_chunk_state_ws(const void* k, const void* v, const la_decay* decay, int normalize, float* state_out,
+                            float* z_out, float* log_g_total, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
+                            void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
+    int kind;
+    const float* log_g;
+    if (check_decay(decay, &kind, &log_g) != LA_OK) return LA_ERR_INVALID_ARG;
+    normalize = normalize ? 1 : 0;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH * 8)) return LA_ERR_INVALID_ARG;
+    if (!state_out || !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if (normalize && (!z_out || !aligned16(z_out))) return LA_ERR_INVALID_ARG;
+    if (log_g_total && !aligned4(log_g_total)) return LA_ERR_INVALID_ARG;
+    if (BH > 0 && T > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
+    if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
+    if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
+    if (BH == 0) return LA_OK;
+    if (dtype == LA_BF16 && T > 0) {
+        const size_t need = la::fwd_state_workspace_bytes(B, H, T, Dk, Dv, normalize != 0);
+        if (!workspace || workspace_bytes < need) return LA_ERR_INVALID_ARG;
+    }
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {  // an empty span: zero state, no decay
+        cudaError_t e = cudaMemsetAsync(state_out, 0, sizeof(float) * static_cast<size_t>(BH) * Dk * Dv, s);
+        if (e == cudaSuccess && normalize) e = cudaMemsetAsync(z_out, 0, sizeof(float) * static_cast<size_t>(BH) * Dk, s);
+        if (e == cudaSuccess && log_g_total) e = cudaMemsetAsync(log_g_total, 0, sizeof(float) * BH, s);
+        return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    }
+    la::FwdArgs a{};
+    a.q = k;  // no read-out is kept: the keys stand in for the queries
+    a.k = k;
+    a.v = v;
+    a.decay_kind = kind;
+    a.log_g = log_g;
+    a.normalize = normalize;
+    a.B = B;
+    a.H = H;
+    a.T = T;
+    a.Dk = Dk;
+    a.Dv = Dv;
+    a.stream = s;
+    a.err_word = err_word_for_current_device();
+    a.q_scale = 1.f;
+    cudaError_t e;
+    if (dtype == LA_F32) {
+        a.out = nullptr;  // the recurrent kernel keeps the state alone
+        a.final_state = state_out;
+        a.final_z = normalize ? z_out : nullptr;
+        e = la::launch_fwd_f32(a);
+        if (e == cudaSuccess && log_g_total)
+            e = la::launch_log_total(log_g, kind, static_cast<int>(BH), H, T, log_g_total, s);
+    } else {
+        a.workspace = workspace;
+        a.workspace_bytes = workspace_bytes;
+        int pieces = 0;
+        e = la::launch_fwd_state(a, &pieces);
+        if (e == cudaErrorNotSupported) return LA_ERR_UNSUPPORTED;
+        if (e == cudaSuccess) {
+            // fold the pieces, in order, into the span's state
+            const long long DkDv = static_cast<long long>(Dk) * Dv;
+            const float* base = static_cast<const float*>(workspace);
+            la::CombineArgs c{};
+            c.S = base;
+            c.S_span = DkDv;
+            c.S_bh = pieces * DkDv;
+            c.z = base + BH * pieces * DkDv;
+            c.z_span = Dk;
+            c.z_bh = static_cast<long long>(pieces) * Dk;
+            c.L = c.z + BH * pieces * Dk;
+            c.L_span = 1;
+            c.L_bh = pieces;
+            c.n = pieces;
+            c.log2_units = 1;
+            c.out_S = state_out;
+            c.out_z = normalize ? z_out : nullptr;
+            c.out_L = log_g_total;
+            c.BH = static_cast<int>(BH);
+            c.Dk = Dk;
+            c.Dv = Dv;
+            c.stream = s;
+            e = la::launch_fold(c);
+        }
+    }
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_state_combine(const float* seg_state, const float* seg_z, const float* seg_log_g, long long state_stride,
+                           long long z_stride, long long log_stride, int n, const float* init_state,
+                           const float* init_z, float* state_out, float* z_out, float* log_g_out, int B, int H,
+                           int Dk, int Dv, la_stream_t stream) {
+    if (B < 0 || H < 0 || Dk < 1 || Dv < 1 || n < 0) return LA_ERR_INVALID_ARG;
+    if (state_stride < 0 || z_stride < 0 || log_stride < 0) return LA_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!fits_int(BH * 8)) return LA_ERR_INVALID_ARG;
+    if (!state_out || !aligned4(state_out)) return LA_ERR_INVALID_ARG;
+    for (const void* p : {static_cast<const void*>(seg_state), static_cast<const void*>(seg_z),
+                          static_cast<const void*>(seg_log_g), static_cast<const void*>(init_state),
+                          static_cast<const void*>(init_z), static_cast<const void*>(z_out),
+                          static_cast<const void*>(log_g_out)})
+        if (p && !aligned4(p)) return LA_ERR_INVALID_ARG;
+    if (n > 0 && (!seg_state || !seg_log_g)) return LA_ERR_INVALID_ARG;
+    if (n > 0 && z_out && !seg_z) return LA_ERR_INVALID_ARG;
+    if (BH == 0) return LA_OK;
+    if (launch_fault_injected()) return LA_ERR_CUDA;
+    la::CombineArgs c{};
+    c.S = seg_state;
+    c.S_span = state_stride;
+    c.S_bh = static_cast<long long>(Dk) * Dv;
+    c.z = seg_z;
+    c.z_span = z_stride;
+    c.z_bh = Dk;
+    c.L = seg_log_g;
+    c.L_span = log_stride;
+    c.L_bh = 1;
+    c.n = n;
+    c.log2_units = 0;
+    c.init_S = init_state;
+    c.init_z = z_out ? init_z : nullptr;
+    c.out_S = state_out;
+    c.out_z = z_out;
+    c.out_L = log_g_out;
+    c.BH = static_cast<int>(BH);
+    c.Dk = Dk;
+    c.Dv = Dv;
+    c.stream = reinterpret_cast<cudaStream_t>(stream);
+    return la::launch_fold(c) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 la_status la_chunk_bidirectional_ws(const void* q, const void* k, const void* v, const la_decay* decay,
                                     int normalize, void* out, int B, int H, int T, int Dk, int Dv, la_dtype dtype,
                                     void* workspace, size_t workspace_bytes, la_stream_t stream) {

@@ -97,8 +97,10 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
                     for (int i = 0; i < Dk; ++i) den += qz[j * Dk + i];
                     y = num / den;
                 }
-                float* o = out + sv + static_cast<size_t>(t0 + j) * Dv + tid;
-                *o = accumulate ? *o + y : y;
+                if (out) {  // (null: the state alone, la_chunk_state_ws)
+                    float* o = out + sv + static_cast<size_t>(t0 + j) * Dv + tid;
+                    *o = accumulate ? *o + y : y;
+                }
             }
         }
     }

@@ -199,6 +199,79 @@ cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const C
 
 }  // namespace
 
+// A span's own state from zero (la_chunk_state_ws): the state pass alone, over
+// `pieces` consecutive pieces of the span per (b, h) (doubled while the CTAs
+// fit on the GPU at once), each writing its state, key sum and total log2
+// decay to the workspace; the caller folds the pieces together.
+namespace {
+
+struct StatePlan {
+    int split, pieces, piece_chunks;
+};
+
+StatePlan plan_state(int BH, int nchunks, int Dk, int Dv, bool norm) {
+    const int sms = sm_count();
+    StatePlan P{};
+    int s = 1;
+    while (!instance_ok(Dk, Dv / s, norm) && Dv / (2 * s) >= 16) s *= 2;
+    int pieces = 1;
+    while (pieces * 2 <= nchunks && static_cast<long long>(BH) * s * pieces * 2 <= sms) pieces *= 2;
+    P.split = s;
+    P.piece_chunks = (nchunks + pieces - 1) / pieces;
+    P.pieces = (nchunks + P.piece_chunks - 1) / P.piece_chunks;  // none empty
+    return P;
+}
+
+}  // namespace
+
+size_t fwd_state_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm) {
+    if (!fwd_tc_supports(Dk, Dv) || B <= 0 || H <= 0 || T <= 0) return 0;
+    const int BH = B * H;
+    return workspace_bytes_for(BH, Dk, Dv, plan_state(BH, (T + ws::C - 1) / ws::C, Dk, Dv, norm).pieces);
+}
+
+cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
+    if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
+    const bool norm = a.normalize != 0;
+    const int BH = a.B * a.H;
+    const int nchunks = (a.T + ws::C - 1) / ws::C;
+    const StatePlan P = plan_state(BH, nchunks, a.Dk, a.Dv, norm);
+    const int nv = a.Dv / P.split;
+    if (a.Dv % P.split != 0 || !width_ok(nv) || !instance_ok(a.Dk, nv, norm)) return cudaErrorNotSupported;
+    if (!a.workspace || a.workspace_bytes < workspace_bytes_for(BH, a.Dk, a.Dv, P.pieces))
+        return cudaErrorInvalidValue;
+    if (pieces_used) *pieces_used = P.pieces;
+    CUtensorMap tmq, tmk, tmv;
+    const int box_k = a.Dk < 64 ? a.Dk : 64;
+    const int box_v = norm ? 16 : (nv < 64 ? nv : 64);
+    // the state pass reads no queries: the key tensor stands in for the map
+    if (!make_map(&tmq, a.k, a.Dk, a.T, BH, box_k) || !make_map(&tmk, a.k, a.Dk, a.T, BH, box_k) ||
+        !make_map(&tmv, a.v, a.Dv, a.T, BH, box_v))
+        return cudaErrorInvalidValue;
+    ws::Params p{};
+    p.log_g = a.log_g;
+    p.decay_kind = a.decay_kind;
+    p.H = a.H;
+    p.T = a.T;
+    p.Dv = a.Dv;
+    p.split = P.split;
+    p.nchunks = nchunks;
+    p.err = a.err_word;
+    p.q_scale = 1.f;
+    p.pdl = kPdlFirst;
+    float* base = static_cast<float*>(a.workspace);
+    p.ws_S = base;
+    p.ws_z = p.ws_S + static_cast<size_t>(BH) * P.pieces * a.Dk * a.Dv;
+    p.ws_L = p.ws_z + static_cast<size_t>(BH) * P.pieces * a.Dk;
+    p.ws_nS = P.pieces;
+    p.ws_per_seg = 1;
+    p.state_pass = 1;
+    p.nseg = P.pieces;
+    p.seg_chunks = P.piece_chunks;
+    return launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, p, BH * P.pieces * P.split, a.stream);
+}
+
+
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used) {
     if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
     if (a.accumulate && !a.reverse) return cudaErrorNotSupported;  // only the reverse instances accumulate

@@ -74,6 +74,39 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
 bool fwd_tc_supports(int Dk, int Dv);
 size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm);
 
+// A span's own state from zero (la_fwd_tc.cu, la_chunk_state_ws): the state
+// pass over consecutive pieces of each (b, h)'s span into a.workspace (at least
+// fwd_state_workspace_bytes), laid out [B H][pieces][Dk][Dv] states, then
+// [B H][pieces][Dk] key sums, then [B H][pieces] total log2 decays;
+// *pieces_used receives the number of pieces.
+cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used);
+size_t fwd_state_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm);
+
+// Left fold of n consecutive spans' states (la_state.cu):
+//   S <- init (or 0);  for j < n:  S <- exp(L_j) S + S_j   (z likewise),
+// out_L = sum_j L_j in natural-log units.  Span j's array for (b, h) starts at
+// base + j * span + bh * bh_stride ([Dk][Dv] states, [Dk] key sums, one L).
+struct CombineArgs {
+    const float* S;
+    long long S_span, S_bh;
+    const float* z;           // may be null when out_z is
+    long long z_span, z_bh;
+    const float* L;
+    long long L_span, L_bh;
+    int n;
+    int log2_units;           // L given in log2 units (the state pass's)
+    const float* init_S;      // may be null (zero)
+    const float* init_z;      // may be null (zero)
+    float* out_S;             // [BH][Dk][Dv]
+    float* out_z;             // [BH][Dk] or null
+    float* out_L;             // [BH] or null
+    int BH, Dk, Dv;
+    cudaStream_t stream;
+};
+cudaError_t launch_fold(const CombineArgs& a);
+// out[bh] = sum over T of the log decay (natural log), summed in double.
+cudaError_t launch_log_total(const float* log_g, int kind, int BH, int H, int T, float* out, cudaStream_t stream);
+
 // Decode step (la_decode.cu).
 cudaError_t launch_decode(const DecodeArgs& a, la_dtype dtype);
 

@@ -380,3 +380,84 @@ def test_ema_validation(L):
     assert ema(C=12) == 2         # bf16 rows: C a multiple of 8
     assert ema(C=6, dtype=0) == 2
     assert ema(B=0) == 0
+
+
+def _state(L, **over):
+    a = dict(k=16, v=16, decay=None, norm=0, S=16, z=None, lg=None, B=1, H=1, T=4, Dk=16, Dv=16, dtype=0,
+             ws=None, nbytes=0)
+    a.update(over)
+    vp = ctypes.c_void_p
+    dec = a["decay"]
+    return L.la_chunk_state_ws(vp(a["k"]), vp(a["v"]), ctypes.byref(dec) if dec is not None else None, a["norm"],
+                               vp(a["S"]), vp(a["z"]), vp(a["lg"]), a["B"], a["H"], a["T"], a["Dk"], a["Dv"],
+                               a["dtype"], vp(a["ws"]), a["nbytes"], None)
+
+
+def test_chunk_state_validation(L):
+    assert _state(L, k=None) == 1
+    assert _state(L, v=8) == 1                   # not 16-byte aligned
+    assert _state(L, S=None) == 1                # the state output is required
+    assert _state(L, norm=1) == 1                # normalize needs z_out
+    assert _state(L, lg=2) == 1                  # not 4-byte aligned
+    assert _state(L, Dk=0) == 1
+    assert _state(L, dtype=3) == 1
+    assert _state(L, decay=la._Decay(7, 16)) == 1
+    assert _state(L, decay=la._Decay(2, 0)) == 1  # a decay without its array
+    assert _state(L, Dk=200) == 2                # fp32: D above 128
+    assert _state(L, Dk=24, dtype=1) == 2        # bf16: D a multiple of 16
+    assert _state(L, dtype=1) == 1               # bf16 needs its workspace
+    need = L.la_chunk_state_workspace_size(1, 1, 4, 16, 16, 1, 0)
+    assert need > 0
+    assert _state(L, dtype=1, ws=256, nbytes=need - 16) == 1
+    assert _state(L, dtype=1, ws=264, nbytes=need) == 1   # misaligned workspace
+    assert _state(L, B=0) == 0
+
+
+def test_chunk_state_workspace_size(L):
+    # 148 SMs (the host default without a device).  32 heads, Dk = Dv = 128:
+    # two value slices; pieces doubled while 32 x 2 x pieces fits: two
+    assert L.la_chunk_state_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 2)
+    # one chunk: one piece
+    assert L.la_chunk_state_workspace_size(1, 1, 100, 64, 32, 1, 0) == _ws_bytes(1, 64, 32, 1)
+    # fp32 and empty inputs: none
+    assert L.la_chunk_state_workspace_size(1, 32, 65536, 128, 128, 0, 0) == 0
+    assert L.la_chunk_state_workspace_size(0, 32, 65536, 128, 128, 1, 0) == 0
+    assert L.la_chunk_state_workspace_size(1, 32, 0, 128, 128, 1, 0) == 0
+
+
+def _combine(L, **over):
+    a = dict(S=16, z=None, lg=16, ss=256, zs=0, ls=1, n=2, S0=None, z0=None, out=16, zo=None, lo=None,
+             B=1, H=1, Dk=4, Dv=4)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return L.la_state_combine(vp(a["S"]), vp(a["z"]), vp(a["lg"]), a["ss"], a["zs"], a["ls"], a["n"], vp(a["S0"]),
+                              vp(a["z0"]), vp(a["out"]), vp(a["zo"]), vp(a["lo"]), a["B"], a["H"], a["Dk"],
+                              a["Dv"], None)
+
+
+def test_state_combine_validation(L):
+    assert _combine(L, n=-1) == 1
+    assert _combine(L, ss=-4) == 1
+    assert _combine(L, out=None) == 1            # the state output is required
+    assert _combine(L, S=None) == 1              # spans without states
+    assert _combine(L, lg=None) == 1             # spans without log decays
+    assert _combine(L, zo=32) == 1               # a key-sum output needs the spans' key sums
+    assert _combine(L, S0=2) == 1                # not 4-byte aligned
+    assert _combine(L, Dv=0) == 1
+    assert _combine(L, B=0) == 0
+
+
+def test_injected_launch_failure_state_entry_points():
+    code = r'''
+import ctypes, sys
+sys.path.insert(0, %r)
+import retention_scan_b200 as la
+L = la.lib()
+vp = ctypes.c_void_p
+r = L.la_chunk_state_ws(vp(16), vp(16), None, 0, vp(16), None, None, 1, 1, 4, 16, 16, 0, None, 0, None)
+r2 = L.la_state_combine(vp(16), None, vp(16), 256, 0, 1, 2, None, None, vp(16), None, None, 1, 1, 4, 4, None)
+print(r, r2)
+''' % ROOT
+    env = dict(os.environ, LA_FAULT_INJECT="launch")
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True)
+    assert out.stdout.split() == ["3", "3"]
