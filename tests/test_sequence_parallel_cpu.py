@@ -137,3 +137,26 @@ def test_record_layout_is_16_byte_aligned():
         s, z, lg, size = sp.record_layout(B, H, Dk, Dv)
         assert s == 0 and z % 4 == 0 and lg % 4 == 0 and size % 4 == 0
         assert z >= B * H * Dk * Dv and lg - z >= B * H * Dk and size - lg >= B * H
+
+
+def test_binding_checks_shapes_before_any_call():
+    """The binding rejects mismatched shapes and dtypes on the host, before
+    it touches the library (CPU tensors: a call would need a device)."""
+    import retention_scan_b200 as la
+    from retention_scan_b200 import sequence_parallel as sp
+    S = torch.zeros(2, 1, 2, 4, 4)
+    with pytest.raises(ValueError):
+        la.state_combine(S, torch.zeros(2, 1, 3))            # log totals of another shape
+    with pytest.raises(TypeError):
+        la.state_combine(S, torch.zeros(2, 1, 2, dtype=torch.float64))
+    with pytest.raises(ValueError):
+        la.state_combine(S, torch.zeros(2, 1, 2), torch.zeros(2, 1, 2, 5))   # key sums of another width
+    with pytest.raises(ValueError):
+        la.state_combine(S.transpose(3, 4), torch.zeros(2, 1, 2))           # spans not contiguous
+    k = torch.zeros(1, 2, 8, 4)
+    with pytest.raises(ValueError):
+        la.chunk_state(k, torch.zeros(1, 2, 7, 4))          # v of another length
+    with pytest.raises(ValueError):
+        la.chunk_state(k, torch.zeros(1, 2, 8, 4), la.DECAY_PER_STEP, torch.zeros(1, 2, 9))
+    with pytest.raises(ValueError):
+        sp.span_forward_with(0, 1, None, None, k, k, k, normalize=True, init_state=torch.zeros(1, 2, 4, 4))
