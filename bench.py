@@ -546,7 +546,9 @@ def run_ours(args, rank, world, dist_on, device):
     bytes_launch = algorithmic_bytes(wl, cfg, args.direction)
     achieved_gbs = bytes_launch / (launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved_gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
+                "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
+                # the committed counters are the forward instances' (other directions: none taken)
+                "traffic": measured_traffic(wl.name) if args.direction == "forward" else None,
                 "peak_source": pk_kind,
                 "kernel": "la_decode (decode_vec_kernel)" if cfg == 5 else
                 ("la_fwd_f32 (fwd_f32_kernel)" if wl.dtype == "f32" else
@@ -775,7 +777,8 @@ def run_wkv4(args, rank, world, dist_on, device):
                    "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels"
                    + (", T-segment)" if job.launches == 2 else ")")},
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": measured_traffic(wl.name),
+                     "frac": round(gbs / pk["hbm_gbs"], 4),
+                     "traffic": measured_traffic(wl.name) if args.direction == "forward" else None,
                      "peak_source": pk_kind,
                      "kernel": "ema_kernel" if ema else
                      ("wkv4_kernel (state pass + output pass)" if job.launches == 2 else "wkv4_kernel"),
