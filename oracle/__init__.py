@@ -11,8 +11,8 @@ cpu_baseline / reference legs may import this package.  The CUDA library
   decode_step(...)       one token of the same recurrence, in place
   backward(...)          gradients of a loss through the forward recurrence,
                          by the chain rule token by token (la_ref.c)
-  wkv4(...)              the RWKV-4 WKV recurrence: the att_seq loop of
-                         BlinkDL/RWKV-LM issue 167, max-shifted (wkv4_ref.c)
+  wkv4(...)              the RWKV-4 WKV recurrence of BlinkDL/RWKV-LM issue
+                         167 (formula 14) as an online weighted mean (wkv4_ref.c)
   wkv4_direct(...)       the same output from its definition, O(T^2), numpy
   ema(...)               the cumulative EMA of RetNet issue 21 (values,
                          factors, reverse), per channel (ema_ref.c)
@@ -173,10 +173,12 @@ WKV4_EMPTY_SCALE = -1e38  # pp of an empty RWKV-4 state (aa = bb = 0)
 
 
 def wkv4(k, v, w, u, init_state=None, lib=None):
-    """RWKV-4 WKV recurrence, float64 (wkv4_ref.c: the att_seq loop of
-    BlinkDL/RWKV-LM issue 167).  k, v [B,T,C]; w (log decay, <= 0), u (bonus)
-    [C]; init_state [B,3,C] (planes aa, bb, pp) or None for an empty state.
-    Returns (out [B,T,C], final_state [B,3,C])."""
+    """RWKV-4 WKV recurrence, float64 (wkv4_ref.c: formula 14 of
+    BlinkDL/RWKV-LM issue 167 evaluated as an online weighted mean).  k, v
+    [B,T,C]; w (log decay, <= 0), u (bonus) [C]; init_state [B,3,C] (planes
+    aa, bb, pp: the sums e^pp aa and e^pp bb) or None for an empty state.
+    Returns (out [B,T,C], final_state [B,3,C]) with the final state written
+    as (weighted mean, 1, log of the total weight)."""
     k, v, w, u, init_state = _f64(k), _f64(v), _f64(w), _f64(u), _f64(init_state)
     B, T, C = k.shape
     out = np.zeros((B, T, C))

@@ -10,9 +10,10 @@
  * collaboration: removing the O(T^2) training cost", the cumulative_ema
  * function: element-wise values and factors of the same shape, scanned
  * along one axis so that each output is the previous output times this
- * step's factor plus this step's value (the docstring's garbled
- * "+ output[i+1]" read as "+ values[i+1]", which the pairing operator of
- * the listing computes); the first output is the first value.  The reverse
+ * step's factor plus this step's value.  (The function's docstring, as
+ * extracted, adds the next output instead of the next value; the pairing
+ * operator that the function applies adds the value, and that reading is
+ * the one taken.)  The first output is the first value.  The reverse
  * flag gives the non-reversed scan of the time-reversed arguments, reversed
  * back, i.e. the same recurrence run from the last step to the first.  A
  * carried state s (0 when absent) enters before the first step of the scan:

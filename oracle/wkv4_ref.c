@@ -7,42 +7,56 @@
  * with the CUDA library and is not a fallback for it.
  *
  * Source: BlinkDL/RWKV-LM issue 167, "Questions about formula 14 and code
- * implementation in the paper" (the att_seq time loop quoted in the opening
- * comment).  Per batch b and channel c, with a time decay w (natural log of
- * the per-step factor, <= 0) and a bonus u for the current token, both per
- * channel, the output at token t is the weighted average
+ * implementation in the paper" (opening comment: formula 14 and the
+ * recurrent form of the WKV operator).  Per batch b and channel c, with a
+ * time decay w (natural log of the per-step factor, <= 0) and a bonus u for
+ * the current token, both per channel, the output at token t is the weighted
+ * average of the values seen so far,
  *
  *   wkv_t = ( sum_{i<t} e^{(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
- *         / ( sum_{i<t} e^{(t-1-i) w + k_i}     + e^{u + k_t}     )
+ *         / ( sum_{i<t} e^{(t-1-i) w + k_i}     + e^{u + k_t}     ).
  *
- * and the loop carries the two sums as (aa, bb) measured against a running
- * log scale pp (the true sums are e^pp aa and e^pp bb), so that no exponential
- * of a large key is ever formed: each step takes the larger of the two log
- * weights it combines as the new scale and exponentiates only differences
- * that are <= 0.  Per token, in the page's order:
- *   1. read-out: combine the state (log weight pp) with the current token
- *      (log weight u + k_t) and divide;
- *   2. update: decay the state (log weight w + pp) and add the current token
- *      (log weight k_t); the larger log weight becomes the new pp.
- * An empty state is aa = bb = 0 with pp = -1e38 (a finite stand-in for
- * minus infinity, so that pp - p stays a number).
+ * This file evaluates that definition directly as an online weighted mean:
+ * before token t it keeps the mean R = N / D of the earlier values under
+ * their weights (N and D the two sums over i < t) and the log of the total
+ * weight, L = log D.  Adding a value x with log weight a to a mean (R, L)
+ * moves the mean towards x by the new value's share of the total weight,
+ * sigma(a - L) = e^a / (e^L + e^a), and the log weight becomes
+ * logaddexp(L, a).  So, per token:
+ *   out_t = R + sigma(u + k_t - L) (v_t - R)           (bonus weight, not kept)
+ *   R    <- R + sigma(k_t - (w + L)) (v_t - R)         (earlier weights decayed by e^w)
+ *   L    <- logaddexp(w + L, k_t)
+ * No exponential of a key is formed, only of differences of log weights;
+ * an empty state (no weight yet) is L = -infinity.
  *
- * Layouts: k, v, out [B, T, C]; w, u [C]; state [B, 3, C] holding the planes
- * aa, bb, pp.  Every (b, c) is an independent sequential loop over t.
+ * State interface: [B, 3, C] with the planes (aa, bb, pp), read as the sums
+ * N = e^pp aa and D = e^pp bb (the representation the library's kernel uses;
+ * it is not unique: (aa e^s, bb e^s, pp - s) is the same state).  On input
+ * R = aa / bb and L = pp + log bb (bb = 0: the empty state); on output
+ * (aa, bb, pp) = (R, 1, L), or (0, 0, -1e38) for a state that is still empty.
+ * Layouts: k, v, out [B, T, C]; w, u [C].  Every (b, c) is an independent
+ * sequential loop over t.
  */
 #include <math.h>
 #include <stddef.h>
 
 #define WKV4_EMPTY_SCALE (-1e38)
 
-/* Weights of two terms with log weights la and lb against their larger log
- * weight: *fa = e^(la - m), *fb = e^(lb - m); returns m. */
-static double shifted_pair(double la, double lb, double* fa, double* fb)
+/* The logistic function 1 / (1 + e^-x), without overflow for large |x|. */
+static double sigmoid(double x)
 {
-    const double m = la > lb ? la : lb;
-    *fa = exp(la - m);
-    *fb = exp(lb - m);
-    return m;
+    if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+    const double e = exp(x);
+    return e / (1.0 + e);
+}
+
+/* log(e^a + e^b), exact for a or b = -infinity. */
+static double logaddexp(double a, double b)
+{
+    if (a == -INFINITY) return b;
+    if (b == -INFINITY) return a;
+    const double hi = a > b ? a : b, lo = a > b ? b : a;
+    return hi + log1p(exp(lo - hi));
 }
 
 /*
@@ -57,26 +71,26 @@ int la_ref_wkv4(const double* k, const double* v, const double* w, const double*
     for (int b = 0; b < B; ++b) {
         for (int c = 0; c < C; ++c) {
             const size_t s = (size_t)b * 3 * C + c;
-            double aa = init_state ? init_state[s] : 0.0;
-            double bb = init_state ? init_state[s + C] : 0.0;
-            double pp = init_state ? init_state[s + 2 * C] : WKV4_EMPTY_SCALE;
+            double mean = 0.0, logw = -INFINITY;  /* R and L: no weight yet */
+            if (init_state && init_state[s + C] > 0.0) {
+                mean = init_state[s] / init_state[s + C];
+                logw = init_state[s + 2 * C] + log(init_state[s + C]);
+            }
             for (int t = 0; t < T; ++t) {
                 const size_t i = ((size_t)b * T + t) * C + c;
                 const double kt = k[i], vt = v[i];
-                double fs, fx;
-                /* 1. read-out: state at log weight pp, this token at u + k_t */
-                shifted_pair(pp, u[c] + kt, &fs, &fx);
-                out[i] = (fs * aa + fx * vt) / (fs * bb + fx);
-                /* 2. update: state decayed to w + pp, this token added at k_t */
-                const double m = shifted_pair(w[c] + pp, kt, &fs, &fx);
-                aa = fs * aa + fx * vt;
-                bb = fs * bb + fx;
-                pp = m;
+                /* the current token joins the earlier ones with the bonus weight */
+                out[i] = mean + sigmoid(u[c] + kt - logw) * (vt - mean);
+                /* then, without the bonus, into the decayed state */
+                const double decayed = logw + w[c];
+                mean += sigmoid(kt - decayed) * (vt - mean);
+                logw = logaddexp(decayed, kt);
             }
             if (final_state) {
-                final_state[s] = aa;
-                final_state[s + C] = bb;
-                final_state[s + 2 * C] = pp;
+                const int empty = logw == -INFINITY;
+                final_state[s] = empty ? 0.0 : mean;
+                final_state[s + C] = empty ? 0.0 : 1.0;
+                final_state[s + 2 * C] = empty ? WKV4_EMPTY_SCALE : logw;
             }
         }
     }

@@ -479,10 +479,11 @@ def backward_parallel_form(bwd, fwd):
 
 
 
-# -- RWKV-4 WKV (BlinkDL/RWKV-LM issue 167, the att_seq loop) ----------------
+# -- RWKV-4 WKV (BlinkDL/RWKV-LM issue 167, formula 14) ----------------------
 #
-#   wkv4_direct_form   the loop against its definition written out (O(T^2),
-#                      numpy exponentials), with and without a carried state
+#   wkv4_direct_form   the online weighted mean against the definition written
+#                      out (O(T^2), numpy exponentials), with and without a
+#                      carried state
 #   wkv4_t1_t2         T = 1: out = v; T = 2 expanded by hand
 #   wkv4_invariants    constant v gives constant out; adding s to every key
 #                      leaves out and (aa, bb) unchanged and moves pp by s

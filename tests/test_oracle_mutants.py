@@ -86,16 +86,19 @@ WKV4_SRC = os.path.join(os.path.dirname(oracle.__file__), "wkv4_ref.c")
 
 # (name, text in wkv4_ref.c, replacement)
 WKV4_MUTANTS = [
-    ("bonus left out of the read-out", "shifted_pair(pp, u[c] + kt, &fs, &fx);", "shifted_pair(pp, kt, &fs, &fx);"),
-    ("state not decayed", "shifted_pair(w[c] + pp, kt, &fs, &fx);", "shifted_pair(pp, kt, &fs, &fx);"),
-    ("bonus used in the update", "shifted_pair(w[c] + pp, kt, &fs, &fx);",
-     "shifted_pair(w[c] + pp, u[c] + kt, &fs, &fx);"),
-    ("denominator without the state", "out[i] = (fs * aa + fx * vt) / (fs * bb + fx);",
-     "out[i] = (fs * aa + fx * vt) / (fs + fx);"),
-    ("scale not carried", "        pp = m;\n", "        pp = 0.0 * m;\n"),
-    ("empty state at scale 0", "init_state[s + 2 * C] : WKV4_EMPTY_SCALE;", "init_state[s + 2 * C] : 0.0;"),
-    ("shift by the smaller log weight", "const double m = la > lb ? la : lb;", "const double m = la < lb ? la : lb;"),
-    ("decay applied twice", "aa = fs * aa + fx * vt;", "aa = fs * fs * aa + fx * vt;"),
+    ("bonus left out of the read-out", "out[i] = mean + sigmoid(u[c] + kt - logw) * (vt - mean);",
+     "out[i] = mean + sigmoid(kt - logw) * (vt - mean);"),
+    ("state not decayed", "const double decayed = logw + w[c];", "const double decayed = logw;"),
+    ("bonus used in the update", "mean += sigmoid(kt - decayed) * (vt - mean);",
+     "mean += sigmoid(u[c] + kt - decayed) * (vt - mean);"),
+    ("read-out ignores the state", "out[i] = mean + sigmoid(u[c] + kt - logw) * (vt - mean);", "out[i] = vt;"),
+    ("total weight not carried", "logw = logaddexp(decayed, kt);", "logw = kt;"),
+    ("empty state at weight 1", "double mean = 0.0, logw = -INFINITY;", "double mean = 0.0, logw = 0.0;"),
+    ("logistic of the wrong sign", "if (x >= 0.0) return 1.0 / (1.0 + exp(-x));", "if (x >= 0.0) return 1.0 / (1.0 + exp(x));"),
+    ("sum of weights as their maximum", "return hi + log1p(exp(lo - hi));", "return hi;"),
+    ("carried state's scale ignored", "logw = init_state[s + 2 * C] + log(init_state[s + C]);",
+     "logw = log(init_state[s + C]);"),
+    ("final mean written as the sum", "final_state[s] = empty ? 0.0 : mean;", "final_state[s] = empty ? 0.0 : mean * exp(logw);"),
 ]
 
 
