@@ -146,11 +146,15 @@ typedef struct {
  *                       without its key sum gives a wrong denominator: the
  *                       defect described in flash-linear-attention issue 268).
  *   LA_ERR_UNSUPPORTED  LA_F32 with Dk or Dv > 128; LA_BF16 with Dk or Dv not
- *                       in {16, 32, 64, 128}.
+ *                       a multiple of 16 in [16, 128].
  *   LA_ERR_CUDA         a launch or CUDA runtime call failed.
  *
  * bf16 runs on tcgen05 tensor cores with fp32 accumulation (chunks of 128
- * tokens); fp32 runs a recurrent kernel on fp32 FMA units (no TF32).
+ * tokens); fp32 runs a recurrent kernel on fp32 FMA units (no TF32).  The
+ * bf16 kernels exist for key widths 16, 32, 64 and 128 and value slices of
+ * 16, 32, 64 or 128 columns; other widths run on the next larger key width,
+ * the tile columns past Dk read as zeros (the TMA loads' fill), and on value
+ * slices of which the last may reach past Dv (nothing is stored there).
  */
 LA_API la_status la_chunk_forward(const void* q, const void* k, const void* v,
                            const la_decay* decay, int normalize,
@@ -379,13 +383,14 @@ LA_API la_status la_chunk_backward_ws(const void* q, const void* k, const void* 
  * la_chunk_forward_pro_ws - la_chunk_forward_ws on phi(q) * q_scale and
  * phi(k) (see la_prologue), with the prologue applied inside the kernels.
  *
- * The fp32 path applies both as it stages q and k.  The bf16 tensor-core
- * path applies q_scale in its epilogue (the output is linear in q, and the
- * normalised output does not depend on the scale of q); it has no feature
- * map: applying elu(x) + 1 to the Q and K tiles in shared memory would put
- * one exponential per element (32768 per 128-token chunk at Dk = 128) on
- * the path from a tile's load to its first MMA, so for bf16 inputs
- * feature_map must be LA_FEATURE_NONE (else LA_ERR_UNSUPPORTED).
+ * The fp32 path applies both as it stages q and k (phi in fp32).  The bf16
+ * tensor-core path applies the feature map to each Q and K tile in shared
+ * memory once it has landed, before the tile's first MMA, at the tiles' own
+ * precision (bf16 arithmetic; within a bf16 rounding step or two of phi
+ * evaluated in fp32 and rounded), leaving the rows past the sequence end and
+ * the columns past Dk at zero; it applies q_scale in its epilogue (the output
+ * is linear in q, and the normalised output does not depend on the scale of
+ * q).  Either way q and k cross HBM once, raw.
  *
  *   prologue        NULL (identity) or a descriptor.
  *   other arguments as la_chunk_forward_ws.
@@ -571,9 +576,20 @@ LA_API la_status la_ema_scan(const void* x, const void* f, const float* init_sta
  * loaded), so that the call itself allocates no device memory.  The pages
  * have no counterpart: this is a property of this library's interface only.
  *
- * The array is shared by every call on a device: calls on one device must
- * not overlap in time (issue them on one stream, or synchronise between the
- * streams).  Arguments, results and errors as la_chunk_forward, plus
+ * It is meant for callers that cannot allocate device memory at the point
+ * of the call: code that runs under a fixed memory budget or behind its own
+ * allocator that must not be bypassed, or host code that must not call
+ * cudaMalloc at all (it can synchronise the device and is not allowed in
+ * some contexts, such as while a stream is being captured).
+ *
+ * The array is shared by every call on a device and keeps what the last call
+ * left in it (every call writes the parts it reads before reading them):
+ * calls on one device that overlap in time on the GPU race on it, so issue
+ * them on one stream, or synchronise between the streams.  The array's
+ * device address is looked up (cudaGetSymbolAddress) by the first call on
+ * each device, with that device current, and again only if that device's
+ * context has been reset since; make that first call before any stream
+ * capture begins.  Arguments, results and errors as la_chunk_forward, plus
  * LA_ERR_UNSUPPORTED (nothing enqueued) when these sizes would need a larger
  * workspace than the array holds (la_chunk_forward_workspace_size), and
  * LA_ERR_CUDA if the array's address cannot be obtained on the current device.

@@ -201,8 +201,8 @@ def chunk_forward(q, k, v, decay_kind=DECAY_NONE, log_g=None, normalize=False,
     as T-segments (a torch allocation on the call's stream), None/False runs
     without, or a CUDA uint8 tensor to use.
     feature_map / q_scale: the input prologue (la_chunk_forward_pro_ws): the
-    kernels read phi(q) * q_scale and phi(k), phi = FEATURE_ELU1 (elu + 1,
-    fp32 inputs only) or FEATURE_NONE.  Forward scans only.
+    kernels read phi(q) * q_scale and phi(k), phi = FEATURE_ELU1 (elu + 1)
+    or FEATURE_NONE.  Forward scans only.
     """
     B, H, T, Dk = q.shape
     Dv = v.shape[-1]

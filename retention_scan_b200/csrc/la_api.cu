@@ -1,9 +1,11 @@
 // la_api.cu - the C ABI (include/la.h): argument validation, dispatch to the
 // kernels, the device error word.  Nothing here allocates device memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <climits>
+#include <mutex>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -12,26 +14,66 @@
 #include "la.h"
 #include "la_internal.h"
 
+namespace la {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// cuCtxGetCurrent, looked up once through the runtime (libcuda is not linked).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+    static std::atomic<CtxGetCurrentFn> fn{nullptr};
+    CtxGetCurrentFn f = fn.load();
+    if (!f) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f = reinterpret_cast<CtxGetCurrentFn>(ptr);
+        fn.store(f);
+    }
+    return f;
+}
+
+void* current_context() {
+    CtxGetCurrentFn f = ctx_get_current();
+    CUcontext c = nullptr;
+    if (!f || f(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+struct SymbolEntry {
+    void* ctx;
+    void* addr;
+};
+std::mutex g_sym_mutex;
+SymbolEntry g_sym[kSymSlots][kMaxDevices];
+
+}  // namespace
+
+void* device_symbol_address(const void* symbol, int slot) {
+    int dev = 0;
+    if (slot < 0 || slot >= kSymSlots || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(g_sym_mutex);
+    SymbolEntry& e = g_sym[slot][dev];
+    void* ctx = current_context();
+    if (e.addr && ctx && e.ctx == ctx) return e.addr;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, symbol) != cudaSuccess) return nullptr;
+    e.ctx = current_context();  // the lookup made the device's primary context current if none was
+    e.addr = addr;
+    return addr;
+}
+
+}  // namespace la
+
 namespace {
 
 // Set by a kernel that gave up waiting on one of its barriers (kErr* codes).
 __device__ int g_err_word;
 
-constexpr int kMaxDevices = 64;
-std::atomic<int*> g_err_ptr[kMaxDevices];
-
-int* err_word_for_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    int* p = g_err_ptr[dev].load();
-    if (!p) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_err_word) != cudaSuccess) return nullptr;
-        p = static_cast<int*>(addr);
-        g_err_ptr[dev].store(p);
-    }
-    return p;
-}
+int* err_word_for_current_device() { return static_cast<int*>(la::device_symbol_address(&g_err_word, la::kSymErrWord)); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -99,7 +141,6 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
     }
     if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
     if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
-    if (dtype == LA_BF16 && fmap != LA_FEATURE_NONE) return LA_ERR_UNSUPPORTED;  // see la.h
     if (BH == 0) return LA_OK;
     if (launch_fault_injected()) return LA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -225,8 +266,8 @@ NormLayout norm_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int 
     return L;
 }
 
-// The normalised backward with the value panel [v | 1 | 0] (W = a supported
-// width > Dv): one scan gives [n | den], and dq, dk each come from one scan
+// The normalised backward with the value panel [v | 1 | 0] (W = Dv + 16 for
+// bf16, Dv + 1 for fp32): one scan gives [n | den], and dq, dk each come from one scan
 // of [dn | dden | 0] against it, so that the cancellation between the
 // numerator's and the denominator's terms happens inside the scores (fp32)
 // instead of between two rounded outputs.  Regions (256-aligned): the
@@ -237,9 +278,7 @@ NormLayout norm_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int 
 // T-segment workspace.
 int panel_width(int Dv, la_dtype dtype) {
     if (dtype == LA_F32) return Dv + 1 <= 128 ? Dv + 1 : 0;
-    for (int w : {32, 64, 128})
-        if (w > Dv) return w;
-    return 0;
+    return Dv + 16 <= 128 ? Dv + 16 : 0;  // bf16 widths are multiples of 16
 }
 
 struct PanelLayout {

@@ -13,11 +13,13 @@
 namespace la {
 namespace ws {
 // instantiated in la_fwd_ws_dk*.cu (one file per key width and direction)
-#define LA_WS_DECL(DK)                                                                                        \
-    extern template cudaError_t launch_dk<DK, false>(int, bool, const CUtensorMap&, const CUtensorMap&,       \
-                                                     const CUtensorMap&, const Params&, int, cudaStream_t);  \
-    extern template cudaError_t launch_dk<DK, true>(int, bool, const CUtensorMap&, const CUtensorMap&,        \
-                                                    const CUtensorMap&, const Params&, int, cudaStream_t);   \
+#define LA_WS_DECL(DK)                                                                                         \
+    extern template cudaError_t launch_dk<DK, false, false>(int, bool, const CUtensorMap&, const CUtensorMap&, \
+                                                            const CUtensorMap&, const Params&, int, cudaStream_t); \
+    extern template cudaError_t launch_dk<DK, true, false>(int, bool, const CUtensorMap&, const CUtensorMap&,  \
+                                                           const CUtensorMap&, const Params&, int, cudaStream_t); \
+    extern template cudaError_t launch_dk<DK, false, true>(int, bool, const CUtensorMap&, const CUtensorMap&,  \
+                                                           const CUtensorMap&, const Params&, int, cudaStream_t); \
     extern template bool supported_dk<DK>(int, bool);
 LA_WS_DECL(16)
 LA_WS_DECL(32)
@@ -43,7 +45,16 @@ EncodeTiledFn encode_tiled() {
 
 namespace {
 
+// Widths with a kernel instance (key width DK, value slice NV).
 bool width_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// The instance key width for a tensor width d (a multiple of 16 up to 128):
+// the smallest instance width >= d; the tile columns past d are zero-filled
+// by the TMA loads, which contributes nothing to scores or states.
+int padded_width(int d) { return d <= 16 ? 16 : d <= 32 ? 32 : d <= 64 ? 64 : 128; }
+
+// Tensor widths the tensor-core path takes.
+bool tensor_width_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 
 CUtensorMapSwizzle swizzle_for(int row_bytes) {
     return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -94,8 +105,9 @@ int env_int(const char* name) {
 }
 
 // How the (b, h) sequences are spread over CTAs (one CTA per SM).
-//  split: CTAs sharing one (b, h, segment), each owning Dv / split value
-//         columns and recomputing the 128 x 128 score tile;
+//  split: CTAs sharing one (b, h, segment), each owning nv value columns
+//         (split = ceil(Dv / nv); the last slice may run past Dv) and
+//         recomputing the 128 x 128 score tile;
 //  nseg:  output segments per (b, h), of seg_chunks chunks each; segment i
 //         starts from the state after segment i - 1, assembled from per_seg
 //         state segments per earlier output segment (computed by a state
@@ -109,7 +121,7 @@ int env_int(const char* name) {
 // and re-multiplies Q and K, a segment only reloads K and V once in the state
 // pass.  The state pass cuts each segment further while SMs stay idle.
 struct Layout {
-    int split, nseg, seg_chunks, per_seg, nS;
+    int split, nv, nseg, seg_chunks, per_seg, nS;
 };
 
 constexpr int kMinSegChunks = 16;
@@ -117,11 +129,13 @@ constexpr int kMinSegChunks = 16;
 Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments) {
     const int sms = sm_count();
     const long long target = sms * 4 / 5;
-    int s = 1;
-    while (!instance_ok(Dk, Dv / s, norm) && Dv / (2 * s) >= 16) s *= 2;
+    const int DK = padded_width(Dk);
+    int nv = padded_width(Dv);
+    while (!instance_ok(DK, nv, norm) && nv / 2 >= 16) nv /= 2;
     const int es = env_int("LA_DV_SPLIT");
-    const bool fixed_split = es >= 1 && Dv % es == 0 && width_ok(Dv / es) && instance_ok(Dk, Dv / es, norm);
-    if (fixed_split) s = es;
+    const bool fixed_split = es >= 1 && Dv % es == 0 && width_ok(Dv / es) && instance_ok(DK, Dv / es, norm);
+    if (fixed_split) nv = Dv / es;
+    int s = (Dv + nv - 1) / nv;
     int nseg = 1;
     if (segments && nchunks >= 2) {
         const int eg = env_int("LA_SEGMENTS");
@@ -133,9 +147,13 @@ Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments
         }
     }
     if (!fixed_split)
-        while (static_cast<long long>(BH) * s * nseg < target && Dv / (2 * s) >= 16) s *= 2;
+        while (static_cast<long long>(BH) * s * nseg < target && nv / 2 >= 16) {
+            nv /= 2;
+            s = (Dv + nv - 1) / nv;
+        }
     Layout L{};
     L.split = s;
+    L.nv = nv;
     L.seg_chunks = (nchunks + nseg - 1) / (nseg > 0 ? nseg : 1);
     if (L.seg_chunks < 1) L.seg_chunks = 1;
     L.nseg = (nchunks + L.seg_chunks - 1) / L.seg_chunks;
@@ -157,7 +175,7 @@ size_t workspace_bytes_for(int BH, int Dk, int Dv, int nS) {
 
 }  // namespace
 
-bool fwd_tc_supports(int Dk, int Dv) { return width_ok(Dk) && width_ok(Dv); }
+bool fwd_tc_supports(int Dk, int Dv) { return tensor_width_ok(Dk) && tensor_width_ok(Dv); }
 
 size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm) {
     if (!fwd_tc_supports(Dk, Dv) || B <= 0 || H <= 0 || T <= 0) return 0;
@@ -177,24 +195,28 @@ namespace {
 constexpr int kPdlFirst = 1;
 constexpr int kPdlOutput = 0;
 
-template <bool REV>
+template <bool REV, bool PHI>
 cudaError_t launch_dir(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
                        const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
     switch (Dk) {
-        case 16: return ws::launch_dk<16, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 32: return ws::launch_dk<32, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 64: return ws::launch_dk<64, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
-        case 128: return ws::launch_dk<128, REV>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 16: return ws::launch_dk<16, REV, PHI>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 32: return ws::launch_dk<32, REV, PHI>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 64: return ws::launch_dk<64, REV, PHI>(nv, norm, tmq, tmk, tmv, p, grid, stream);
+        case 128: return ws::launch_dk<128, REV, PHI>(nv, norm, tmq, tmk, tmv, p, grid, stream);
         default: return cudaErrorNotSupported;
     }
 }
 
-// The direction picks the instance: the forward instances carry no code of
-// the reverse scan (its index mapping, mask and accumulating epilogue).
+// The direction and the feature map pick the instance: the forward
+// instances carry no code of the reverse scan (its index mapping, mask and
+// accumulating epilogue), and only the feature-map instances map tiles.
 cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk,
                       const CUtensorMap& tmv, const ws::Params& p, int grid, cudaStream_t stream) {
-    return p.reverse ? launch_dir<true>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream)
-                     : launch_dir<false>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream);
+    if (p.feature_map == LA_FEATURE_ELU1)
+        return p.reverse ? cudaErrorNotSupported
+                         : launch_dir<false, true>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream);
+    return p.reverse ? launch_dir<true, false>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream)
+                     : launch_dir<false, false>(Dk, nv, norm, tmq, tmk, tmv, p, grid, stream);
 }
 
 }  // namespace
@@ -206,14 +228,16 @@ cudaError_t launch_ws(int Dk, int nv, bool norm, const CUtensorMap& tmq, const C
 namespace {
 
 struct StatePlan {
-    int split, pieces, piece_chunks;
+    int split, nv, pieces, piece_chunks;
 };
 
 StatePlan plan_state(int BH, int nchunks, int Dk, int Dv, bool norm) {
     const int sms = sm_count();
     StatePlan P{};
-    int s = 1;
-    while (!instance_ok(Dk, Dv / s, norm) && Dv / (2 * s) >= 16) s *= 2;
+    int nv = padded_width(Dv);
+    while (!instance_ok(padded_width(Dk), nv, norm) && nv / 2 >= 16) nv /= 2;
+    const int s = (Dv + nv - 1) / nv;
+    P.nv = nv;
     int pieces = 1;
     while (pieces * 2 <= nchunks && static_cast<long long>(BH) * s * pieces * 2 <= sms) pieces *= 2;
     P.split = s;
@@ -236,13 +260,13 @@ cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
     const int BH = a.B * a.H;
     const int nchunks = (a.T + ws::C - 1) / ws::C;
     const StatePlan P = plan_state(BH, nchunks, a.Dk, a.Dv, norm);
-    const int nv = a.Dv / P.split;
-    if (a.Dv % P.split != 0 || !width_ok(nv) || !instance_ok(a.Dk, nv, norm)) return cudaErrorNotSupported;
+    const int nv = P.nv, DK = padded_width(a.Dk);
+    if (!width_ok(nv) || !instance_ok(DK, nv, norm)) return cudaErrorNotSupported;
     if (!a.workspace || a.workspace_bytes < workspace_bytes_for(BH, a.Dk, a.Dv, P.pieces))
         return cudaErrorInvalidValue;
     if (pieces_used) *pieces_used = P.pieces;
     CUtensorMap tmq, tmk, tmv;
-    const int box_k = a.Dk < 64 ? a.Dk : 64;
+    const int box_k = DK < 64 ? DK : 64;
     const int box_v = norm ? 16 : (nv < 64 ? nv : 64);
     // the state pass reads no queries: the key tensor stands in for the map
     if (!make_map(&tmq, a.k, a.Dk, a.T, BH, box_k) || !make_map(&tmk, a.k, a.Dk, a.T, BH, box_k) ||
@@ -253,6 +277,7 @@ cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
     p.decay_kind = a.decay_kind;
     p.H = a.H;
     p.T = a.T;
+    p.Dk = a.Dk;
     p.Dv = a.Dv;
     p.split = P.split;
     p.nchunks = nchunks;
@@ -268,7 +293,7 @@ cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
     p.state_pass = 1;
     p.nseg = P.pieces;
     p.seg_chunks = P.piece_chunks;
-    return launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, p, BH * P.pieces * P.split, a.stream);
+    return launch_ws(DK, nv, norm, tmq, tmk, tmv, p, BH * P.pieces * P.split, a.stream);
 }
 
 
@@ -281,13 +306,13 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     Layout L = plan_layout(BH, nchunks, a.Dk, a.Dv, norm, a.workspace != nullptr);
     if (L.nS > 0 && a.workspace_bytes < workspace_bytes_for(BH, a.Dk, a.Dv, L.nS))
         L = plan_layout(BH, nchunks, a.Dk, a.Dv, norm, false);  // too small: one segment
-    const int split = L.split, nv = a.Dv / split;
-    if (a.Dv % split != 0 || !width_ok(nv) || !instance_ok(a.Dk, nv, norm)) return cudaErrorNotSupported;
+    const int split = L.split, nv = L.nv, DK = padded_width(a.Dk);
+    if (!width_ok(nv) || !instance_ok(DK, nv, norm)) return cudaErrorNotSupported;
     if (split_used) *split_used = split;
     if (segments_used) *segments_used = L.nseg;
 
     CUtensorMap tmq, tmk, tmv;
-    const int box_k = a.Dk < 64 ? a.Dk : 64;
+    const int box_k = DK < 64 ? DK : 64;
     const int box_v = norm ? 16 : (nv < 64 ? nv : 64);  // the normaliser instances use 16-column panels
     if (!make_map(&tmq, a.q, a.Dk, a.T, BH, box_k) || !make_map(&tmk, a.k, a.Dk, a.T, BH, box_k) ||
         !make_map(&tmv, a.v, a.Dv, a.T, BH, box_v))
@@ -303,6 +328,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     p.final_z = a.final_z;
     p.H = a.H;
     p.T = a.T;
+    p.Dk = a.Dk;
     p.Dv = a.Dv;
     p.split = split;
     p.nchunks = nchunks;
@@ -310,6 +336,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     p.reverse = a.reverse;
     p.accumulate = a.accumulate;
     p.q_scale = a.q_scale;
+    p.feature_map = a.feature_map;
     p.pdl = kPdlFirst;
     if (L.nS > 0) {
         float* base = static_cast<float*>(a.workspace);
@@ -323,14 +350,14 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
         ps.state_pass = 1;
         ps.nseg = L.nS;
         ps.seg_chunks = L.seg_chunks / L.per_seg;
-        const cudaError_t e = launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, ps, BH * L.nS * split, a.stream);
+        const cudaError_t e = launch_ws(DK, nv, norm, tmq, tmk, tmv, ps, BH * L.nS * split, a.stream);
         if (e != cudaSuccess) return e;
     }
     p.state_pass = 0;
     if (L.nS > 0) p.pdl = kPdlOutput;
     p.nseg = L.nseg;
     p.seg_chunks = L.seg_chunks;
-    return launch_ws(a.Dk, nv, norm, tmq, tmk, tmv, p, BH * L.nseg * split, a.stream);
+    return launch_ws(DK, nv, norm, tmq, tmk, tmv, p, BH * L.nseg * split, a.stream);
 }
 
 }  // namespace la

@@ -93,8 +93,9 @@ enum Bar : int {
     B_DSEMPTY = 42,  // [2] state warps done with it
     B_SBFULL = 44,   // [2] bf16 state copy written
     B_SBEMPTY = 46,  // [2] Q S done reading it
-    B_DRAIN = 48,
-    B_COUNT = 49
+    B_PHI = 48,      // [4] feature map applied to the chunk's Q and K tiles
+    B_DRAIN = 52,
+    B_COUNT = 53
 };
 
 template <int DK, int NV, bool NORM>
@@ -209,7 +210,11 @@ struct Params {
     __nv_bfloat16* out;
     float* final_state;
     float* final_z;
-    int H, T, Dv, split, nchunks;
+    // Dk and Dv are the tensors' widths.  The instance's key width DK is the
+    // smallest one >= Dk: the key and query tiles' columns past Dk are the
+    // TMA's zero fill, and so are the value columns past Dv in the last value
+    // slice; rows of S past Dk and columns past Dv are neither read nor written.
+    int H, T, Dk, Dv, split, nchunks;
     int* err;
     // T-segments: each (b, h, slice) is cut into nseg segments of seg_chunks
     // chunks, one CTA each.  The output pass starts segment i from the state
@@ -230,6 +235,8 @@ struct Params {
     int accumulate;      // reverse instances only: add y to the values already in out (fp32 add)
     float q_scale;       // the output of an unnormalised scan is linear in q: y *= q_scale
                          // (the normalised output does not depend on the scale of q)
+    int feature_map;     // LA_FEATURE_ELU1: the prep warps replace each landed Q and K tile
+                         // by phi(x) = elu(x) + 1 before the chunk's first MMA (forward only)
     int pdl;             // (host) launch with programmatic stream serialisation
 };
 
@@ -364,6 +371,46 @@ __device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&o)
         uint4* d4 = reinterpret_cast<uint4*>(dst);
         d4[0] = make_uint4(u[0], u[1], u[2], u[3]);
         d4[1] = make_uint4(u[4], u[5], u[6], u[7]);
+    }
+}
+
+// phi(x) = elu(x) + 1 = max(x, 0) + e^min(x, 0) (flash-linear-attention
+// issue 268's feature map) on two bf16 values, in bf16x2 arithmetic: the
+// exponential is the tensor-core tile's own precision (ex2.approx on a bf16
+// pair, its argument min(x, 0) log2(e) rounded to bf16), within a few bf16
+// rounding steps of phi computed in fp32 and then rounded; for x > 0 it is
+// exactly the bf16 rounding of x + 1.
+__device__ __forceinline__ uint32_t elu1_pair(uint32_t u) {
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u);
+    const __nv_bfloat162 zero = __float2bfloat162_rn(0.f), log2e = __float2bfloat162_rn(kLog2e);
+    const __nv_bfloat162 arg = __hmul2(__hmin2(x, zero), log2e);
+    uint32_t e;
+    asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(*reinterpret_cast<const uint32_t*>(&arg)));
+    const __nv_bfloat162 r = __hadd2(__hmax2(x, zero), *reinterpret_cast<const __nv_bfloat162*>(&e));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// phi on row `row` of a landed [C x DK] Q or K tile (DK / (W / 2) swizzled
+// panels of C rows of W bytes), in place; the columns at or past dk (the
+// TMA's zero fill of a padded key width) stay zero, since phi(0) = 1.  One
+// thread per row, so that the direct-form row scaling of the same thread
+// follows it without a barrier.
+template <int DK>
+__device__ __noinline__ void elu1_row(uint8_t* tile, int row, int dk) {
+    constexpr int W = row_bytes_for(DK), NP = DK * 2 / W, NCH = W / 16;
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) {
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+            if (pn * (W / 2) + ch * 8 >= dk) continue;
+            uint4* q = reinterpret_cast<uint4*>(tile + pn * C * W + swz(row, ch * 16, W));
+            uint4 v = *q;
+            v.x = elu1_pair(v.x);
+            v.y = elu1_pair(v.y);
+            v.z = elu1_pair(v.z);
+            v.w = elu1_pair(v.w);
+            *q = v;
+        }
     }
 }
 
@@ -511,7 +558,7 @@ __device__ __noinline__ void mma_state_pass(const Ctx x) {
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
 }
 
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
 __device__ __noinline__ void role_mma(const Ctx x) {
     LA_ROLE_PRELUDE
     if (p.state_pass) {
@@ -531,7 +578,9 @@ __device__ __noinline__ void role_mma(const Ctx x) {
     // One snapshot per pass of every barrier a queue head may wait on: the
     // issuing lane runs the tests back to back (their latencies overlap; no
     // test waits for another's answer) and broadcasts the bits to the warp.
-    enum : uint32_t { kP = 1, kQ = 2, kK = 4, kA = 8, kPrep = 16, kDir = 32, kDse = 64, kOe = 128, kSb = 256 };
+    enum : uint32_t { kP = 1, kQ = 2, kK = 4, kA = 8, kPrep = 16, kDir = 32, kDse = 64, kOe = 128, kSb = 256,
+                      kPhi = 512 };
+    constexpr bool phi = PHI;  // Q K^T (c) also awaits the feature map of c
     auto snapshot = [&]() -> uint32_t {
         uint32_t b = 0;
         if (leader) {
@@ -540,6 +589,9 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             b |= mbar_test(&bar[B_KFULL + m1 % G::NK], (m1 / G::NK) & 1) ? kK : 0u;
             b |= (m1 < G::NA || mbar_test(&bar[B_AEMPTY + m1 % G::NA], ((m1 / G::NA) - 1) & 1)) ? kA : 0u;
             b |= mbar_test(&bar[B_PREP + kv % G::NVS], (kv / G::NVS) & 1) ? kPrep : 0u;
+            // the feature map of chunk m1 (its slot is unambiguous: the map of
+            // m1 - 4 preceded the issued Q K^T (m1 - 4))
+            if (phi) b |= mbar_test(&bar[B_PHI + m1 % 4], (m1 / 4) & 1) ? kPhi : 0u;
             b |= (kv < G::NDS || mbar_test(&bar[B_DSEMPTY + kv % G::NDS], ((kv / G::NDS) - 1) & 1)) ? kDse : 0u;
             b |= (qs < G::NO || mbar_test(&bar[B_OEMPTY + qs % G::NO], ((qs / G::NO) - 1) & 1)) ? kOe : 0u;
             b |= mbar_test(&bar[B_SBFULL + qs % G::NSB], (qs / G::NSB) & 1) ? kSb : 0u;
@@ -557,7 +609,8 @@ __device__ __noinline__ void role_mma(const Ctx x) {
         }
         // Q K^T of chunk m1
         auto issue_qk = [&]() {
-            if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA)) {
+            const bool phi_done = !phi || (bits & kPhi) != 0;
+            if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA) && phi_done) {
                 tc_fence_after_sync();
                 const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
                 const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
@@ -719,7 +772,7 @@ __device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint6
     fence_async_smem();
 }
 
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
 __device__ __noinline__ void role_prep_mask(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_PM) / 4;  // 0: score columns 0-63, V rows; 1: columns 64-127, weights
@@ -746,6 +799,14 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     // rows; warpgroup 1 writes the normaliser weights, or has nothing to do.
     auto prep = [&](int c) -> bool {
         const int s = c % G::NVS, rem = min(C, T - mem_chunk(c) * C);
+        if (PHI && p.state_pass && wg == 0) {
+            // the state pass has no Q tile and no mask: warpgroup 0 maps the
+            // chunk's key rows here (before it decays them, for a direct-form
+            // chunk), before the prep arrival that the chunk's K^T V' awaits
+            if (!waitw(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, abort, p, kErrTmaWait)) return false;
+            if (t < rem) elu1_row<DK>(sm + G::OFF_K + (c % G::NK) * G::Q_STAGE, t, p.Dk);
+            fence_async_smem();
+        }
         if (!NORM && wg == 1) {
             // nothing to prepare; in the state pass (no mask to pace this
             // warpgroup) wait for the tile so that its arrivals never run a
@@ -918,8 +979,9 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst = out_row(c);
+        const int npiece = min(NV, p.Dv - x.j0) / 16;  // the last slice may run past Dv
 #pragma unroll 1
-        for (int piece = 0; piece < NV / 16; ++piece) {
+        for (int piece = 0; piece < npiece; ++piece) {
             float o[16];
             tmem_ld16(oa + 16 * piece, o);
             tmem_wait_ld();
@@ -937,12 +999,33 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         }
         return;
     }
+    // Feature map (output pass): warpgroup 0 maps the chunk's Q tile and
+    // warpgroup 1 its K tile, one row per thread, rows past the sequence end
+    // left at the TMA's zero fill (phi(0) = 1 would add them to the key
+    // sum); the chunk's Q K^T awaits the arrival.
+    auto phi = [&](int c) -> bool {
+        const int rem = min(C, T - mem_chunk(c) * C);
+        if (wg == 0) {
+            if (!waitw(&bar[B_QFULL + c % G::NQ], (c / G::NQ) & 1, abort, p, kErrTmaWait)) return false;
+            if (t < rem) elu1_row<DK>(sm + (c % G::NQ) * G::Q_STAGE, t, p.Dk);
+        } else {
+            if (!waitw(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, abort, p, kErrTmaWait)) return false;
+            if (t < rem) elu1_row<DK>(sm + G::OFF_K + (c % G::NK) * G::Q_STAGE, t, p.Dk);
+        }
+        fence_async_smem();
+        warp_arrive(&bar[B_PHI + c % 4]);
+        return true;
+    };
+    constexpr bool map = PHI;
     // prep runs one chunk ahead of the mask, the epilogue one chunk behind
-    // it (one call site each keeps the loop small in the instruction cache)
+    // it, and the feature map of the next chunk right after the mask (off the
+    // path from a chunk's scores to its mask); one call site each keeps the
+    // loop small in the instruction cache
 #pragma unroll 1
     for (int c = -1; c <= n; ++c) {
         if (c + 1 < n && !prep(c + 1)) break;
         if (c >= 0 && c < n && !pmask(c)) break;
+        if (map && c + 1 < n && !phi(c + 1)) break;
         if (G::EPI_MASK && wg == 1 && c >= 1 && !epilogue(c - 1)) break;
     }
 }
@@ -957,9 +1040,12 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     const int wg = (warp - G::W_ES) / 4;
     const int wq = warp & 3;
     const int d = 32 * wq + lane;          // key row of S; also token row t of O
-    const bool warp_rows = 32 * wq < DK;   // this warp holds real rows of S
-    const bool row_ok = d < DK;
+    const bool warp_rows = 32 * wq < DK;   // this warp holds rows of S (past Dk they stay zero)
+    const bool row_ok = d < p.Dk;
     const int cb = wg * G::NVW;            // first column (within the slice) of this warpgroup
+    // columns of this warpgroup inside the tensor (a multiple of 16: the last
+    // value slice may run past Dv)
+    const int ncols = min(G::NVW, max(0, p.Dv - (x.j0 + cb)));
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * wq) << 16);
     const int bh = x.bh, j0 = x.j0;
     float S[G::NVW];
@@ -968,9 +1054,10 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     for (int j = 0; j < G::NVW; ++j) S[j] = 0.f;
     float ltot = 0.f;  // state pass: total log2 decay of the segment
     if (row_ok && p.init_state && !p.state_pass) {
-        const float* src = p.init_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
+        const float* src = p.init_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
         for (int j = 0; j < G::NVW; j += 4) {
+            if (j >= ncols) break;
             const float4 v4 = *reinterpret_cast<const float4*>(src + j);
             S[j] = v4.x;
             S[j + 1] = v4.y;
@@ -978,30 +1065,34 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             S[j + 3] = v4.w;
         }
     }
-    if (NORM && row_ok && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * DK + d];
+    if (NORM && row_ok && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * p.Dk + d];
     if (row_ok && !p.state_pass && x.seg > 0) {
         // state entering this segment: fold in every earlier state segment j,
         // S <- 2^(L_j) S + S_j (the combination of two consecutive spans)
         for (int j = 0; j < x.seg * p.ws_per_seg; ++j) {
             const size_t sj = static_cast<size_t>(bh) * p.ws_nS + j;
             const float e = ex2_approx(p.ws_L[sj]);
-            const float* src = p.ws_S + (sj * DK + d) * p.Dv + j0 + cb;
+            const float* src = p.ws_S + (sj * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
             for (int i = 0; i < G::NVW; i += 4) {
+                if (i >= ncols) break;
                 const float4 v4 = *reinterpret_cast<const float4*>(src + i);
                 S[i] = fmaf(e, S[i], v4.x);
                 S[i + 1] = fmaf(e, S[i + 1], v4.y);
                 S[i + 2] = fmaf(e, S[i + 2], v4.z);
                 S[i + 3] = fmaf(e, S[i + 3], v4.w);
             }
-            if (NORM) z = fmaf(e, z, p.ws_z[sj * DK + d]);
+            if (NORM) z = fmaf(e, z, p.ws_z[sj * p.Dk + d]);
         }
     }
 
     auto write_copy = [&](int k) {  // bf16 copy of S (and z) for production index k
         const int buf = k % G::NSB;
         uint8_t* sb = sm + G::OFF_SB + buf * G::SB_BYTES;
-        if (row_ok) {
+        // every row of the tile, the zero rows past Dk included: Q S reads
+        // them (against zero query columns, but whatever else sat in shared
+        // memory there could be an infinity or a NaN)
+        if (d < DK) {
 #pragma unroll
             for (int j = 0; j < G::NVW; j += 8) {
                 const int col = cb + j;
@@ -1087,7 +1178,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst = out_row(c);
 #pragma unroll 1
-        for (int piece = 0; piece < G::NVW / 16; ++piece) {
+        for (int piece = 0; piece < ncols / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
             tmem_wait_ld();
@@ -1104,11 +1195,11 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         if (ok && !*abort) {
             const size_t sj = static_cast<size_t>(bh) * p.ws_nS + x.seg;
             if (row_ok) {
-                float* dst = p.ws_S + (sj * DK + d) * p.Dv + j0 + cb;
+                float* dst = p.ws_S + (sj * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
                 for (int j = 0; j < G::NVW; j += 4)
-                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-                if (NORM && x.slice == 0 && wg == 0) p.ws_z[sj * DK + d] = z;
+                    if (j < ncols) *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                if (NORM && x.slice == 0 && wg == 0) p.ws_z[sj * p.Dk + d] = z;
             }
             if (x.slice == 0 && wg == 0 && d == 0) p.ws_L[sj] = ltot;
         }
@@ -1134,16 +1225,16 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     }
     if (ok && !*abort && row_ok && x.seg == p.nseg - 1) {
         if (p.final_state) {
-            float* fs = p.final_state + (static_cast<size_t>(bh) * DK + d) * p.Dv + j0 + cb;
+            float* fs = p.final_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
             for (int j = 0; j < G::NVW; j += 4)
-                *reinterpret_cast<float4*>(fs + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                if (j < ncols) *reinterpret_cast<float4*>(fs + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
-        if (NORM && p.final_z && x.slice == 0 && wg == 0) p.final_z[static_cast<size_t>(bh) * DK + d] = z;
+        if (NORM && p.final_z && x.slice == 0 && wg == 0) p.final_z[static_cast<size_t>(bh) * p.Dk + d] = z;
     }
 }
 
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
 __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     fwd_ws_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ Params p) {
@@ -1176,17 +1267,18 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
             mbar_init(&bar[B_PREP + s], 8);
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar[B_OFULL + i], 1);
+            mbar_init(&bar[B_OEMPTY + i], G::EPI_MASK ? 4 : 4 * G::NSW);
             mbar_init(&bar[B_AFULL + i], 1);
             mbar_init(&bar[B_AEMPTY + i], 8);
             mbar_init(&bar[B_PFULL + i], 8);
             mbar_init(&bar[B_PEMPTY + i], 1);
-            mbar_init(&bar[B_OFULL + i], 1);
-            mbar_init(&bar[B_OEMPTY + i], G::EPI_MASK ? 4 : 4 * G::NSW);
             mbar_init(&bar[B_DSFULL + i], 1);
             mbar_init(&bar[B_DSEMPTY + i], 4 * G::NSW);
             mbar_init(&bar[B_SBFULL + i], 4 * G::NSW);
             mbar_init(&bar[B_SBEMPTY + i], 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&bar[B_PHI + i], 8);
         mbar_init(&bar[B_DRAIN], 1);
         *abort = 0;
         fence_barrier_init();
@@ -1215,9 +1307,9 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_TMA) {
         role_tma_q<DK, NV, NORM, REV>(x, &tmq);
     } else if (warp == G::W_MMA) {
-        role_mma<DK, NV, NORM, REV>(x);
+        role_mma<DK, NV, NORM, REV, PHI>(x);
     } else if (warp < G::W_ES) {
-        role_prep_mask<DK, NV, NORM, REV>(x);
+        role_prep_mask<DK, NV, NORM, REV, PHI>(x);
     } else if (warp < G::W_TMAV) {
         role_state_epilogue<DK, NV, NORM, REV>(x);
     } else {
@@ -1231,7 +1323,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_MMA) tmem_dealloc(tmem, G::TMEM_COLS);
 }
 
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
 cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                             const Params& p, int grid, cudaStream_t stream) {
     using G = Plan<DK, NV, NORM>;
@@ -1241,7 +1333,7 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         // at least 116 KB so that one CTA (512 TMEM columns) owns each SM
         const int smem = G::SMEM > 116 * 1024 ? G::SMEM : 116 * 1024;
         cudaError_t e =
-            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM, REV, PHI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         // programmatic serialisation: this grid's prologue (barriers, TMEM,
         // descriptor prefetch) overlaps the tail of the previous kernel
@@ -1255,7 +1347,7 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = p.pdl ? 1 : 0;
-        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM, REV>, tmq, tmk, tmv, p);
+        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM, REV, PHI>, tmq, tmk, tmv, p);
     }
 }
 
@@ -1265,25 +1357,29 @@ constexpr bool supported() {
 }
 
 // Dispatch on the value slice and the normaliser for one key width and one
-// direction; each instantiation file (la_fwd_ws_dk*.cu) instantiates these
-// for its key width, so that the build compiles the widths in parallel.
-template <int DK, bool REV, bool NORM>
+// direction (and feature map); each instantiation file (la_fwd_ws_dk*.cu)
+// instantiates these for its key width, so that the build compiles the
+// widths in parallel.
+template <int DK, bool REV, bool NORM, bool PHI>
 cudaError_t launch_nv(int nv, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                       const Params& p, int grid, cudaStream_t stream) {
     switch (nv) {
-        case 16: return launch_instance<DK, 16, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
-        case 32: return launch_instance<DK, 32, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
-        case 64: return launch_instance<DK, 64, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
-        case 128: return launch_instance<DK, 128, NORM, REV>(tmq, tmk, tmv, p, grid, stream);
+        case 16: return launch_instance<DK, 16, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 32: return launch_instance<DK, 32, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 64: return launch_instance<DK, 64, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 128: return launch_instance<DK, 128, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
         default: return cudaErrorNotSupported;
     }
 }
 
-template <int DK, bool REV>
+// PHI: the instances that apply the feature map to the Q and K tiles
+// (forward scans only; the others carry none of its code).
+template <int DK, bool REV, bool PHI>
 cudaError_t launch_dk(int nv, bool norm, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                       const Params& p, int grid, cudaStream_t stream) {
-    return norm ? launch_nv<DK, REV, true>(nv, tmq, tmk, tmv, p, grid, stream)
-                : launch_nv<DK, REV, false>(nv, tmq, tmk, tmv, p, grid, stream);
+    static_assert(!(REV && PHI), "the feature map applies to forward scans");
+    return norm ? launch_nv<DK, REV, true, PHI>(nv, tmq, tmk, tmv, p, grid, stream)
+                : launch_nv<DK, REV, false, PHI>(nv, tmq, tmk, tmv, p, grid, stream);
 }
 
 template <int DK>

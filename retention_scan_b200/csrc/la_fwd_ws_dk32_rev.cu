@@ -1,13 +1,13 @@
 // la_fwd_ws_dk32_rev.cu - instantiations of the warp-specialised tensor-core kernel for
-// Dk = 32, reverse (anti-causal) scan (one file per key width and direction, so that
-// the build compiles them in parallel).
+// Dk = 32, reverse (anti-causal) scan (one file per key width and variant, so that the build
+// compiles them in parallel).
 #include "la_fwd_ws.cuh"
 
 namespace la {
 namespace ws {
 
-template cudaError_t launch_dk<32, true>(int, bool, const CUtensorMap&, const CUtensorMap&,
-                                             const CUtensorMap&, const Params&, int, cudaStream_t);
+template cudaError_t launch_dk<32, true, false>(int, bool, const CUtensorMap&, const CUtensorMap&,
+                                                 const CUtensorMap&, const Params&, int, cudaStream_t);
 
 }  // namespace ws
 }  // namespace la

@@ -15,6 +15,14 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_tiled();
 
+// Device address of one of this library's __device__ variables in the
+// current device's current context (`slot` names the variable: one cache
+// entry per slot and device).  The lookup (cudaGetSymbolAddress) runs once per
+// device and is repeated only when the device's context has changed since,
+// for instance after cudaDeviceReset; null if it fails.
+enum SymbolSlot : int { kSymErrWord = 0, kSymStaticScratch = 1, kSymSlots = 2 };
+void* device_symbol_address(const void* symbol, int slot);
+
 // Device error codes written by kernels that give up waiting on a barrier.
 enum DeviceError : int {
     kErrNone = 0,
@@ -41,7 +49,7 @@ struct FwdArgs {
     size_t workspace_bytes;
     int reverse;              // 1: anti-causal scan, t = T-1 down to 0
     int accumulate;           // 1: add y to the values already in out
-    int feature_map;          // la_feature_map on q and k (fp32 path only)
+    int feature_map;          // la_feature_map on q and k (forward scans)
     float q_scale;            // q <- q_scale * phi(q)
 };
 

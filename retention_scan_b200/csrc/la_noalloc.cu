@@ -3,8 +3,6 @@
 // instead of from the caller, so that a call allocates no device memory.
 #include <cuda_runtime.h>
 
-#include <atomic>
-
 #include "la.h"
 #include "la_internal.h"
 
@@ -13,20 +11,12 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t{16} << 20;  // 16 MiB per device
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
-
-// Device address of the array in the current device's context (looked up
-// once per device; the symbol has a different address on every device).
+// Device address of the array in the current device's context: the symbol
+// has a different address on every device, and in host code its name is only
+// a host-side stand-in.  Looked up with cudaGetSymbolAddress on the first
+// call on each device (and again if that device's context was reset since).
 void* static_scratch_for_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    void* p = g_scratch_ptr[dev].load();
-    if (!p) {
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev].store(p);
-    }
-    return p;
+    return la::device_symbol_address(&g_static_scratch, la::kSymStaticScratch);
 }
 
 }  // namespace

@@ -72,7 +72,8 @@ def _fwd(L, **over):
     (dict(Dk=0), 1),
     (dict(dtype=7), 1),
     (dict(normalize=1, init_state=32, init_z=None), 1),   # carried state without its key sum
-    (dict(Dk=48), 2),                     # bf16 tensor-core path: widths 16/32/64/128
+    (dict(Dk=40), 2),                     # bf16 tensor-core path: multiples of 16 up to 128
+    (dict(Dk=144), 2),
     (dict(Dv=256), 2),
     (dict(dtype=0, Dk=129), 2),
 ], ids=str)
@@ -185,7 +186,7 @@ def test_reverse_and_bidirectional_validate_like_the_forward(L):
         assert f(out=8) == 1
         assert f(T=-1) == 1
         assert f(dtype=9) == 1
-        assert f(Dk=48) == 2
+        assert f(Dk=40) == 2
         assert f(dtype=0, Dv=200) == 2
         assert f(B=0) == 0
     assert rev(normalize=1, init_state=32, init_z=None) == 1
@@ -239,7 +240,7 @@ def _bwd(L, **over):
     (dict(dS0=8), 1),
     (dict(T=-1), 1),
     (dict(dtype=5), 1),
-    (dict(Dk=48), 2),
+    (dict(Dk=40), 2),
     (dict(dtype=0, Dv=130), 2),
     (dict(B=0), 0),                           # empty batch: a no-op
 ], ids=str)
@@ -336,7 +337,12 @@ def test_prologue_validation(L):
     assert fwd(P(2, 1.0)) == 1                   # feature map out of range
     assert fwd(P(0, float("inf"))) == 1          # q scale not finite
     assert fwd(P(0, float("nan"))) == 1
-    assert fwd(P(1, 1.0)) == 2                   # bf16 tensor-core path: no feature map
+    # the bf16 tensor-core path takes the feature map too: its argument
+    # checks pass, and an unsupported width still gives LA_ERR_UNSUPPORTED
+    assert L.la_chunk_forward_pro_ws(vp(16), vp(16), vp(16), None, 0, ctypes.byref(P(1, 1.0)), None, None, vp(16),
+                                     None, None, 1, 1, 4, 40, 16, 1, None, 0, None) == 2
+    assert L.la_chunk_forward_pro_ws(None, None, None, None, 0, ctypes.byref(P(1, 1.0)), None, None, None, None,
+                                     None, 0, 1, 4, 16, 16, 1, None, 0, None) == 0
     assert dec(P(-1, 1.0)) == 1
     assert dec(P(0, float("inf"))) == 1
     # B = 0 with valid prologues: no-ops (the fp32 path takes the feature map)

@@ -112,7 +112,7 @@ def test_backward_tc(kind, init, final, D):
     check_backward(inp, S0, dSf, seed=7 + kind)
 
 
-@pytest.mark.parametrize("Dk,Dv", [(16, 128), (128, 32), (64, 16), (32, 64)])
+@pytest.mark.parametrize("Dk,Dv", [(16, 128), (128, 32), (64, 16), (32, 64), (48, 80), (112, 96), (96, 48)])
 def test_backward_widths(Dk, Dv):
     inp, S0, _ = gen_case(1, 3, 333, Dk, Dv, kind=2, init=True, seed=3200 + Dk + Dv)
     dSf = torch.randn(1, 3, Dk, Dv, generator=torch.Generator().manual_seed(41))

@@ -138,7 +138,7 @@ def test_backward_norm_tc(kind, init, final, D):
     check(inp, S0, z0, dSf, dzf, seed=9 + kind)
 
 
-@pytest.mark.parametrize("Dk,Dv", [(16, 128), (128, 32), (64, 16)])
+@pytest.mark.parametrize("Dk,Dv", [(16, 128), (128, 32), (64, 16), (80, 48), (48, 112)])
 def test_backward_norm_widths(Dk, Dv):
     inp, S0, z0 = gen_case(1, 3, 333, Dk, Dv, kind=2, normalize=True, init=True, seed=6200 + Dk + Dv)
     check(inp, S0, z0, None, torch.randn(1, 3, Dk) * 0.1, seed=19)

@@ -131,7 +131,10 @@ def test_fp32_flags(kind, normalize):
 
 # ---------------------------------------------------------------- tensor-core path
 
-WIDTHS = [16, 32, 64, 128]
+# every multiple of 16 up to 128: 16, 32, 64 and 128 have kernel instances of
+# their own; the others run on the next larger key width (zero-filled
+# columns) and on value slices whose last one reaches past Dv
+WIDTHS = [16, 32, 48, 64, 80, 96, 112, 128]
 
 
 @pytest.mark.parametrize("Dk", WIDTHS)
@@ -232,6 +235,17 @@ def test_segments_direct_form(monkeypatch, decay_mean):
     check_case(inp, True, S0, z0)
 
 
+@pytest.mark.parametrize("Dk,Dv", [(48, 112), (80, 48), (112, 80)])
+@pytest.mark.parametrize("normalize", [False, True])
+def test_segments_odd_widths(monkeypatch, Dk, Dv, normalize):
+    # T-segments with padded key columns and a last value slice past Dv: the
+    # state pass's workspace and the fold use the tensors' own widths
+    monkeypatch.setenv("LA_SEGMENTS", "3")
+    inp, S0, z0 = gen_case(1, 2, 2048 + 77, Dk, Dv, kind=2, normalize=normalize, init=True, seed=Dk * 7 + Dv,
+                           decay_mean=4.0)
+    check_case(inp, normalize, S0, z0)
+
+
 def test_segments_match_one_segment():
     # the default plan segments this shape; without a workspace it runs as one segment
     inp, S0, _ = gen_case(1, 4, 4096, 64, 64, kind=1, init=True, seed=930)
@@ -289,7 +303,7 @@ def test_empty_and_zero_sizes():
 
 
 def test_invalid_arguments_raise():
-    q = torch.randn(1, 1, 8, 48, device="cuda", dtype=torch.bfloat16)
+    q = torch.randn(1, 1, 8, 40, device="cuda", dtype=torch.bfloat16)  # bf16: not a multiple of 16
     with pytest.raises(la().LAError) as ei:
         la().chunk_forward(q, q, q)
     assert ei.value.status == 2
@@ -402,3 +416,43 @@ def test_decode_workload_sampled_heads():
         assert rel_err(y.view(-1, wl.Dv)[heads][None], yr) <= 2e-2
     assert rel_err(S.view(-1, wl.Dk, wl.Dv)[heads][None], Sref) <= 1e-5
     assert rel_err(z.view(-1, wl.Dk)[heads][None], zref) <= 1e-5
+
+
+def test_decode_workload_1024_tokens_sampled_heads():
+    """The decode workload as the benchmark runs it: the full-size state
+    [256, 32, 128, 128], 1024 token calls in a row (tokens drawn on the
+    device), y checked at every step and the state and key sum after the last
+    one, on sampled heads whose tokens and initial state the oracle reads bit
+    for bit.  The outputs are bf16 (bar 2e-2 per step and head).  The fp32
+    state and key sum meet 1e-4: each step rounds the update once (2^-24) and
+    the per-head decay is rounded once to fp32 (at most 2^-25 relative), so
+    1024 steps stay below 1024 * 3 * 2^-25 ~ 9e-5 even if every rounding went
+    the same way."""
+    wl = W.DECODE
+    steps, Dk, Dv = wl.steps, wl.Dk, wl.Dv
+    heads = [0, 31, 1000, 2047, 4100, 6150, 7000, wl.B * wl.H - 1]
+    S0, z0 = W.decode_initial_state(wl)
+    S, z = S0.cuda(), z0.cuda()
+    q, k, v = W.decode_pool_device(wl, steps, torch.device("cuda"))
+    lg = W.per_head_log_gamma(wl.H).cuda()
+    idx = torch.tensor(heads, device="cuda")
+    out = torch.empty(wl.B, wl.H, Dv, dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty(steps, len(heads), Dv, dtype=torch.bfloat16, device="cuda")
+    for t in range(steps):
+        la().decode_step(q[t], k[t], v[t], S, z, 1, lg, True, out=out)
+        ys[t] = out.view(-1, Dv).index_select(0, idx)
+    torch.cuda.synchronize()
+    qs = q.view(steps, -1, Dk).index_select(1, idx).cpu()
+    ks = k.view(steps, -1, Dk).index_select(1, idx).cpu()
+    vs = v.view(steps, -1, Dv).index_select(1, idx).cpu()
+    del q, k, v
+    Sref = S0.view(-1, Dk, Dv)[heads][None].double().numpy()
+    zref = z0.view(-1, Dk)[heads][None].double().numpy()
+    lgs = W.per_head_log_gamma(wl.H)[[bh % wl.H for bh in heads]]
+    yref = np.zeros((steps, len(heads), Dv))
+    for t in range(steps):
+        yr, Sref, zref = oracle.decode_step(qs[t][None], ks[t][None], vs[t][None], Sref, zref, 1, lgs, True)
+        yref[t] = yr[0]
+    assert rel_err(ys, yref) <= 2e-2  # every (step, head) slice
+    assert rel_err(S.view(-1, Dk, Dv)[heads][None], Sref) <= 1e-4
+    assert rel_err(z.view(-1, Dk)[heads][None], zref) <= 1e-4

@@ -79,6 +79,61 @@ def test_bf16_forward_with_q_scale(kind, normalize, T):
     assert max(errs.values()) <= TOL[torch.bfloat16], errs
 
 
+@pytest.mark.parametrize("kind", [0, 1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+@pytest.mark.parametrize("T", [300, 4096 + 77])
+def test_bf16_forward_with_feature_map(kind, normalize, T):
+    """phi = elu + 1 on the Q and K tiles inside the tensor-core kernel (the
+    raw q, k cross HBM once), with the q scale; long T also runs T-segments,
+    whose state pass maps its K tiles the same way."""
+    inp, S0, z0 = gen_case(1, 2, T, 64, 64, kind=kind, normalize=False, init=True,
+                           seed=5300 + kind * 2 + normalize + T)
+    if normalize:
+        z0 = torch.rand(1, 2, 64) * 4 + 0.5
+    scale = 0.37
+    d = to_dev(inp)
+    y, S, z = la().chunk_forward(d["q"], d["k"], d["v"], kind, d["log_g"], normalize, S0.cuda(),
+                                 z0.cuda() if normalize else None, feature_map=la().FEATURE_ELU1, q_scale=scale)
+    torch.cuda.synchronize()
+    yr, Sr, zr = oracle.forward(scale * elu1(inp["q"]), elu1(inp["k"]), inp["v"], kind, inp["log_g"], normalize,
+                                S0, z0 if normalize else None)
+    errs = {"y": rel_err(y, yr), "S": rel_err(S, Sr)}
+    if normalize:
+        errs["z"] = rel_err(z, zr)
+    assert max(errs.values()) <= TOL[torch.bfloat16], errs
+
+
+@pytest.mark.parametrize("Dk,Dv", [(48, 80), (128, 128), (16, 32), (112, 64)])
+def test_bf16_feature_map_widths(Dk, Dv):
+    """Padded key widths: the zero columns past Dk must stay zero (phi(0) = 1)."""
+    inp, S0, _ = gen_case(2, 3, 333, Dk, Dv, kind=2, normalize=False, init=True, seed=5400 + Dk + Dv)
+    z0 = torch.rand(2, 3, Dk) * 4 + 0.5
+    d = to_dev(inp)
+    y, S, z = la().chunk_forward(d["q"], d["k"], d["v"], 2, d["log_g"], True, S0.cuda(), z0.cuda(),
+                                 feature_map=la().FEATURE_ELU1)
+    torch.cuda.synchronize()
+    yr, Sr, zr = oracle.forward(elu1(inp["q"]), elu1(inp["k"]), inp["v"], 2, inp["log_g"], True, S0, z0)
+    errs = {"y": rel_err(y, yr), "S": rel_err(S, Sr), "z": rel_err(z, zr)}
+    assert max(errs.values()) <= TOL[torch.bfloat16], errs
+
+
+def test_bf16_feature_map_equals_caller_side_map():
+    """The normalised workload's recipe: phi in the kernel on the raw bf16
+    q, k against phi applied by the caller in fp32 and rounded to bf16.  The
+    kernel evaluates the exponential at the tiles' bf16 precision (argument
+    and result), a bf16 rounding step or two from the fp32 value, so the
+    outputs agree to about 0.3 %, far inside the bar."""
+    g = torch.Generator().manual_seed(5500)
+    B, H, T, D = 2, 4, 1000, 128
+    q, k, v = (torch.randn(B, H, T, D, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    y1, S1, z1 = la().chunk_forward(q, k, v, normalize=True, feature_map=la().FEATURE_ELU1)
+    phi = lambda x: (torch.nn.functional.elu(x.float()) + 1).to(torch.bfloat16)  # noqa: E731
+    y2, S2, z2 = la().chunk_forward(phi(q), phi(k), v, normalize=True)
+    torch.cuda.synchronize()
+    for a, b in ((y1, y2), (S1, S2), (z1, z2)):
+        assert rel_err(a, b.cpu().double().numpy()) <= 1e-2
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("normalize", [False, True])
 @pytest.mark.parametrize("D", [64, 128, 40])

@@ -77,8 +77,8 @@ def test_reverse_tc_flags(kind, normalize, init, D):
     check_reverse(inp, normalize, S0, z0)
 
 
-@pytest.mark.parametrize("Dk", [16, 32, 64, 128])
-@pytest.mark.parametrize("Dv", [16, 32, 64, 128])
+@pytest.mark.parametrize("Dk", [16, 32, 48, 64, 112, 128])
+@pytest.mark.parametrize("Dv", [16, 32, 80, 64, 96, 128])
 def test_reverse_tc_widths(Dk, Dv):
     inp, S0, _ = gen_case(1, 2, 300, Dk, Dv, kind=2, init=True, seed=2200 + Dk + Dv)
     check_reverse(inp, False, S0)

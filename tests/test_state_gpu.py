@@ -111,7 +111,7 @@ def test_span_state_empty():
 def test_fold_of_spans_is_the_concatenated_forward(dtype, kind, normalize):
     """Ragged spans' states folded onto an initial state equal the final
     state of one forward over the whole sequence from that state."""
-    B, H, Dk, Dv = 2, 2, 32, 64
+    B, H, Dk, Dv = 2, 2, 32, 48
     cuts = [0, 150, 151, 400, 640, 1001]
     T = cuts[-1]
     inp, S0, z0 = gen_case(B, H, T, Dk, Dv, dtype=dtype, kind=kind, normalize=normalize, init=True,
