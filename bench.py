@@ -5,11 +5,13 @@
 
 One step is one pass of the hot path over one batch of the workload:
 
-  config 2 (default): retention, per-head gamma_h = 1 - 2^(-5-h), bf16,
-      B=4, H=8, T=2048, Dk=Dv=64 -> one la_chunk_forward call
+  config 4 (the headline of the default run): gated per-step decay,
+      B=1, H=32, T=65536, D=128 -> one la_chunk_forward call (the largest
+      single-GPU workload)
   config 1: plain linear attention, fp32, B=1, H=1, T=64, D=16
+  config 2: retention, per-head gamma_h = 1 - 2^(-5-h), bf16,
+      B=4, H=8, T=2048, Dk=Dv=64
   config 3: normalised, elu+1 feature map, carried state, B=8, H=16, T=4096, D=128
-  config 4: gated per-step decay, B=1, H=32, T=65536, D=128
   config 5: decode, B=256, H=32, D=128, normalised, 1024 la_decode_step calls
   config 6: the RWKV-4 WKV recurrence, B=8, T=4096, C=2048, bf16 -> one
       la_wkv4_forward call (tokens = B*T; a different recurrence)
@@ -25,12 +27,22 @@ log-decay gradient and, with a carried state, the initial state's and key
 sum's) for a seeded upstream gradient dy.  Configs 1-4; config 7 takes
 forward or reverse (la_ema_scan's reverse flag).
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
-on the launching stream; the L2 cache (126 MB) is flushed by writing a 512 MB
-buffer before every step whose inputs fit in L2, outside the events.  A
-barrier and a device synchronisation bracket the timed region; the time is
-the maximum over ranks.  Under torchrun every rank runs the same per-GPU
-workload (weak scaling, no collective on the data path).
+Without --config the run times config 4 for the JSON line's headline
+fields and adds a "configs" record with the same measurement of configs 3
+(normalised, T=4096), 5 (decode, per token) and 2 (retention, T=2048), each
+with its own roofline, clocks, e2e and cpu_baseline.
+
+Timing: W untimed warm-up steps, then untimed steps until the GPU has run
+the step for at least half a second (its clocks leave their idle state:
+short runs otherwise time the ramp), then K steps, each bracketed by CUDA
+events on the launching stream; the L2 cache (126 MB) is flushed by writing
+a 512 MB buffer before every step whose inputs fit in L2, outside the events.
+A barrier and a device synchronisation bracket the timed region; the time is
+the maximum over ranks; ms_per_step is its mean, and the median, minimum and
+maximum of the per-step times are reported beside it.  `--gpus N` without
+torchrun's environment starts N local ranks itself (torch.distributed.run);
+every rank runs the same per-GPU workload (weak scaling, no collective on
+the data path).
 
 Extra keys: roofline (dominant kernel, algorithmic bytes / event time against
 the measured HBM copy bandwidth), e2e (the same metric through the public API
@@ -104,24 +116,26 @@ def tokens_per_step(wl, cfg):
     return wl.B * wl.H * (wl.steps if cfg == 5 else wl.T)
 
 
-def kernel_source_sha():
+def kernel_source_sha(files):
+    """Hash of the kernel source files (names under csrc/, and include/la.h)
+    that a measured kernel is built from."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "retention_scan_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
+    for f in sorted(files):
+        path = os.path.join(ROOT, "include", f) if f == "la.h" else os.path.join(ROOT, "retention_scan_b200", "csrc", f)
+        with open(path, "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(workload_name):
     """DRAM bytes per launch of the dominant kernel from a committed ncu
-    summary, if it was taken on the current kernel sources; else None."""
+    summary, if it was taken on the kernel's current sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(path)).get(workload_name)
-    except (OSError, ValueError):
-        return None
-    if not rec or rec.get("kernel_sha") != kernel_source_sha():
+        if not rec or rec.get("kernel_sha") != kernel_source_sha(rec["sources"]):
+            return None
+    except (OSError, ValueError, KeyError):
         return None
     return rec.get("bytes_per_launch")
 
@@ -203,13 +217,17 @@ def bus_id_of(device):
 class Job:
     """Device-resident inputs and the step function of one workload."""
 
-    def __init__(self, cfg, device, wl=None, rank=0, direction="forward"):
+    def __init__(self, cfg, device, wl=None, rank=0, direction="forward", prologue=False):
         import retention_scan_b200 as la
         self.la = la
         self.cfg = cfg
         self.direction = direction
         self.wl = wl = wl or W.WORKLOADS[cfg]
         self.dev = device
+        # prologue: q, k handed over raw and the feature map applied inside
+        # the forward kernel (la_chunk_forward_pro_ws) instead of by the caller
+        self.prologue = prologue and wl.feature_map == "elu1"
+        self.fmap = la.FEATURE_ELU1 if self.prologue else la.FEATURE_NONE
         if cfg == 5:
             S0, z0 = W.decode_initial_state(wl)
             self.S0, self.z0 = S0.to(device), z0.to(device)
@@ -218,7 +236,7 @@ class Job:
             self.log_g = W.per_head_log_gamma(wl.H).to(device)
             self.out = torch.empty(wl.B, wl.H, wl.Dv, dtype=wl.torch_dtype, device=device)
             return
-        inp = W.forward_inputs(wl, seed=rank_seed(wl, rank))
+        inp = W.forward_inputs(wl.with_sizes(feature_map=None) if self.prologue else wl, seed=rank_seed(wl, rank))
         self.host = inp
         self.q, self.k, self.v = (inp[n].to(device) for n in ("q", "k", "v"))
         self.kind = inp["decay_kind"]
@@ -248,9 +266,10 @@ class Job:
             self.fwd_launches = backward_launches(la, wl, self.kind, wl.prefix_T > 0)
         if wl.prefix_T and direction != "bidirectional":
             # carried state of the workload: the library's own forward over the seeded prefix
-            pre = W.prefix_inputs(wl)
+            pre = W.prefix_inputs(wl.with_sizes(feature_map=None) if self.prologue else wl)
             _, self.S0, self.z0 = la.chunk_forward(pre["q"].to(device), pre["k"].to(device),
-                                                   pre["v"].to(device), pre["decay_kind"], None, True)
+                                                   pre["v"].to(device), pre["decay_kind"], None, True,
+                                                   feature_map=self.fmap)
 
     def step(self):
         la, wl = self.la, self.wl
@@ -270,8 +289,16 @@ class Job:
         else:
             la.chunk_forward(self.q, self.k, self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
                              out=self.out, final_state=self.S, final_z=self.z,
-                             reverse=self.direction == "reverse")
+                             reverse=self.direction == "reverse", feature_map=self.fmap)
         return self.fwd_launches
+
+    def caller_mapped_step(self):
+        """The step as a caller without the prologue runs it: elu + 1 on q and
+        k by a torch pass (fp32, stored as bf16), then the forward on them."""
+        la, wl = self.la, self.wl
+        phi = lambda x: (torch.nn.functional.elu(x.float()) + 1.0).to(x.dtype)  # noqa: E731
+        la.chunk_forward(phi(self.q), phi(self.k), self.v, self.kind, self.log_g, wl.normalize, self.S0, self.z0,
+                         out=self.out, final_state=self.S, final_z=self.z)
 
     E2E_DECODE_TOKENS = 64
 
@@ -307,7 +334,7 @@ class Job:
             return tokens_per_step(wl, self.cfg)
         y, S, _ = la.chunk_forward(q, k, v, self.kind, lg, wl.normalize, self.S0, self.z0,
                                    out=self.out, final_state=self.S, final_z=self.z,
-                                   reverse=self.direction == "reverse")
+                                   reverse=self.direction == "reverse", feature_map=self.fmap)
         pinned["y"].copy_(y, non_blocking=True)
         pinned["S"].copy_(S, non_blocking=True)
         return tokens_per_step(wl, self.cfg)
@@ -356,7 +383,7 @@ def backward_launches(la, wl, kind, carried):
         return (n + (1 if carried else 0) + (2 if carried else 0) + 1 + scan(wl.Dk, wl.Dv) + scan(wl.Dk, 16) + 1
                 + scan(wl.Dv, wl.Dk) + scan(16, wl.Dk) + 1 + scan(wl.Dv, wl.Dk) + scan(16, wl.Dk)
                 + scan(wl.Dk, wl.Dv) + 1)
-    W = next(w for w in (32, 64, 128) if w > wl.Dv) if wl.dtype != "f32" else wl.Dv + 1
+    W = wl.Dv + 16 if wl.dtype != "f32" else wl.Dv + 1
     return (n + (2 if carried else 0) + 1 + scan(wl.Dk, W) + 1 + 2 * scan(W, wl.Dk) + scan(wl.Dk, wl.Dv) + 1)
 
 
@@ -412,6 +439,46 @@ def rank_seed(wl, rank):
     """Each rank processes its own batch of independent sequences (weak
     scaling): same shapes and distributions, rank-specific seed."""
     return wl.seed + 7919 * rank
+
+
+SPIN_UP_S = 0.5
+
+
+def spin_up(job, flush, device, min_s=SPIN_UP_S):
+    """Untimed steps until the GPU has run them for min_s seconds of wall
+    time (at least one), so that the timed steps do not see the SM clock
+    ramping up from idle.  Returns the number of steps run."""
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        if flush is not None:
+            flush.add_(1)
+        job.step()
+        n += 1
+        if n % 4 == 0 or n == 1:
+            torch.cuda.synchronize(device)
+            if time.perf_counter() - t0 >= min_s:
+                return n
+
+
+def step_stats(per):
+    """Median, minimum and maximum of the per-step event times (ms)."""
+    return {"median": round(statistics.median(per), 5), "min": round(min(per), 5), "max": round(max(per), 5)}
+
+
+def config_dict(wl, cfg, direction, world):
+    """The JSON line's `config`: the workload and how it is timed (shared by
+    both arms, so that their lines name the same configuration)."""
+    if cfg == 5:
+        in_l2 = False
+    else:
+        in_l2 = algorithmic_bytes(wl, cfg, direction) < 2 * L2_BYTES
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
+            "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
+            "direction": direction,
+            "decode_steps": wl.steps if cfg == 5 else None,
+            "l2": "flushed before every step (512 MB write)" if in_l2 else "inputs larger than L2",
+            "parallelism": f"replicas x{world}; batch sharded across GPUs (weak scaling), no collective"}
 
 
 def time_steps(job, steps, flush, dist_on, device):
@@ -496,21 +563,23 @@ def cpu_baseline(cfg, budget_s=15.0, direction="forward"):
             "sample": f"{nh} of {total} (b,h) sequences, all {wl.T} tokens each, {threads} threads"}
 
 
-def sized_workload(args):
-    """The workload of --config, with --tokens / --batch overrides (smaller
-    cases for profiler captures); an override renames the workload."""
-    wl = W.WORKLOADS[args.config]
-    if args.tokens and args.config != 5:
+def sized_workload(args, cfg):
+    """The workload of config `cfg`, with --tokens / --batch overrides
+    (smaller cases for profiler captures); an override renames the workload."""
+    wl = W.WORKLOADS[cfg]
+    if args.tokens and cfg != 5:
         wl = wl.with_sizes(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.batch:
         wl = wl.with_sizes(B=args.batch, name=f"{wl.name}_B{args.batch}")
     return wl
 
 
-def run_ours(args, rank, world, dist_on, device):
-    cfg = args.config
-    wl = sized_workload(args)
-    job = Job(cfg, device, wl, rank, args.direction)
+def run_ours(args, rank, world, dist_on, device, cfg=None, prologue=False):
+    cfg = args.config if cfg is None else cfg
+    wl = sized_workload(args, cfg)
+    job = Job(cfg, device, wl, rank, args.direction, prologue=prologue)
+    if job.prologue:
+        wl = job.wl = wl.with_sizes(name=wl.name + "_raw_qk_elu1_in_kernel")
     torch.cuda.synchronize()
     in_bytes = algorithmic_bytes(wl, cfg, args.direction) * (wl.steps if cfg == 5 else 1)
     flush = None
@@ -522,6 +591,7 @@ def run_ours(args, rank, world, dist_on, device):
             flush.add_(1)
         job.step()
     torch.cuda.synchronize()
+    spun = spin_up(job, flush, device)
     assert job.la.device_error(device) == 0
 
     sampler = ClockSampler(bus_id_of(device)) if rank == 0 else None
@@ -582,25 +652,43 @@ def run_ours(args, rank, world, dist_on, device):
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
 
     clocks = sampler.summary(w0, w1) if sampler else None
+    # per-step statistics, the slowest rank's (max over ranks of each)
+    stats = {k: max_over_ranks(v, dist_on, device) for k, v in step_stats(per).items()}
     line = {
         "metric": metric_for(args.direction), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if wl.dtype == "f32" else "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
-                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
-                   "direction": args.direction,
-                   "decode_steps": wl.steps if cfg == 5 else None,
-                   "l2": "flushed before every step (512 MB write)" if flush is not None
-                   else "inputs larger than L2",
-                   "parallelism": f"replicas x{world}; per GPU (b,h) spread over CTAs by value slices"
-                   + (" and T-segments" if cfg != 5 and job.fwd_launches in (2, 4) and
-                      (args.direction != "bidirectional" or job.fwd_launches == 4) else "")},
+        "config": config_dict(wl, cfg, args.direction, world),
         "roofline": roofline, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches,
+        "ms_per_step_stats": stats,
+        "spin_up": {"steps": spun, "min_s": SPIN_UP_S},
+        "plan": ("decode: one CTA per (b, h)" if cfg == 5 else
+                 "one CTA per (b, h)" if wl.dtype == "f32" else
+                 "per GPU (b, h) spread over CTAs by value slices"
+                 + (" and T-segments (state pass + output pass)" if job.fwd_launches in (2, 4) and
+                    (args.direction != "bidirectional" or job.fwd_launches == 4) else "")),
     }
     if graph:
         line["decode_graph"] = graph
+    if job.prologue:
+        # the same step with the feature map applied by a caller pass instead
+        # (it reads and writes q and k once more: 4 B H T Dk bf16 bytes)
+        for _ in range(3):
+            job.caller_mapped_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(torch.cuda.current_stream(device))
+        for _ in range(args.steps):
+            job.caller_mapped_step()
+        e1.record(torch.cuda.current_stream(device))
+        barrier(dist_on)
+        caller_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist_on, device)
+        line["feature_map"] = {"where": "in the forward kernel (la_chunk_forward_pro_ws, FEATURE_ELU1) on raw q, k",
+                               "caller_pass_ms_per_step": round(caller_ms, 5),
+                               "caller_pass_extra_hbm_bytes": 4 * wl.B * wl.H * wl.T * wl.Dk * 2,
+                               "saving_ms_per_step": round(caller_ms - ms_per_step, 5)}
     return line
 
 
@@ -746,6 +834,7 @@ def run_wkv4(args, rank, world, dist_on, device):
             flush.add_(1)
         job.step()
     torch.cuda.synchronize()
+    spun = spin_up(job, flush, device)
     assert job.la.device_error(device) == 0
     sampler = ClockSampler(bus_id_of(device)) if rank == 0 else None
     if sampler:
@@ -757,6 +846,7 @@ def run_wkv4(args, rank, world, dist_on, device):
         sampler.stop()
     assert job.la.device_error(device) == 0
     ms = max_over_ranks(sum(per), dist_on, device) / args.steps
+    stats = {k: max_over_ranks(v, dist_on, device) for k, v in step_stats(per).items()}
     pk, pk_kind = peaks()
     gbs = nbytes / (ms / 1e3) / 1e9
     e2e = None
@@ -774,8 +864,8 @@ def run_wkv4(args, rank, world, dist_on, device):
                    **({"direction": args.direction} if ema else {}),
                    "l2": "flushed before every step (512 MB write)" if flush is not None
                    else "inputs larger than L2",
-                   "parallelism": f"replicas x{world}; per GPU one CTA per (batch row, 64 channels"
-                   + (", T-segment)" if job.launches == 2 else ")")},
+                   "parallelism": f"replicas x{world}; batch sharded across GPUs (weak scaling), no collective"},
+        "plan": "per GPU one CTA per (batch row, 64 channels" + (", T-segment)" if job.launches == 2 else ")"),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4),
                      "traffic": measured_traffic(wl.name) if args.direction == "forward" else None,
@@ -784,51 +874,103 @@ def run_wkv4(args, rank, world, dist_on, device):
                      ("wkv4_kernel (state pass + output pass)" if job.launches == 2 else "wkv4_kernel"),
                      "algorithmic_bytes_per_launch": nbytes},
         "e2e": e2e, "clocks": sampler.summary(w0, w1) if sampler else None, "gpu_launches": launches,
+        "ms_per_step_stats": stats, "spin_up": {"steps": spun, "min_s": SPIN_UP_S},
     }
 
 
 # ---------------------------------------------------------------- reference arm (the oracle)
 
-def run_reference(args):
+def run_reference(args, world):
+    """The oracle as it stands on the host cores: each step a bounded sample of
+    the workload, sized so that W + K steps take about two and a half minutes."""
     cfg = args.config
+    per_step_s = min(8.0, max(1.0, 150.0 / max(1, args.steps + args.warmup)))
     if cfg in (6, 7):
         wl = W.WKV4 if cfg == 6 else W.EMA
         base = cpu_baseline_wkv4 if cfg == 6 else cpu_baseline_ema
         for _ in range(args.warmup):
-            base(wl, budget_s=2.0)
-        vals = [base(wl, budget_s=8.0) for _ in range(args.steps)]
+            base(wl, budget_s=min(2.0, per_step_s))
+        vals = [base(wl, budget_s=per_step_s) for _ in range(args.steps)]
         v = statistics.median(x["value"] for x in vals)
         cb = dict(vals[-1])
         cb["value"] = v
         return {"impl": "reference", "metric": WKV4_METRIC if cfg == 6 else EMA_METRIC, "value": v, "unit": "tokens/s",
-                "n_gpus": 1,
+                "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.B * wl.T / v * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C},
+                "data": "synthetic",
+                "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+                           **({"direction": args.direction} if cfg == 7 else {}),
+                           "l2": "flushed before every step (512 MB write)"
+                           if (ema_bytes if cfg == 7 else wkv4_bytes)(wl) < 2 * L2_BYTES else "inputs larger than L2",
+                           "parallelism": f"replicas x{world}; batch sharded across GPUs (weak scaling), no collective"},
                 "cpu_baseline": cb,
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                 "gpu_launches": 0}
     wl = W.WORKLOADS[cfg]
     for _ in range(args.warmup):
-        cpu_baseline(cfg, budget_s=2.0, direction=args.direction)
+        cpu_baseline(cfg, budget_s=min(2.0, per_step_s), direction=args.direction)
     vals = []
     for _ in range(args.steps):
-        vals.append(cpu_baseline(cfg, budget_s=8.0, direction=args.direction))
+        vals.append(cpu_baseline(cfg, budget_s=per_step_s, direction=args.direction))
     v = statistics.median(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = v
     return {
-        "impl": "reference", "metric": metric_for(args.direction), "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "impl": "reference", "metric": metric_for(args.direction), "value": v, "unit": "tokens/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tokens_per_step(wl, cfg) / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T if cfg != 5 else 1,
-                   "Dk": wl.Dk, "Dv": wl.Dv, "decay": wl.decay, "normalize": wl.normalize,
-                   "direction": args.direction},
+        "config": config_dict(wl, cfg, args.direction, world),
         "cpu_baseline": cb,
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+
+
+EXTRA_CONFIGS = (3, 5, 2)  # measured beside the headline config 4 by the default run
+
+
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def launch_ranks(n):
+    """`--gpus N` outside torchrun: run this command as N local ranks under
+    torch.distributed.run (rank 0 prints the line) and return its status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+    env = dict(os.environ, OMP_NUM_THREADS=os.environ.get("OMP_NUM_THREADS", "1"))
+    return subprocess.run(cmd, env=env).returncode
+
+
+def cpu_selftest(rank, world):
+    """The multi-rank timing path without a GPU (gloo): rank r times a host
+    busy loop of (r + 1) * 20 ms per step, between barriers; the reported
+    time is the maximum over ranks, as for the GPU steps."""
+    import datetime
+    torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        torch.distributed.barrier()
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 0.02 * (rank + 1):
+            pass
+        ms = (time.perf_counter() - t0) * 1e3
+        torch.distributed.barrier()
+        t = torch.tensor([ms], dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        mine = torch.tensor([ms], dtype=torch.float64)
+        every = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
+        torch.distributed.all_gather(every, mine)
+        if rank == 0:
+            print(json.dumps({"selftest": True, "n_gpus": world, "ms_per_step": float(t.item()),
+                              "per_rank_ms": [float(x.item()) for x in every]}), flush=True)
+    finally:
+        torch.distributed.destroy_process_group()
 
 
 def main():
@@ -836,18 +978,25 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5, 6, 7],
+                    help="time one workload only (default: config 4 with configs 3, 5 and 2 beside it)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling a smaller case)")
     ap.add_argument("--direction", default="forward", choices=["forward", "reverse", "bidirectional", "backward"])
+    ap.add_argument("--cpu-selftest", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
+    combined = args.config is None
+    if combined:
+        args.config = 4
     if args.config in (5, 6) and args.direction != "forward":
         ap.error("--direction applies to the whole-sequence configs 1-4 and 7")
     if args.config == 7 and args.direction not in ("forward", "reverse"):
         ap.error("the cumulative EMA (config 7) scans forward or reverse")
+    if combined and args.direction != "forward":
+        combined = False  # the extra configs are forward lines
     default_steps = {1: 2000, 2: 2000, 3: 200, 4: 50, 5: 3, 6: 200, 7: 200}
     if args.steps is None:
         args.steps = default_steps[args.config] if args.impl == "ours" else 3
@@ -855,13 +1004,20 @@ def main():
         args.warmup = max(3, args.steps // 20) if args.impl == "ours" else 1
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(launch_ranks(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but {world} ranks were launched")
 
+    if args.cpu_selftest:
+        cpu_selftest(rank, world)
+        return
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
 
     device = torch.device("cuda", local_rank)
@@ -873,12 +1029,29 @@ def main():
                                              timeout=datetime.timedelta(seconds=120))
     try:
         line = (run_wkv4 if args.config in (6, 7) else run_ours)(args, rank, world, dist_on, device)
+        extra = {}
+        if combined:
+            for cfg in EXTRA_CONFIGS:
+                sub = run_ours(args, rank, world, dist_on, device, cfg=cfg)
+                extra[sub["config"]["workload"]] = sub
+                torch.cuda.empty_cache()
+                if cfg == 3:  # the normalised workload once more, with the feature map in the kernel
+                    sub = run_ours(args, rank, world, dist_on, device, cfg=cfg, prologue=True)
+                    extra[sub["config"]["workload"]] = sub
+                    torch.cuda.empty_cache()
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
                 line["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4) if args.config == 6 else
                                         cpu_baseline_ema(W.EMA, reverse=args.direction == "reverse")
                                         if args.config == 7 else
                                         cpu_baseline(args.config, direction=args.direction))
+                for sub in extra.values():
+                    cfg = next(c for c, w in W.WORKLOADS.items() if sub["config"]["workload"].startswith(w.name))
+                    sub["cpu_baseline"] = cpu_baseline(cfg, budget_s=8.0)
+            if extra:
+                line["configs"] = {name: {k: v for k, v in sub.items()
+                                          if k not in ("metric", "higher_is_better", "scaling", "data", "unit")}
+                                   for name, sub in extra.items()}
             print(json.dumps(line), flush=True)
     finally:
         if dist_on:

@@ -55,3 +55,30 @@ def test_single_process_needs_no_collective():
     assert bench.max_over_ranks(3.25, False, torch.device("cpu")) == 3.25
     import workloads as W
     assert bench.rank_seed(W.RETENTION, 0) == W.RETENTION.seed
+
+
+def test_bench_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` outside torchrun launches two ranks (gloo standing
+    in for NCCL in the timing self-test); rank 0 reports n_gpus = 2 and the
+    slowest rank's time."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--cpu-selftest"],
+                       capture_output=True, text=True, timeout=240, env=dict(os.environ, OMP_NUM_THREADS="1"))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and len(line["per_rank_ms"]) == 2
+    assert line["ms_per_step"] == max(line["per_rank_ms"])
+    assert line["per_rank_ms"][1] > line["per_rank_ms"][0]  # rank 1 works twice as long
+
+
+def test_bench_refuses_a_rank_count_that_disagrees_with_gpus():
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--cpu-selftest"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0 and "ranks were launched" in r.stderr
