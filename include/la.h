@@ -152,9 +152,9 @@ typedef struct {
  * bf16 runs on tcgen05 tensor cores with fp32 accumulation (chunks of 128
  * tokens); fp32 runs a recurrent kernel on fp32 FMA units (no TF32).  The
  * bf16 kernels exist for key widths 16, 32, 64 and 128 and value slices of
- * 16, 32, 64 or 128 columns; other widths run on the next larger key width,
- * the tile columns past Dk read as zeros (the TMA loads' fill), and on value
- * slices of which the last may reach past Dv (nothing is stored there).
+ * 16, 32, 64 or 128 columns; other key widths run on the next larger one,
+ * the tile columns past Dk read as zeros (the TMA loads' fill), and the
+ * value columns run in slices of a width that divides Dv.
  */
 LA_API la_status la_chunk_forward(const void* q, const void* k, const void* v,
                            const la_decay* decay, int normalize,

@@ -56,6 +56,14 @@ int padded_width(int d) { return d <= 16 ? 16 : d <= 32 ? 32 : d <= 64 ? 64 : 12
 // Tensor widths the tensor-core path takes.
 bool tensor_width_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 
+// The widest value slice that divides Dv (a multiple of 16): halving it
+// keeps it a divisor, so no slice ever runs past Dv.
+int widest_slice(int Dv) {
+    for (int w : {128, 64, 32})
+        if (Dv % w == 0) return w;
+    return 16;
+}
+
 CUtensorMapSwizzle swizzle_for(int row_bytes) {
     return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                             : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -106,8 +114,9 @@ int env_int(const char* name) {
 
 // How the (b, h) sequences are spread over CTAs (one CTA per SM).
 //  split: CTAs sharing one (b, h, segment), each owning nv value columns
-//         (split = ceil(Dv / nv); the last slice may run past Dv) and
-//         recomputing the 128 x 128 score tile;
+//         (a slice width that divides Dv: Dv is a multiple of 16, and the
+//         slices are 16, 32, 64 or 128 wide) and recomputing the 128 x 128
+//         score tile;
 //  nseg:  output segments per (b, h), of seg_chunks chunks each; segment i
 //         starts from the state after segment i - 1, assembled from per_seg
 //         state segments per earlier output segment (computed by a state
@@ -130,12 +139,12 @@ Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments
     const int sms = sm_count();
     const long long target = sms * 4 / 5;
     const int DK = padded_width(Dk);
-    int nv = padded_width(Dv);
+    int nv = widest_slice(Dv);
     while (!instance_ok(DK, nv, norm) && nv / 2 >= 16) nv /= 2;
     const int es = env_int("LA_DV_SPLIT");
     const bool fixed_split = es >= 1 && Dv % es == 0 && width_ok(Dv / es) && instance_ok(DK, Dv / es, norm);
     if (fixed_split) nv = Dv / es;
-    int s = (Dv + nv - 1) / nv;
+    int s = Dv / nv;
     int nseg = 1;
     if (segments && nchunks >= 2) {
         const int eg = env_int("LA_SEGMENTS");
@@ -149,7 +158,7 @@ Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments
     if (!fixed_split)
         while (static_cast<long long>(BH) * s * nseg < target && nv / 2 >= 16) {
             nv /= 2;
-            s = (Dv + nv - 1) / nv;
+            s = Dv / nv;
         }
     Layout L{};
     L.split = s;
@@ -234,9 +243,9 @@ struct StatePlan {
 StatePlan plan_state(int BH, int nchunks, int Dk, int Dv, bool norm) {
     const int sms = sm_count();
     StatePlan P{};
-    int nv = padded_width(Dv);
+    int nv = widest_slice(Dv);
     while (!instance_ok(padded_width(Dk), nv, norm) && nv / 2 >= 16) nv /= 2;
-    const int s = (Dv + nv - 1) / nv;
+    const int s = Dv / nv;
     P.nv = nv;
     int pieces = 1;
     while (pieces * 2 <= nchunks && static_cast<long long>(BH) * s * pieces * 2 <= sms) pieces *= 2;

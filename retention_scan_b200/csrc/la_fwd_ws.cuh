@@ -212,8 +212,8 @@ struct Params {
     float* final_z;
     // Dk and Dv are the tensors' widths.  The instance's key width DK is the
     // smallest one >= Dk: the key and query tiles' columns past Dk are the
-    // TMA's zero fill, and so are the value columns past Dv in the last value
-    // slice; rows of S past Dk and columns past Dv are neither read nor written.
+    // TMA's zero fill, and the rows of S past Dk are neither read nor written
+    // in global memory.  The value slices divide Dv exactly.
     int H, T, Dk, Dv, split, nchunks;
     int* err;
     // T-segments: each (b, h, slice) is cut into nseg segments of seg_chunks
@@ -979,9 +979,8 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         const int rem = min(C, T - mem_chunk(c) * C);
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst = out_row(c);
-        const int npiece = min(NV, p.Dv - x.j0) / 16;  // the last slice may run past Dv
 #pragma unroll 1
-        for (int piece = 0; piece < npiece; ++piece) {
+        for (int piece = 0; piece < NV / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + 16 * piece, o);
             tmem_wait_ld();
@@ -1041,11 +1040,11 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
     const int wq = warp & 3;
     const int d = 32 * wq + lane;          // key row of S; also token row t of O
     const bool warp_rows = 32 * wq < DK;   // this warp holds rows of S (past Dk they stay zero)
-    const bool row_ok = d < p.Dk;
+    // rows of S past Dk (a padded key width) are never read or written in
+    // global memory; evaluated at each use (a long-lived predicate here costs
+    // registers in the chunk loop)
+    auto row_ok = [&]() { return d < p.Dk; };
     const int cb = wg * G::NVW;            // first column (within the slice) of this warpgroup
-    // columns of this warpgroup inside the tensor (a multiple of 16: the last
-    // value slice may run past Dv)
-    const int ncols = min(G::NVW, max(0, p.Dv - (x.j0 + cb)));
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * wq) << 16);
     const int bh = x.bh, j0 = x.j0;
     float S[G::NVW];
@@ -1053,11 +1052,10 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
 #pragma unroll
     for (int j = 0; j < G::NVW; ++j) S[j] = 0.f;
     float ltot = 0.f;  // state pass: total log2 decay of the segment
-    if (row_ok && p.init_state && !p.state_pass) {
+    if (row_ok() && p.init_state && !p.state_pass) {
         const float* src = p.init_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
         for (int j = 0; j < G::NVW; j += 4) {
-            if (j >= ncols) break;
             const float4 v4 = *reinterpret_cast<const float4*>(src + j);
             S[j] = v4.x;
             S[j + 1] = v4.y;
@@ -1065,8 +1063,8 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             S[j + 3] = v4.w;
         }
     }
-    if (NORM && row_ok && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * p.Dk + d];
-    if (row_ok && !p.state_pass && x.seg > 0) {
+    if (NORM && row_ok() && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * p.Dk + d];
+    if (row_ok() && !p.state_pass && x.seg > 0) {
         // state entering this segment: fold in every earlier state segment j,
         // S <- 2^(L_j) S + S_j (the combination of two consecutive spans)
         for (int j = 0; j < x.seg * p.ws_per_seg; ++j) {
@@ -1075,7 +1073,6 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             const float* src = p.ws_S + (sj * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
             for (int i = 0; i < G::NVW; i += 4) {
-                if (i >= ncols) break;
                 const float4 v4 = *reinterpret_cast<const float4*>(src + i);
                 S[i] = fmaf(e, S[i], v4.x);
                 S[i + 1] = fmaf(e, S[i + 1], v4.y);
@@ -1178,7 +1175,7 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
         __nv_bfloat16* dst = out_row(c);
 #pragma unroll 1
-        for (int piece = 0; piece < ncols / 16; ++piece) {
+        for (int piece = 0; piece < G::NVW / 16; ++piece) {
             float o[16];
             tmem_ld16(oa + cb + 16 * piece, o);
             tmem_wait_ld();
@@ -1194,11 +1191,11 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         for (int c = 0; c < n && ok; ++c) ok = state(c);
         if (ok && !*abort) {
             const size_t sj = static_cast<size_t>(bh) * p.ws_nS + x.seg;
-            if (row_ok) {
+            if (row_ok()) {
                 float* dst = p.ws_S + (sj * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
                 for (int j = 0; j < G::NVW; j += 4)
-                    if (j < ncols) *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
                 if (NORM && x.slice == 0 && wg == 0) p.ws_z[sj * p.Dk + d] = z;
             }
             if (x.slice == 0 && wg == 0 && d == 0) p.ws_L[sj] = ltot;
@@ -1223,12 +1220,12 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
             if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
         }
     }
-    if (ok && !*abort && row_ok && x.seg == p.nseg - 1) {
+    if (ok && !*abort && row_ok() && x.seg == p.nseg - 1) {
         if (p.final_state) {
             float* fs = p.final_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
             for (int j = 0; j < G::NVW; j += 4)
-                if (j < ncols) *reinterpret_cast<float4*>(fs + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                *reinterpret_cast<float4*>(fs + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
         if (NORM && p.final_z && x.slice == 0 && wg == 0) p.final_z[static_cast<size_t>(bh) * p.Dk + d] = z;
     }
