@@ -40,15 +40,17 @@
 //
 // Roles (one CTA = one (b, h) and NV of its Dv columns; Dv / NV CTAs share a
 // head and read its q, k through L2):
-//   warp 0       TMA producer of the Q ring
-//   warp 1       MMA issuer (one elected lane) and TMEM owner
+//   warp 0       MMA issuer B (one elected lane): Q S and P V (a ready P V
+//                first: it completes a chunk, and so frees its O buffer)
+//   warp 1       MMA issuer A (one elected lane): Q K^T and K^T V'; TMEM owner
 //   warps 2-9    two warpgroups: prep (decay prefix, value-row scaling,
 //                normaliser weights) and mask (scores -> P in TMEM); warpgroup
 //                0 owns score columns 0-63, warpgroup 1 columns 64-127 and
-//                writes the outputs (epilogue)
+//                writes the outputs (epilogue); with the feature map, the
+//                warpgroups map the Q and K tiles
 //   warps 10-..  state: fp32 S in registers and its bf16 copy (one warpgroup
 //                per 64 value columns)
-//   last warp    TMA producer of the K and V rings
+//   last warp    TMA producer of the Q, K and V rings
 // Every hand-off is an mbarrier; every wait gives up after kWaitLimitNs (then
 // the CTA sets the device error word and unwinds).
 #pragma once
@@ -64,6 +66,7 @@ namespace ws {
 
 constexpr int C = 128;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr unsigned kTmaIdleSleepNs = 64;  // the producer's pause after a pass that issued nothing
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kFoldLimit = 64.f;
 constexpr int kSmemLimit = 232448;
@@ -94,8 +97,9 @@ enum Bar : int {
     B_SBFULL = 44,   // [2] bf16 state copy written
     B_SBEMPTY = 46,  // [2] Q S done reading it
     B_PHI = 48,      // [4] feature map applied to the chunk's Q and K tiles
-    B_DRAIN = 52,
-    B_COUNT = 53
+    B_DRAIN = 52,    // MMA warp A's issued MMAs complete
+    B_DRAINB = 53,   // MMA warp B's
+    B_COUNT = 54
 };
 
 template <int DK, int NV, bool NORM>
@@ -178,7 +182,7 @@ struct Plan {
     // warps
     static constexpr int NSW = NV > 64 ? 2 : 1;
     static constexpr int NVW = NV / NSW;
-    static constexpr int W_TMA = 0, W_MMA = 1, W_PM = 2, W_ES = 10;
+    static constexpr int W_MMAB = 0, W_MMA = 1, W_PM = 2, W_ES = 10;
     static constexpr int W_TMAV = W_ES + 4 * NSW;
     static constexpr int NWARPS = W_TMAV + 1;
     static constexpr int THREADS = 32 * NWARPS;
@@ -186,7 +190,6 @@ struct Plan {
     static constexpr uint32_t Q_TX = Q_BYTES;
     static constexpr uint32_t V_TX = V_BYTES;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, 0, 0);
-    static constexpr bool EPI_MASK = NORM;  // outputs written by mask warpgroup 1 (else by the state warps)
     static constexpr int NOUT = NV + (NORM ? 16 : 0);  // value columns plus the normaliser panel
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, NOUT, 0, 1);
     static constexpr uint32_t IDESC_KV = make_idesc_bf16(128, NOUT, 1, 1);
@@ -232,7 +235,7 @@ struct Params {
     // takes the direction from its REV template argument (the forward
     // instances carry no reverse-scan code); this field selects the instance.
     int reverse;
-    int accumulate;      // reverse instances only: add y to the values already in out (fp32 add)
+    int accumulate;      // reverse or 16-wide key instances: add y to the values in out (fp32 add)
     float q_scale;       // the output of an unnormalised scan is linear in q: y *= q_scale
                          // (the normalised output does not depend on the scale of q)
     int feature_map;     // LA_FEATURE_ELU1: the prep warps replace each landed Q and K tile
@@ -434,7 +437,7 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
         return REV ? p.nchunks - 1 - (x.c0 + c) : x.c0 + c;                                          \
     };                                                                                               \
     (void)mem_chunk;                                                                                 \
-    const bool accumulate = REV && p.accumulate != 0; /* only the reverse scan accumulates */        \
+    const bool accumulate = (REV || DK == 16) && p.accumulate != 0; /* reverse, or 16-wide keys */   \
     (void)accumulate;                                                                                \
     (void)sa;                                                                                        \
     (void)tmem;                                                                                      \
@@ -442,39 +445,30 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
     (void)T;                                                                                         \
     (void)lane;
 
-// ------------------------------------------------------------ TMA producers
-// Q ring: one thread, blocking on each stage in turn.
+// ------------------------------------------------------------ TMA producer
+// Q, K and V rings: one thread polls all three, so that none waits behind
+// another's free stage (the state pass reads no queries).  K and V run as
+// far ahead as their rings allow: the prep of chunk c + 1 (which needs V)
+// runs before the mask of chunk c.
 template <int DK, int NV, bool NORM, bool REV>
-__device__ __noinline__ void role_tma_q(const Ctx x, const CUtensorMap* tmq) {
-    LA_ROLE_PRELUDE
-    if (lane != 0 || p.state_pass) return;  // the state pass reads no queries
-    int issued = 0;
-    for (int c = 0; c < n; ++c) {
-        const int s = c % G::NQ;
-        if (c >= G::NQ && !wait1(&bar[B_QEMPTY + s], ((c / G::NQ) - 1) & 1, abort, p, kErrTmaWait)) break;
-        mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
-        uint8_t* st = sm + s * G::Q_STAGE;
-        for (int pp = 0; pp < G::PK; ++pp)
-            tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * (G::WK / 2), mem_chunk(c) * C, x.bh);
-        ++issued;
-    }
-    if (*abort) {  // let issued copies land before the CTA's shared memory goes away
-        for (int c = issued > G::NQ ? issued - G::NQ : 0; c < issued; ++c)
-            mbar_wait_bounded(&bar[B_QFULL + c % G::NQ], (c / G::NQ) & 1, kWaitLimitNs);
-    }
-}
-
-// K and V rings: one thread polls both, so that neither waits behind the
-// other's free stage.  V runs as far ahead as its ring allows: the prep of
-// chunk c + 1 (which needs V) runs before the mask of chunk c.
-template <int DK, int NV, bool NORM, bool REV>
-__device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, const CUtensorMap* tmv) {
+__device__ __noinline__ void role_tma(const Ctx x, const CUtensorMap* tmq, const CUtensorMap* tmk,
+                                      const CUtensorMap* tmv) {
     LA_ROLE_PRELUDE
     if (lane != 0) return;
-    int ck = 0, cv = 0;
+    const int nq = p.state_pass ? 0 : n;
+    int cq = 0, ck = 0, cv = 0;
     uint64_t last = global_timer_ns();
-    while (ck < n || cv < n) {
+    while (cq < nq || ck < n || cv < n) {
         bool moved = false;
+        if (cq < nq && (cq < G::NQ || mbar_test(&bar[B_QEMPTY + cq % G::NQ], ((cq / G::NQ) - 1) & 1))) {
+            const int s = cq % G::NQ;
+            mbar_arrive_expect_tx(&bar[B_QFULL + s], G::Q_TX);
+            uint8_t* st = sm + s * G::Q_STAGE;
+            for (int pp = 0; pp < G::PK; ++pp)
+                tma_load_3d(st + pp * C * G::WK, tmq, &bar[B_QFULL + s], pp * (G::WK / 2), mem_chunk(cq) * C, x.bh);
+            ++cq;
+            moved = true;
+        }
         if (ck < n &&
             (ck < G::NK || mbar_test(&bar[B_KEMPTY + ck % G::NK], ((ck / G::NK) - 1) & 1))) {
             const int s = ck % G::NK;
@@ -504,10 +498,12 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
                 fail(p, abort, kErrTmaWait);
                 break;
             }
-            __nanosleep(128);
+            __nanosleep(kTmaIdleSleepNs);
         }
     }
-    if (*abort) {
+    if (*abort) {  // let issued copies land before the CTA's shared memory goes away
+        for (int c = cq > G::NQ ? cq - G::NQ : 0; c < cq; ++c)
+            mbar_wait_bounded(&bar[B_QFULL + c % G::NQ], (c / G::NQ) & 1, kWaitLimitNs);
         for (int c = ck > G::NK ? ck - G::NK : 0; c < ck; ++c)
             mbar_wait_bounded(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, kWaitLimitNs);
         for (int c = cv > G::NVS ? cv - G::NVS : 0; c < cv; ++c)
@@ -515,19 +511,26 @@ __device__ __noinline__ void role_tma_kv(const Ctx x, const CUtensorMap* tmk, co
     }
 }
 
-// ------------------------------------------------------------ MMA issuer
-// Four in-order queues, each issued as soon as its inputs are there:
-//   Q K^T (c)   Q and K tiles of c landed, its score buffer free
-//   K^T V' (j)  after Q K^T (j) and the prep of j; a direct-form chunk also
-//               after its mask, which decays Q and K; K^T V' buffer free;
-//               releases the K stage
-//   Q S (j)     after K^T V' (j); O buffer free; bf16 state after j - 1
-//               written; releases the Q stage
-//   P V (j)     after Q S (j), which opened the accumulator; P (j) written
-// The warp polls the barriers (never blocking on one while another queue
-// could move) and gives up after kWaitLimitNs without progress.
-// State pass: only K^T V' (and K^T W), in order; each also releases its K and
-// V stages.
+// ------------------------------------------------------------ MMA issuers
+// Two warps issue the MMAs, one elected lane each, so that neither queue
+// waits behind the other's blocked issue:
+//   warp A (W_MMA):  Q K^T (c)  Q and K tiles of c landed (and mapped), its
+//                               score buffer free
+//                    K^T V' (c) after Q K^T (c) and the prep of c; a
+//                               direct-form chunk also after its mask, which
+//                               decays Q and K; K^T V' buffer free;
+//                               releases the K stage
+//   warp B (W_MMAB): Q S (c)    Q tile of c landed (and mapped); the prep of
+//                               c done, and the mask too for a direct-form
+//                               chunk (it decays the Q tile); O buffer free;
+//                               bf16 state after c - 1 written
+//                    P V (c)    after Q S (c), which opened the accumulator;
+//                               P (c) written
+// A Q stage is free once Q K^T (warp A) and Q S (warp B) of its chunk have
+// run: two commits.  Each warp polls its barriers (a snapshot per pass) and
+// gives up after kWaitLimitNs without progress.
+// State pass: warp A issues K^T V' (and K^T W) in order; each also releases
+// its K and V stages.
 template <int DK, int NV, bool NORM, bool REV>
 __device__ __noinline__ void mma_state_pass(const Ctx x) {
     LA_ROLE_PRELUDE
@@ -558,29 +561,39 @@ __device__ __noinline__ void mma_state_pass(const Ctx x) {
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
 }
 
+// One pass without progress: give up after kWaitLimitNs (or on abort);
+// returns false when the issuer should stop.
+__device__ __forceinline__ bool idle_pass(bool moved, uint64_t& idle_since, volatile int* abort, const Params& p) {
+    if (moved) {
+        idle_since = 0;
+        return true;
+    }
+    const uint64_t now = global_timer_ns();
+    if (idle_since == 0) idle_since = now;
+    bool give_up = *abort != 0;
+    if (!give_up && now - idle_since > kWaitLimitNs) {
+        give_up = true;
+        if ((threadIdx.x & 31) == 0) fail(p, abort, kErrMmaWait);
+    }
+    if (__any_sync(0xffffffffu, give_up)) return false;
+    __nanosleep(64);
+    return true;
+}
+
 template <int DK, int NV, bool NORM, bool REV, bool PHI>
-__device__ __noinline__ void role_mma(const Ctx x) {
+__device__ __noinline__ void role_mma_a(const Ctx x) {
     LA_ROLE_PRELUDE
     if (p.state_pass) {
         mma_state_pass<DK, NV, NORM, REV>(x);
         return;
     }
     const bool leader = elect_one();
+    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
     auto mode_of = [&](int j) {
         return *reinterpret_cast<volatile int*>(sm + G::OFF_V + (j % G::NVS) * G::V_STAGE + G::VS_META + 4);
     };
-    auto q_addr = [&](int j) { return sa + (j % G::NQ) * G::Q_STAGE; };
-    auto k_addr = [&](int j) { return sa + G::OFF_K + (j % G::NK) * G::Q_STAGE; };
-    auto v_addr = [&](int j) { return sa + G::OFF_V + (j % G::NVS) * G::V_STAGE; };
-    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
-
-    int m1 = 0, kv = 0, qs = 0, pv = 0, pseen = 0;  // next chunk of each queue; P (j) seen for j < pseen
-    // One snapshot per pass of every barrier a queue head may wait on: the
-    // issuing lane runs the tests back to back (their latencies overlap; no
-    // test waits for another's answer) and broadcasts the bits to the warp.
-    enum : uint32_t { kP = 1, kQ = 2, kK = 4, kA = 8, kPrep = 16, kDir = 32, kDse = 64, kOe = 128, kSb = 256,
-                      kPhi = 512 };
-    constexpr bool phi = PHI;  // Q K^T (c) also awaits the feature map of c
+    int m1 = 0, kv = 0, pseen = 0;  // next Q K^T, next K^T V'; P (j) seen for j < pseen
+    enum : uint32_t { kP = 1, kQ = 2, kK = 4, kA = 8, kPrep = 16, kDir = 32, kDse = 64, kPhi = 128 };
     auto snapshot = [&]() -> uint32_t {
         uint32_t b = 0;
         if (leader) {
@@ -588,144 +601,144 @@ __device__ __noinline__ void role_mma(const Ctx x) {
             b |= mbar_test(&bar[B_QFULL + m1 % G::NQ], (m1 / G::NQ) & 1) ? kQ : 0u;
             b |= mbar_test(&bar[B_KFULL + m1 % G::NK], (m1 / G::NK) & 1) ? kK : 0u;
             b |= (m1 < G::NA || mbar_test(&bar[B_AEMPTY + m1 % G::NA], ((m1 / G::NA) - 1) & 1)) ? kA : 0u;
+            if (PHI) b |= mbar_test(&bar[B_PHI + m1 % 4], (m1 / 4) & 1) ? kPhi : 0u;
             b |= mbar_test(&bar[B_PREP + kv % G::NVS], (kv / G::NVS) & 1) ? kPrep : 0u;
-            // the feature map of chunk m1 (its slot is unambiguous: the map of
-            // m1 - 4 preceded the issued Q K^T (m1 - 4))
-            if (phi) b |= mbar_test(&bar[B_PHI + m1 % 4], (m1 / 4) & 1) ? kPhi : 0u;
             b |= (kv < G::NDS || mbar_test(&bar[B_DSEMPTY + kv % G::NDS], ((kv / G::NDS) - 1) & 1)) ? kDse : 0u;
-            b |= (qs < G::NO || mbar_test(&bar[B_OEMPTY + qs % G::NO], ((qs / G::NO) - 1) & 1)) ? kOe : 0u;
-            b |= mbar_test(&bar[B_SBFULL + qs % G::NSB], (qs / G::NSB) & 1) ? kSb : 0u;
             if ((b & kPrep) && mode_of(kv) == kModeDirect) b |= kDir;  // the mode is valid once prep is done
         }
         return __shfl_sync(0xffffffffu, b, leader_lane);
     };
-    uint64_t idle_since = 0;  // start of the current run of passes without progress
-    while (pv < n) {
+    uint64_t idle_since = 0;
+    while (kv < n) {
         bool moved = false;
         const uint32_t bits = snapshot();
         if (pseen < m1 && (bits & kP)) {
             ++pseen;
             moved = true;
         }
-        // Q K^T of chunk m1
-        auto issue_qk = [&]() {
-            const bool phi_done = !phi || (bits & kPhi) != 0;
-            if (m1 < n && (bits & kQ) && (bits & kK) && (bits & kA) && phi_done) {
-                tc_fence_after_sync();
-                const uint64_t dq = make_smem_desc(q_addr(m1), 16, 8 * G::WK, G::WK);
-                const uint64_t dk = make_smem_desc(k_addr(m1), 16, 8 * G::WK, G::WK);
-                if (leader) {
+        const bool kv_ok = kv < m1 && (bits & kPrep) && (!(bits & kDir) || kv < pseen) && (bits & kDse);
+        const bool qk_ok = m1 < n && (bits & kQ) && (bits & kK) && (bits & kA) && (!PHI || (bits & kPhi));
+        if (qk_ok) {
+            tc_fence_after_sync();
+            const uint64_t dq = make_smem_desc(sa + (m1 % G::NQ) * G::Q_STAGE, 16, 8 * G::WK, G::WK);
+            const uint64_t dk = make_smem_desc(sa + G::OFF_K + (m1 % G::NK) * G::Q_STAGE, 16, 8 * G::WK, G::WK);
+            if (leader) {
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16(tmem + 128 * (m1 % G::NA), dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4),
-                                  G::IDESC_QK, kk > 0);
-                    umma_commit(&bar[B_AFULL + m1 % G::NA]);
-                }
-                __syncwarp();
-                ++m1;
-                moved = true;
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16(tmem + 128 * (m1 % G::NA), dq + (kstep(kk, G::WK) >> 4), dk + (kstep(kk, G::WK) >> 4),
+                              G::IDESC_QK, kk > 0);
+                umma_commit(&bar[B_AFULL + m1 % G::NA]);
+                umma_commit(&bar[B_QEMPTY + m1 % G::NQ]);  // one of the Q stage's two releases
             }
-        };
-        // K^T V' of chunk kv
-        auto issue_kv = [&]() {
-            if (kv < m1 && (bits & kPrep) && (!(bits & kDir) || kv < pseen) && (bits & kDse)) {
-                // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
-                // repeats the key panel when Dk < 128
-                tc_fence_after_sync();
-                const int b = kv % G::NDS;
-                const uint64_t dk = make_smem_desc(k_addr(kv), DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
-                const uint64_t dv = make_smem_desc(v_addr(kv), C * G::WV, 8 * G::WV, G::WV);
-                const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
-                if (leader) {
+            __syncwarp();
+            ++m1;
+            moved = true;
+        } else if (kv_ok) {
+            // DS = K^T V' (and K^T W); M = 128 key rows, a zero panel offset
+            // repeats the key panel when Dk < 128
+            tc_fence_after_sync();
+            const int b = kv % G::NDS;
+            const uint64_t dk =
+                make_smem_desc(sa + G::OFF_K + (kv % G::NK) * G::Q_STAGE, DK == 128 ? C * G::WK : 0, 8 * G::WK, G::WK);
+            const uint64_t dv = make_smem_desc(sa + G::OFF_V + (kv % G::NVS) * G::V_STAGE, C * G::WV, 8 * G::WV, G::WV);
+            const uint32_t d = tmem + G::COL_DS0 + b * G::OCOLS;
+            if (leader) {
 #pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
-                    umma_commit(&bar[B_DSFULL + b]);
-                    umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
-                }
-                __syncwarp();
-                ++kv;
-                moved = true;
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(d, dk + ((kk * 16 * G::WK) >> 4), dv + ((kk * 16 * G::WV) >> 4), G::IDESC_KV, kk > 0);
+                umma_commit(&bar[B_DSFULL + b]);
+                umma_commit(&bar[B_KEMPTY + kv % G::NK]);  // Q K^T and K^T V' of this chunk have run
             }
-        };
-        // Q S of chunk qs
-        auto issue_qs = [&]() {
-            if (qs < kv && (bits & kOe) && (bits & kSb)) {
-                // O = Q S (and den = Q z), opening the accumulator of chunk qs
-                tc_fence_after_sync();
-                const int ro = qs % G::NO, sbb = qs % G::NSB;
-                const uint64_t dq = make_smem_desc(q_addr(qs), 16, 8 * G::WK, G::WK);
-                // B = [S | z] panels of the bf16 state copy
-                const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
-                const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
-                    umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // Q K^T and Q S of this chunk have run
-                    umma_commit(&bar[B_SBEMPTY + sbb]);
-                }
-                __syncwarp();
-                ++qs;
-                moved = true;
-            }
-        };
-        // P V of chunk pv
-        auto issue_pv = [&]() {
-            if (pv < qs && pv < pseen) {
-                // P V (and P W) accumulate into the O that Q S opened
-                tc_fence_after_sync();
-                const int pb = pv % G::NPB, ro = pv % G::NO;
-                const uint64_t dv = make_smem_desc(v_addr(pv), C * G::WV, 8 * G::WV, G::WV);
-                const uint32_t pa = tmem + G::COL_P0 + 64 * pb;
-                const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
-                    umma_commit(&bar[B_OFULL + ro]);
-                    umma_commit(&bar[B_PEMPTY + pb]);
-                    umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
-                }
-                __syncwarp();
-                ++pv;
-                moved = true;
-            }
-        };
-        // Order within a pass: the newest chunks' Q K^T and K^T V' first for
-        // Dk = 128.  With Dk <= 64 the chunk period is set by the Q ring (a
-        // stage is held until the chunk's Q S) and the issuing thread waits
-        // behind the MMAs already queued, so Q S and P V of the older chunks
-        // go first (measured: 3% faster at Dk = 64, slower at Dk = 128).
-        if constexpr (DK <= 64) {
-            issue_qs();
-            issue_pv();
-            issue_qk();
-            issue_kv();
-        } else {
-            issue_qk();
-            issue_kv();
-            issue_qs();
-            issue_pv();
+            __syncwarp();
+            ++kv;
+            moved = true;
         }
-        if (moved) {
-            idle_since = 0;
-        } else {
-            const uint64_t now = global_timer_ns();
-            if (idle_since == 0) idle_since = now;
-            bool give_up = *abort != 0;
-            if (!give_up && now - idle_since > kWaitLimitNs) {
-                give_up = true;
-                if (lane == 0) fail(p, abort, kErrMmaWait);
-            }
-            if (__any_sync(0xffffffffu, give_up)) break;
-            __nanosleep(64);
-        }
+        if (!idle_pass(moved, idle_since, abort, p)) break;
     }
     // everything issued has completed before TMEM is released
     if (leader) umma_commit(&bar[B_DRAIN]);
     __syncwarp();
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
+}
+
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
+__device__ __noinline__ void role_mma_b(const Ctx x) {
+    LA_ROLE_PRELUDE
+    if (p.state_pass) return;  // no queries, no outputs
+    const bool leader = elect_one();
+    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+    auto mode_of = [&](int j) {
+        return *reinterpret_cast<volatile int*>(sm + G::OFF_V + (j % G::NVS) * G::V_STAGE + G::VS_META + 4);
+    };
+    int qs = 0, pv = 0, pseen = 0;  // next Q S, next P V; P (j) seen for j < pseen
+    enum : uint32_t { kP = 1, kQ = 2, kPhi = 4, kPrep = 8, kDir = 16, kOe = 32, kSb = 64 };
+    auto snapshot = [&]() -> uint32_t {
+        uint32_t b = 0;
+        if (leader) {
+            b |= mbar_test(&bar[B_PFULL + pseen % G::NPB], (pseen / G::NPB) & 1) ? kP : 0u;
+            b |= mbar_test(&bar[B_QFULL + qs % G::NQ], (qs / G::NQ) & 1) ? kQ : 0u;
+            if (PHI) b |= mbar_test(&bar[B_PHI + qs % 4], (qs / 4) & 1) ? kPhi : 0u;
+            b |= mbar_test(&bar[B_PREP + qs % G::NVS], (qs / G::NVS) & 1) ? kPrep : 0u;
+            b |= (qs < G::NO || mbar_test(&bar[B_OEMPTY + qs % G::NO], ((qs / G::NO) - 1) & 1)) ? kOe : 0u;
+            b |= mbar_test(&bar[B_SBFULL + qs % G::NSB], (qs / G::NSB) & 1) ? kSb : 0u;
+            if ((b & kPrep) && mode_of(qs) == kModeDirect) b |= kDir;
+        }
+        return __shfl_sync(0xffffffffu, b, leader_lane);
+    };
+    uint64_t idle_since = 0;
+    while (pv < n) {
+        bool moved = false;
+        const uint32_t bits = snapshot();
+        // masks are in order, so P (pseen) is tested only after P (pseen - 1)
+        if (pseen < n && (bits & kP)) {
+            ++pseen;
+            moved = true;
+        }
+        const bool pv_ok = pv < qs && pv < pseen;
+        const bool qs_ok = qs < n && (bits & kQ) && (!PHI || (bits & kPhi)) && (bits & kPrep) &&
+                           (!(bits & kDir) || qs < pseen) && (bits & kOe) && (bits & kSb);
+        if (pv_ok) {
+            // P V (and P W) accumulate into the O that Q S opened
+            tc_fence_after_sync();
+            const int pb = pv % G::NPB, ro = pv % G::NO;
+            const uint64_t dv = make_smem_desc(sa + G::OFF_V + (pv % G::NVS) * G::V_STAGE, C * G::WV, 8 * G::WV, G::WV);
+            const uint32_t pa = tmem + G::COL_P0 + 64 * pb;
+            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16_ts(d, pa + 8 * kk, dv + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, 1);
+                umma_commit(&bar[B_OFULL + ro]);
+                umma_commit(&bar[B_PEMPTY + pb]);
+                umma_commit(&bar[B_VEMPTY + pv % G::NVS]);
+            }
+            __syncwarp();
+            ++pv;
+            moved = true;
+        } else if (qs_ok) {
+            // O = Q S (and den = Q z), opening the accumulator of chunk qs
+            tc_fence_after_sync();
+            const int ro = qs % G::NO, sbb = qs % G::NSB;
+            const uint64_t dq = make_smem_desc(sa + (qs % G::NQ) * G::Q_STAGE, 16, 8 * G::WK, G::WK);
+            // B = [S | z] panels of the bf16 state copy
+            const uint64_t dsb = make_smem_desc(sa + G::OFF_SB + sbb * G::SB_BYTES, DK * G::WV, 8 * G::WV, G::WV);
+            const uint32_t d = tmem + G::COL_O0 + ro * G::OCOLS;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16(d, dq + (kstep(kk, G::WK) >> 4), dsb + ((kk * 16 * G::WV) >> 4), G::IDESC_PV, kk > 0);
+                umma_commit(&bar[B_QEMPTY + qs % G::NQ]);  // the Q stage's other release
+                umma_commit(&bar[B_SBEMPTY + sbb]);
+            }
+            __syncwarp();
+            ++qs;
+            moved = true;
+        }
+        if (!idle_pass(moved, idle_since, abort, p)) break;
+    }
+    if (leader) umma_commit(&bar[B_DRAINB]);
+    __syncwarp();
+    mbar_wait_bounded(&bar[B_DRAINB], 0, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------ prep + mask
@@ -1025,7 +1038,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         if (c + 1 < n && !prep(c + 1)) break;
         if (c >= 0 && c < n && !pmask(c)) break;
         if (map && c + 1 < n && !phi(c + 1)) break;
-        if (G::EPI_MASK && wg == 1 && c >= 1 && !epilogue(c - 1)) break;
+        if (wg == 1 && c >= 1 && !epilogue(c - 1)) break;
     }
 }
 
@@ -1034,7 +1047,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
 // chunk c: the state update of chunk c, then its bf16 copy, which the next
 // chunk's Q S reads.
 template <int DK, int NV, bool NORM, bool REV>
-__device__ __noinline__ void role_state_epilogue(const Ctx x) {
+__device__ __noinline__ void role_state(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_ES) / 4;
     const int wq = warp & 3;
@@ -1148,43 +1161,6 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
         return true;
     };
 
-    // Epilogue (unnormalised instances): y = O times the row factor 2^(L_t)
-    // for this warpgroup's columns.
-    auto out_row = [&](int c) {
-        return p.out + (static_cast<size_t>(bh) * T + static_cast<size_t>(mem_chunk(c)) * C + d) * p.Dv + j0 + cb;
-    };
-    auto epilogue = [&](int c) -> bool {
-        const int ro = c % G::NO, t = d;
-        if (accumulate) {  // the rows this epilogue and the next read back
-            if (c == 0 && t < min(C, T - mem_chunk(0) * C)) prefetch_row_l2(out_row(0), G::NVW);
-            if (c + 1 < n && t < min(C, T - mem_chunk(c + 1) * C)) prefetch_row_l2(out_row(c + 1), G::NVW);
-        }
-        if (!waitw(&bar[B_OFULL + ro], (c / G::NO) & 1, abort, p, kErrMmaWait)) return false;
-        tc_fence_after_sync();
-        const uint32_t oa = lane_addr + G::COL_O0 + ro * G::OCOLS;
-        float inv;  // y = O * inv
-        if (NORM) {
-            float dd[16];
-            tmem_ld16(oa + NV, dd);
-            tmem_wait_ld();
-            inv = 1.f / (dd[0] + dd[1]);
-        } else {
-            inv = reinterpret_cast<const float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] * p.q_scale;
-        }
-        const int rem = min(C, T - mem_chunk(c) * C);
-        const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;  // 32-byte stores allowed
-        __nv_bfloat16* dst = out_row(c);
-#pragma unroll 1
-        for (int piece = 0; piece < G::NVW / 16; ++piece) {
-            float o[16];
-            tmem_ld16(oa + cb + 16 * piece, o);
-            tmem_wait_ld();
-            if (t < rem) store_row16(dst + 16 * piece, o, inv, wide, accumulate);
-        }
-        tc_fence_before_sync();
-        warp_arrive(&bar[B_OEMPTY + ro]);
-        return true;
-    };
     if (p.state_pass) {
         bool ok = true;
 #pragma unroll 1
@@ -1205,21 +1181,8 @@ __device__ __noinline__ void role_state_epilogue(const Ctx x) {
 
     write_copy(0);
     bool ok = true;
-    if constexpr (G::EPI_MASK) {
 #pragma unroll 1
-        for (int c = 0; c < n && ok; ++c) ok = state(c);
-    } else {
-        // The state update of chunk c gates the next chunk's Q S, so it goes
-        // first, unless both the O buffer and the state copy are single: then
-        // Q S (c) waits for the epilogue of c - 1 and the state of c for Q S (c).
-        constexpr bool kStateFirst = G::NO >= 2 || G::NSB >= 2;
-#pragma unroll 1
-        for (int c = 0; c <= n && ok; ++c) {
-            if (!kStateFirst && c >= 1) ok = epilogue(c - 1);
-            if (ok && c < n) ok = state(c);
-            if (ok && kStateFirst && c >= 1) ok = epilogue(c - 1);
-        }
-    }
+    for (int c = 0; c < n && ok; ++c) ok = state(c);
     if (ok && !*abort && row_ok() && x.seg == p.nseg - 1) {
         if (p.final_state) {
             float* fs = p.final_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
@@ -1256,7 +1219,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
         prefetch_tensormap(&tmv);
         for (int s = 0; s < 4; ++s) {
             mbar_init(&bar[B_QFULL + s], 1);
-            mbar_init(&bar[B_QEMPTY + s], 1);
+            mbar_init(&bar[B_QEMPTY + s], 2);  // Q K^T (warp A) and Q S (warp B)
             mbar_init(&bar[B_KFULL + s], 1);
             mbar_init(&bar[B_KEMPTY + s], 1);
             mbar_init(&bar[B_VFULL + s], 1);
@@ -1265,7 +1228,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar[B_OFULL + i], 1);
-            mbar_init(&bar[B_OEMPTY + i], G::EPI_MASK ? 4 : 4 * G::NSW);
+            mbar_init(&bar[B_OEMPTY + i], 4);  // the epilogue warpgroup
             mbar_init(&bar[B_AFULL + i], 1);
             mbar_init(&bar[B_AEMPTY + i], 8);
             mbar_init(&bar[B_PFULL + i], 8);
@@ -1277,6 +1240,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
         }
         for (int i = 0; i < 4; ++i) mbar_init(&bar[B_PHI + i], 8);
         mbar_init(&bar[B_DRAIN], 1);
+        mbar_init(&bar[B_DRAINB], 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -1301,16 +1265,16 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     grid_launch_dependents();
 
     const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice, seg, c0, nloc};
-    if (warp == G::W_TMA) {
-        role_tma_q<DK, NV, NORM, REV>(x, &tmq);
+    if (warp == G::W_MMAB) {
+        role_mma_b<DK, NV, NORM, REV, PHI>(x);
     } else if (warp == G::W_MMA) {
-        role_mma<DK, NV, NORM, REV, PHI>(x);
+        role_mma_a<DK, NV, NORM, REV, PHI>(x);
     } else if (warp < G::W_ES) {
         role_prep_mask<DK, NV, NORM, REV, PHI>(x);
     } else if (warp < G::W_TMAV) {
-        role_state_epilogue<DK, NV, NORM, REV>(x);
+        role_state<DK, NV, NORM, REV>(x);
     } else {
-        role_tma_kv<DK, NV, NORM, REV>(x, &tmk, &tmv);
+        role_tma<DK, NV, NORM, REV>(x, &tmq, &tmk, &tmv);
     }
 
     __syncwarp();  // lanes that idled while lane 0 ran a single-thread role rejoin it
