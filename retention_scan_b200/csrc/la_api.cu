@@ -232,7 +232,7 @@ BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int ki
 // the numerator n, dn, the dden panel and the key-sum part of dq.
 struct NormLayout {
     BwdLayout base;
-    size_t z0p, z0t, dzft, ztp, dz1p, ones, denp, num, dn, ddp, dq2, scan, scan_bytes, total;
+    size_t z0p, z0t, dzft, ztp, dz1p, ones, denp, y, dn, ddp, scan, scan_bytes, total;
 };
 
 NormLayout norm_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind) {
@@ -248,16 +248,15 @@ NormLayout norm_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int 
     L.dz1p = L.ztp + panel;
     L.ones = L.dz1p + panel;
     L.denp = L.ones + tok16;
-    L.num = L.denp + tok16;
-    L.dn = L.num + round256(es * BH * T * Dv);
+    L.y = L.denp + tok16;
+    L.dn = L.y + round256(es * BH * T * Dv);
     L.ddp = L.dn + round256(es * BH * T * Dv);
-    L.dq2 = L.ddp + tok16;
-    L.scan = L.dq2 + round256(es * BH * T * Dk);
+    L.scan = L.ddp + tok16;
     L.scan_bytes = 0;
     if (dtype == LA_BF16) {
-        const int dims[6][2] = {{Dk, Dv}, {Dk, 16}, {Dv, Dk}, {16, Dk}, {Dk, Dv}, {Dv, Dk}};
+        const int dims[5][3] = {{Dk, Dv, 1}, {Dk, 16, 0}, {Dv, Dk, 0}, {16, Dk, 0}, {Dk, Dv, 0}};
         for (const auto& d : dims) {
-            const size_t b = la::fwd_tc_workspace_bytes(B, H, T, d[0], d[1], false);
+            const size_t b = la::fwd_tc_workspace_bytes(B, H, T, d[0], d[1], d[2] != 0);
             if (b > L.scan_bytes) L.scan_bytes = b;
         }
         L.scan_bytes = round256(L.scan_bytes);
@@ -780,7 +779,8 @@ la_status la_chunk_backward_norm_ws(const void* q, const void* k, const void* v,
         return LA_OK;
     }
     // Dv + 1 above the widest panel: the numerator's and the denominator's
-    // terms of dq and dk come from separate scans and are added
+    // terms of dq and dk come from separate scans, the second adding into the
+    // first's output (fp32 add, one rounding)
     float* s0t = init_state ? at(L.base.s0t) : nullptr;
     float* dsft = d_final_state ? at(L.base.dsft) : nullptr;
     const bool need_st = d_log_g && d_final_state;
@@ -793,10 +793,9 @@ la_status la_chunk_backward_norm_ws(const void* q, const void* k, const void* v,
     float* dz1p = d_init_z ? at(L.dz1p) : nullptr;
     void* ones = ws + L.ones;
     void* denp = ws + L.denp;
-    void* num = ws + L.num;
+    void* y = ws + L.y;
     void* dn = ws + L.dn;
     void* ddp = ws + L.ddp;
-    void* dq2 = ws + L.dq2;
     void* scan_ws = L.scan_bytes ? ws + L.scan : nullptr;
     const size_t sw = L.scan_bytes;
 
@@ -809,17 +808,18 @@ la_status la_chunk_backward_norm_ws(const void* q, const void* k, const void* v,
     if (!ok(la::launch_ones_panel(ones, ntok, dtype, s))) return LA_ERR_CUDA;
     const la_decay shifted{LA_DECAY_PER_STEP, lsh};
     const la_decay* rdecay = lsh ? &shifted : nullptr;
-    // numerator n_t = q_t^T S_t and denominator q_t . z_t (ones value panel, column 0)
-    LA_SCAN(q, k, v, decay, 0, init_state, nullptr, num, nullptr, nullptr, B, H, T, Dk, Dv, dtype, scan_ws, sw,
-            stream, 0, 0);
+    // the normalised output y_t = n_t / den_t (one rounding of the ratio, whose
+    // numerator and denominator share the kernel's scores) and the
+    // denominator q_t . z_t (ones value panel, column 0)
+    LA_SCAN(q, k, v, decay, 1, init_state, init_z, y, nullptr, nullptr, B, H, T, Dk, Dv, dtype, scan_ws, sw, stream,
+            0, 0);
     LA_SCAN(q, k, ones, decay, 0, z0p, nullptr, denp, ztp, nullptr, B, H, T, Dk, 16, dtype, scan_ws, sw, stream, 0,
             0);
-    if (!ok(la::launch_norm_grad(dy, num, denp, dn, ddp, Dv, ntok, dtype, s))) return LA_ERR_CUDA;
-    // dq = S_t dn_t + dden_t z_t
+    if (!ok(la::launch_norm_grad(dy, y, denp, dn, ddp, Dv, ntok, dtype, s))) return LA_ERR_CUDA;
+    // dq = S_t dn_t + dden_t z_t (the second scan adds into dq)
     LA_SCAN(dn, v, k, decay, 0, s0t, nullptr, dq, st, nullptr, B, H, T, Dv, Dk, dtype, scan_ws, sw, stream, 0, 0);
-    LA_SCAN(ddp, ones, k, decay, 0, z0t, nullptr, dq2, nullptr, nullptr, B, H, T, 16, Dk, dtype, scan_ws, sw,
-            stream, 0, 0);
-    if (!ok(la::launch_add_into(dq, dq2, ntok * Dk, dtype, s))) return LA_ERR_CUDA;
+    LA_SCAN(ddp, ones, k, decay, 0, z0t, nullptr, dq, nullptr, nullptr, B, H, T, 16, Dk, dtype, scan_ws, sw, stream,
+            0, 1);
     // dk = dS_t v_t + dz_t (the second scan adds into dk), dv = dS_t^T k_t
     LA_SCAN(v, dn, q, rdecay, 0, dsft, nullptr, dk, nullptr, nullptr, B, H, T, Dv, Dk, dtype, scan_ws, sw, stream,
             1, 0);

@@ -270,10 +270,11 @@ __global__ void vec_panel_kernel(const float* __restrict__ x, float* __restrict_
 }
 
 // Normalised output y = n / den: per token, dn = dy / den and
-// dden = -(dy . n) / den^2 (the latter as column 0 of a 16-wide panel).
-// One warp per token.
+// dden = -(dy . y) / den = -(dy . n) / den^2 (the latter as column 0 of a
+// 16-wide panel); from y, whose rounding is one of the ratio, a rounding of
+// den scales dn and dden alike.  One warp per token.
 template <typename E>
-__global__ void norm_grad_kernel(const E* __restrict__ dy, const E* __restrict__ num,
+__global__ void norm_grad_kernel(const E* __restrict__ dy, const E* __restrict__ y,
                                  const E* __restrict__ den_panel, E* __restrict__ dn, E* __restrict__ dden_panel,
                                  int Dv, long long ntok) {
     const int lane = threadIdx.x % 32;
@@ -286,12 +287,12 @@ __global__ void norm_grad_kernel(const E* __restrict__ dy, const E* __restrict__
         float dot = 0.f;
         for (int c = lane; c < Dv; c += 32) {
             const float g = to_f(dy[row + c]);
-            dot = fmaf(g, to_f(num[row + c]), dot);
+            dot = fmaf(g, to_f(y[row + c]), dot);
             dn[row + c] = static_cast<E>(g * inv);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane < 16) dden_panel[t * 16 + lane] = static_cast<E>(lane == 0 ? -dot * inv * inv : 0.f);
+        if (lane < 16) dden_panel[t * 16 + lane] = static_cast<E>(lane == 0 ? -dot * inv : 0.f);
     }
 }
 
@@ -345,13 +346,6 @@ __global__ void norm_grad_panel_kernel(const E* __restrict__ dy, const E* __rest
     }
 }
 
-template <typename E>
-__global__ void add_into_kernel(E* __restrict__ a, const E* __restrict__ b, long long n) {
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<long long>(gridDim.x) * blockDim.x)
-        a[i] = static_cast<E>(to_f(a[i]) + to_f(b[i]));
-}
-
 // out[bh][i] = g_1 * panel[bh * rows * Dk + row * Dk + i] (one row of a
 // [rows][Dk] state panel), g_1 the decay of the sequence's first token (1
 // without a decay).
@@ -385,16 +379,16 @@ cudaError_t launch_vec_panel(const float* x, float* out, int BH, int Dk, bool ro
     return cudaGetLastError();
 }
 
-cudaError_t launch_norm_grad(const void* dy, const void* num, const void* den_panel, void* dn, void* dden_panel,
+cudaError_t launch_norm_grad(const void* dy, const void* y, const void* den_panel, void* dn, void* dden_panel,
                              int Dv, long long ntok, la_dtype dtype, cudaStream_t stream) {
     const int grid = grid_for(ntok * 32, 256);
     if (dtype == LA_BF16)
         norm_grad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(num),
+            static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(y),
             static_cast<const __nv_bfloat16*>(den_panel), static_cast<__nv_bfloat16*>(dn),
             static_cast<__nv_bfloat16*>(dden_panel), Dv, ntok);
     else
-        norm_grad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dy), static_cast<const float*>(num),
+        norm_grad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dy), static_cast<const float*>(y),
                                                          static_cast<const float*>(den_panel), static_cast<float*>(dn),
                                                          static_cast<float*>(dden_panel), Dv, ntok);
     return cudaGetLastError();
@@ -430,16 +424,6 @@ cudaError_t launch_norm_grad_panel(const void* dy, const void* nd, void* pq, voi
         norm_grad_panel_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dy),
                                                                static_cast<const float*>(nd), static_cast<float*>(pq),
                                                                static_cast<float*>(dn), Dv, W, ntok);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_add_into(void* a, const void* b, long long n, la_dtype dtype, cudaStream_t stream) {
-    if (dtype == LA_BF16)
-        add_into_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, stream>>>(
-            static_cast<__nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), n);
-    else
-        add_into_kernel<float><<<grid_for(n, 256), 256, 0, stream>>>(static_cast<float*>(a),
-                                                                    static_cast<const float*>(b), n);
     return cudaGetLastError();
 }
 

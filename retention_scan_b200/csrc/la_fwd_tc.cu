@@ -308,7 +308,8 @@ cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used) {
     if (!fwd_tc_supports(a.Dk, a.Dv)) return cudaErrorNotSupported;
-    if (a.accumulate && !a.reverse) return cudaErrorNotSupported;  // only the reverse instances accumulate
+    // the reverse instances and the forward ones of 16-wide keys accumulate
+    if (a.accumulate && !a.reverse && padded_width(a.Dk) != 16) return cudaErrorNotSupported;
     const bool norm = a.normalize != 0;
     const int BH = a.B * a.H;
     const int nchunks = (a.T + ws::C - 1) / ws::C;

@@ -159,11 +159,10 @@ cudaError_t launch_ones_panel(void* out, long long n, la_dtype dtype, cudaStream
 //   per (b, h) the Dk vector x (null: zeros) into column 0 of [Dk][16]
 //   (rows = true) or row 0 of [16][Dk] (rows = false), fp32
 cudaError_t launch_vec_panel(const float* x, float* out, int BH, int Dk, bool rows, cudaStream_t stream);
-//   dn = dy / den, dden panel column 0 = -(dy . n) / den^2, per token
-cudaError_t launch_norm_grad(const void* dy, const void* num, const void* den_panel, void* dn, void* dden_panel,
+//   dn = dy / den, dden panel column 0 = -(dy . y) / den, per token (y the
+//   normalised output n / den)
+cudaError_t launch_norm_grad(const void* dy, const void* y, const void* den_panel, void* dn, void* dden_panel,
                              int Dv, long long ntok, la_dtype dtype, cudaStream_t stream);
-//   a += b elementwise (`dtype`)
-cudaError_t launch_add_into(void* a, const void* b, long long n, la_dtype dtype, cudaStream_t stream);
 //   out[b,h,:] = g_1 * row `row` of panel [B,H,rows,Dk]
 cudaError_t launch_panel_row_scaled(const float* panel, float* out, const float* log_g, int kind, int B, int H,
                                     int T, int Dk, int rows, int row, cudaStream_t stream);

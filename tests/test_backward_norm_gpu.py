@@ -7,10 +7,12 @@ and dk carry along the undecayed suffix sum.
 dq_t = S_t dn_t + dden_t z_t and dk_t = dS_t v_t + dz_t are differences of
 comparable terms.  For Dv + 1 <= 128 the library forms each with one scan
 whose scores hold both terms (fp32), and the bar above holds.  For Dv = 128
-the two terms come from two scans, each rounded to the output type before
-the sum, so the bar adds 4 u (|first| + |second|) elementwise (u = 2^-8 for
-bf16, 2^-20 for fp32), the terms' sizes taken from the float64 oracle's
-scans."""
+the two terms come from two scans: the second adds its fp32 result into the
+first's rounded output, and each scan rounds its own scores and state copy
+to bf16 before the terms meet.  Those roundings are relative to each term,
+not to their difference, so the bar adds 4 u (|first| + |second|)
+elementwise (u = 2^-8 for bf16, 2^-20 for fp32), the terms' sizes taken
+from the float64 oracle's scans."""
 import numpy as np
 import pytest
 import torch
