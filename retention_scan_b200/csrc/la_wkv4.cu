@@ -1,5 +1,5 @@
 // la_wkv4.cu - the RWKV-4 WKV recurrence (BlinkDL/RWKV-LM issue 167, the
-// att_seq time loop), one thread per channel.
+// att_seq time loop), two channels per thread.
 //
 // Per batch b and channel c, with time decay w (log of the per-step factor)
 // and bonus u, the output is the decayed average
@@ -13,11 +13,13 @@
 //
 // Data movement: a CTA owns one batch row, kCW consecutive channels and one
 // T-segment.  One producer thread streams [TT tokens x kCW channels] tiles
-// of k and v into a ring of kStages shared-memory stages with TMA (eight CTAs
+// of k and v into a ring of kStages shared-memory stages with TMA (four CTAs
 // per SM, about 200 KB in flight per SM), so the HBM latency is hidden
-// behind the sequential per-token work; each consumer thread reads its
-// channel's column of the tile and writes its output directly (a warp writes
-// 32 consecutive values).
+// behind the sequential per-token work; each consumer thread reads its two
+// channels' columns of the tile as one pair and writes its two outputs as
+// one pair (a warp writes 64 consecutive values).  The two channels' chains
+// are independent, and their adds, multiplies and fmas issue as packed
+// fp32x2 instructions.
 //
 // Parallelism: a channel's recurrence is sequential in t, and B x C channels
 // alone leave each scheduler about one warp.  With a workspace, each sequence
@@ -39,11 +41,11 @@
 namespace la {
 namespace {
 
-constexpr int kCW = 64;                 // channels per CTA (one per consumer thread)
-constexpr int kStages = 3;              // 3 x 8 KB: eight CTAs per SM
-constexpr int kConsumerWarps = kCW / 32;
+constexpr int kConsumerWarps = 2;
+constexpr int kCW = 64 * kConsumerWarps;  // channels per CTA: two per consumer thread
+constexpr int kStages = 3;                // 3 x 16 KB: four CTAs per SM
 constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one producer warp
-constexpr int kCtasPerSm = 8;
+constexpr int kCtasPerSm = 4;
 constexpr int kMinSegTokens = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -82,10 +84,23 @@ __device__ __forceinline__ void shifted_pair(float a, float b, float& fa, float&
     fb = d >= 0.f ? t : 1.f;
 }
 
-__device__ __forceinline__ float load_f(const float* p) { return *p; }
-__device__ __forceinline__ float load_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-__device__ __forceinline__ void store_e(float* p, float x) { *p = x; }
-__device__ __forceinline__ void store_e(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+// The same weights from the difference d = a - b.
+__device__ __forceinline__ void shifted_diff(float d, float& fa, float& fb) {
+    const float t = ex2_approx(-fabsf(d));
+    fa = d >= 0.f ? 1.f : t;
+    fb = d >= 0.f ? t : 1.f;
+}
+
+// Two adjacent channels' values as fp32 pairs.
+__device__ __forceinline__ float2 load_f2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 load_f2(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ void store_e2(float* p, float2 y) { *reinterpret_cast<float2*>(p) = y; }
+__device__ __forceinline__ void store_e2(__nv_bfloat16* p, float2 y) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(y.x, y.y);
+}
+
 
 template <typename E>
 __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -142,62 +157,78 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
         return;
     }
 
-    // consumer: thread = channel
-    const int c = c0 + threadIdx.x;
+    // consumer: thread = two adjacent channels (C is even, so a pair never
+    // straddles the end)
+    const int c = c0 + 2 * threadIdx.x;
     const bool live = c < C;
-    const float W = live ? p.w[c] * kLog2e : 0.f;
-    const float U = live ? p.u[c] * kLog2e : 0.f;
     const size_t plane = static_cast<size_t>(C);
-    float aa = 0.f, bb = 0.f, P = kEmptyScale * kLog2e;
+    float W[2], U[2], aa[2], bb[2], P[2];
     float* slot0 = p.ws ? p.ws + static_cast<size_t>(b) * p.nseg * 3 * plane + c : nullptr;
-    if (live) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        W[e] = live ? p.w[c + e] * kLog2e : 0.f;
+        U[e] = live ? p.u[c + e] * kLog2e : 0.f;
+        aa[e] = 0.f;
+        bb[e] = 0.f;
+        P[e] = kEmptyScale * kLog2e;
+        if (!live) continue;
         if (p.state_pass) {
             if (seg == 0) {  // keep the initial state for the output pass
-                const float* s0 = p.init_state ? p.init_state + static_cast<size_t>(b) * 3 * plane + c : nullptr;
-                slot0[0] = s0 ? s0[0] : 0.f;
-                slot0[plane] = s0 ? s0[plane] : 0.f;
-                slot0[2 * plane] = s0 ? s0[2 * plane] : kEmptyScale;
+                const float* s0 = p.init_state ? p.init_state + static_cast<size_t>(b) * 3 * plane + c + e : nullptr;
+                slot0[e] = s0 ? s0[0] : 0.f;
+                slot0[e + plane] = s0 ? s0[plane] : 0.f;
+                slot0[e + 2 * plane] = s0 ? s0[2 * plane] : kEmptyScale;
             }
         } else if (p.ws) {
             // the initial state, then each earlier segment: decayed over that
             // segment's tokens, plus the segment's own state (max-shifted add)
-            aa = slot0[0];
-            bb = slot0[plane];
-            P = slot0[2 * plane] * kLog2e;
+            aa[e] = slot0[e];
+            bb[e] = slot0[e + plane];
+            P[e] = slot0[e + 2 * plane] * kLog2e;
             for (int j = 0; j < seg; ++j) {
-                const float* sj = slot0 + static_cast<size_t>(j + 1) * 3 * plane;
-                const float Pd = P + W * static_cast<float>(p.seg_len);
+                const float* sj = slot0 + e + static_cast<size_t>(j + 1) * 3 * plane;
+                const float Pd = P[e] + W[e] * static_cast<float>(p.seg_len);
                 const float Pj = sj[2 * plane] * kLog2e;
                 float fa, fb;
                 shifted_pair(Pd, Pj, fa, fb);
-                aa = fmaf(fa, aa, fb * sj[0]);
-                bb = fmaf(fa, bb, fb * sj[plane]);
-                P = fmaxf(Pd, Pj);
+                aa[e] = fmaf(fa, aa[e], fb * sj[0]);
+                bb[e] = fmaf(fa, bb[e], fb * sj[plane]);
+                P[e] = fmaxf(Pd, Pj);
             }
         } else if (p.init_state) {
-            const float* s0 = p.init_state + static_cast<size_t>(b) * 3 * plane + c;
-            aa = s0[0];
-            bb = s0[plane];
-            P = s0[2 * plane] * kLog2e;
+            const float* s0 = p.init_state + static_cast<size_t>(b) * 3 * plane + c + e;
+            aa[e] = s0[0];
+            bb[e] = s0[plane];
+            P[e] = s0[2 * plane] * kLog2e;
         }
     }
     E* o = static_cast<E*>(p.out) + (static_cast<size_t>(b) * T + t0) * C + c;
-    // one token: read-out (the state at log weight P, this token at U + K),
-    // then update (the state decayed to W + P, this token at K)
-    auto update = [&](float K, float v) {
-        const float d = W + P;
-        float f1, f2;
-        shifted_pair(d, K, f1, f2);
-        aa = fmaf(f1, aa, f2 * v);
-        bb = fmaf(f1, bb, f2);
-        P = fmaxf(d, K);
+    // One token on both channels: read-out (the state at log weight P, this
+    // token at U + K), then update (the state decayed to W + P, this token at
+    // K).  Adds, multiplies and fmas in packed fp32x2 arithmetic (each lane
+    // rounded as its scalar form would be); exponentials, compares and
+    // maxima per channel.
+    const float2 W2 = make_float2(W[0], W[1]), U2 = make_float2(U[0], U[1]);
+    const float2 m1 = make_float2(-1.f, -1.f), l2e = make_float2(kLog2e, kLog2e);
+    float2 aa2 = make_float2(aa[0], aa[1]), bb2 = make_float2(bb[0], bb[1]), P2 = make_float2(P[0], P[1]);
+    auto update = [&](float2 K, float2 v) {
+        const float2 d = __fadd2_rn(W2, P2);
+        const float2 x = __ffma2_rn(K, m1, d);  // d - K
+        float2 f1, f2;
+        shifted_diff(x.x, f1.x, f2.x);
+        shifted_diff(x.y, f1.y, f2.y);
+        aa2 = __ffma2_rn(f1, aa2, __fmul2_rn(f2, v));
+        bb2 = __ffma2_rn(f1, bb2, f2);
+        P2 = make_float2(fmaxf(d.x, K.x), fmaxf(d.y, K.y));
     };
-    auto step = [&](float K, float v) -> float {
-        float e1, e2;
-        shifted_pair(P, U + K, e1, e2);
-        const float y = __fdividef(fmaf(e1, aa, e2 * v), fmaf(e1, bb, e2));
+    auto step = [&](float2 K, float2 v) -> float2 {
+        const float2 x = __ffma2_rn(__fadd2_rn(U2, K), m1, P2);  // P - (U + K)
+        float2 e1, e2;
+        shifted_diff(x.x, e1.x, e2.x);
+        shifted_diff(x.y, e1.y, e2.y);
+        const float2 num = __ffma2_rn(e1, aa2, __fmul2_rn(e2, v)), den = __ffma2_rn(e1, bb2, e2);
         update(K, v);
-        return y;
+        return make_float2(__fdividef(num.x, den.x), __fdividef(num.y, den.y));
     };
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
@@ -221,37 +252,37 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
             }
             if (!ok) break;
         }
-        const E* tk = reinterpret_cast<const E*>(sm + s * G::STAGE) + threadIdx.x;
-        const E* tv = reinterpret_cast<const E*>(sm + s * G::STAGE + G::BYTES) + threadIdx.x;
+        const E* tk = reinterpret_cast<const E*>(sm + s * G::STAGE) + 2 * threadIdx.x;
+        const E* tv = reinterpret_cast<const E*>(sm + s * G::STAGE + G::BYTES) + 2 * threadIdx.x;
         const int n = min(G::TT, t1 - (j0 + j) * G::TT);
         if (live && p.state_pass) {
 #pragma unroll 8
-            for (int i = 0; i < n; ++i) update(load_f(tk + i * kCW) * kLog2e, load_f(tv + i * kCW));
+            for (int i = 0; i < n; ++i) update(__fmul2_rn(load_f2(tk + i * kCW), l2e), load_f2(tv + i * kCW));
         } else if (live) {
             // batches of 8 tokens: the next batch's tile reads are issued
             // before this batch's dependent steps, the outputs stored after
             // them, so that memory latency stays off the recurrence's path
             const int nb = n / 8;
-            float kk[8], vv[8];
+            float2 kk[8], vv[8];
             if (nb > 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    kk[e] = load_f(tk + e * kCW);
-                    vv[e] = load_f(tv + e * kCW);
+                    kk[e] = load_f2(tk + e * kCW);
+                    vv[e] = load_f2(tv + e * kCW);
                 }
             }
             for (int bi = 0; bi < nb; ++bi) {
-                float kn[8], vn[8], yy[8];
+                float2 kn[8], vn[8], yy[8];
                 const int nxt = bi + 1 < nb ? (bi + 1) * 8 : bi * 8;  // (a harmless re-read at the end)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    kn[e] = load_f(tk + (nxt + e) * kCW);
-                    vn[e] = load_f(tv + (nxt + e) * kCW);
+                    kn[e] = load_f2(tk + (nxt + e) * kCW);
+                    vn[e] = load_f2(tv + (nxt + e) * kCW);
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) yy[e] = step(kk[e] * kLog2e, vv[e]);
+                for (int e = 0; e < 8; ++e) yy[e] = step(__fmul2_rn(kk[e], l2e), vv[e]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) store_e(o + static_cast<size_t>(e) * C, yy[e]);
+                for (int e = 0; e < 8; ++e) store_e2(o + static_cast<size_t>(e) * C, yy[e]);
                 o += static_cast<size_t>(8) * C;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -260,7 +291,7 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
                 }
             }
             for (int i = nb * 8; i < n; ++i) {
-                store_e(o, step(load_f(tk + i * kCW) * kLog2e, load_f(tv + i * kCW)));
+                store_e2(o, step(__fmul2_rn(load_f2(tk + i * kCW), l2e), load_f2(tv + i * kCW)));
                 o += C;
             }
         }
@@ -274,9 +305,12 @@ __global__ void __launch_bounds__(kThreads) wkv4_kernel(const __grid_constant__ 
     else if (seg == p.nseg - 1 && p.final_state)
         dst = p.final_state + static_cast<size_t>(b) * 3 * plane + c;
     if (dst) {
-        dst[0] = aa;
-        dst[plane] = bb;
-        dst[2 * plane] = P * (1.f / kLog2e);
+        dst[0] = aa2.x;
+        dst[1] = aa2.y;
+        dst[plane] = bb2.x;
+        dst[plane + 1] = bb2.y;
+        dst[2 * plane] = P2.x * (1.f / kLog2e);
+        dst[2 * plane + 1] = P2.y * (1.f / kLog2e);
     }
 }
 
