@@ -442,6 +442,7 @@ def rank_seed(wl, rank):
 
 
 SPIN_UP_S = 0.5
+SPACER_CYCLES = 2_000_000  # about 1 ms at the B200's clocks
 
 
 def spin_up(job, flush, device, min_s=SPIN_UP_S):
@@ -490,6 +491,10 @@ def time_steps(job, steps, flush, dist_on, device):
     launches = 0
     barrier(dist_on)
     wall0 = time.time()
+    # the device waits about a millisecond (no memory traffic) while the host
+    # enqueues the first steps, so that the first step's events time its
+    # kernels, not the host's launch latency (the steady state of a queue)
+    torch.cuda._sleep(SPACER_CYCLES)
     for i in range(steps):
         if flush is not None:
             flush.add_(1)
