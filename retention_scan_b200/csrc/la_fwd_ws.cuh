@@ -102,7 +102,7 @@ enum Bar : int {
     B_COUNT = 54
 };
 
-template <int DK, int NV, bool NORM>
+template <int DK, int NV, bool NORM, bool SP = false>
 struct Plan {
     static constexpr int WK = row_bytes_for(DK), PK = panels_for(DK);
     // Value tiles (and the bf16 state copy, whose columns are value columns):
@@ -140,28 +140,51 @@ struct Plan {
         if (450 / nvs > b) b = 450 / nvs;
         return b + (nsb == 1 ? 20 : 0);
     }
+    // A state pass (SP) reads no queries and keeps no state copy: its shared
+    // memory holds only K and V rings, as deep as fit (at most 4, the
+    // barrier slots per ring).  A K stage stays busy from its load to K^T V'
+    // and a V stage a little longer (the state warps read its decay), about
+    // equally long, so the deepest balanced rings win.
+    static constexpr int bound_sp(int nk, int nvs) {
+        const int a = 500 / nk, b = 520 / nvs;
+        return a > b ? a : b;
+    }
     static constexpr int pick() {
         int best = 0, bb = 1 << 30;
-        for (int nq = 4; nq >= 2; --nq)
+        if (SP) {
             for (int nk = 4; nk >= 2; --nk)
                 for (int nvs = 4; nvs >= 2; --nvs)
-                    for (int nsb = 2; nsb >= 1; --nsb)
-                        if (fits(nq, nk, nvs, nsb) && bound(nq, nk, nvs, nsb) < bb) {
-                            bb = bound(nq, nk, nvs, nsb);
-                            best = nq * 1000 + nk * 100 + nvs * 10 + nsb;
-                        }
+                    if (fits(0, nk, nvs, 0) && bound_sp(nk, nvs) < bb) {
+                        bb = bound_sp(nk, nvs);
+                        best = nk * 100 + nvs * 10;
+                    }
+        } else {
+            for (int nq = 4; nq >= 2; --nq)
+                for (int nk = 4; nk >= 2; --nk)
+                    for (int nvs = 4; nvs >= 2; --nvs)
+                        for (int nsb = 2; nsb >= 1; --nsb)
+                            if (fits(nq, nk, nvs, nsb) && bound(nq, nk, nvs, nsb) < bb) {
+                                bb = bound(nq, nk, nvs, nsb);
+                                best = nq * 1000 + nk * 100 + nvs * 10 + nsb;
+                            }
+        }
         return best;
     }
     static constexpr int PICK = pick();
     static constexpr bool OK = PICK != 0;
-    static constexpr int NQ = OK ? PICK / 1000 : 2;
+    // stages allocated (a state pass allocates no Q stage and no state copy)
+    static constexpr int NQA = OK ? PICK / 1000 : 2;
+    static constexpr int NSBA = OK ? PICK % 10 : 1;
+    // ring lengths for the index arithmetic (at least 1; a state pass never
+    // touches the Q ring or the state copy)
+    static constexpr int NQ = NQA > 0 ? NQA : 1;
     static constexpr int NK = OK ? (PICK / 100) % 10 : 2;
     static constexpr int NVS = OK ? (PICK / 10) % 10 : 2;
-    static constexpr int NSB = OK ? PICK % 10 : 1;
-    static constexpr int OFF_K = NQ * Q_STAGE;
+    static constexpr int NSB = NSBA > 0 ? NSBA : 1;
+    static constexpr int OFF_K = NQA * Q_STAGE;
     static constexpr int OFF_V = OFF_K + NK * Q_STAGE;
     static constexpr int OFF_SB = OFF_V + NVS * V_STAGE;
-    static constexpr int OFF_MISC = OFF_SB + NSB * SB_BYTES;
+    static constexpr int OFF_MISC = OFF_SB + NSBA * SB_BYTES;
     static constexpr int OFF_ROWF = OFF_MISC + 1024;  // float[kRowfRing][C]: 2^(L_t) per token
     static constexpr int SMEM = OFF_MISC + MISC + 1024;
     // TMEM columns: scores 128 per buffer | P (bf16 pairs) 64 per buffer | O | K^T V'.
@@ -425,7 +448,7 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
 }
 
 #define LA_ROLE_PRELUDE                                                                              \
-    using G = Plan<DK, NV, NORM>;                                                                    \
+    using G = Plan<DK, NV, NORM, SP>;                                                                \
     const Params& p = *x.p;                                                                          \
     uint8_t* const sm = x.sm;                                                                        \
     const uint32_t sa = x.sa, tmem = x.tmem;                                                         \
@@ -450,12 +473,12 @@ __device__ __forceinline__ void prefetch_row_l2(const __nv_bfloat16* p, int n) {
 // another's free stage (the state pass reads no queries).  K and V run as
 // far ahead as their rings allow: the prep of chunk c + 1 (which needs V)
 // runs before the mask of chunk c.
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool SP>
 __device__ __noinline__ void role_tma(const Ctx x, const CUtensorMap* tmq, const CUtensorMap* tmk,
                                       const CUtensorMap* tmv) {
     LA_ROLE_PRELUDE
     if (lane != 0) return;
-    const int nq = p.state_pass ? 0 : n;
+    const int nq = SP ? 0 : n;
     int cq = 0, ck = 0, cv = 0;
     uint64_t last = global_timer_ns();
     while (cq < nq || ck < n || cv < n) {
@@ -531,7 +554,7 @@ __device__ __noinline__ void role_tma(const Ctx x, const CUtensorMap* tmq, const
 // gives up after kWaitLimitNs without progress.
 // State pass: warp A issues K^T V' (and K^T W) in order; each also releases
 // its K and V stages.
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool SP>
 __device__ __noinline__ void mma_state_pass(const Ctx x) {
     LA_ROLE_PRELUDE
     const bool leader = elect_one();
@@ -580,11 +603,11 @@ __device__ __forceinline__ bool idle_pass(bool moved, uint64_t& idle_since, vola
     return true;
 }
 
-template <int DK, int NV, bool NORM, bool REV, bool PHI>
+template <int DK, int NV, bool NORM, bool REV, bool PHI, bool SP>
 __device__ __noinline__ void role_mma_a(const Ctx x) {
     LA_ROLE_PRELUDE
-    if (p.state_pass) {
-        mma_state_pass<DK, NV, NORM, REV>(x);
+    if constexpr (SP) {
+        mma_state_pass<DK, NV, NORM, REV, SP>(x);
         return;
     }
     const bool leader = elect_one();
@@ -661,10 +684,10 @@ __device__ __noinline__ void role_mma_a(const Ctx x) {
     mbar_wait_bounded(&bar[B_DRAIN], 0, kWaitLimitNs);
 }
 
-template <int DK, int NV, bool NORM, bool REV, bool PHI>
+template <int DK, int NV, bool NORM, bool REV, bool PHI, bool SP>
 __device__ __noinline__ void role_mma_b(const Ctx x) {
     LA_ROLE_PRELUDE
-    if (p.state_pass) return;  // no queries, no outputs
+    if constexpr (SP) return;  // no queries, no outputs
     const bool leader = elect_one();
     const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
     auto mode_of = [&](int j) {
@@ -785,7 +808,7 @@ __device__ __noinline__ void mask_direct(uint32_t s_addr, uint32_t p_addr, uint6
     fence_async_smem();
 }
 
-template <int DK, int NV, bool NORM, bool REV, bool PHI>
+template <int DK, int NV, bool NORM, bool REV, bool PHI, bool SP>
 __device__ __noinline__ void role_prep_mask(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_PM) / 4;  // 0: score columns 0-63, V rows; 1: columns 64-127, weights
@@ -812,7 +835,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
     // rows; warpgroup 1 writes the normaliser weights, or has nothing to do.
     auto prep = [&](int c) -> bool {
         const int s = c % G::NVS, rem = min(C, T - mem_chunk(c) * C);
-        if (PHI && p.state_pass && wg == 0) {
+        if (PHI && SP && wg == 0) {
             // the state pass has no Q tile and no mask: warpgroup 0 maps the
             // chunk's key rows here (before it decays them, for a direct-form
             // chunk), before the prep arrival that the chunk's K^T V' awaits
@@ -824,7 +847,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
             // nothing to prepare; in the state pass (no mask to pace this
             // warpgroup) wait for the tile so that its arrivals never run a
             // ring's length ahead
-            if (p.state_pass && !waitw(&bar[B_VFULL + s], (c / G::NVS) & 1, abort, p, kErrTmaWait)) return false;
+            if (SP && !waitw(&bar[B_VFULL + s], (c / G::NVS) & 1, abort, p, kErrTmaWait)) return false;
             warp_arrive(&bar[B_PREP + s]);
             return true;
         }
@@ -876,7 +899,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
                 reinterpret_cast<float*>(sm + G::OFF_ROWF)[(c % G::kRowfRing) * C + t] =
                     md == kModeFolded ? ex2_approx(lt) : 1.f;
             if (md == kModeFolded) scale_row<NV, G::WV>(st, t, ex2_approx(-lt));
-            if (md == kModeDirect && p.state_pass) {
+            if (md == kModeDirect && SP) {
                 // no mask in the state pass: decay this key row here, K~ = 2^(L_C - L_t) K
                 if (!waitw(&bar[B_KFULL + c % G::NK], (c / G::NK) & 1, abort, p, kErrTmaWait)) return false;
                 scale_row<DK>(sm + G::OFF_K + (c % G::NK) * G::Q_STAGE, t, ex2_approx(lc - lt));
@@ -1003,7 +1026,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
         warp_arrive(&bar[B_OEMPTY + ro]);
         return true;
     };
-    if (p.state_pass) {  // prep only; nothing reads the V stage's prefix later
+    if constexpr (SP) {  // prep only; nothing reads the V stage's prefix later
 #pragma unroll 1
         for (int c = 0; c < n; ++c) {
             if (!prep(c)) break;
@@ -1046,7 +1069,7 @@ __device__ __noinline__ void role_prep_mask(const Ctx x) {
 // Warpgroup wg owns value columns [wg NVW, (wg + 1) NVW) of the slice.  Per
 // chunk c: the state update of chunk c, then its bf16 copy, which the next
 // chunk's Q S reads.
-template <int DK, int NV, bool NORM, bool REV>
+template <int DK, int NV, bool NORM, bool REV, bool SP>
 __device__ __noinline__ void role_state(const Ctx x) {
     LA_ROLE_PRELUDE
     const int wg = (warp - G::W_ES) / 4;
@@ -1065,7 +1088,7 @@ __device__ __noinline__ void role_state(const Ctx x) {
 #pragma unroll
     for (int j = 0; j < G::NVW; ++j) S[j] = 0.f;
     float ltot = 0.f;  // state pass: total log2 decay of the segment
-    if (row_ok() && p.init_state && !p.state_pass) {
+    if (row_ok() && p.init_state && !SP) {
         const float* src = p.init_state + (static_cast<size_t>(bh) * p.Dk + d) * p.Dv + j0 + cb;
 #pragma unroll
         for (int j = 0; j < G::NVW; j += 4) {
@@ -1076,8 +1099,8 @@ __device__ __noinline__ void role_state(const Ctx x) {
             S[j + 3] = v4.w;
         }
     }
-    if (NORM && row_ok() && p.init_z && !p.state_pass) z = p.init_z[static_cast<size_t>(bh) * p.Dk + d];
-    if (row_ok() && !p.state_pass && x.seg > 0) {
+    if (NORM && row_ok() && p.init_z && !SP) z = p.init_z[static_cast<size_t>(bh) * p.Dk + d];
+    if (row_ok() && !SP && x.seg > 0) {
         // state entering this segment: fold in every earlier state segment j,
         // S <- 2^(L_j) S + S_j (the combination of two consecutive spans)
         for (int j = 0; j < x.seg * p.ws_per_seg; ++j) {
@@ -1153,7 +1176,7 @@ __device__ __noinline__ void role_state(const Ctx x) {
         tc_fence_before_sync();
         warp_arrive(&bar[B_DSEMPTY + b]);
         warp_arrive(&bar[B_VEMPTY + s]);
-        if (c == n - 1 || p.state_pass) return true;
+        if (c == n - 1 || SP) return true;
         const int k = c + 1;
         if (k >= G::NSB && !waitw(&bar[B_SBEMPTY + k % G::NSB], ((k / G::NSB) - 1) & 1, abort, p, kErrMmaWait))
             return false;
@@ -1161,7 +1184,7 @@ __device__ __noinline__ void role_state(const Ctx x) {
         return true;
     };
 
-    if (p.state_pass) {
+    if constexpr (SP) {
         bool ok = true;
 #pragma unroll 1
         for (int c = 0; c < n && ok; ++c) ok = state(c);
@@ -1194,11 +1217,11 @@ __device__ __noinline__ void role_state(const Ctx x) {
     }
 }
 
-template <int DK, int NV, bool NORM, bool REV, bool PHI>
-__global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
+template <int DK, int NV, bool NORM, bool REV, bool PHI, bool SP>
+__global__ void __launch_bounds__(Plan<DK, NV, NORM, SP>::THREADS, 1)
     fwd_ws_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ Params p) {
-    using G = Plan<DK, NV, NORM>;
+    using G = Plan<DK, NV, NORM, SP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sa = smem_u32(sm);
@@ -1245,7 +1268,7 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
         fence_barrier_init();
     }
     if (warp == G::W_MMA) tmem_alloc(tmem_slot, G::TMEM_COLS);
-    if (NORM && warp >= G::W_ES && warp < G::W_ES + 4) {
+    if (NORM && !SP && warp >= G::W_ES && warp < G::W_ES + 4) {
         // zeroed key-sum tiles (only their first two columns are ever written)
         for (int i = tid - 32 * G::W_ES; i < G::NSB * DK * 2; i += 128)  // 16-byte pieces
             reinterpret_cast<uint4*>(sm + G::OFF_SB + (i / (DK * 2)) * G::SB_BYTES + G::SB_ZB)[i % (DK * 2)] =
@@ -1266,15 +1289,15 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
 
     const Ctx x{&p, sm, sa, tmem, bh, bh % p.H, slice * NV, slice, seg, c0, nloc};
     if (warp == G::W_MMAB) {
-        role_mma_b<DK, NV, NORM, REV, PHI>(x);
+        role_mma_b<DK, NV, NORM, REV, PHI, SP>(x);
     } else if (warp == G::W_MMA) {
-        role_mma_a<DK, NV, NORM, REV, PHI>(x);
+        role_mma_a<DK, NV, NORM, REV, PHI, SP>(x);
     } else if (warp < G::W_ES) {
-        role_prep_mask<DK, NV, NORM, REV, PHI>(x);
+        role_prep_mask<DK, NV, NORM, REV, PHI, SP>(x);
     } else if (warp < G::W_TMAV) {
-        role_state<DK, NV, NORM, REV>(x);
+        role_state<DK, NV, NORM, REV, SP>(x);
     } else {
-        role_tma<DK, NV, NORM, REV>(x, &tmq, &tmk, &tmv);
+        role_tma<DK, NV, NORM, REV, SP>(x, &tmq, &tmk, &tmv);
     }
 
     __syncwarp();  // lanes that idled while lane 0 ran a single-thread role rejoin it
@@ -1284,17 +1307,17 @@ __global__ void __launch_bounds__(Plan<DK, NV, NORM>::THREADS, 1)
     if (warp == G::W_MMA) tmem_dealloc(tmem, G::TMEM_COLS);
 }
 
-template <int DK, int NV, bool NORM, bool REV, bool PHI>
+template <int DK, int NV, bool NORM, bool REV, bool PHI, bool SP>
 cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                             const Params& p, int grid, cudaStream_t stream) {
-    using G = Plan<DK, NV, NORM>;
+    using G = Plan<DK, NV, NORM, SP>;
     if constexpr (!G::OK) {
         return cudaErrorNotSupported;
     } else {
         // at least 116 KB so that one CTA (512 TMEM columns) owns each SM
         const int smem = G::SMEM > 116 * 1024 ? G::SMEM : 116 * 1024;
         cudaError_t e =
-            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM, REV, PHI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaFuncSetAttribute(fwd_ws_kernel<DK, NV, NORM, REV, PHI, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         // programmatic serialisation: this grid's prologue (barriers, TMEM,
         // descriptor prefetch) overlaps the tail of the previous kernel
@@ -1308,13 +1331,21 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = p.pdl ? 1 : 0;
-        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM, REV, PHI>, tmq, tmk, tmv, p);
+        return cudaLaunchKernelEx(&cfg, fwd_ws_kernel<DK, NV, NORM, REV, PHI, SP>, tmq, tmk, tmv, p);
     }
 }
 
 template <int DK, int NV, bool NORM>
 constexpr bool supported() {
     return Plan<DK, NV, NORM>::OK;
+}
+
+template <int DK, int NV, bool NORM, bool REV, bool PHI>
+cudaError_t launch_pass(const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv, const Params& p,
+                        int grid, cudaStream_t stream) {
+    // a state pass runs its own instance (no Q ring, deeper K and V rings)
+    return p.state_pass ? launch_instance<DK, NV, NORM, REV, PHI, true>(tmq, tmk, tmv, p, grid, stream)
+                        : launch_instance<DK, NV, NORM, REV, PHI, false>(tmq, tmk, tmv, p, grid, stream);
 }
 
 // Dispatch on the value slice and the normaliser for one key width and one
@@ -1325,10 +1356,10 @@ template <int DK, bool REV, bool NORM, bool PHI>
 cudaError_t launch_nv(int nv, const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                       const Params& p, int grid, cudaStream_t stream) {
     switch (nv) {
-        case 16: return launch_instance<DK, 16, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
-        case 32: return launch_instance<DK, 32, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
-        case 64: return launch_instance<DK, 64, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
-        case 128: return launch_instance<DK, 128, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 16: return launch_pass<DK, 16, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 32: return launch_pass<DK, 32, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 64: return launch_pass<DK, 64, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
+        case 128: return launch_pass<DK, 128, NORM, REV, PHI>(tmq, tmk, tmv, p, grid, stream);
         default: return cudaErrorNotSupported;
     }
 }
