@@ -20,7 +20,7 @@ namespace ws {
                                                            const CUtensorMap&, const Params&, int, cudaStream_t); \
     extern template cudaError_t launch_dk<DK, false, true>(int, bool, const CUtensorMap&, const CUtensorMap&,  \
                                                            const CUtensorMap&, const Params&, int, cudaStream_t); \
-    extern template bool supported_dk<DK>(int, bool);
+    extern template bool supported_dk<DK>(int, bool, bool);
 LA_WS_DECL(16)
 LA_WS_DECL(32)
 LA_WS_DECL(64)
@@ -97,14 +97,23 @@ int sm_count() {
     return v;
 }
 
-bool instance_ok(int Dk, int nv, bool norm) {
+// sp: the state-pass instance
+bool instance_ok(int Dk, int nv, bool norm, bool sp = false) {
     switch (Dk) {
-        case 16: return ws::supported_dk<16>(nv, norm);
-        case 32: return ws::supported_dk<32>(nv, norm);
-        case 64: return ws::supported_dk<64>(nv, norm);
-        case 128: return ws::supported_dk<128>(nv, norm);
+        case 16: return ws::supported_dk<16>(nv, norm, sp);
+        case 32: return ws::supported_dk<32>(nv, norm, sp);
+        case 64: return ws::supported_dk<64>(nv, norm, sp);
+        case 128: return ws::supported_dk<128>(nv, norm, sp);
         default: return false;
     }
+}
+
+// The widest value slice of the state-pass instance: it holds no Q ring, so
+// wider slices fit than in the output pass, and each slice reloads K.
+int state_slice(int Dk, int Dv, bool norm) {
+    int nv = widest_slice(Dv);
+    while (!instance_ok(padded_width(Dk), nv, norm, true) && nv / 2 >= 16) nv /= 2;
+    return nv;
 }
 
 int env_int(const char* name) {
@@ -131,6 +140,7 @@ int env_int(const char* name) {
 // pass.  The state pass cuts each segment further while SMs stay idle.
 struct Layout {
     int split, nv, nseg, seg_chunks, per_seg, nS;
+    int split_sp, nv_sp;  // the state pass's slices
 };
 
 constexpr int kMinSegChunks = 16;
@@ -167,10 +177,12 @@ Layout plan_layout(int BH, int nchunks, int Dk, int Dv, bool norm, bool segments
     if (L.seg_chunks < 1) L.seg_chunks = 1;
     L.nseg = (nchunks + L.seg_chunks - 1) / L.seg_chunks;
     if (L.nseg < 1) L.nseg = 1;
+    L.nv_sp = state_slice(Dk, Dv, norm);
+    L.split_sp = Dv / L.nv_sp;
     L.per_seg = 1;
     if (L.nseg > 1)
         while (L.seg_chunks % (2 * L.per_seg) == 0 &&
-               static_cast<long long>(BH) * s * (L.nseg - 1) * L.per_seg * 2 <= sms)
+               static_cast<long long>(BH) * L.split_sp * (L.nseg - 1) * L.per_seg * 2 <= sms)
             L.per_seg *= 2;
     L.nS = (L.nseg - 1) * L.per_seg;
     return L;
@@ -243,8 +255,7 @@ struct StatePlan {
 StatePlan plan_state(int BH, int nchunks, int Dk, int Dv, bool norm) {
     const int sms = sm_count();
     StatePlan P{};
-    int nv = widest_slice(Dv);
-    while (!instance_ok(padded_width(Dk), nv, norm) && nv / 2 >= 16) nv /= 2;
+    const int nv = state_slice(Dk, Dv, norm);
     const int s = Dv / nv;
     P.nv = nv;
     int pieces = 1;
@@ -270,7 +281,7 @@ cudaError_t launch_fwd_state(const FwdArgs& a, int* pieces_used) {
     const int nchunks = (a.T + ws::C - 1) / ws::C;
     const StatePlan P = plan_state(BH, nchunks, a.Dk, a.Dv, norm);
     const int nv = P.nv, DK = padded_width(a.Dk);
-    if (!width_ok(nv) || !instance_ok(DK, nv, norm)) return cudaErrorNotSupported;
+    if (!width_ok(nv) || !instance_ok(DK, nv, norm, true)) return cudaErrorNotSupported;
     if (!a.workspace || a.workspace_bytes < workspace_bytes_for(BH, a.Dk, a.Dv, P.pieces))
         return cudaErrorInvalidValue;
     if (pieces_used) *pieces_used = P.pieces;
@@ -360,7 +371,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
         ps.state_pass = 1;
         ps.nseg = L.nS;
         ps.seg_chunks = L.seg_chunks / L.per_seg;
-        const cudaError_t e = launch_ws(DK, nv, norm, tmq, tmk, tmv, ps, BH * L.nS * split, a.stream);
+        ps.split = L.split_sp;
+        // the value tiles of the state pass's own slice width
+        CUtensorMap tmv_sp;
+        if (!make_map(&tmv_sp, a.v, a.Dv, a.T, BH, norm ? 16 : (L.nv_sp < 64 ? L.nv_sp : 64)))
+            return cudaErrorInvalidValue;
+        const cudaError_t e = launch_ws(DK, L.nv_sp, norm, tmq, tmk, tmv_sp, ps, BH * L.nS * L.split_sp, a.stream);
         if (e != cudaSuccess) return e;
     }
     p.state_pass = 0;

@@ -196,10 +196,11 @@ struct Plan {
     static constexpr int NPB = tmem_need(1, 2, 2, 1) <= 512 ? 2 : 1;
     static constexpr int NO = tmem_need(1, NPB, 2, 1) <= 512 ? 2 : 1;
     static constexpr int NA = tmem_need(2, NPB, NO, 1) <= 512 ? 2 : 1;
-    static constexpr int NDS = tmem_need(NA, NPB, NO, 2) <= 512 ? 2 : 1;
+    // a state pass keeps only K^T V' in tensor memory: two buffers from column 0
+    static constexpr int NDS = SP ? 2 : (tmem_need(NA, NPB, NO, 2) <= 512 ? 2 : 1);
     static constexpr int COL_P0 = 128 * NA;
     static constexpr int COL_O0 = COL_P0 + 64 * NPB;
-    static constexpr int COL_DS0 = COL_O0 + NO * OCOLS;
+    static constexpr int COL_DS0 = SP ? 0 : COL_O0 + NO * OCOLS;
     static constexpr int TMEM_USED = COL_DS0 + NDS * OCOLS;
     static constexpr int TMEM_COLS = 512;
     // warps
@@ -1335,9 +1336,10 @@ cudaError_t launch_instance(const CUtensorMap& tmq, const CUtensorMap& tmk, cons
     }
 }
 
-template <int DK, int NV, bool NORM>
-constexpr bool supported() {
-    return Plan<DK, NV, NORM>::OK;
+template <int DK, int NV>
+constexpr bool supported(bool norm, bool sp) {
+    return norm ? (sp ? Plan<DK, NV, true, true>::OK : Plan<DK, NV, true>::OK)
+                : (sp ? Plan<DK, NV, false, true>::OK : Plan<DK, NV, false>::OK);
 }
 
 template <int DK, int NV, bool NORM, bool REV, bool PHI>
@@ -1374,13 +1376,14 @@ cudaError_t launch_dk(int nv, bool norm, const CUtensorMap& tmq, const CUtensorM
                 : launch_nv<DK, REV, false, PHI>(nv, tmq, tmk, tmv, p, grid, stream);
 }
 
+// sp: the state-pass instance (its plan fits wider slices: no Q ring)
 template <int DK>
-bool supported_dk(int nv, bool norm) {
+bool supported_dk(int nv, bool norm, bool sp) {
     switch (nv) {
-        case 16: return norm ? supported<DK, 16, true>() : supported<DK, 16, false>();
-        case 32: return norm ? supported<DK, 32, true>() : supported<DK, 32, false>();
-        case 64: return norm ? supported<DK, 64, true>() : supported<DK, 64, false>();
-        case 128: return norm ? supported<DK, 128, true>() : supported<DK, 128, false>();
+        case 16: return supported<DK, 16>(norm, sp);
+        case 32: return supported<DK, 32>(norm, sp);
+        case 64: return supported<DK, 64>(norm, sp);
+        case 128: return supported<DK, 128>(norm, sp);
         default: return false;
     }
 }

@@ -8,7 +8,7 @@ namespace ws {
 
 template cudaError_t launch_dk<128, false, false>(int, bool, const CUtensorMap&, const CUtensorMap&,
                                                  const CUtensorMap&, const Params&, int, cudaStream_t);
-template bool supported_dk<128>(int, bool);
+template bool supported_dk<128>(int, bool, bool);
 
 }  // namespace ws
 }  // namespace la

@@ -138,12 +138,14 @@ def test_workspace_size_follows_the_segment_plan(L, monkeypatch):
     monkeypatch.delenv("LA_DV_SPLIT", raising=False)
     assert L.la_chunk_forward_workspace_size(4, 8, 2048, 64, 64, 1, 0) == 0
     # 8 heads of 64 chunks, Dk = Dv = 64: four segments of 16 chunks, then
-    # four value slices (8 x 4 x 4 = 128 CTAs); a state pass of 8 x 4 x 3 =
-    # 96 CTAs, one state segment for each of the first three segments
-    assert L.la_chunk_forward_workspace_size(1, 8, 8192, 64, 64, 1, 0) == _ws_bytes(8, 64, 64, 3)
-    # 32 heads of 512 chunks, Dk = Dv = 128: two value slices, two segments,
-    # the first cut into two state segments
-    assert L.la_chunk_forward_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 2)
+    # four value slices (8 x 4 x 4 = 128 CTAs); the state pass runs one
+    # 64-column slice, each of the first three segments cut into four state
+    # segments (8 x 1 x 3 x 4 = 96 CTAs)
+    assert L.la_chunk_forward_workspace_size(1, 8, 8192, 64, 64, 1, 0) == _ws_bytes(8, 64, 64, 12)
+    # 32 heads of 512 chunks, Dk = Dv = 128: two value slices, two segments;
+    # the state pass runs one 128-column slice, the first segment cut into
+    # four state segments (32 x 4 = 128 CTAs)
+    assert L.la_chunk_forward_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 4)
     # 128 heads fill the GPU: no segments
     assert L.la_chunk_forward_workspace_size(8, 16, 4096, 128, 128, 1, 1) == 0
     # fp32, empty or too short inputs: none
@@ -421,8 +423,9 @@ def test_chunk_state_validation(L):
 
 def test_chunk_state_workspace_size(L):
     # 148 SMs (the host default without a device).  32 heads, Dk = Dv = 128:
-    # two value slices; pieces doubled while 32 x 2 x pieces fits: two
-    assert L.la_chunk_state_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 2)
+    # one 128-column slice (the state-pass instance); pieces doubled while
+    # 32 x 1 x pieces fits: four
+    assert L.la_chunk_state_workspace_size(1, 32, 65536, 128, 128, 1, 0) == _ws_bytes(32, 128, 128, 4)
     # one chunk: one piece
     assert L.la_chunk_state_workspace_size(1, 1, 100, 64, 32, 1, 0) == _ws_bytes(1, 64, 32, 1)
     # fp32 and empty inputs: none
