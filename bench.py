@@ -935,6 +935,8 @@ def run_reference(args, world):
 
 
 EXTRA_CONFIGS = (3, 5, 2)  # measured beside the headline config 4 by the default run
+# and, beside them, the gated workload's backward and the two per-channel scans
+EXTRA_LINES = (("backward", 4), ("forward", 6), ("forward", 7))
 
 
 def free_port():
@@ -984,7 +986,8 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5, 6, 7],
-                    help="time one workload only (default: config 4 with configs 3, 5 and 2 beside it)")
+                    help="time one workload only (default: config 4 with configs 3, 5 and 2 beside it, "
+                         "the backward of config 4, and configs 6 and 7)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -1034,29 +1037,39 @@ def main():
                                              timeout=datetime.timedelta(seconds=120))
     try:
         line = (run_wkv4 if args.config in (6, 7) else run_ours)(args, rank, world, dist_on, device)
-        extra = {}
+        extra = {}   # name -> (line, config, direction)
         if combined:
             for cfg in EXTRA_CONFIGS:
                 sub = run_ours(args, rank, world, dist_on, device, cfg=cfg)
-                extra[sub["config"]["workload"]] = sub
+                extra[sub["config"]["workload"]] = (sub, cfg, "forward")
                 torch.cuda.empty_cache()
                 if cfg == 3:  # the normalised workload once more, with the feature map in the kernel
                     sub = run_ours(args, rank, world, dist_on, device, cfg=cfg, prologue=True)
-                    extra[sub["config"]["workload"]] = sub
+                    extra[sub["config"]["workload"]] = (sub, cfg, "forward")
                     torch.cuda.empty_cache()
+            for direction, cfg in EXTRA_LINES:
+                a2 = argparse.Namespace(**vars(args))
+                a2.config, a2.direction = cfg, direction
+                sub = (run_wkv4 if cfg in (6, 7) else run_ours)(a2, rank, world, dist_on, device)
+                name = sub["config"]["workload"] + ("" if direction == "forward" else "_" + direction)
+                extra[name] = (sub, cfg, direction)
+                torch.cuda.empty_cache()
         if rank == 0:
             if world == 1 and not args.skip_cpu_baseline:
                 line["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4) if args.config == 6 else
                                         cpu_baseline_ema(W.EMA, reverse=args.direction == "reverse")
                                         if args.config == 7 else
                                         cpu_baseline(args.config, direction=args.direction))
-                for sub in extra.values():
-                    cfg = next(c for c, w in W.WORKLOADS.items() if sub["config"]["workload"].startswith(w.name))
-                    sub["cpu_baseline"] = cpu_baseline(cfg, budget_s=8.0)
+                for sub, cfg, direction in extra.values():
+                    sub["cpu_baseline"] = (cpu_baseline_wkv4(W.WKV4, budget_s=8.0) if cfg == 6 else
+                                           cpu_baseline_ema(W.EMA, budget_s=8.0) if cfg == 7 else
+                                           cpu_baseline(cfg, budget_s=8.0, direction=direction))
             if extra:
+                # each record keeps its metric and unit where they differ from the headline's
                 line["configs"] = {name: {k: v for k, v in sub.items()
-                                          if k not in ("metric", "higher_is_better", "scaling", "data", "unit")}
-                                   for name, sub in extra.items()}
+                                          if k not in ("higher_is_better", "scaling", "data")
+                                          and not (k in ("metric", "unit") and v == line[k])}
+                                   for name, (sub, _, _) in extra.items()}
             print(json.dumps(line), flush=True)
     finally:
         if dist_on:
