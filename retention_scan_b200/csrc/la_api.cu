@@ -116,7 +116,8 @@ la_status check_decay(const la_decay* decay, int* kind, const float** log_g) {
 la_status scan(const void* q, const void* k, const void* v, const la_decay* decay, int normalize,
                const float* init_state, const float* init_z, void* out, float* final_state, float* final_z,
                int B, int H, int T, int Dk, int Dv, la_dtype dtype, void* workspace, size_t workspace_bytes,
-               la_stream_t stream, int reverse, int accumulate, const la_prologue* pro = nullptr) {
+               la_stream_t stream, int reverse, int accumulate, const la_prologue* pro = nullptr,
+               int states_ready = 0) {
     if (B < 0 || H < 0 || T < 0 || Dk < 1 || Dv < 1) return LA_ERR_INVALID_ARG;
     int fmap;
     float qscale;
@@ -181,6 +182,7 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
     a.accumulate = accumulate;
     a.feature_map = fmap;
     a.q_scale = qscale;
+    a.states_ready = states_ready;
     cudaError_t e;
     if (dtype == LA_F32) {
         e = la::launch_fwd_f32(a);
@@ -200,12 +202,18 @@ la_status scan(const void* q, const void* k, const void* v, const la_decay* deca
 //   decay-gradient scratch          la::dlog_scratch_doubles doubles
 //   T-segment workspace of the scans (the larger of the two key/value widths' orders)
 struct BwdLayout {
-    size_t s0t, dsft, st, lsh, dlog, scan, scan_bytes, total;
+    size_t s0t, dsft, st, lsh, dlog, scan, scan_bytes, scan2, scan2_bytes, total;
+    int shared_pieces;  // state pieces per (b, h) that the dk and dv scans share (0: none)
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind) {
+// share_states (the unnormalised backward): the dk and dv reverse scans
+// compute the same state, transposed (sum q dy^T and sum dy q^T, with the
+// same decay); when their plans cut T alike, the dv scan takes the dk scan's
+// state pieces, transposed into a second scan workspace, instead of running
+// its own state pass.
+BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int kind, bool share_states = false) {
     const size_t BH = static_cast<size_t>(B) * H;
     const size_t state = round256(sizeof(float) * BH * Dk * Dv);
     BwdLayout L{};
@@ -220,8 +228,16 @@ BwdLayout bwd_layout(int B, int H, int T, int Dk, int Dv, la_dtype dtype, int ki
         const size_t a = la::fwd_tc_workspace_bytes(B, H, T, Dv, Dk, false);  // dq, dk scans
         const size_t b = la::fwd_tc_workspace_bytes(B, H, T, Dk, Dv, false);  // dv scan
         L.scan_bytes = round256(a > b ? a : b);
+        long long key_k = 0, key_v = 0;
+        const int nk = la::fwd_tc_state_pieces(B, H, T, Dv, Dk, false, &key_k);
+        const int nv = la::fwd_tc_state_pieces(B, H, T, Dk, Dv, false, &key_v);
+        if (share_states && nk > 0 && nk == nv && key_k == key_v) {
+            L.shared_pieces = nk;
+            L.scan2_bytes = round256(b);
+        }
     }
-    L.total = L.scan + L.scan_bytes;
+    L.scan2 = L.scan + L.scan_bytes;
+    L.total = L.scan2 + L.scan2_bytes;
     return L;
 }
 
@@ -524,7 +540,7 @@ size_t la_chunk_backward_workspace_size(int B, int H, int T, int Dk, int Dv, la_
     if ((dtype != LA_F32 && dtype != LA_BF16) || B < 1 || H < 1 || T < 1 || Dk < 1 || Dv < 1) return 0;
     if (decay_kind < LA_DECAY_NONE || decay_kind > LA_DECAY_PER_STEP) return 0;
     if (!fits_int(static_cast<long long>(B) * H * 8)) return 0;
-    return bwd_layout(B, H, T, Dk, Dv, dtype, decay_kind).total;
+    return bwd_layout(B, H, T, Dk, Dv, dtype, decay_kind, true).total;
 }
 
 // dq, dk, dv by three scans on the forward and reverse scan kernels (the
@@ -554,7 +570,7 @@ la_status la_chunk_backward_ws(const void* q, const void* k, const void* v, cons
     if (dtype == LA_F32 && (Dk > 128 || Dv > 128)) return LA_ERR_UNSUPPORTED;
     if (dtype == LA_BF16 && !la::fwd_tc_supports(Dk, Dv)) return LA_ERR_UNSUPPORTED;
     if (work && (T + 255) / 256 > 65535) return LA_ERR_UNSUPPORTED;
-    const BwdLayout L = work ? bwd_layout(B, H, T, Dk, Dv, dtype, kind) : BwdLayout{};
+    const BwdLayout L = work ? bwd_layout(B, H, T, Dk, Dv, dtype, kind, true) : BwdLayout{};
     if (work && workspace_bytes < L.total) return LA_ERR_INVALID_ARG;
     if (BH == 0) return LA_OK;
     if (launch_fault_injected()) return LA_ERR_CUDA;
@@ -596,8 +612,24 @@ la_status la_chunk_backward_ws(const void* q, const void* k, const void* v, cons
              L.scan_bytes, stream, 1, 0);
     if (r != LA_OK) return r;
     // dv = reverse scan of (k, q, dy) from d_final_state; its final state is dS_1
-    r = scan(k, q, dy, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype,
-             scan_ws, L.scan_bytes, stream, 1, 0);
+    if (L.shared_pieces > 0) {
+        // its state pieces are the dk scan's ([B H][pieces][Dv][Dk], then the
+        // key sums, then the log decays), transposed, with the same log decays
+        const int np = L.shared_pieces;
+        const size_t n_s = static_cast<size_t>(BH) * np * Dk * Dv;
+        const float* from = static_cast<const float*>(scan_ws);
+        float* to = reinterpret_cast<float*>(ws + L.scan2);
+        if (!cuda_ok(la::launch_transpose(from, to, bh * np, Dv, Dk, s)) ||
+            !cuda_ok(cudaMemcpyAsync(to + n_s + static_cast<size_t>(BH) * np * Dk,
+                                     from + n_s + static_cast<size_t>(BH) * np * Dv,
+                                     sizeof(float) * static_cast<size_t>(BH) * np, cudaMemcpyDeviceToDevice, s)))
+            return LA_ERR_CUDA;
+        r = scan(k, q, dy, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype,
+                 ws + L.scan2, L.scan2_bytes, stream, 1, 0, nullptr, 1);
+    } else {
+        r = scan(k, q, dy, rdecay, 0, d_final_state, nullptr, dv, d_init_state, nullptr, B, H, T, Dk, Dv, dtype,
+                 scan_ws, L.scan_bytes, stream, 1, 0);
+    }
     if (r != LA_OK) return r;
     if (d_init_state && kind != LA_DECAY_NONE &&
         !cuda_ok(la::launch_scale_by_first_decay(d_init_state, log_g, kind, B, H, T, Dk * Dv, s)))

@@ -198,6 +198,14 @@ size_t workspace_bytes_for(int BH, int Dk, int Dv, int nS) {
 
 bool fwd_tc_supports(int Dk, int Dv) { return tensor_width_ok(Dk) && tensor_width_ok(Dv); }
 
+int fwd_tc_state_pieces(int B, int H, int T, int Dk, int Dv, bool norm, long long* plan_key) {
+    if (!fwd_tc_supports(Dk, Dv) || B <= 0 || H <= 0 || T <= 0) return 0;
+    const Layout L = plan_layout(B * H, (T + ws::C - 1) / ws::C, Dk, Dv, norm, true);
+    if (plan_key)
+        *plan_key = ((static_cast<long long>(L.nseg) * 65536 + L.seg_chunks) * 64 + L.per_seg) * 64 + L.nS;
+    return L.nS;
+}
+
 size_t fwd_tc_workspace_bytes(int B, int H, int T, int Dk, int Dv, bool norm) {
     if (!fwd_tc_supports(Dk, Dv) || B <= 0 || H <= 0 || T <= 0) return 0;
     const int BH = B * H;
@@ -359,6 +367,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
     p.q_scale = a.q_scale;
     p.feature_map = a.feature_map;
     p.pdl = kPdlFirst;
+    if (a.states_ready && L.nS == 0) return cudaErrorInvalidValue;
     if (L.nS > 0) {
         float* base = static_cast<float*>(a.workspace);
         p.ws_S = base;
@@ -366,6 +375,8 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, int* split_used, int* segments_used)
         p.ws_L = p.ws_z + static_cast<size_t>(BH) * L.nS * a.Dk;
         p.ws_nS = L.nS;
         p.ws_per_seg = L.per_seg;
+    }
+    if (L.nS > 0 && !a.states_ready) {
         // state pass: the contribution of each state segment before the last output segment
         ws::Params ps = p;
         ps.state_pass = 1;

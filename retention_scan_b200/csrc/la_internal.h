@@ -51,7 +51,15 @@ struct FwdArgs {
     int accumulate;           // 1: add y to the values already in out
     int feature_map;          // la_feature_map on q and k (forward scans)
     float q_scale;            // q <- q_scale * phi(q)
+    int states_ready;         // 1: the workspace already holds this call's state
+                              // segments (fwd_tc_state_pieces); no state pass
 };
+
+// The T-segment state pieces that launch_fwd_tc plans for these sizes with a
+// workspace (0: none): their count per (b, h), and the plan's segmentation as
+// one number that equal plans share (for reusing one scan's state pieces,
+// transposed, in another).
+int fwd_tc_state_pieces(int B, int H, int T, int Dk, int Dv, bool norm, long long* plan_key);
 
 struct DecodeArgs {
     const void* q;

@@ -252,17 +252,19 @@ def test_backward_validation(L, over, status):
 
 def test_backward_workspace_size(L):
     # S_0^T, d_final_state^T, S_T^T, the shifted decay, the decay-gradient
-    # scratch and the scans' T-segment workspace, each rounded to 256 bytes
+    # scratch and the scans' T-segment workspace, each rounded to 256 bytes,
+    # then a second scan workspace: the dk and dv scans share their state
+    # pieces (same plan), which the dv scan takes transposed
     def r(x):
         return (x + 255) // 256 * 256
     B, H, T, D = 1, 8, 8192, 64
     state = r(4 * B * H * D * D)
     nblk = (T + 255) // 256
     scan = L.la_chunk_forward_workspace_size(B, H, T, D, D, 1, 0)
-    want = 3 * state + r(4 * B * H * T) + r(8 * (B * H + 3 * B * H * nblk)) + r(scan)
+    want = 3 * state + r(4 * B * H * T) + r(8 * (B * H + 3 * B * H * nblk)) + 2 * r(scan)
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 2) == want
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 0) == want - r(4 * B * H * T)
-    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 0, 2) == want - r(scan)  # fp32: no segments
+    assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 0, 2) == want - 2 * r(scan)  # fp32: no segments
     assert L.la_chunk_backward_workspace_size(0, H, T, D, D, 1, 0) == 0
     assert L.la_chunk_backward_workspace_size(B, H, T, D, D, 1, 3) == 0
 
