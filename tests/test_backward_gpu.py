@@ -129,6 +129,17 @@ def test_backward_t_segments(kind):
     check_backward(inp, S0, dSf, seed=13)
 
 
+@pytest.mark.parametrize("Dk,Dv", [(128, 128), (64, 128), (128, 64), (32, 96)])
+def test_backward_t_segments_widths(Dk, Dv):
+    """T-segments with square and mixed widths: the dv scan reuses the dk
+    scan's state pieces (transposed) when the two plans cut T alike, and
+    runs its own state pass otherwise."""
+    inp, S0, _ = gen_case(1, 2, 4096 + 77, Dk, Dv, kind=2, init=True, seed=3310 + Dk + Dv, decay_mean=4.0)
+    dSf = torch.randn(1, 2, Dk, Dv, generator=torch.Generator().manual_seed(47))
+    assert la().workspace_size(1, 2, 4096 + 77, Dk, Dv) > 0
+    check_backward(inp, S0, dSf, seed=17)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("T", [1, 2, 129])
 def test_backward_short(dtype, T):
