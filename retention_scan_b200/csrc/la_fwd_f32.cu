@@ -5,14 +5,16 @@
 // "CS336 L04 linear attention duality" recurrent form, with the per-step
 // decay of RetNet issue 21 and the key-sum normaliser of
 // flash-linear-attention issue 268; the reverse scan is the same recurrence
-// from the last token back to the first).  The fp32 state S [Dk, Dv] lives in
-// shared memory; thread c owns value column c, so the update of column c
-// and its read-out q_t^T S_t[:, c] need no synchronisation.  Tokens are
-// staged kTile at a time: one coalesced load of the tile's q, k, v and
-// decays, then the tile's steps run without a barrier (with the normaliser,
-// the threads that own z write q_t,i z_t,i for the whole tile first and one
-// barrier later every thread sums its token's row).  No TF32: every product
-// is an fp32 FMA.
+// from the last token back to the first).  Thread c owns value column c of
+// the fp32 state S [Dk, Dv] and holds it in registers (the key width padded
+// to a compile-time bound), so the update of column c and its read-out
+// q_t^T S_t[:, c] touch no shared memory and need no synchronisation; the
+// read-out's sum runs as four interleaved chains.  Tokens are staged kTile
+// at a time: one coalesced load of the tile's q, k, v and decays, then the
+// tile's steps run without a barrier (with the normaliser, the threads that
+// own z write q_t,i z_t,i for the whole tile first and one barrier later
+// every thread sums its token's row).  No TF32: every product is an fp32
+// FMA.
 #include <cuda_runtime.h>
 
 #include "la_internal.h"
@@ -28,6 +30,7 @@ __device__ __forceinline__ float feature(float x, int fmap) {
     return fmap == LA_FEATURE_ELU1 ? (x > 0.f ? x + 1.f : expf(x)) : x;
 }
 
+template <int DKP>
 __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     int decay_kind, const float* __restrict__ log_g, int normalize,
@@ -35,22 +38,23 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
     float* __restrict__ out, float* __restrict__ final_state, float* __restrict__ final_z,
     int H, int T, int Dk, int Dv, int reverse, int accumulate, int fmap, float qscale) {
     extern __shared__ float smem[];
-    float* S = smem;                    // [Dk][Dv]
-    float* qs = S + Dk * Dv;            // [kTile][Dk]
+    float* qs = smem;                   // [kTile][Dk]
     float* ks = qs + kTile * Dk;        // [kTile][Dk]
     float* vs = ks + kTile * Dk;        // [kTile][Dv]
     float* gs = vs + kTile * Dv;        // [kTile]
-    float* zs = gs + kTile;             // [Dk]
-    float* qz = zs + Dk;                // [kTile][Dk]: q_t,i z_t,i (normaliser only)
+    float* qz = gs + kTile;             // [kTile][Dk]: q_t,i z_t,i (normaliser only)
 
     const int bh = blockIdx.x;
     const int h = bh % H;
     const int tid = threadIdx.x;
+    const bool own = tid < Dv;  // thread c owns value column c
     const size_t sq = static_cast<size_t>(bh) * T * Dk;
     const size_t sv = static_cast<size_t>(bh) * T * Dv;
+    const size_t s0 = static_cast<size_t>(bh) * Dk * Dv;
 
-    for (int e = tid; e < Dk * Dv; e += kThreads)
-        S[e] = init_state ? init_state[static_cast<size_t>(bh) * Dk * Dv + e] : 0.f;
+    float S[DKP];  // S[i][tid], i < Dk
+#pragma unroll
+    for (int i = 0; i < DKP; ++i) S[i] = (own && i < Dk && init_state) ? init_state[s0 + static_cast<size_t>(i) * Dv + tid] : 0.f;
     float zi = 0.f;  // z_i, owned by thread i < Dk
     if (normalize && init_z && tid < Dk) zi = init_z[static_cast<size_t>(bh) * Dk + tid];
     const float g_head = decay_kind == LA_DECAY_PER_HEAD ? expf(log_g[h]) : 1.f;
@@ -78,24 +82,25 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
                 }
             __syncthreads();
         }
-        // thread c owns value column c (Dv <= kThreads)
-        if (tid < Dv) {
+        if (own) {
             for (int jj = 0; jj < nt; ++jj) {
                 const int j = reverse ? nt - 1 - jj : jj;
                 const float vc = vs[j * Dv + tid], g = gs[j];
                 const float* qj = qs + j * Dk;
                 const float* kj = ks + j * Dk;
-                float num = 0.f;
-                for (int i = 0; i < Dk; ++i) {
-                    const float s = fmaf(kj[i], vc, g * S[i * Dv + tid]);
-                    S[i * Dv + tid] = s;
-                    num = fmaf(qj[i], s, num);
+                float num[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < DKP; ++i) {
+                    if (i < Dk) {
+                        S[i] = fmaf(kj[i], vc, g * S[i]);
+                        num[i & 3] = fmaf(qj[i], S[i], num[i & 3]);
+                    }
                 }
-                float y = num;
+                float y = (num[0] + num[1]) + (num[2] + num[3]);
                 if (normalize) {
                     float den = 0.f;
                     for (int i = 0; i < Dk; ++i) den += qz[j * Dk + i];
-                    y = num / den;
+                    y = y / den;
                 }
                 if (out) {  // (null: the state alone, la_chunk_state_ws)
                     float* o = out + sv + static_cast<size_t>(t0 + j) * Dv + tid;
@@ -104,26 +109,34 @@ __global__ void __launch_bounds__(kThreads) fwd_f32_kernel(
             }
         }
     }
-    __syncthreads();
-    if (final_state)
-        for (int e = tid; e < Dk * Dv; e += kThreads)
-            final_state[static_cast<size_t>(bh) * Dk * Dv + e] = S[e];
+    if (final_state && own)
+#pragma unroll
+        for (int i = 0; i < DKP; ++i)
+            if (i < Dk) final_state[s0 + static_cast<size_t>(i) * Dv + tid] = S[i];
     if (final_z && normalize && tid < Dk) final_z[static_cast<size_t>(bh) * Dk + tid] = zi;
+}
+
+template <int DKP>
+cudaError_t launch_f32(const FwdArgs& a) {
+    const size_t smem = sizeof(float) * (3 * kTile * static_cast<size_t>(a.Dk) + kTile * a.Dv + kTile);
+    cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<DKP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    fwd_f32_kernel<DKP><<<a.B * a.H, kThreads, smem, a.stream>>>(
+        static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
+        a.decay_kind, a.log_g, a.normalize, a.init_state, a.init_z, static_cast<float*>(a.out),
+        a.final_state, a.final_z, a.H, a.T, a.Dk, a.Dv, a.reverse, a.accumulate, a.feature_map, a.q_scale);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_f32(const FwdArgs& a) {
-    const size_t smem = sizeof(float) * (static_cast<size_t>(a.Dk) * a.Dv + 3 * kTile * a.Dk +
-                                         kTile * a.Dv + kTile + a.Dk);
-    cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    fwd_f32_kernel<<<a.B * a.H, kThreads, smem, a.stream>>>(
-        static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
-        a.decay_kind, a.log_g, a.normalize, a.init_state, a.init_z, static_cast<float*>(a.out),
-        a.final_state, a.final_z, a.H, a.T, a.Dk, a.Dv, a.reverse, a.accumulate, a.feature_map, a.q_scale);
-    return cudaGetLastError();
+    // the state column's registers: the key width padded to 16, 32, 64 or 128
+    if (a.Dk <= 16) return launch_f32<16>(a);
+    if (a.Dk <= 32) return launch_f32<32>(a);
+    if (a.Dk <= 64) return launch_f32<64>(a);
+    return launch_f32<128>(a);
 }
 
 }  // namespace la
