@@ -363,9 +363,10 @@ LA_API size_t la_chunk_backward_workspace_size(int B, int H, int T, int Dk, int 
  *                  aligned, used on `stream` only.  Required (for T > 0).
  *
  * Several launches on `stream`: three scans (each possibly a state pass and
- * an output pass) and small kernels for the transposed carried states, the
- * shifted decay, d_init_state and d_log_g.  Outputs must not overlap inputs
- * or each other.
+ * an output pass; the dv scan takes the dk scan's state pieces, transposed,
+ * when the two scans cut T alike) and small kernels for the transposed
+ * carried states, the shifted decay, d_init_state and d_log_g.  Outputs must
+ * not overlap inputs or each other.
  *
  * Errors: as la_chunk_forward_ws, plus LA_ERR_INVALID_ARG for a NULL
  * required pointer (dy, dq, dk, dv, workspace), a workspace smaller than
