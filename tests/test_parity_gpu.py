@@ -224,15 +224,17 @@ def test_segments_with_value_split(monkeypatch, split):
 
 
 @pytest.mark.parametrize("decay_mean", [1.0, -30.0])
-def test_segments_direct_form(monkeypatch, decay_mean):
+@pytest.mark.parametrize("D,normalize", [(64, True), (128, False), (128, True)])
+def test_segments_direct_form(monkeypatch, decay_mean, D, normalize):
     # chunks whose total decay passes the fold limit run in the direct form,
-    # in the state pass too (there the key rows are decayed by the prep warps)
+    # in the state pass too (there the key rows are decayed by the prep warps;
+    # at D = 128 the state pass is its own instance of one 128-column slice)
     monkeypatch.setenv("LA_SEGMENTS", "4")
-    inp, S0, z0 = gen_case(1, 2, 1024, 64, 64, kind=2, normalize=True, init=True, seed=920,
+    inp, S0, z0 = gen_case(1, 2, 1024, D, D, kind=2, normalize=normalize, init=True, seed=920 + D,
                            decay_mean=decay_mean)
     if decay_mean < 0:
         inp["log_g"] = torch.full_like(inp["log_g"], decay_mean)
-    check_case(inp, True, S0, z0)
+    check_case(inp, normalize, S0, z0)
 
 
 @pytest.mark.parametrize("Dk,Dv", [(48, 112), (80, 48), (112, 80)])

@@ -111,14 +111,27 @@ def test_reverse_segments(monkeypatch, nseg, kind, normalize):
 
 @pytest.mark.parametrize("decay_mean", [1.0, -30.0])
 @pytest.mark.parametrize("nseg", [1, 4])
-def test_reverse_direct_form(monkeypatch, decay_mean, nseg):
-    # chunks whose total decay passes the fold limit take the direct form
+@pytest.mark.parametrize("D", [64, 128])
+def test_reverse_direct_form(monkeypatch, decay_mean, nseg, D):
+    # chunks whose total decay passes the fold limit take the direct form (at
+    # D = 128 with segments, in the state pass's one 128-column slice too)
     monkeypatch.setenv("LA_SEGMENTS", str(nseg))
-    inp, S0, z0 = gen_case(1, 2, 1000, 64, 64, kind=2, normalize=True, init=True, seed=2600 + nseg,
+    inp, S0, z0 = gen_case(1, 2, 1000, D, D, kind=2, normalize=True, init=True, seed=2600 + nseg + D,
                            decay_mean=decay_mean)
     if decay_mean < 0:
         inp["log_g"] = torch.full_like(inp["log_g"], decay_mean)
     check_reverse(inp, True, S0, z0)
+
+
+@pytest.mark.parametrize("nseg", [2, 4])
+@pytest.mark.parametrize("normalize", [False, True])
+def test_reverse_segments_d128(monkeypatch, nseg, normalize):
+    # the reverse scan's state pass as one 128-column slice (the output pass
+    # in two 64-column slices)
+    monkeypatch.setenv("LA_SEGMENTS", str(nseg))
+    inp, S0, z0 = gen_case(1, 2, 1100, 128, 128, kind=2, normalize=normalize, init=True,
+                           seed=2700 + nseg * 2 + normalize)
+    check_reverse(inp, normalize, S0, z0)
 
 
 def test_reverse_is_forward_of_flipped_inputs():
